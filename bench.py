@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Selective-scan forward benchmark on B200: Gelem/s (elements = batch*L*D) and the
+achieved fraction of the HBM / MUFU roofline at the Mamba-2.8B layer shape
+(batch 8, L 2048, D 5120, N 16, bf16 I/O, fp32 state), on seeded synthetic inputs.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1).  Each rank runs its own replica of the
+workload (the scan has no cross-rank step), so per-GPU work is fixed: weak scaling.
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle on the
+host cores instead (the reference arm: a plain sequential scan, never tuned).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_33_b200 import workloads as W  # noqa: E402
+
+METRIC = "selective-scan fwd Gelem/s (B·L·D) & % of HBM/MUFU roofline at 2.8B-layer shape"
+UNIT = "Gelem/s"
+DEFAULT_WORKLOAD = "mamba2.8b"
+SM_COUNT = 148
+MUFU_PER_SM_CLK = 16          # ex2 results per SM per clock (4 per sub-partition)
+HBM_FALLBACK_GBS = 6650.0     # used only when MEASURED_PEAKS.json is absent
+
+
+# ----------------------------------------------------------------------------- ranks
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    world, rank, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a scalar over all ranks (the step time every rank waits for)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(elements_per_rank_step: int, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job throughput in Gelem/s: every rank's elements over the slowest rank's time."""
+    return elements_per_rank_step * steps * world / max_seconds / 1e9
+
+
+# ----------------------------------------------------------------------------- model
+def roofline_units(w: W.Workload) -> dict:
+    """Algorithmic bytes and exponentials of one forward pass.
+
+    bytes: read u, delta_raw, z and write out (4 * E * s), read B and C
+    (2 * batch * L * N * s), read A, bias, D_skip once (fp32); the (batch, L, D, N)
+    state is never moved (the method keeps it on chip).
+    exps: N per element for Abar = exp(delta A), plus one for softplus and one for
+    the SiLU gate (Bbar reuses Abar's exponential)."""
+    s = 2 if w.io == "bf16" else 4
+    E = w.batch * w.seqlen * w.dim
+    bytes_ = 4 * E * s + 2 * w.batch * w.seqlen * w.dstate * s + (w.dim * w.dstate + 2 * w.dim) * 4
+    return {"elements": E, "bytes": bytes_, "exps": E * (w.dstate + 2)}
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f)
+    return {}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of this GPU's SM clock and throttle reasons every 200 ms."""
+
+    FIELDS = ["uuid", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [[c.strip() for c in line.split(",")] for line in self.file if line.strip()]
+        self.file.close()
+        os.unlink(self.file.name)
+        mine = [r for r in rows if len(r) == len(self.FIELDS) and (not self.uuid or r[0] == self.uuid)]
+        sm = [float(r[1]) for r in mine if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in mine if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        for r in mine:
+            for name, col in (("hw_slowdown", 5), ("hw_thermal_slowdown", 6), ("sw_thermal_slowdown", 7),
+                              ("sw_power_cap", 8)):
+                if r[col].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(mine)}
+
+
+# ----------------------------------------------------------------------------- CPU arms
+def cpu_oracle_rate(x: dict, w: W.Workload, target_s: float, seed: int = 0):
+    """Time the fp64 oracle on a random sample of (batch, channel) rows, each the full
+    sequence; the sample is sized for about ``target_s`` seconds.  Returns
+    (Gelem/s, threads, rows, seconds)."""
+    import oracle
+    threads = oracle.set_threads(0)
+    rng = np.random.default_rng(seed)
+    total_rows = w.batch * w.dim
+
+    def run(k):
+        rows = np.sort(rng.choice(total_rows, size=k, replace=False))
+        t0 = time.perf_counter()
+        oracle.fwd(x["u"], x["delta_raw"], x["A"], x["B"], x["C"], delta_bias=x["delta_bias"],
+                   D_skip=x["D_skip"], z=x.get("z"), rows=rows)
+        return time.perf_counter() - t0
+
+    k0 = min(total_rows, 8 * threads)
+    dt0 = run(k0)
+    k = int(min(total_rows, max(k0, k0 * target_s / max(dt0, 1e-6))))
+    dt = run(k)
+    return k * w.seqlen / dt / 1e9, threads, k, dt
+
+
+def reference_arm(args, w: W.Workload):
+    """The oracle as it stands, timed on the host cores: K timed steps (after W
+    warm-up steps), each a bounded random sample of the workload's rows."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    x = W.make_inputs(w)
+    threads = oracle.set_threads(0)
+    total_rows = w.batch * w.dim
+    rng = np.random.default_rng(1234)
+    rate0, _, _, _ = cpu_oracle_rate(x, w, 2.0)
+    per_step_rows = int(min(total_rows, max(threads, rate0 * 1e9 * 4.0 / w.seqlen)))  # ~4 s per step
+
+    def step():
+        rows = np.sort(rng.choice(total_rows, size=per_step_rows, replace=False))
+        oracle.fwd(x["u"], x["delta_raw"], x["A"], x["B"], x["C"], delta_bias=x["delta_bias"],
+                   D_skip=x["D_skip"], z=x.get("z"), rows=rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = per_step_rows * w.seqlen * args.steps / dt / 1e9
+    sample = f"{per_step_rows} random rows x L={w.seqlen} per step ({per_step_rows * w.seqlen} elements)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def workload_config(w: W.Workload, world: int) -> dict:
+    return {"workload": f"{w.name}: {w.description}", "batch": w.batch, "seq_len": w.seqlen,
+            "d_inner": w.dim, "d_state": w.dstate, "io_dtype": w.io, "state_dtype": "f32",
+            "global_batch": w.batch * world, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (no flush needed)"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def ex2_probe(torch, lib, device, repeats=5):
+    """Measured MUFU ex2 rate (exps/s) of the whole GPU."""
+    import ctypes
+    blocks, threads, iters = SM_COUNT * 8, 256, 4096
+    sink = torch.empty(blocks * threads, dtype=torch.float32, device=device)
+    st = torch.cuda.current_stream()
+    lib.sscan_probe_ex2.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    lib.sscan_probe_ex2.restype = ctypes.c_int
+    best = None
+    for _ in range(repeats):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        rc = lib.sscan_probe_ex2(ctypes.c_void_p(sink.data_ptr()), iters, blocks, threads,
+                                 ctypes.c_void_p(st.cuda_stream))
+        b.record(st)
+        if rc != 0:
+            return None
+        b.synchronize()
+        ms = a.elapsed_time(b)
+        best = ms if best is None else min(best, ms)
+    return blocks * threads * 8 * iters / (best * 1e-3)
+
+
+def gpu_arm(args, w: W.Workload):
+    import torch
+
+    from selective_state_space_33_b200 import binding as sb
+    world, rank = init_dist("nccl" if int(os.environ.get("WORLD_SIZE", "1")) > 1 else "gloo")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lib = sb.load_library()
+
+    x = W.make_inputs(w.with_(seed=w.seed + rank)) if world > 1 else W.make_inputs(w)
+    t = W.to_device(x, dev)
+    out = torch.empty_like(t["u"])
+    prob = sb.make_problem(w.batch, w.seqlen, w.dim, w.dstate, sb.SSCAN_BF16 if w.io == "bf16" else sb.SSCAN_F32)
+    ws_bytes = sb.sscan_workspace_size(prob, sb.SSCAN_OP_FWD)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+
+    def step():
+        sb.sscan_fwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["delta_bias"], t["D_skip"], t.get("z"),
+                     out=out, workspace=ws, stream=st)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    uuid = ""
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    time.sleep(0.4)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        starts[i].record(st)
+        step()
+        ends[i].record(st)
+    torch.cuda.synchronize()
+    barrier()
+    # keep the GPU busy while the sampler takes a few more readings under load
+    for _ in range(max(1, int(0.6 / max(starts[0].elapsed_time(ends[0]) * 1e-3, 1e-4)))):
+        step()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    per_launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_s = starts[0].elapsed_time(ends[-1]) * 1e-3
+    max_s = reduce_max(total_s, dev if world > 1 else None)
+    units = roofline_units(w)
+    value = aggregate(units["elements"], args.steps, world, max_s)
+
+    # end to end through the C ABI from pinned host buffers: H2D inputs, scan, D2H output
+    host = {k: v.cpu().pin_memory() for k, v in t.items()}
+    dev_in = {k: torch.empty_like(v) for k, v in t.items()}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for k in host:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        sb.sscan_fwd(dev_in["u"], dev_in["delta_raw"], dev_in["A"], dev_in["B"], dev_in["C"], dev_in["delta_bias"],
+                     dev_in["D_skip"], dev_in.get("z"), out=out, workspace=ws, stream=st)
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(st)
+    for _ in range(args.steps):
+        e2e_step()
+    eb.record(st)
+    torch.cuda.synchronize()
+    e2e_s = reduce_max(ea.elapsed_time(eb) * 1e-3, dev if world > 1 else None)
+    e2e_value = aggregate(units["elements"], args.steps, world, e2e_s)
+
+    if rank != 0:
+        return
+    peaks = measured_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", HBM_FALLBACK_GBS))
+    hbm_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    mufu_nominal = SM_COUNT * MUFU_PER_SM_CLK * sm_max * 1e6
+    mufu_probe = ex2_probe(torch, lib, dev)
+    launch_s = statistics.mean(per_launch_ms) * 1e-3
+    exps_rate = units["exps"] / launch_s
+    gbs = units["bytes"] / launch_s / 1e9
+    t_roof = max(units["bytes"] / (hbm_peak * 1e9), units["exps"] / mufu_nominal)
+    launches_per_step = 1 if ws_bytes == 0 else 3
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rate, cores, rows, secs = cpu_oracle_rate(x, w, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{rows} random rows of {w.batch * w.dim} x L={w.seqlen} ({rows * w.seqlen} elements, "
+                         f"{secs:.1f} s)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": max_s / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w, world),
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "roofline": {
+            "bound": "alu", "pipe": "MUFU ex2", "achieved": exps_rate / 1e9, "peak": mufu_nominal / 1e9,
+            "unit": "Gexp/s", "frac": exps_rate / mufu_nominal, "traffic": None,
+            "peak_source": f"derived: {SM_COUNT} SMs x {MUFU_PER_SM_CLK} ex2/clk x {sm_max:.0f} MHz",
+            "peak_probe_gexps": None if mufu_probe is None else mufu_probe / 1e9,
+            "frac_of_probe": None if mufu_probe is None else exps_rate / mufu_probe,
+            "hbm": {"achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                    "source": hbm_src},
+            "roofline_frac": t_roof / launch_s,
+            "per_launch_ms": launch_s * 1e3,
+            "alg_bytes_per_launch": units["bytes"], "alg_exps_per_launch": units["exps"],
+        },
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        reference_arm(args, w)
+    else:
+        gpu_arm(args, w)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,137 @@
+/*
+ * sscan.h -- C ABI of libsscan, a B200 (sm_100a) implementation of the selective
+ * state-space scan (S6) from "Mamba: Linear-Time Sequence Modeling with Selective
+ * State Spaces" (Gu & Dao, 2023).
+ *
+ * The operation (technical summary page "Mamba 状态空间模型原理与 Transformer 对比",
+ * kb.agiseed.tech, sec. 2.1 eqs. (2), (3a), (3b); sec. 3.2; sec. 4.1; Fig. 3):
+ *   delta_t = softplus(delta_raw_t + delta_bias_d)     (flag SSCAN_DELTA_SOFTPLUS,
+ *                                                        else delta_raw_t + bias_d)
+ *   Abar_tn = exp(delta_t A_dn)                          eq. (2)
+ *   Bbar_tn = expm1(delta_t A_dn) / A_dn * B_tn          eq. (2), diagonal A;
+ *                                                        the limit delta_t B_tn at A_dn = 0
+ *   h_tn    = Abar_tn h_{t-1,n} + Bbar_tn x_t            eq. (3a), x = u
+ *   y_t     = sum_n C_tn h_tn + D_skip_d x_t             eq. (3b) plus a skip term
+ *   out_t   = y_t * SiLU(z_t)                            Fig. 3 gate (when z is given)
+ * for every batch b and channel d independently; h_{-1} = h0 (zero when NULL).
+ * The (batch, L, D, N) state is never written to memory (sec. 4.1).
+ *
+ * Layouts (dense, row-major, no padding):
+ *   u, delta_raw, z, out, du, ddelta_raw, dz, dout : (batch, L, D)
+ *   B, C, dB, dC                                    : (batch, L, N), shared by all D channels
+ *   A, dA                                           : (D, N)
+ *   delta_bias, D_skip, ddelta_bias, dD             : (D)
+ *   h0, h_last, dh0                                 : (batch, D, N)
+ * Element types: the tensors in the first two rows (and their gradients) use
+ * problem->io_dtype (fp32 or bf16); A, delta_bias, D_skip, states and their
+ * gradients are always fp32.  All arithmetic is fp32; bf16 results are rounded
+ * to nearest-even once.
+ *
+ * Ownership and execution: every pointer is a device pointer owned by the caller
+ * (except `problem`, a host pointer read during the call).  The library never
+ * allocates, frees or synchronises; it enqueues its kernels on `stream` (a
+ * cudaStream_t, NULL = legacy default stream) and returns.  Outputs are
+ * overwritten, never accumulated into.  Inputs must not alias outputs.
+ *
+ * Errors: arguments are checked on the host before anything is launched; a
+ * rejected call returns a non-zero status and enqueues nothing.  Launch failures
+ * return SSCAN_ERR_CUDA.  sscan_last_error() gives a one-line reason for the most
+ * recent failure on the calling thread.
+ */
+#ifndef SSCAN_H
+#define SSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSCAN_API __attribute__((visibility("default")))
+#else
+#define SSCAN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sscan_status {
+    SSCAN_OK = 0,
+    SSCAN_ERR_INVALID_ARG = 1, /* NULL required pointer, negative size, unknown dtype or flag */
+    SSCAN_ERR_UNSUPPORTED = 2, /* a well-formed problem this build does not handle (dstate > 16) */
+    SSCAN_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than sscan_workspace_size() */
+    SSCAN_ERR_CUDA = 4         /* a CUDA runtime call or kernel launch failed */
+} sscan_status;
+
+typedef enum sscan_dtype { SSCAN_F32 = 0, SSCAN_BF16 = 1 } sscan_dtype;
+
+/* problem->flags */
+#define SSCAN_DELTA_SOFTPLUS 1u
+
+typedef struct sscan_problem {
+    int64_t batch;    /* >= 0 */
+    int64_t seqlen;   /* L >= 0 */
+    int64_t dim;      /* D >= 0, channels */
+    int64_t dstate;   /* N, 1..16 */
+    int32_t io_dtype; /* sscan_dtype of the (batch,L,D) and (batch,L,N) tensors */
+    uint32_t flags;   /* SSCAN_DELTA_SOFTPLUS or 0 */
+} sscan_problem;
+
+typedef enum sscan_op { SSCAN_OP_FWD = 0, SSCAN_OP_LAST_STATE = 1, SSCAN_OP_BWD = 2 } sscan_op;
+
+/* Bytes of device workspace the operation needs for this problem (0 when none).
+ * The size depends only on the problem and the op.  Returns 0 for an invalid
+ * problem (the operation itself then reports the error). */
+SSCAN_API size_t sscan_workspace_size(const sscan_problem* problem, int op);
+
+/*
+ * Forward scan: writes out (batch, L, D) in io_dtype and, when h_last is not
+ * NULL, the final state h_{L-1} (batch, D, N) fp32.  delta_bias, D_skip, z and h0
+ * may be NULL (zero bias, no skip term, no gate, zero initial state).  out may be
+ * NULL only if h_last is not (that is the last-state operation).
+ * Sec. 2.1 eqs. (2)-(3), sec. 3.2, sec. 4.1, Fig. 3 of the page cited above.
+ */
+SSCAN_API sscan_status sscan_fwd(const sscan_problem* problem, const void* u, const void* delta_raw,
+                       const float* delta_bias, const float* A, const void* B, const void* C,
+                       const float* D_skip, const void* z, const float* h0, void* out,
+                       float* h_last, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Final state only: h_last = h_{L-1} (batch, D, N) fp32, without reading C or z
+ * and without writing any (batch, L, D) output.  With h0 this chains sequence
+ * segments: running [0,k) then [k,L) from its h_last equals one run over [0,L)
+ * (eq. (3a) is a recurrence; sec. 5: constant-size state for generation).
+ */
+SSCAN_API sscan_status sscan_last_state(const sscan_problem* problem, const void* u, const void* delta_raw,
+                              const float* delta_bias, const float* A, const void* B,
+                              const float* h0, float* h_last, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
+ * Backward scan: gradients of sum(out * dout) with respect to every input of
+ * sscan_fwd, recomputing the states on chip instead of storing them (sec. 4.1,
+ * item 3).  du, ddelta_raw, dB, dC (and dz) are in io_dtype; dA, ddelta_bias, dD,
+ * dh0 are fp32.  ddelta_bias, dD, dz and dh0 may be NULL when not wanted; dz must
+ * be given exactly when z is, dD only when D_skip is.  The argument list of the
+ * forward pass must be repeated exactly as it was given to sscan_fwd.
+ */
+SSCAN_API sscan_status sscan_bwd(const sscan_problem* problem, const void* u, const void* delta_raw,
+                       const float* delta_bias, const float* A, const void* B, const void* C,
+                       const float* D_skip, const void* z, const float* h0, const void* dout,
+                       void* du, void* ddelta_raw, float* ddelta_bias, float* dA, void* dB,
+                       void* dC, float* dD, void* dz, float* dh0, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Static, human-readable name of a status code. */
+SSCAN_API const char* sscan_status_string(sscan_status status);
+
+/* One-line reason for the most recent failed call on this thread ("" if none). */
+SSCAN_API const char* sscan_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+SSCAN_API int sscan_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSCAN_H */

@@ -1,0 +1,200 @@
+"""Thin Python binding of libsscan (include/sscan.h): argument marshalling only.
+
+Each function takes CUDA ``torch.Tensor``s, checks their dtypes, shapes and
+contiguity, allocates any output or workspace the caller did not pass (PyTorch
+is the allocator), and calls the C function of the same name on the current
+CUDA stream.  All arithmetic runs in the library's kernels; there is no CPU or
+PyTorch fallback, and a missing library is an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsscan.so")
+
+SSCAN_F32, SSCAN_BF16 = 0, 1
+SSCAN_DELTA_SOFTPLUS = 1
+SSCAN_OP_FWD, SSCAN_OP_LAST_STATE, SSCAN_OP_BWD = 0, 1, 2
+
+_IO_CODES = {torch.float32: SSCAN_F32, torch.bfloat16: SSCAN_BF16}
+_lib = None
+
+
+class SscanError(RuntimeError):
+    """A libsscan call returned a non-zero sscan_status."""
+
+    def __init__(self, status: int, name: str, detail: str):
+        super().__init__(f"{name}: {detail}" if detail else name)
+        self.status = status
+        self.name = name
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("dim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("io_dtype", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libsscan.so (built in-tree by ``selective_state_space_33_b200/build.py``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise SscanError(-1, "SSCAN_LIBRARY_MISSING",
+                         f"{p} not found; build it with python selective_state_space_33_b200/build.py")
+    lib = ctypes.CDLL(p)
+    vp, sz, pp = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(Problem)
+    lib.sscan_workspace_size.argtypes = [pp, ctypes.c_int]
+    lib.sscan_workspace_size.restype = sz
+    lib.sscan_fwd.argtypes = [pp] + [vp] * 12 + [sz, vp]
+    lib.sscan_fwd.restype = ctypes.c_int
+    lib.sscan_last_state.argtypes = [pp] + [vp] * 8 + [sz, vp]
+    lib.sscan_last_state.restype = ctypes.c_int
+    lib.sscan_bwd.argtypes = [pp] + [vp] * 20 + [sz, vp]
+    lib.sscan_bwd.restype = ctypes.c_int
+    lib.sscan_status_string.argtypes = [ctypes.c_int]
+    lib.sscan_status_string.restype = ctypes.c_char_p
+    lib.sscan_last_error.argtypes = []
+    lib.sscan_last_error.restype = ctypes.c_char_p
+    lib.sscan_version.argtypes = []
+    lib.sscan_version.restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != 0:
+        lib = load_library()
+        raise SscanError(status, lib.sscan_status_string(status).decode(), lib.sscan_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_problem(batch, seqlen, dim, dstate, io_dtype, delta_softplus=True) -> Problem:
+    return Problem(int(batch), int(seqlen), int(dim), int(dstate), int(io_dtype),
+                   SSCAN_DELTA_SOFTPLUS if delta_softplus else 0)
+
+
+def _io_problem(u, B, delta_softplus):
+    if u.dim() != 3 or B.dim() != 3:
+        raise ValueError("u must be (batch, L, D) and B (batch, L, N)")
+    if u.dtype not in _IO_CODES:
+        raise TypeError(f"I/O tensors must be float32 or bfloat16, got {u.dtype}")
+    batch, L, D = u.shape
+    if B.shape[0] != batch or B.shape[1] != L:
+        raise ValueError(f"B has shape {tuple(B.shape)}, expected ({batch}, {L}, N)")
+    return make_problem(batch, L, D, B.shape[2], _IO_CODES[u.dtype], delta_softplus)
+
+
+def _expect(t, name, shape, dtype, device):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def sscan_workspace_size(problem: Problem, op: int) -> int:
+    return int(load_library().sscan_workspace_size(ctypes.byref(problem), int(op)))
+
+
+def _workspace(problem, op, workspace, device):
+    need = sscan_workspace_size(problem, op)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return workspace, nbytes
+
+
+def _check_inputs(prob, u, delta_raw, A, B, C, delta_bias, D_skip, z, h0):
+    dev, io = u.device, u.dtype
+    if dev.type != "cuda":
+        raise ValueError("libsscan works on CUDA tensors only")
+    bld, bln = (prob.batch, prob.seqlen, prob.dim), (prob.batch, prob.seqlen, prob.dstate)
+    _expect(u, "u", bld, io, dev)
+    _expect(delta_raw, "delta_raw", bld, io, dev)
+    _expect(B, "B", bln, io, dev)
+    _expect(C, "C", bln, io, dev)
+    _expect(z, "z", bld, io, dev)
+    _expect(A, "A", (prob.dim, prob.dstate), torch.float32, dev)
+    _expect(delta_bias, "delta_bias", (prob.dim,), torch.float32, dev)
+    _expect(D_skip, "D_skip", (prob.dim,), torch.float32, dev)
+    _expect(h0, "h0", (prob.batch, prob.dim, prob.dstate), torch.float32, dev)
+
+
+def sscan_fwd(u, delta_raw, A, B, C, delta_bias=None, D_skip=None, z=None, h0=None, *,
+              delta_softplus=True, out=None, h_last=None, return_last_state=False,
+              workspace=None, stream=None):
+    """Forward selective scan.  Returns ``out`` or ``(out, h_last)``."""
+    prob = _io_problem(u, B, delta_softplus)
+    _check_inputs(prob, u, delta_raw, A, B, C, delta_bias, D_skip, z, h0)
+    if out is None:
+        out = torch.empty_like(u)
+    _expect(out, "out", u.shape, u.dtype, u.device)
+    if return_last_state and h_last is None:
+        h_last = torch.empty((prob.batch, prob.dim, prob.dstate), dtype=torch.float32, device=u.device)
+    _expect(h_last, "h_last", (prob.batch, prob.dim, prob.dstate), torch.float32, u.device)
+    ws, nbytes = _workspace(prob, SSCAN_OP_FWD, workspace, u.device)
+    _check(load_library().sscan_fwd(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias),
+                                    _ptr(A), _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h0),
+                                    _ptr(out), _ptr(h_last), _ptr(ws), nbytes, _stream(stream)))
+    return (out, h_last) if (return_last_state or h_last is not None) else out
+
+
+def sscan_last_state(u, delta_raw, A, B, delta_bias=None, h0=None, *, delta_softplus=True,
+                     h_last=None, workspace=None, stream=None):
+    """Final state h_{L-1} (batch, D, N) only."""
+    prob = _io_problem(u, B, delta_softplus)
+    _check_inputs(prob, u, delta_raw, A, B, None, delta_bias, None, None, h0)
+    if h_last is None:
+        h_last = torch.empty((prob.batch, prob.dim, prob.dstate), dtype=torch.float32, device=u.device)
+    _expect(h_last, "h_last", (prob.batch, prob.dim, prob.dstate), torch.float32, u.device)
+    ws, nbytes = _workspace(prob, SSCAN_OP_LAST_STATE, workspace, u.device)
+    _check(load_library().sscan_last_state(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias),
+                                           _ptr(A), _ptr(B), _ptr(h0), _ptr(h_last), _ptr(ws), nbytes,
+                                           _stream(stream)))
+    return h_last
+
+
+def sscan_bwd(u, delta_raw, A, B, C, dout, delta_bias=None, D_skip=None, z=None, h0=None, *,
+              delta_softplus=True, want_dh0=True, workspace=None, stream=None):
+    """Gradients of sum(out * dout).  Returns a dict keyed du, ddelta_raw, dA, dB, dC and,
+    when the matching input is given, ddelta_bias, dD, dz; dh0 when ``want_dh0``."""
+    prob = _io_problem(u, B, delta_softplus)
+    _check_inputs(prob, u, delta_raw, A, B, C, delta_bias, D_skip, z, h0)
+    _expect(dout, "dout", u.shape, u.dtype, u.device)
+    f32 = dict(dtype=torch.float32, device=u.device)
+    g = {"du": torch.empty_like(u), "ddelta_raw": torch.empty_like(u),
+         "dA": torch.empty((prob.dim, prob.dstate), **f32), "dB": torch.empty_like(B),
+         "dC": torch.empty_like(C)}
+    g["ddelta_bias"] = torch.empty(prob.dim, **f32) if delta_bias is not None else None
+    g["dD"] = torch.empty(prob.dim, **f32) if D_skip is not None else None
+    g["dz"] = torch.empty_like(u) if z is not None else None
+    g["dh0"] = torch.empty((prob.batch, prob.dim, prob.dstate), **f32) if want_dh0 else None
+    ws, nbytes = _workspace(prob, SSCAN_OP_BWD, workspace, u.device)
+    _check(load_library().sscan_bwd(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias), _ptr(A),
+                                    _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h0), _ptr(dout),
+                                    _ptr(g["du"]), _ptr(g["ddelta_raw"]), _ptr(g["ddelta_bias"]),
+                                    _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]),
+                                    _ptr(g["dz"]), _ptr(g["dh0"]), _ptr(ws), nbytes, _stream(stream)))
+    return {k: v for k, v in g.items() if v is not None}

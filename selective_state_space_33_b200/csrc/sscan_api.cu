@@ -1,0 +1,297 @@
+// sscan_api.cu -- the C ABI of libsscan (declared in include/sscan.h): argument
+// checks, workspace planning and kernel dispatch.  Everything is enqueued on the
+// caller's stream; nothing here allocates, frees or synchronises.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+
+#include "sscan.h"
+#include "sscan_generic.cuh"
+#include "sscan_generic_bwd.cuh"
+#include "sscan_plan.h"
+
+namespace {
+
+thread_local char g_err[256] = "";
+
+sscan_status fail(sscan_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+sscan_status cuda_check(const char* what) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return SSCAN_OK;
+}
+
+sscan_status check_problem(const sscan_problem* p) {
+    if (!p) return fail(SSCAN_ERR_INVALID_ARG, "problem is NULL");
+    if (p->batch < 0 || p->seqlen < 0 || p->dim < 0)
+        return fail(SSCAN_ERR_INVALID_ARG, "negative size (batch %lld, seqlen %lld, dim %lld)",
+                    (long long)p->batch, (long long)p->seqlen, (long long)p->dim);
+    if (p->dstate < 1) return fail(SSCAN_ERR_INVALID_ARG, "dstate must be >= 1");
+    if (p->dstate > sscan::kMaxState)
+        return fail(SSCAN_ERR_UNSUPPORTED, "dstate %lld > %d", (long long)p->dstate, sscan::kMaxState);
+    if (p->io_dtype != SSCAN_F32 && p->io_dtype != SSCAN_BF16)
+        return fail(SSCAN_ERR_INVALID_ARG, "unknown io_dtype %d", (int)p->io_dtype);
+    if (p->flags & ~SSCAN_DELTA_SOFTPLUS)
+        return fail(SSCAN_ERR_INVALID_ARG, "unknown flag bits 0x%x", (unsigned)p->flags);
+    return SSCAN_OK;
+}
+
+sscan_status check_workspace(size_t need, const void* ws, size_t bytes) {
+    if (need == 0) return SSCAN_OK;
+    if (!ws || bytes < need)
+        return fail(SSCAN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given%s", need, bytes,
+                    ws ? "" : " (NULL)");
+    if (reinterpret_cast<uintptr_t>(ws) % 256 != 0)
+        return fail(SSCAN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    return SSCAN_OK;
+}
+
+inline unsigned blocks_for(int64_t n, int threads) { return (unsigned)((n + threads - 1) / threads); }
+
+template <typename T, int NMAX>
+void launch_fwd_rows(const sscan::ScanArgs& a, int mode, cudaStream_t st) {
+    const int64_t n = a.batch * a.D * a.nchunks;
+    if (mode == sscan::kModeOutput)
+        sscan::fwd_rows_kernel<T, NMAX, sscan::kModeOutput><<<blocks_for(n, 128), 128, 0, st>>>(a);
+    else
+        sscan::fwd_rows_kernel<T, NMAX, sscan::kModeAggregate><<<blocks_for(n, 128), 128, 0, st>>>(a);
+}
+
+template <typename T>
+void dispatch_fwd_rows(const sscan::ScanArgs& a, int mode, cudaStream_t st) {
+    if (a.N <= 4) launch_fwd_rows<T, 4>(a, mode, st);
+    else if (a.N <= 8) launch_fwd_rows<T, 8>(a, mode, st);
+    else launch_fwd_rows<T, 16>(a, mode, st);
+}
+
+void fwd_rows(const sscan::ScanArgs& a, int io, int mode, cudaStream_t st) {
+    if (io == SSCAN_BF16) dispatch_fwd_rows<__nv_bfloat16>(a, mode, st);
+    else dispatch_fwd_rows<float>(a, mode, st);
+}
+
+// L == 0: no steps, h_last = h0 (or zero); nothing else to write.
+sscan_status empty_sequence(const sscan_problem* p, const float* h0, float* h_last, cudaStream_t st) {
+    if (!h_last) return SSCAN_OK;
+    const size_t bytes = (size_t)(p->batch * p->dim * p->dstate) * sizeof(float);
+    if (bytes == 0) return SSCAN_OK;
+    const cudaError_t e = h0 ? cudaMemcpyAsync(h_last, h0, bytes, cudaMemcpyDeviceToDevice, st)
+                             : cudaMemsetAsync(h_last, 0, bytes, st);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "copying h0 to h_last: %s", cudaGetErrorString(e));
+    return SSCAN_OK;
+}
+
+sscan::ScanArgs make_args(const sscan_problem* p, const void* u, const void* delta_raw,
+                          const float* delta_bias, const float* A, const void* B, const void* C,
+                          const float* D_skip, const void* z, const float* h0, void* out,
+                          float* h_last) {
+    sscan::ScanArgs a{};
+    a.batch = p->batch;
+    a.L = p->seqlen;
+    a.D = p->dim;
+    a.N = p->dstate;
+    a.u = u;
+    a.delta_raw = delta_raw;
+    a.bias = delta_bias;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.Dskip = D_skip;
+    a.z = z;
+    a.h0 = h0;
+    a.out = out;
+    a.h_last = h_last;
+    a.softplus = (p->flags & SSCAN_DELTA_SOFTPLUS) ? 1 : 0;
+    a.chunk_len = p->seqlen;
+    a.nchunks = 1;
+    return a;
+}
+
+// Forward or last-state through the row kernels, split along L when there are
+// too few rows to fill the GPU (chunk aggregates, carry, then the chunk outputs).
+sscan_status run_rows(const sscan_problem* p, sscan::ScanArgs a, void* ws, cudaStream_t st) {
+    const sscan::FwdPlan plan = sscan::plan_fwd(p->batch, p->seqlen, p->dim, p->dstate);
+    a.nchunks = plan.nchunks;
+    a.chunk_len = plan.chunk_len;
+    const bool want_out = a.out != nullptr;
+    if (plan.nchunks > 1) {
+        a.ws_state = static_cast<float*>(ws);
+        a.ws_dsum = a.ws_state + plan.state_floats;
+        fwd_rows(a, p->io_dtype, sscan::kModeAggregate, st);
+        if (sscan_status s = cuda_check("chunk aggregate kernel")) return s;
+        sscan::ScanArgs c = a;
+        if (want_out) c.h_last = nullptr;  // the output pass writes h_last itself
+        sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate, 128), 128, 0, st>>>(c);
+        if (sscan_status s = cuda_check("carry kernel")) return s;
+        if (!want_out) return SSCAN_OK;
+    }
+    fwd_rows(a, p->io_dtype, sscan::kModeOutput, st);
+    return cuda_check("forward kernel");
+}
+
+template <typename T, int NMAX>
+void launch_bwd_rows(const sscan::BwdArgs& g, cudaStream_t st) {
+    sscan::bwd_rows_kernel<T, NMAX><<<blocks_for(g.f.batch * g.f.D, 128), 128, 0, st>>>(g);
+}
+
+template <typename T>
+void dispatch_bwd_rows(const sscan::BwdArgs& g, cudaStream_t st) {
+    if (g.f.N <= 4) launch_bwd_rows<T, 4>(g, st);
+    else if (g.f.N <= 8) launch_bwd_rows<T, 8>(g, st);
+    else launch_bwd_rows<T, 16>(g, st);
+}
+
+template <typename T>
+void cast_out(const float* src, void* dst, int64_t n, cudaStream_t st) {
+    if (n > 0) sscan::cast_kernel<T><<<blocks_for(n, 256), 256, 0, st>>>(src, static_cast<T*>(dst), n);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sscan_workspace_size(const sscan_problem* p, int op) {
+    if (check_problem(p) != SSCAN_OK) return 0;
+    switch (op) {
+        case SSCAN_OP_FWD:
+        case SSCAN_OP_LAST_STATE:
+            return sscan::plan_fwd(p->batch, p->seqlen, p->dim, p->dstate).workspace_bytes;
+        case SSCAN_OP_BWD:
+            return sscan::plan_bwd(p->batch, p->seqlen, p->dim, p->dstate).workspace_bytes;
+        default:
+            return 0;
+    }
+}
+
+sscan_status sscan_fwd(const sscan_problem* p, const void* u, const void* delta_raw,
+                       const float* delta_bias, const float* A, const void* B, const void* C,
+                       const float* D_skip, const void* z, const float* h0, void* out,
+                       float* h_last, void* workspace, size_t workspace_bytes, void* stream) {
+    g_err[0] = 0;
+    if (sscan_status s = check_problem(p)) return s;
+    if (!out && !h_last) return fail(SSCAN_ERR_INVALID_ARG, "out and h_last are both NULL");
+    const bool any = p->batch * p->dim > 0;
+    if (any && p->seqlen > 0) {
+        if (!u || !delta_raw || !A || !B) return fail(SSCAN_ERR_INVALID_ARG, "u, delta_raw, A, B are required");
+        if (out && !C) return fail(SSCAN_ERR_INVALID_ARG, "C is required when out is written");
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!any) return SSCAN_OK;
+    if (p->seqlen == 0) return empty_sequence(p, h0, h_last, st);
+    if (sscan_status s = check_workspace(sscan_workspace_size(p, SSCAN_OP_FWD), workspace, workspace_bytes))
+        return s;
+    return run_rows(p, make_args(p, u, delta_raw, delta_bias, A, B, C, D_skip, z, h0, out, h_last),
+                    workspace, st);
+}
+
+sscan_status sscan_last_state(const sscan_problem* p, const void* u, const void* delta_raw,
+                              const float* delta_bias, const float* A, const void* B,
+                              const float* h0, float* h_last, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    g_err[0] = 0;
+    if (sscan_status s = check_problem(p)) return s;
+    if (!h_last) return fail(SSCAN_ERR_INVALID_ARG, "h_last is required");
+    const bool any = p->batch * p->dim > 0;
+    if (any && p->seqlen > 0 && (!u || !delta_raw || !A || !B))
+        return fail(SSCAN_ERR_INVALID_ARG, "u, delta_raw, A, B are required");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!any) return SSCAN_OK;
+    if (p->seqlen == 0) return empty_sequence(p, h0, h_last, st);
+    if (sscan_status s = check_workspace(sscan_workspace_size(p, SSCAN_OP_LAST_STATE), workspace,
+                                         workspace_bytes))
+        return s;
+    return run_rows(p, make_args(p, u, delta_raw, delta_bias, A, B, nullptr, nullptr, nullptr, h0,
+                                 nullptr, h_last),
+                    workspace, st);
+}
+
+sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_raw,
+                       const float* delta_bias, const float* A, const void* B, const void* C,
+                       const float* D_skip, const void* z, const float* h0, const void* dout,
+                       void* du, void* ddelta_raw, float* ddelta_bias, float* dA, void* dB,
+                       void* dC, float* dD, void* dz, float* dh0, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    g_err[0] = 0;
+    if (sscan_status s = check_problem(p)) return s;
+    if ((z == nullptr) != (dz == nullptr)) return fail(SSCAN_ERR_INVALID_ARG, "dz must be given exactly when z is");
+    if (dD && !D_skip) return fail(SSCAN_ERR_INVALID_ARG, "dD needs D_skip");
+    const int64_t rows = p->batch * p->dim;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (rows > 0 && p->seqlen > 0 &&
+        (!u || !delta_raw || !A || !B || !C || !dout || !du || !ddelta_raw || !dB || !dC))
+        return fail(SSCAN_ERR_INVALID_ARG, "u, delta_raw, A, B, C, dout, du, ddelta_raw, dB, dC are required");
+    if (p->dim > 0 && !dA) return fail(SSCAN_ERR_INVALID_ARG, "dA is required");
+    const size_t need = sscan_workspace_size(p, SSCAN_OP_BWD);
+    if (sscan_status s = check_workspace(need, workspace, workspace_bytes)) return s;
+    const int64_t DN = p->dim * p->dstate, BLN = p->batch * p->seqlen * p->dstate;
+    // parameter gradients are sums: start them at zero
+    cudaError_t e = cudaSuccess;
+    if (DN > 0) e = cudaMemsetAsync(dA, 0, (size_t)DN * sizeof(float), st);
+    if (e == cudaSuccess && dD && p->dim > 0) e = cudaMemsetAsync(dD, 0, (size_t)p->dim * sizeof(float), st);
+    if (e == cudaSuccess && ddelta_bias && p->dim > 0)
+        e = cudaMemsetAsync(ddelta_bias, 0, (size_t)p->dim * sizeof(float), st);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing gradients: %s", cudaGetErrorString(e));
+    if (rows == 0) {
+        return SSCAN_OK;
+    }
+    if (p->seqlen == 0) {
+        if (dh0) {
+            e = cudaMemsetAsync(dh0, 0, (size_t)(rows * p->dstate) * sizeof(float), st);
+            if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing dh0: %s", cudaGetErrorString(e));
+        }
+        return SSCAN_OK;
+    }
+    const sscan::BwdPlan plan = sscan::plan_bwd(p->batch, p->seqlen, p->dim, p->dstate);
+    sscan::BwdArgs g{};
+    g.f = make_args(p, u, delta_raw, delta_bias, A, B, C, D_skip, z, h0, nullptr, nullptr);
+    g.dout = dout;
+    g.du = du;
+    g.ddelta_raw = ddelta_raw;
+    g.dbias = ddelta_bias;
+    g.dA = dA;
+    g.dD = dD;
+    g.dz = dz;
+    g.dh0 = dh0;
+    g.nseg = plan.nseg;
+    float* ws = static_cast<float*>(workspace);
+    g.dB32 = ws;
+    g.dC32 = ws + BLN;
+    g.ckpt = ws + 2 * BLN;
+    e = cudaMemsetAsync(ws, 0, (size_t)(2 * BLN) * sizeof(float), st);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing workspace: %s", cudaGetErrorString(e));
+    if (p->io_dtype == SSCAN_BF16) dispatch_bwd_rows<__nv_bfloat16>(g, st);
+    else dispatch_bwd_rows<float>(g, st);
+    if (sscan_status s = cuda_check("backward kernel")) return s;
+    if (p->io_dtype == SSCAN_BF16) {
+        cast_out<__nv_bfloat16>(g.dB32, dB, BLN, st);
+        cast_out<__nv_bfloat16>(g.dC32, dC, BLN, st);
+    } else {
+        cast_out<float>(g.dB32, dB, BLN, st);
+        cast_out<float>(g.dC32, dC, BLN, st);
+    }
+    return cuda_check("gradient cast kernel");
+}
+
+const char* sscan_status_string(sscan_status s) {
+    switch (s) {
+        case SSCAN_OK: return "SSCAN_OK";
+        case SSCAN_ERR_INVALID_ARG: return "SSCAN_ERR_INVALID_ARG";
+        case SSCAN_ERR_UNSUPPORTED: return "SSCAN_ERR_UNSUPPORTED";
+        case SSCAN_ERR_WORKSPACE: return "SSCAN_ERR_WORKSPACE";
+        case SSCAN_ERR_CUDA: return "SSCAN_ERR_CUDA";
+        default: return "SSCAN_ERR_UNKNOWN";
+    }
+}
+
+const char* sscan_last_error(void) { return g_err; }
+
+int sscan_version(void) { return 100; }
+
+}  // extern "C"

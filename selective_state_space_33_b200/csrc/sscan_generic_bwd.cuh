@@ -1,0 +1,195 @@
+// sscan_generic_bwd.cuh -- general-purpose backward of the selective scan: one
+// thread per (batch, channel) row.  States are never stored for the whole
+// sequence (sec. 4.1, item 3: recomputation): a forward sweep keeps one state
+// every kSeg steps, and the reverse sweep recomputes each segment's states
+// from its checkpoint before walking it backwards.
+//
+// With lam_t = dLoss/dh_t = C_t dy_t + Abar_{t+1} lam_{t+1} and
+// dAbar = lam_t h_{t-1}, dbeta = lam_t B_t x_t (beta = Bbar / B = expm1(delta A)/A):
+//   d delta += dAbar A Abar + dbeta Abar            (d beta / d delta = Abar)
+//   dA      += dAbar delta Abar + dbeta delta^2 psi(delta A)
+//   dx      += lam beta B,   dB += lam beta x,   dC += dy h_t
+// with psi(q) = (q e^q - expm1(q)) / q^2; dy = dout SiLU(z), dz = dout y SiLU'(z).
+#pragma once
+
+#include "sscan_generic.cuh"
+#include "sscan_plan.h"
+
+namespace sscan {
+
+constexpr int kSeg = kBwdSeg;
+
+struct BwdArgs {
+    ScanArgs f;            // forward inputs (out, h_last, chunking unused)
+    const void* dout;      // (batch, L, D)
+    void* du;              // (batch, L, D)
+    void* ddelta_raw;      // (batch, L, D)
+    float* dbias;          // (D) or null, pre-zeroed
+    float* dA;             // (D, N), pre-zeroed
+    float* dB32;           // (batch, L, N) fp32, pre-zeroed
+    float* dC32;           // (batch, L, N) fp32, pre-zeroed
+    float* dD;             // (D) or null, pre-zeroed
+    void* dz;              // (batch, L, D) or null
+    float* dh0;            // (batch, D, N) or null
+    float* ckpt;           // [rows][nseg][N]
+    int64_t nseg;
+};
+
+// psi(q) = (q e^q - expm1(q)) / q^2 = sum_{m>=2} (m-1)/m! q^(m-2).
+//   |q| <= 1 : the series through q^7 (dropped tail < 2.5e-6 q^8, ~5e-6 relative)
+//   |q| > 1  : the closed form from abar = e^q; 1 - abar (1 - q) >= 0.26 there, so
+//              the subtraction costs < 1e-6 relative
+__device__ __forceinline__ float psi(float q, float abar) {
+    if (fabsf(q) <= 1.f) {
+        float p = 1.f / 45360.f;
+        p = fmaf(p, q, 1.f / 5760.f);
+        p = fmaf(p, q, 1.f / 840.f);
+        p = fmaf(p, q, 1.f / 144.f);
+        p = fmaf(p, q, 1.f / 30.f);
+        p = fmaf(p, q, 1.f / 8.f);
+        p = fmaf(p, q, 1.f / 3.f);
+        return fmaf(p, q, 0.5f);
+    }
+    return (fmaf(q, abar, -abar) + 1.f) / (q * q);
+}
+
+template <typename T, int NMAX>
+__global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
+    const ScanArgs& a = g.f;
+    const int64_t rows = a.batch * a.D;
+    const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (row >= rows) return;
+    const int64_t b = row / a.D, d = row - b * a.D;
+    const int N = (int)a.N;
+    const T* u = static_cast<const T*>(a.u);
+    const T* dr = static_cast<const T*>(a.delta_raw);
+    const T* Bm = static_cast<const T*>(a.B);
+    const T* Cm = static_cast<const T*>(a.C);
+    const T* z = static_cast<const T*>(a.z);
+    const T* dout = static_cast<const T*>(g.dout);
+
+    float Al[NMAX], A2[NMAX], invA[NMAX], h[NMAX];
+#pragma unroll
+    for (int n = 0; n < NMAX; ++n) {
+        const float An = n < N ? __ldg(a.A + d * N + n) : 0.f;
+        Al[n] = An;
+        A2[n] = An * kLog2e;
+        invA[n] = An != 0.f ? 1.f / An : 0.f;
+        h[n] = (a.h0 && n < N) ? __ldg(a.h0 + row * N + n) : 0.f;
+    }
+    const float bias = a.bias ? __ldg(a.bias + d) : 0.f;
+    const float dsk = a.Dskip ? __ldg(a.Dskip + d) : 0.f;
+    float* ck = g.ckpt + row * g.nseg * N;
+
+    // forward sweep: checkpoint h_{t-1} at the start of every segment
+    for (int64_t t = 0; t < a.L; ++t) {
+        if (t % kSeg == 0) {
+#pragma unroll
+            for (int n = 0; n < NMAX; ++n)
+                if (n < N) ck[(t / kSeg) * N + n] = h[n];
+        }
+        const int64_t e = (b * a.L + t) * a.D + d, s = (b * a.L + t) * N;
+        const float x = IO<T>::load(u, e);
+        const float r = IO<T>::load(dr, e) + bias;
+        const float delta = a.softplus ? softplus(r) : r;
+#pragma unroll
+        for (int n = 0; n < NMAX; ++n) {
+            if (n < N) {
+                const float abar = ex2(delta * A2[n]);
+                const float beta = bbar_coef(delta, delta * Al[n], abar, invA[n]);
+                h[n] = fmaf(abar, h[n], beta * IO<T>::load(Bm, s + n) * x);
+            }
+        }
+    }
+
+    // reverse sweep over segments
+    float lam[NMAX], dAacc[NMAX];
+#pragma unroll
+    for (int n = 0; n < NMAX; ++n) lam[n] = dAacc[n] = 0.f;  // lam holds Abar_{t+1} lam_{t+1}
+    float dDacc = 0.f, dbacc = 0.f;
+    float hs[kSeg + 1][NMAX];
+    for (int64_t sg = g.nseg - 1; sg >= 0; --sg) {
+        const int64_t t0 = sg * kSeg;
+        const int len = (int)(a.L - t0 < kSeg ? a.L - t0 : kSeg);
+#pragma unroll
+        for (int n = 0; n < NMAX; ++n) hs[0][n] = n < N ? ck[sg * N + n] : 0.f;
+        for (int k = 0; k < len; ++k) {
+            const int64_t t = t0 + k;
+            const int64_t e = (b * a.L + t) * a.D + d, s = (b * a.L + t) * N;
+            const float x = IO<T>::load(u, e);
+            const float r = IO<T>::load(dr, e) + bias;
+            const float delta = a.softplus ? softplus(r) : r;
+#pragma unroll
+            for (int n = 0; n < NMAX; ++n) {
+                if (n < N) {
+                    const float abar = ex2(delta * A2[n]);
+                    const float beta = bbar_coef(delta, delta * Al[n], abar, invA[n]);
+                    hs[k + 1][n] = fmaf(abar, hs[k][n], beta * IO<T>::load(Bm, s + n) * x);
+                }
+            }
+        }
+        for (int k = len - 1; k >= 0; --k) {
+            const int64_t t = t0 + k;
+            const int64_t e = (b * a.L + t) * a.D + d, s = (b * a.L + t) * N;
+            const float x = IO<T>::load(u, e);
+            const float r = IO<T>::load(dr, e) + bias;
+            const float delta = a.softplus ? softplus(r) : r;
+            const float go = IO<T>::load(dout, e);
+            float dy = go;
+            if (z) {
+                float y = 0.f;
+#pragma unroll
+                for (int n = 0; n < NMAX; ++n)
+                    if (n < N) y = fmaf(IO<T>::load(Cm, s + n), hs[k + 1][n], y);
+                y = fmaf(dsk, x, y);
+                const float zz = IO<T>::load(z, e);
+                const float sg = sigmoid(zz);
+                dy = go * zz * sg;
+                IO<T>::store(static_cast<T*>(g.dz), e, go * y * sg * fmaf(zz, 1.f - sg, 1.f));
+            }
+            float dx = dsk * dy;
+            dDacc = fmaf(dy, x, dDacc);
+            float ddelta = 0.f;
+#pragma unroll
+            for (int n = 0; n < NMAX; ++n) {
+                if (n < N) {
+                    const float q = delta * Al[n];
+                    const float abar = ex2(delta * A2[n]);
+                    const float beta = bbar_coef(delta, q, abar, invA[n]);
+                    const float Bn = IO<T>::load(Bm, s + n), Cn = IO<T>::load(Cm, s + n);
+                    const float l = fmaf(Cn, dy, lam[n]);
+                    const float dab = l * hs[k][n];
+                    const float dbeta = l * Bn * x;
+                    atomicAdd(g.dC32 + s + n, dy * hs[k + 1][n]);
+                    atomicAdd(g.dB32 + s + n, l * beta * x);
+                    dx = fmaf(l * beta, Bn, dx);
+                    ddelta = fmaf(dab * Al[n] + dbeta, abar, ddelta);
+                    dAacc[n] += dab * delta * abar + dbeta * delta * delta * psi(q, abar);
+                    lam[n] = abar * l;
+                }
+            }
+            const float drr = a.softplus ? ddelta * sigmoid(r) : ddelta;
+            IO<T>::store(static_cast<T*>(g.du), e, dx);
+            IO<T>::store(static_cast<T*>(g.ddelta_raw), e, drr);
+            dbacc += drr;
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < NMAX; ++n) {
+        if (n < N) {
+            if (g.dh0) g.dh0[row * N + n] = lam[n];
+            atomicAdd(g.dA + d * N + n, dAacc[n]);
+        }
+    }
+    if (g.dD) atomicAdd(g.dD + d, dDacc);
+    if (g.dbias) atomicAdd(g.dbias + d, dbacc);
+}
+
+// fp32 accumulator -> I/O type (dB, dC)
+template <typename T>
+__global__ void cast_kernel(const float* src, T* dst, int64_t n) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) IO<T>::store(dst, i, src[i]);
+}
+
+}  // namespace sscan

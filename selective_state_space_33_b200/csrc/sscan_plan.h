@@ -1,0 +1,63 @@
+// sscan_plan.h -- host-side planning: how a problem is split across the GPU and
+// how much workspace each operation needs.  Pure integer arithmetic, identical
+// for sscan_workspace_size() and the operations themselves.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+namespace sscan {
+
+constexpr int kMaxState = 16;
+constexpr int kSmCount = 148;               // B200
+constexpr int64_t kRowsFillGpu = 16384;     // rows that keep every sub-partition busy
+constexpr int64_t kTargetThreads = (int64_t)kSmCount * 4 * 32 * 4;  // 4 warps per sub-partition
+constexpr int64_t kMinChunk = 512;          // shortest sequence chunk worth a carry
+constexpr int kBwdSeg = 16;                 // steps between backward checkpoints
+
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+struct FwdPlan {
+    int64_t nchunks;
+    int64_t chunk_len;
+    int64_t state_floats;  // floats of chunk end states (then carry-ins)
+    size_t workspace_bytes;
+};
+
+// Split L into chunks only when the rows alone cannot fill the GPU; each extra
+// chunk costs one more pass over its steps (the chunk aggregate), so chunks are
+// kept long.
+inline FwdPlan plan_fwd(int64_t batch, int64_t L, int64_t D, int64_t N) {
+    FwdPlan p{1, L, 0, 0};
+    const int64_t rows = batch * D;
+    if (rows <= 0 || L <= 0 || rows >= kRowsFillGpu) return p;
+    int64_t want = (kTargetThreads + rows - 1) / rows;
+    const int64_t most = L / kMinChunk;
+    if (want > most) want = most;
+    if (want <= 1) return p;
+    p.chunk_len = (L + want - 1) / want;
+    p.nchunks = (L + p.chunk_len - 1) / p.chunk_len;
+    if (p.nchunks <= 1) return FwdPlan{1, L, 0, 0};
+    p.state_floats = batch * p.nchunks * D * N;
+    const int64_t dsum_floats = batch * p.nchunks * D;
+    p.workspace_bytes = align256((size_t)(p.state_floats + dsum_floats) * sizeof(float));
+    return p;
+}
+
+struct BwdPlan {
+    int64_t nseg;
+    size_t workspace_bytes;
+};
+
+// fp32 accumulators for dB and dC (batch, L, N), then one checkpointed state
+// every kBwdSeg steps of every row.
+inline BwdPlan plan_bwd(int64_t batch, int64_t L, int64_t D, int64_t N) {
+    BwdPlan p{0, 0};
+    if (batch * D <= 0 || L <= 0) return p;
+    p.nseg = (L + kBwdSeg - 1) / kBwdSeg;
+    const size_t floats = (size_t)(2 * batch * L * N) + (size_t)(batch * D * p.nseg * N);
+    p.workspace_bytes = align256(floats * sizeof(float));
+    return p;
+}
+
+}  // namespace sscan

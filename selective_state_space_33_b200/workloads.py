@@ -127,3 +127,16 @@ def small_case(batch: int, seqlen: int, dim: int, dstate: int, io: str = "f32", 
     """Inputs of any shape drawn with the same recipe (for tails and edge cases)."""
     return make_inputs(Workload("custom", batch, seqlen, dim, dstate, io, dt_min, dt_max,
                                 dskip, seed, backward=backward))
+
+
+def to_device(x: dict, device) -> dict:
+    """Copy drawn inputs to torch tensors on ``device`` (uint16 arrays become bfloat16
+    tensors with the same bits)."""
+    import torch
+    out = {}
+    for k, v in x.items():
+        t = torch.from_numpy(np.ascontiguousarray(v))
+        if v.dtype == np.uint16:
+            t = t.view(torch.bfloat16)
+        out[k] = t.to(device)
+    return out

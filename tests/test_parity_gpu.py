@@ -1,0 +1,240 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 CPU oracle on
+the same seeded inputs.  Tolerance (normwise, per tensor): max|gpu - ref| / max|ref|
+<= 1e-4 for fp32 I/O and <= 2e-2 for bf16 I/O."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_33_b200 import binding as sb
+from selective_state_space_33_b200 import workloads as W
+
+from .helpers import TOL, normwise, to_f64, to_torch
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_fwd(x, rows=None, **kw):
+    return oracle.fwd(x["u"], x["delta_raw"], x["A"], x["B"], x["C"], delta_bias=x.get("delta_bias"),
+                      D_skip=x.get("D_skip"), z=x.get("z"), rows=rows, **kw)
+
+
+def _gpu_fwd(t, **kw):
+    return sb.sscan_fwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t.get("delta_bias"),
+                        t.get("D_skip"), t.get("z"), t.get("h0"), **kw)
+
+
+def _check_full(x, io, dev, h0=None, **kw):
+    t = to_torch(x, dev)
+    if h0 is not None:
+        t["h0"] = torch.from_numpy(h0.astype(np.float32)).to(dev)
+    out, hl = _gpu_fwd(t, return_last_state=True, **kw)
+    torch.cuda.synchronize()
+    ref, ref_h = oracle.fwd(x["u"], x["delta_raw"], x["A"], x["B"], x["C"], delta_bias=x.get("delta_bias"),
+                            D_skip=x.get("D_skip"), z=x.get("z"),
+                            h0=None if h0 is None else h0.astype(np.float32).astype(np.float64), **kw)
+    e_out, e_h = normwise(to_f64(out), ref), normwise(to_f64(hl), ref_h)
+    assert e_out <= TOL[io], e_out
+    assert e_h <= TOL[io], e_h
+    return e_out, e_h
+
+
+# ---------------------------------------------------------------- configs at full size
+def test_tiny_fp32(cuda_device):
+    x = W.make_inputs(W.WORKLOADS["tiny"])
+    _check_full(x, "f32", cuda_device)
+
+
+def test_mamba130m_bf16_full(cuda_device):
+    x = W.make_inputs(W.WORKLOADS["mamba130m"])
+    _check_full(x, "bf16", cuda_device)
+
+
+def _sampled_rows(w, k, seed):
+    rng = np.random.default_rng(seed)
+    rows = rng.choice(w.batch * w.dim, size=k, replace=False)
+    # always include the first and last channel of the first and last batch
+    extra = [0, w.dim - 1, (w.batch - 1) * w.dim, w.batch * w.dim - 1]
+    return np.unique(np.concatenate([rows, extra]))
+
+
+def _check_sampled(w, dev, k=96):
+    x = W.make_inputs(w)
+    t = to_torch(x, dev)
+    out, hl = _gpu_fwd(t, return_last_state=True)
+    torch.cuda.synchronize()
+    rows = _sampled_rows(w, k, w.seed)
+    ref, ref_h = _oracle_fwd(x, rows=rows)
+    b, d = rows // w.dim, rows % w.dim
+    got = to_f64(out[b, :, d])                     # (rows, L)
+    got_h = to_f64(hl.reshape(-1, w.dstate)[rows])
+    e_out, e_h = normwise(got, ref), normwise(got_h, ref_h)
+    assert e_out <= TOL[w.io], e_out
+    assert e_h <= TOL[w.io], e_h
+    assert torch.isfinite(out.float()).all()
+
+
+def test_mamba2p8b_bf16_sampled(cuda_device):
+    _check_sampled(W.WORKLOADS["mamba2.8b"], cuda_device)
+
+
+def test_mamba2p8b_fp32_sampled(cuda_device):
+    _check_sampled(W.WORKLOADS["mamba2.8b-f32"], cuda_device)
+
+
+def test_million_length_sampled(cuda_device):
+    _check_sampled(W.WORKLOADS["million"], cuda_device, k=16)
+
+
+# ---------------------------------------------------------------- tails, options, N
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 100, 37, 16), (1, 257, 8, 4), (3, 33, 5, 1), (2, 64, 40, 7),
+                                   (1, 1, 3, 16), (2, 1030, 24, 8)])
+def test_shapes_and_tails(cuda_device, io, shape):
+    batch, L, D, N = shape
+    x = W.small_case(batch, L, D, N, io=io, seed=sum(shape))
+    _check_full(x, io, cuda_device)
+
+
+@pytest.mark.parametrize("variant", ["no_gate", "no_skip", "no_bias", "no_softplus", "h0", "bare"])
+def test_optional_inputs(cuda_device, variant):
+    x = W.small_case(2, 96, 19, 16, io="f32", seed=31)
+    kw, h0 = {}, None
+    if variant in ("no_gate", "bare"):
+        del x["z"]
+    if variant in ("no_skip", "bare"):
+        del x["D_skip"]
+    if variant in ("no_bias", "bare"):
+        del x["delta_bias"]
+    if variant == "no_softplus":
+        x["delta_raw"] = np.abs(x["delta_raw"]) * 0.05
+        kw["delta_softplus"] = False
+    if variant == "h0":
+        h0 = np.random.default_rng(3).standard_normal((2, 19, 16))
+    _check_full(x, "f32", cuda_device, h0=h0, **kw)
+
+
+def test_general_A_values(cuda_device):
+    """A with zeros (the delta B limit), tiny and large magnitudes, and positive entries."""
+    x = W.small_case(2, 80, 12, 16, io="f32", seed=41)
+    rng = np.random.default_rng(41)
+    A = -np.exp(rng.uniform(-6, 3, size=(12, 16))).astype(np.float32)
+    A[0, :4] = 0.0
+    A[1, 5] = 0.25
+    A[2, 7] = -1e-7
+    x["A"] = A
+    _check_full(x, "f32", cuda_device)
+
+
+# ---------------------------------------------------------------- pins through the ABI
+def test_hand_case_through_abi(cuda_device):
+    ln2 = math.log(2.0)
+    t = {"u": torch.tensor([1.0, 2, 3, 4]).reshape(1, 4, 1), "delta_raw": torch.tensor([1.0, 2, 1, 0]).reshape(1, 4, 1),
+         "A": torch.tensor([[-ln2]]), "B": torch.full((1, 4, 1), ln2), "C": torch.tensor([1.0, 1, 2, 1]).reshape(1, 4, 1)}
+    t = {k: v.float().to(cuda_device) for k, v in t.items()}
+    out, hl = _gpu_fwd(t, delta_softplus=False, return_last_state=True)
+    np.testing.assert_allclose(to_f64(out).ravel(), [0.5, 1.625, 4.625, 2.3125], rtol=1e-5)
+    np.testing.assert_allclose(to_f64(hl).ravel(), [2.3125], rtol=1e-5)
+
+
+@pytest.mark.parametrize("k", [1, 255, 256, 257, 700])
+def test_split_with_carry_on_gpu(cuda_device, k):
+    x = W.small_case(2, 1024, 24, 16, io="f32", seed=51)
+    t = to_torch(x, cuda_device)
+    full, hl = _gpu_fwd(t, return_last_state=True)
+    cut = lambda v, s: v[:, s].contiguous()
+    s1, s2 = slice(0, k), slice(k, None)
+    a = {n: (cut(v, s1) if n in ("u", "delta_raw", "z", "B", "C") else v) for n, v in t.items()}
+    o1, h1 = _gpu_fwd(a, return_last_state=True)
+    b = {n: (cut(v, s2) if n in ("u", "delta_raw", "z", "B", "C") else v) for n, v in t.items()}
+    b["h0"] = h1
+    o2, h2 = _gpu_fwd(b, return_last_state=True)
+    assert normwise(to_f64(torch.cat([o1, o2], 1)), to_f64(full)) <= 1e-5
+    assert normwise(to_f64(h2), to_f64(hl)) <= 1e-5
+
+
+def test_last_state_matches_oracle(cuda_device):
+    for w in (W.small_case(2, 3000, 16, 16, io="bf16", seed=61),
+              W.small_case(1, 5000, 4, 8, io="f32", seed=62)):
+        t = to_torch(w, cuda_device)
+        hl = sb.sscan_last_state(t["u"], t["delta_raw"], t["A"], t["B"], t["delta_bias"])
+        torch.cuda.synchronize()
+        _, ref_h = oracle.fwd(w["u"], w["delta_raw"], w["A"], w["B"], w["C"], delta_bias=w["delta_bias"],
+                              want_out=False)
+        io = "bf16" if w["u"].dtype == np.uint16 else "f32"
+        assert normwise(to_f64(hl), ref_h) <= TOL[io]
+
+
+def test_delta_to_zero_on_gpu(cuda_device):
+    x = W.small_case(2, 50, 9, 16, io="f32", seed=71)
+    x["delta_raw"] = np.full_like(x["delta_raw"], -40.0)
+    h0 = np.random.default_rng(71).standard_normal((2, 9, 16))
+    _check_full(x, "f32", cuda_device, h0=h0)
+
+
+# ---------------------------------------------------------------- edge cases
+def test_empty_sequence_returns_h0(cuda_device):
+    t = to_torch(W.small_case(2, 0, 5, 4, io="f32", seed=1), cuda_device)
+    h0 = torch.randn(2, 5, 4, device=cuda_device)
+    out, hl = sb.sscan_fwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], h0=h0, return_last_state=True)
+    torch.cuda.synchronize()
+    assert out.numel() == 0 and torch.equal(hl, h0)
+    hl = sb.sscan_last_state(t["u"], t["delta_raw"], t["A"], t["B"])
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(hl) == 0
+
+
+def test_empty_batch_and_channels(cuda_device):
+    for shape in ((0, 10, 4, 4), (2, 10, 0, 4)):
+        t = to_torch(W.small_case(*shape, io="f32", seed=2), cuda_device)
+        out = sb.sscan_fwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"])
+        torch.cuda.synchronize()
+        assert out.numel() == 0
+
+
+def test_errors_through_binding(cuda_device):
+    t = to_torch(W.small_case(1, 16, 4, 4, io="f32", seed=3), cuda_device)
+    with pytest.raises(sb.SscanError) as e:
+        sb.sscan_fwd(t["u"], t["delta_raw"], torch.zeros(4, 17, device=cuda_device),
+                     torch.zeros(1, 16, 17, device=cuda_device), torch.zeros(1, 16, 17, device=cuda_device))
+    assert e.value.name == "SSCAN_ERR_UNSUPPORTED"
+    big = to_torch(W.small_case(1, 4096, 8, 4, io="f32", seed=4), cuda_device)
+    prob = sb.make_problem(1, 4096, 8, 4, sb.SSCAN_F32)
+    need = sb.sscan_workspace_size(prob, sb.SSCAN_OP_FWD)
+    assert need > 0
+    with pytest.raises(sb.SscanError) as e:
+        sb.sscan_fwd(big["u"], big["delta_raw"], big["A"], big["B"], big["C"],
+                     workspace=torch.empty(need // 2, dtype=torch.uint8, device=cuda_device))
+    assert e.value.name == "SSCAN_ERR_WORKSPACE"
+
+
+# ---------------------------------------------------------------- backward
+def _check_bwd(x, io, dev, h0=None):
+    t = to_torch(x, dev)
+    if h0 is not None:
+        t["h0"] = torch.from_numpy(h0.astype(np.float32)).to(dev)
+    g = sb.sscan_bwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t.get("delta_bias"),
+                     t.get("D_skip"), t.get("z"), t.get("h0"))
+    torch.cuda.synchronize()
+    ref = oracle.bwd(x["u"], x["delta_raw"], x["A"], x["B"], x["C"], x["dout"], delta_bias=x.get("delta_bias"),
+                     D_skip=x.get("D_skip"), z=x.get("z"),
+                     h0=None if h0 is None else h0.astype(np.float32).astype(np.float64))
+    errs = {k: normwise(to_f64(g[k]), ref[k]) for k in ref}
+    bad = {k: e for k, e in errs.items() if not e <= TOL[io]}
+    assert not bad, errs
+    return errs
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 64, 4, 4), (2, 100, 37, 16), (1, 33, 5, 1), (2, 70, 9, 7)])
+def test_backward_small(cuda_device, io, shape):
+    x = W.small_case(*shape, io=io, seed=sum(shape) + 1, backward=True)
+    h0 = np.random.default_rng(5).standard_normal((shape[0], shape[2], shape[3])) * 0.3
+    _check_bwd(x, io, cuda_device, h0=h0)
+
+
+def test_backward_mamba130m_full(cuda_device):
+    x = W.make_inputs(W.WORKLOADS["bwd130m"])
+    _check_bwd(x, "bf16", cuda_device)
