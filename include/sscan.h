@@ -127,6 +127,15 @@ SSCAN_API const char* sscan_status_string(sscan_status status);
 /* One-line reason for the most recent failed call on this thread ("" if none). */
 SSCAN_API const char* sscan_last_error(void);
 
+/*
+ * Device-side status of the library's kernels on the current device: *flags
+ * receives the OR of every error bit raised since the last clear (bit 0: a
+ * bounded wait for an asynchronous tile copy gave up, so that kernel stopped
+ * early and its outputs are incomplete).  clear != 0 resets the word after
+ * reading.  Synchronous: it waits for work already submitted to the device.
+ */
+SSCAN_API sscan_status sscan_device_status(int clear, unsigned int* flags);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 SSCAN_API int sscan_version(void);
 

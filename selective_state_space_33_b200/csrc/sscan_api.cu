@@ -9,6 +9,7 @@
 #include "sscan.h"
 #include "sscan_generic.cuh"
 #include "sscan_generic_bwd.cuh"
+#include "sscan_launch.h"
 #include "sscan_plan.h"
 
 namespace {
@@ -136,6 +137,64 @@ sscan_status run_rows(const sscan_problem* p, sscan::ScanArgs a, void* ws, cudaS
     return cuda_check("forward kernel");
 }
 
+bool aligned16(const void* q) { return q == nullptr || reinterpret_cast<uintptr_t>(q) % 16 == 0; }
+
+// The tiled kernel reads rows of the (batch, L, D) tensors through TMA, which needs
+// 16-byte aligned bases and row pitches.
+bool tiled_ok(const sscan_problem* p, const sscan::ScanArgs& a) {
+    const int64_t es = p->io_dtype == SSCAN_BF16 ? 2 : 4;
+    return (p->dim * es) % 16 == 0 && aligned16(a.u) && aligned16(a.delta_raw) && aligned16(a.z) &&
+           aligned16(a.out) && p->seqlen < (int64_t(1) << 31) && p->dim < (int64_t(1) << 31);
+}
+
+sscan_status run_tiled(const sscan_problem* p, const sscan::ScanArgs& a, void* ws, cudaStream_t st) {
+    const int64_t DC = sscan::tiled_channels_per_cta(p->dstate);
+    const sscan::FwdPlan plan = sscan::plan_tiled(p->batch, p->seqlen, p->dim, p->dstate, DC);
+    sscan::TiledArgs t{};
+    t.batch = p->batch;
+    t.L = p->seqlen;
+    t.D = p->dim;
+    t.N = (int)p->dstate;
+    t.softplus = a.softplus;
+    t.has_z = a.z != nullptr;
+    t.bias = a.bias;
+    t.A = a.A;
+    t.Dskip = a.Dskip;
+    t.h0 = a.h0;
+    t.B = a.B;
+    t.C = a.C;
+    t.h_last = a.h_last;
+    t.chunk_len = plan.chunk_len;
+    t.nchunks = plan.nchunks;
+    sscan::TiledPtrs ptr{a.u, a.delta_raw, a.z, a.out};
+    const int bf16 = p->io_dtype == SSCAN_BF16;
+    const bool want_out = a.out != nullptr;
+    cudaError_t e;
+    if (plan.nchunks > 1) {
+        t.ws_state = static_cast<float*>(ws);
+        t.ws_dsum = t.ws_state + plan.state_floats;
+        e = sscan::launch_fwd_tiled(t, ptr, bf16, sscan::kTiledAgg, st);
+        if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "chunk aggregate kernel: %s", cudaGetErrorString(e));
+        sscan::ScanArgs c = a;
+        c.nchunks = plan.nchunks;
+        c.chunk_len = plan.chunk_len;
+        c.ws_state = t.ws_state;
+        c.ws_dsum = t.ws_dsum;
+        if (want_out) c.h_last = nullptr;
+        sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate, 128), 128, 0, st>>>(c);
+        if (sscan_status s = cuda_check("carry kernel")) return s;
+        if (!want_out) return SSCAN_OK;
+    }
+    e = sscan::launch_fwd_tiled(t, ptr, bf16, want_out ? sscan::kTiledOut : sscan::kTiledLast, st);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "tiled forward kernel: %s", cudaGetErrorString(e));
+    return SSCAN_OK;
+}
+
+sscan_status run_fwd(const sscan_problem* p, const sscan::ScanArgs& a, void* ws, cudaStream_t st) {
+    if (tiled_ok(p, a)) return run_tiled(p, a, ws, st);
+    return run_rows(p, a, ws, st);
+}
+
 template <typename T, int NMAX>
 void launch_bwd_rows(const sscan::BwdArgs& g, cudaStream_t st) {
     sscan::bwd_rows_kernel<T, NMAX><<<blocks_for(g.f.batch * g.f.D, 128), 128, 0, st>>>(g);
@@ -161,8 +220,14 @@ size_t sscan_workspace_size(const sscan_problem* p, int op) {
     if (check_problem(p) != SSCAN_OK) return 0;
     switch (op) {
         case SSCAN_OP_FWD:
-        case SSCAN_OP_LAST_STATE:
-            return sscan::plan_fwd(p->batch, p->seqlen, p->dim, p->dstate).workspace_bytes;
+        case SSCAN_OP_LAST_STATE: {
+            // enough for either path (the choice also depends on pointer alignment)
+            const size_t g = sscan::plan_fwd(p->batch, p->seqlen, p->dim, p->dstate).workspace_bytes;
+            const size_t t = sscan::plan_tiled(p->batch, p->seqlen, p->dim, p->dstate,
+                                               sscan::tiled_channels_per_cta(p->dstate))
+                                 .workspace_bytes;
+            return g > t ? g : t;
+        }
         case SSCAN_OP_BWD:
             return sscan::plan_bwd(p->batch, p->seqlen, p->dim, p->dstate).workspace_bytes;
         default:
@@ -187,8 +252,8 @@ sscan_status sscan_fwd(const sscan_problem* p, const void* u, const void* delta_
     if (p->seqlen == 0) return empty_sequence(p, h0, h_last, st);
     if (sscan_status s = check_workspace(sscan_workspace_size(p, SSCAN_OP_FWD), workspace, workspace_bytes))
         return s;
-    return run_rows(p, make_args(p, u, delta_raw, delta_bias, A, B, C, D_skip, z, h0, out, h_last),
-                    workspace, st);
+    return run_fwd(p, make_args(p, u, delta_raw, delta_bias, A, B, C, D_skip, z, h0, out, h_last),
+                   workspace, st);
 }
 
 sscan_status sscan_last_state(const sscan_problem* p, const void* u, const void* delta_raw,
@@ -207,9 +272,9 @@ sscan_status sscan_last_state(const sscan_problem* p, const void* u, const void*
     if (sscan_status s = check_workspace(sscan_workspace_size(p, SSCAN_OP_LAST_STATE), workspace,
                                          workspace_bytes))
         return s;
-    return run_rows(p, make_args(p, u, delta_raw, delta_bias, A, B, nullptr, nullptr, nullptr, h0,
-                                 nullptr, h_last),
-                    workspace, st);
+    return run_fwd(p, make_args(p, u, delta_raw, delta_bias, A, B, nullptr, nullptr, nullptr, h0,
+                                nullptr, h_last),
+                   workspace, st);
 }
 
 sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_raw,
@@ -291,6 +356,14 @@ const char* sscan_status_string(sscan_status s) {
 }
 
 const char* sscan_last_error(void) { return g_err; }
+
+sscan_status sscan_device_status(int clear, unsigned int* flags) {
+    g_err[0] = 0;
+    if (!flags) return fail(SSCAN_ERR_INVALID_ARG, "flags is NULL");
+    const cudaError_t e = sscan::read_device_error(flags, clear);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+    return SSCAN_OK;
+}
 
 int sscan_version(void) { return 100; }
 

@@ -44,6 +44,31 @@ inline FwdPlan plan_fwd(int64_t batch, int64_t L, int64_t D, int64_t N) {
     return p;
 }
 
+// Plan of the tiled forward kernel: CTAs cover DC channels of one batch; the
+// sequence is split only when there are too few CTA columns to occupy the GPU.
+constexpr int64_t kTiledMinCols = 2 * kSmCount;     // below this, split the sequence
+constexpr int64_t kTiledTargetCtas = 8 * kSmCount;  // CTAs resident at once (8 per SM)
+constexpr int64_t kTiledMinChunk = 1024;            // steps
+constexpr int64_t kTiledStep = 16;                  // chunk lengths are whole tiles
+
+inline FwdPlan plan_tiled(int64_t batch, int64_t L, int64_t D, int64_t N, int64_t DC) {
+    FwdPlan p{1, L, 0, 0};
+    const int64_t cols = batch * ((D + DC - 1) / DC);
+    if (cols <= 0 || L <= 0 || cols >= kTiledMinCols) return p;
+    int64_t want = (kTiledTargetCtas + cols - 1) / cols;
+    const int64_t most = L / kTiledMinChunk;
+    if (want > most) want = most;
+    if (want <= 1) return p;
+    int64_t len = (L + want - 1) / want;
+    len = (len + kTiledStep - 1) / kTiledStep * kTiledStep;
+    p.chunk_len = len;
+    p.nchunks = (L + len - 1) / len;
+    if (p.nchunks <= 1) return FwdPlan{1, L, 0, 0};
+    p.state_floats = batch * p.nchunks * D * N;
+    p.workspace_bytes = align256((size_t)(p.state_floats + batch * p.nchunks * D) * sizeof(float));
+    return p;
+}
+
 struct BwdPlan {
     int64_t nseg;
     size_t workspace_bytes;

@@ -109,7 +109,9 @@ def test_optional_inputs(cuda_device, variant):
     if variant in ("no_bias", "bare"):
         del x["delta_bias"]
     if variant == "no_softplus":
+        # delta = delta_raw directly, so keep it positive and drop the (negative) bias
         x["delta_raw"] = np.abs(x["delta_raw"]) * 0.05
+        del x["delta_bias"]
         kw["delta_softplus"] = False
     if variant == "h0":
         h0 = np.random.default_rng(3).standard_normal((2, 19, 16))
@@ -238,3 +240,43 @@ def test_backward_small(cuda_device, io, shape):
 def test_backward_mamba130m_full(cuda_device):
     x = W.make_inputs(W.WORKLOADS["bwd130m"])
     _check_bwd(x, "bf16", cuda_device)
+
+
+# ---------------------------------------------------------------- both kernel paths
+def _misaligned_copy(t):
+    """Same values, contiguous, but starting one element past a 16-byte boundary, which
+    sends the call down the general row kernels instead of the TMA-tiled kernel."""
+    buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+    v = buf[1:].view(t.shape)
+    v.copy_(t)
+    return v
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_general_path_matches_tiled_path(cuda_device, io):
+    x = W.small_case(2, 300, 64, 16, io=io, seed=81)
+    t = to_torch(x, cuda_device)
+    fast, hf = _gpu_fwd(t, return_last_state=True)
+    m = dict(t)
+    for k in ("u", "delta_raw", "z"):
+        m[k] = _misaligned_copy(t[k])
+    slow, hs = _gpu_fwd(m, return_last_state=True)
+    torch.cuda.synchronize()
+    ref, ref_h = _oracle_fwd(x)
+    for got, gh in ((fast, hf), (slow, hs)):
+        assert normwise(to_f64(got), ref) <= TOL[io]
+        assert normwise(to_f64(gh), ref_h) <= TOL[io]
+    assert normwise(to_f64(fast), to_f64(slow)) <= (1e-5 if io == "f32" else 1e-2)
+
+
+def test_device_status_is_clear(cuda_device):
+    import ctypes
+    lib = sb.load_library()
+    lib.sscan_device_status.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_uint)]
+    lib.sscan_device_status.restype = ctypes.c_int
+    x = W.small_case(2, 100, 64, 16, io="bf16", seed=82)
+    t = to_torch(x, cuda_device)
+    _gpu_fwd(t)
+    flags = ctypes.c_uint(123)
+    assert lib.sscan_device_status(1, ctypes.byref(flags)) == 0
+    assert flags.value == 0
