@@ -16,9 +16,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -101,50 +99,68 @@ def measured_peaks() -> dict:
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of this GPU's SM clock and throttle reasons every 200 ms."""
+    """Samples this GPU's SM clock and clock-event (throttle) reasons through NVML
+    every 10 ms on a host thread; read-only.  ``mark()`` brackets the timed region
+    so the summary uses the samples taken during it (plus a short busy tail when
+    the region is shorter than a few sample periods)."""
 
-    FIELDS = ["uuid", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
-              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
-              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, uuid: str):
-        self.uuid = uuid
-        self.proc = None
-        self.file = None
+    def __init__(self, uuid: str, period_s: float = 0.01):
+        self.uuid, self.period = uuid, period_s
+        self.samples = []          # (host time, sm MHz, max MHz, reasons mask)
+        self.marks = []
+        self._stop = None
+        self._thread = None
+        self.error = None
 
     def start(self):
+        import threading
         try:
-            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else nv.nvmlDeviceGetHandleByIndex(0)
+            getr = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.error = f"nvml unavailable: {e}"
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                    rs = getr(h)
+                    self.samples.append((time.perf_counter(), sm, mx, rs))
+                except Exception as e:
+                    self.error = str(e)
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+
+    def mark(self):
+        self.marks.append(time.perf_counter())
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.file.flush()
-        self.file.seek(0)
-        rows = [[c.strip() for c in line.split(",")] for line in self.file if line.strip()]
-        self.file.close()
-        os.unlink(self.file.name)
-        mine = [r for r in rows if len(r) == len(self.FIELDS) and (not self.uuid or r[0] == self.uuid)]
-        sm = [float(r[1]) for r in mine if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in mine if r[2].replace(".", "").isdigit()]
-        reasons = set()
-        for r in mine:
-            for name, col in (("hw_slowdown", 5), ("hw_thermal_slowdown", 6), ("sw_thermal_slowdown", 7),
-                              ("sw_power_cap", 8)):
-                if r[col].lower().startswith("active"):
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(mine)}
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "no samples"]}
+        self._stop.set()
+        self._thread.join(timeout=2)
+        t0, t1 = (self.marks[0], self.marks[-1]) if len(self.marks) >= 2 else (0.0, float("inf"))
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if len(inside) < 5:  # short region: add the busy tail that follows it
+            inside = [s for s in self.samples if s[0] >= t0]
+        mask = 0
+        for s in inside:
+            mask |= int(s[3])
+        reasons = sorted(name for bit, name in self.REASONS.items() if mask & bit)
+        return {"sm_mhz": statistics.median([s[1] for s in inside]) if inside else None,
+                "sm_max_mhz": max(s[2] for s in inside) if inside else None,
+                "reasons": reasons, "samples": len(inside)}
 
 
 # ----------------------------------------------------------------------------- CPU arms
@@ -272,21 +288,25 @@ def gpu_arm(args, w: W.Workload):
         pass
     clocks = ClockSampler(uuid)
     clocks.start()
-    time.sleep(0.4)
+    time.sleep(0.05)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
+    clocks.mark()
     for i in range(args.steps):
         starts[i].record(st)
         step()
         ends[i].record(st)
     torch.cuda.synchronize()
+    clocks.mark()
     barrier()
-    # keep the GPU busy while the sampler takes a few more readings under load
-    for _ in range(max(1, int(0.6 / max(starts[0].elapsed_time(ends[0]) * 1e-3, 1e-4)))):
-        step()
-    torch.cuda.synchronize()
+    if not args.profile_run:
+        # a short busy tail so that a brief timed region still has clock samples under load
+        tail = min(2000, max(1, int(0.3 / max(starts[0].elapsed_time(ends[0]) * 1e-3, 1e-5))))
+        for _ in range(tail):
+            step()
+        torch.cuda.synchronize()
     clk = clocks.stop()
     per_launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_s = starts[0].elapsed_time(ends[-1]) * 1e-3
@@ -294,6 +314,11 @@ def gpu_arm(args, w: W.Workload):
     units = roofline_units(w)
     value = aggregate(units["elements"], args.steps, world, max_s)
 
+    if args.profile_run:
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "workload": w.name, "value": value, "unit": UNIT,
+                              "per_launch_ms": statistics.mean(per_launch_ms)}), flush=True)
+        return
     # end to end through the C ABI from pinned host buffers: H2D inputs, scan, D2H output
     host = {k: v.cpu().pin_memory() for k, v in t.items()}
     dev_in = {k: torch.empty_like(v) for k, v in t.items()}
@@ -368,12 +393,15 @@ def gpu_arm(args, w: W.Workload):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile-run", action="store_true",
+                    help="timed steps only (no clock tail, end-to-end leg, probe or CPU baseline): "
+                         "the command line used under ncu")
     args = ap.parse_args(argv)
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":

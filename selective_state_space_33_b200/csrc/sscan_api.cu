@@ -241,9 +241,9 @@ sscan_status sscan_fwd(const sscan_problem* p, const void* u, const void* delta_
                        float* h_last, void* workspace, size_t workspace_bytes, void* stream) {
     g_err[0] = 0;
     if (sscan_status s = check_problem(p)) return s;
-    if (!out && !h_last) return fail(SSCAN_ERR_INVALID_ARG, "out and h_last are both NULL");
     const bool any = p->batch * p->dim > 0;
     if (any && p->seqlen > 0) {
+        if (!out && !h_last) return fail(SSCAN_ERR_INVALID_ARG, "out and h_last are both NULL");
         if (!u || !delta_raw || !A || !B) return fail(SSCAN_ERR_INVALID_ARG, "u, delta_raw, A, B are required");
         if (out && !C) return fail(SSCAN_ERR_INVALID_ARG, "C is required when out is written");
     }
@@ -262,8 +262,8 @@ sscan_status sscan_last_state(const sscan_problem* p, const void* u, const void*
                               size_t workspace_bytes, void* stream) {
     g_err[0] = 0;
     if (sscan_status s = check_problem(p)) return s;
-    if (!h_last) return fail(SSCAN_ERR_INVALID_ARG, "h_last is required");
     const bool any = p->batch * p->dim > 0;
+    if (any && !h_last) return fail(SSCAN_ERR_INVALID_ARG, "h_last is required");
     if (any && p->seqlen > 0 && (!u || !delta_raw || !A || !B))
         return fail(SSCAN_ERR_INVALID_ARG, "u, delta_raw, A, B are required");
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -64,6 +64,7 @@ def test_fwd_rejects_bad_arguments(lib):
     assert _fwd(lib, _p(flags=6)) == 1
     assert _fwd(lib, _p(), u=None) == 1
     assert _fwd(lib, _p(), out=None, h_last=None) == 1
+    assert b"both NULL" in lib.sscan_last_error()
     assert _fwd(lib, _p(), C=None) == 1
 
 

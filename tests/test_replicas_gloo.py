@@ -1,0 +1,79 @@
+"""Multi-process plumbing of bench.py on CPU (gloo, world size 2): the slowest rank's
+time is what every rank reports, whole-job throughput counts every rank's work,
+and the reference arm runs on rank 0 only."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    w, r = bench.init_dist("gloo")
+    t = bench.reduce_max(1.5 + rank)          # rank 1 is slower
+    v = bench.aggregate(1000, 10, w, t)
+    bench.barrier()
+    import torch.distributed as dist
+    dist.destroy_process_group()
+    q.put((r, w, t, v))
+
+
+def test_max_over_ranks_and_aggregate():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in ps)
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, world, t, v in res:
+        assert world == 2
+        assert t == pytest.approx(2.5)                   # the slowest rank's time
+        assert v == pytest.approx(1000 * 10 * 2 / 2.5 / 1e9)
+
+
+def _ref_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import contextlib
+    import io
+
+    import bench
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"])
+    q.put((rank, buf.getvalue()))
+
+
+def test_reference_arm_prints_on_rank0_only():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_ref_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    res = dict(q.get(timeout=300) for _ in ps)
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    import json
+    line = json.loads(res[0].strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert res[1].strip() == ""
