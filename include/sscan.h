@@ -107,6 +107,36 @@ SSCAN_API sscan_status sscan_last_state(const sscan_problem* problem, const void
                               size_t workspace_bytes, void* stream);
 
 /*
+ * Forward scan without a caller workspace (the paper has no counterpart: this
+ * is plumbing for callers that cannot allocate device memory).  Same arguments
+ * and results as sscan_fwd, minus workspace / workspace_bytes.
+ *
+ * Who needs it: code that may not call cudaMalloc or any allocator -- a plugin
+ * hosted by a framework that owns every byte of device memory and forbids
+ * outside allocations, or a latency-critical caller that cannot afford
+ * cudaMalloc's implicit device synchronisation.  Such callers still pass their
+ * own inputs and outputs; only the scratch moves inside the library.
+ *
+ * Scratch: a fixed 4 MiB array in the library's device memory (every GPU that
+ * loads libsscan holds it until the process exits).  It covers every problem
+ * whose (batch, L, D) tensors have 16-byte aligned bases and row pitches (the
+ * TMA-tiled path needs at most 3.8 MB).  A call whose path needs more scratch
+ * than that (possible only on the general path for unaligned tensors) returns
+ * SSCAN_ERR_WORKSPACE before anything is launched.  The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress, with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents; the kernels overwrite every scratch byte they later read, so nothing
+ * needs clearing.  Calls whose work overlaps on the GPU (different streams, or
+ * different host threads without ordering) race on the scratch: serialise them.
+ * No allocation or free of any kind happens in this call.
+ */
+SSCAN_API sscan_status sscan_fwd_noalloc(const sscan_problem* problem, const void* u, const void* delta_raw,
+                                         const float* delta_bias, const float* A, const void* B, const void* C,
+                                         const float* D_skip, const void* z, const float* h0, void* out,
+                                         float* h_last, void* stream);
+
+/*
  * Backward scan: gradients of sum(out * dout) with respect to every input of
  * sscan_fwd, recomputing the states on chip instead of storing them (sec. 4.1,
  * item 3).  du, ddelta_raw, dB, dC (and dz) are in io_dtype; dA, ddelta_bias, dD,

@@ -5,6 +5,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 
 #include "sscan.h"
 #include "sscan_generic.cuh"
@@ -212,6 +213,38 @@ void cast_out(const float* src, void* dst, int64_t n, cudaStream_t st) {
     if (n > 0) sscan::cast_kernel<T><<<blocks_for(n, 256), 256, 0, st>>>(src, static_cast<T*>(dst), n);
 }
 
+// Fixed device scratch for sscan_fwd_noalloc.  Every GPU that loads this library
+// holds these bytes until the process exits.  In host code the array's name is
+// only a host-side stand-in; its device address comes from cudaGetSymbolAddress.
+// 4 MiB covers every plan of the tiled path: fewer than kTiledMinCols CTA columns
+// times at most ceil(kTiledTargetCtas / cols) chunks bounds the chunk states by
+// 1480 * DC * (N + 1) floats, at most 3.8 MB for N <= 16.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device, looked up once per device
+// (with that device current) and cached.
+sscan_status noalloc_scratch(void** ptr) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(SSCAN_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(SSCAN_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return SSCAN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -275,6 +308,38 @@ sscan_status sscan_last_state(const sscan_problem* p, const void* u, const void*
     return run_fwd(p, make_args(p, u, delta_raw, delta_bias, A, B, nullptr, nullptr, nullptr, h0,
                                 nullptr, h_last),
                    workspace, st);
+}
+
+sscan_status sscan_fwd_noalloc(const sscan_problem* p, const void* u, const void* delta_raw,
+                               const float* delta_bias, const float* A, const void* B, const void* C,
+                               const float* D_skip, const void* z, const float* h0, void* out,
+                               float* h_last, void* stream) {
+    g_err[0] = 0;
+    if (sscan_status s = check_problem(p)) return s;
+    const bool any = p->batch * p->dim > 0;
+    if (any && p->seqlen > 0) {
+        if (!out && !h_last) return fail(SSCAN_ERR_INVALID_ARG, "out and h_last are both NULL");
+        if (!u || !delta_raw || !A || !B) return fail(SSCAN_ERR_INVALID_ARG, "u, delta_raw, A, B are required");
+        if (out && !C) return fail(SSCAN_ERR_INVALID_ARG, "C is required when out is written");
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!any) return SSCAN_OK;
+    if (p->seqlen == 0) return empty_sequence(p, h0, h_last, st);
+    const sscan::ScanArgs a = make_args(p, u, delta_raw, delta_bias, A, B, C, D_skip, z, h0, out, h_last);
+    // scratch of the path this call takes (run_fwd makes the same choice)
+    const size_t need =
+        tiled_ok(p, a) ? sscan::plan_tiled(p->batch, p->seqlen, p->dim, p->dstate,
+                                           sscan::tiled_channels_per_cta(p->dstate))
+                             .workspace_bytes
+                       : sscan::plan_fwd(p->batch, p->seqlen, p->dim, p->dstate).workspace_bytes;
+    if (need > kNoAllocScratchBytes)
+        return fail(SSCAN_ERR_WORKSPACE, "problem needs %zu bytes of scratch; the static scratch holds %zu", need,
+                    kNoAllocScratchBytes);
+    void* ws = nullptr;
+    if (need > 0) {
+        if (sscan_status s = noalloc_scratch(&ws)) return s;
+    }
+    return run_fwd(p, a, ws, st);
 }
 
 sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_raw,
