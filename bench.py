@@ -13,6 +13,7 @@ host cores instead (the reference arm: a plain sequential scan, never tuned).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -27,6 +28,8 @@ sys.path.insert(0, ROOT)
 from selective_state_space_33_b200 import workloads as W  # noqa: E402
 
 METRIC = "selective-scan fwd Gelem/s (B·L·D) & % of HBM/MUFU roofline at 2.8B-layer shape"
+METRIC_BWD = "selective-scan bwd Gelem/s (B·L·D), states recomputed on chip"
+METRIC_STEP = "selective-scan generation step Gelem/s (batch·D per token), state read and written in HBM"
 UNIT = "Gelem/s"
 DEFAULT_WORKLOAD = "mamba2.8b"
 SM_COUNT = 148
@@ -85,7 +88,19 @@ def roofline_units(w: W.Workload) -> dict:
     the SiLU gate (Bbar reuses Abar's exponential)."""
     s = 2 if w.io == "bf16" else 4
     E = w.batch * w.seqlen * w.dim
-    bytes_ = 4 * E * s + 2 * w.batch * w.seqlen * w.dstate * s + (w.dim * w.dstate + 2 * w.dim) * 4
+    BLN = w.batch * w.seqlen * w.dstate
+    if w.decode:
+        # one token: read and write the fp32 state (the dominant term), read u, delta_raw,
+        # z and write out (batch, D), read B, C (batch, N) and the parameters.
+        bytes_ = 2 * w.batch * w.dim * w.dstate * 4 + 4 * E * s + 2 * BLN * s + (w.dim * w.dstate + 2 * w.dim) * 4
+        return {"elements": E, "bytes": bytes_, "exps": E * (w.dstate + 2)}
+    if w.backward:
+        # read u, delta_raw, z, dout, write du, ddelta_raw, dz; read B, C, write dB, dC;
+        # A, bias, D_skip in and their gradients out.  Exponentials: Abar once per state
+        # (recomputed on chip), softplus, the gate's sigmoid, softplus' derivative.
+        bytes_ = 7 * E * s + 4 * BLN * s + 2 * (w.dim * w.dstate + 2 * w.dim) * 4
+        return {"elements": E, "bytes": bytes_, "exps": E * (w.dstate + 3)}
+    bytes_ = 4 * E * s + 2 * BLN * s + (w.dim * w.dstate + 2 * w.dim) * 4
     return {"elements": E, "bytes": bytes_, "exps": E * (w.dstate + 2)}
 
 
@@ -234,7 +249,6 @@ def workload_config(w: W.Workload, world: int) -> dict:
 # ----------------------------------------------------------------------------- GPU arm
 def ex2_probe(torch, lib, device, repeats=5):
     """Measured MUFU ex2 rate (exps/s) of the whole GPU."""
-    import ctypes
     blocks, threads, iters = SM_COUNT * 8, 256, 4096
     sink = torch.empty(blocks * threads, dtype=torch.float32, device=device)
     st = torch.cuda.current_stream()
@@ -269,17 +283,35 @@ def gpu_arm(args, w: W.Workload):
     t = W.to_device(x, dev)
     out = torch.empty_like(t["u"])
     prob = sb.make_problem(w.batch, w.seqlen, w.dim, w.dstate, sb.SSCAN_BF16 if w.io == "bf16" else sb.SSCAN_F32)
-    ws_bytes = sb.sscan_workspace_size(prob, sb.SSCAN_OP_FWD)
+    op = sb.SSCAN_OP_BWD if w.backward else sb.SSCAN_OP_FWD
+    ws_bytes = sb.sscan_workspace_size(prob, op)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream()
+    grads = None
+    if w.backward:
+        grads = sb.sscan_bwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t["delta_bias"],
+                             t["D_skip"], t.get("z"), workspace=ws)
+
+    if w.decode:
+        sq = {k: (v[:, 0].contiguous() if k in ("u", "delta_raw", "z", "B", "C") else v) for k, v in t.items()}
+        out = torch.empty_like(sq["u"])
 
     def step():
-        sb.sscan_fwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["delta_bias"], t["D_skip"], t.get("z"),
-                     out=out, workspace=ws, stream=st)
+        if w.decode:
+            sb.sscan_step(sq["u"], sq["delta_raw"], sq["A"], sq["B"], sq["C"], sq["state"], sq["delta_bias"],
+                          sq["D_skip"], sq.get("z"), out=out, stream=st)
+        elif w.backward:
+            sb.sscan_bwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t["delta_bias"], t["D_skip"],
+                         t.get("z"), grads=grads, workspace=ws, stream=st)
+        else:
+            sb.sscan_fwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["delta_bias"], t["D_skip"], t.get("z"),
+                         out=out, workspace=ws, stream=st)
 
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
+    lib.sscan_last_launch_count.restype = ctypes.c_int
+    launches_per_step = int(lib.sscan_last_launch_count())  # kernels one step enqueues
 
     uuid = ""
     try:
@@ -319,7 +351,22 @@ def gpu_arm(args, w: W.Workload):
             print(json.dumps({"profile_run": True, "workload": w.name, "value": value, "unit": UNIT,
                               "per_launch_ms": statistics.mean(per_launch_ms)}), flush=True)
         return
-    # end to end through the C ABI from pinned host buffers: H2D inputs, scan, D2H output
+    if w.backward or w.decode:
+        e2e_value, h2d, d2h = None, 0, 0
+    else:
+        e2e_value, h2d, d2h = e2e_leg(args, t, out, ws, st, units, world, dev)
+    if rank != 0:
+        return
+    finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk, e2e_value, h2d, d2h,
+           launches_per_step, world)
+
+
+def e2e_leg(args, t, out, ws, st, units, world, dev):
+    """End to end through the C ABI from pinned host buffers: every step copies the
+    inputs host -> device, runs the scan and copies the output back."""
+    import torch
+
+    from selective_state_space_33_b200 import binding as sb
     host = {k: v.cpu().pin_memory() for k, v in t.items()}
     dev_in = {k: torch.empty_like(v) for k, v in t.items()}
     host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -344,10 +391,11 @@ def gpu_arm(args, w: W.Workload):
     eb.record(st)
     torch.cuda.synchronize()
     e2e_s = reduce_max(ea.elapsed_time(eb) * 1e-3, dev if world > 1 else None)
-    e2e_value = aggregate(units["elements"], args.steps, world, e2e_s)
+    return aggregate(units["elements"], args.steps, world, e2e_s), h2d, d2h
 
-    if rank != 0:
-        return
+
+def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk, e2e_value, h2d, d2h,
+           launches_per_step, world):
     peaks = measured_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", HBM_FALLBACK_GBS))
     hbm_src = "measured" if "hbm_gbs" in peaks else "fallback"
@@ -358,22 +406,22 @@ def gpu_arm(args, w: W.Workload):
     exps_rate = units["exps"] / launch_s
     gbs = units["bytes"] / launch_s / 1e9
     t_roof = max(units["bytes"] / (hbm_peak * 1e9), units["exps"] / mufu_nominal)
-    launches_per_step = 1 if ws_bytes == 0 else 3
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not w.backward and not w.decode:
         rate, cores, rows, secs = cpu_oracle_rate(x, w, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{rows} random rows of {w.batch * w.dim} x L={w.seqlen} ({rows * w.seqlen} elements, "
                          f"{secs:.1f} s)"}
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_BWD if w.backward else (METRIC_STEP if w.decode else METRIC), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": max_s / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(w, world),
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": None if e2e_value is None else {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                                               "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
-        "roofline": {
+        "roofline": hbm_roofline(units, launch_s, hbm_peak, hbm_src) if w.decode else {
             "bound": "alu", "pipe": "MUFU ex2", "achieved": exps_rate / 1e9, "peak": mufu_nominal / 1e9,
             "unit": "Gexp/s", "frac": exps_rate / mufu_nominal, "traffic": None,
             "peak_source": f"derived: {SM_COUNT} SMs x {MUFU_PER_SM_CLK} ex2/clk x {sm_max:.0f} MHz",
@@ -388,6 +436,13 @@ def gpu_arm(args, w: W.Workload):
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
+
+
+def hbm_roofline(units, launch_s, hbm_peak, hbm_src):
+    gbs = units["bytes"] / launch_s / 1e9
+    return {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+            "traffic": None, "source": hbm_src, "per_launch_ms": launch_s * 1e3,
+            "alg_bytes_per_launch": units["bytes"]}
 
 
 def main(argv=None):

@@ -151,17 +151,37 @@ SSCAN_API sscan_status sscan_bwd(const sscan_problem* problem, const void* u, co
                        void* dC, float* dD, void* dz, float* dh0, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/*
+ * One recurrence step for autoregressive generation: every (batch, channel)
+ * advances its state by one token, h <- Abar h + Bbar x, and emits
+ * out = (C.h + D_skip x) SiLU(z) -- constant time and memory per token with no
+ * cache that grows with the context (sec. 5; sec. 2.1 eqs. (2), (3a), (3b) at one t).
+ * problem->seqlen must be 1; u, delta_raw, z, out are (batch, D) and B, C are
+ * (batch, N) in io_dtype; state (batch, D, N) fp32 is read and overwritten in
+ * place.  The result equals sscan_fwd with seqlen 1, h0 = state, h_last = state.
+ * delta_bias, D_skip and z may be NULL.  No workspace.
+ */
+SSCAN_API sscan_status sscan_step(const sscan_problem* problem, const void* u, const void* delta_raw,
+                                  const float* delta_bias, const float* A, const void* B, const void* C,
+                                  const float* D_skip, const void* z, float* state, void* out, void* stream);
+
 /* Static, human-readable name of a status code. */
 SSCAN_API const char* sscan_status_string(sscan_status status);
 
 /* One-line reason for the most recent failed call on this thread ("" if none). */
 SSCAN_API const char* sscan_last_error(void);
 
+/* Number of kernels the most recent sscan_fwd / sscan_fwd_noalloc /
+ * sscan_last_state / sscan_bwd call on this thread enqueued (memsets and copies
+ * not counted). */
+SSCAN_API int sscan_last_launch_count(void);
+
 /*
  * Device-side status of the library's kernels on the current device: *flags
- * receives the OR of every error bit raised since the last clear (bit 0: a
- * bounded wait for an asynchronous tile copy gave up, so that kernel stopped
- * early and its outputs are incomplete).  clear != 0 resets the word after
+ * receives the OR of every error bit raised since the last clear (bit 0: in a
+ * forward kernel, bit 1: in the backward kernel, a bounded wait for an
+ * asynchronous tile copy gave up, so that kernel stopped early and its outputs
+ * are incomplete).  clear != 0 resets the word after
  * reading.  Synchronous: it waits for work already submitted to the device.
  */
 SSCAN_API sscan_status sscan_device_status(int clear, unsigned int* flags);

@@ -57,6 +57,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sscan_last_state.restype = ctypes.c_int
     lib.sscan_bwd.argtypes = [pp] + [vp] * 20 + [sz, vp]
     lib.sscan_bwd.restype = ctypes.c_int
+    lib.sscan_step.argtypes = [pp] + [vp] * 10 + [vp]
+    lib.sscan_step.restype = ctypes.c_int
     lib.sscan_status_string.argtypes = [ctypes.c_int]
     lib.sscan_status_string.restype = ctypes.c_char_p
     lib.sscan_last_error.argtypes = []
@@ -177,20 +179,36 @@ def sscan_last_state(u, delta_raw, A, B, delta_bias=None, h0=None, *, delta_soft
 
 
 def sscan_bwd(u, delta_raw, A, B, C, dout, delta_bias=None, D_skip=None, z=None, h0=None, *,
-              delta_softplus=True, want_dh0=True, workspace=None, stream=None):
+              delta_softplus=True, want_dh0=True, grads=None, workspace=None, stream=None):
     """Gradients of sum(out * dout).  Returns a dict keyed du, ddelta_raw, dA, dB, dC and,
-    when the matching input is given, ddelta_bias, dD, dz; dh0 when ``want_dh0``."""
+    when the matching input is given, ddelta_bias, dD, dz; dh0 when ``want_dh0``.
+    ``grads`` may supply preallocated outputs under the same keys."""
     prob = _io_problem(u, B, delta_softplus)
     _check_inputs(prob, u, delta_raw, A, B, C, delta_bias, D_skip, z, h0)
     _expect(dout, "dout", u.shape, u.dtype, u.device)
     f32 = dict(dtype=torch.float32, device=u.device)
-    g = {"du": torch.empty_like(u), "ddelta_raw": torch.empty_like(u),
-         "dA": torch.empty((prob.dim, prob.dstate), **f32), "dB": torch.empty_like(B),
-         "dC": torch.empty_like(C)}
-    g["ddelta_bias"] = torch.empty(prob.dim, **f32) if delta_bias is not None else None
-    g["dD"] = torch.empty(prob.dim, **f32) if D_skip is not None else None
-    g["dz"] = torch.empty_like(u) if z is not None else None
-    g["dh0"] = torch.empty((prob.batch, prob.dim, prob.dstate), **f32) if want_dh0 else None
+    pre = grads or {}
+    g = {"du": pre.get("du", None), "ddelta_raw": pre.get("ddelta_raw", None), "dA": pre.get("dA", None),
+         "dB": pre.get("dB", None), "dC": pre.get("dC", None)}
+    g["du"] = g["du"] if g["du"] is not None else torch.empty_like(u)
+    g["ddelta_raw"] = g["ddelta_raw"] if g["ddelta_raw"] is not None else torch.empty_like(u)
+    g["dA"] = g["dA"] if g["dA"] is not None else torch.empty((prob.dim, prob.dstate), **f32)
+    g["dB"] = g["dB"] if g["dB"] is not None else torch.empty_like(B)
+    g["dC"] = g["dC"] if g["dC"] is not None else torch.empty_like(C)
+    g["ddelta_bias"] = (pre.get("ddelta_bias") if pre.get("ddelta_bias") is not None
+                        else torch.empty(prob.dim, **f32)) if delta_bias is not None else None
+    g["dD"] = (pre.get("dD") if pre.get("dD") is not None else torch.empty(prob.dim, **f32)) \
+        if D_skip is not None else None
+    g["dz"] = (pre.get("dz") if pre.get("dz") is not None else torch.empty_like(u)) if z is not None else None
+    g["dh0"] = (pre.get("dh0") if pre.get("dh0") is not None
+                else torch.empty((prob.batch, prob.dim, prob.dstate), **f32)) if want_dh0 else None
+    for k, ref in (("du", u), ("ddelta_raw", u), ("dB", B), ("dC", C), ("dz", u)):
+        if g[k] is not None:
+            _expect(g[k], k, ref.shape, ref.dtype, u.device)
+    _expect(g["dA"], "dA", (prob.dim, prob.dstate), torch.float32, u.device)
+    _expect(g["ddelta_bias"], "ddelta_bias", (prob.dim,), torch.float32, u.device)
+    _expect(g["dD"], "dD", (prob.dim,), torch.float32, u.device)
+    _expect(g["dh0"], "dh0", (prob.batch, prob.dim, prob.dstate), torch.float32, u.device)
     ws, nbytes = _workspace(prob, SSCAN_OP_BWD, workspace, u.device)
     _check(load_library().sscan_bwd(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias), _ptr(A),
                                     _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h0), _ptr(dout),
@@ -198,3 +216,33 @@ def sscan_bwd(u, delta_raw, A, B, C, dout, delta_bias=None, D_skip=None, z=None,
                                     _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]),
                                     _ptr(g["dz"]), _ptr(g["dh0"]), _ptr(ws), nbytes, _stream(stream)))
     return {k: v for k, v in g.items() if v is not None}
+
+
+def sscan_step(u, delta_raw, A, B, C, state, delta_bias=None, D_skip=None, z=None, *, delta_softplus=True,
+               out=None, stream=None):
+    """One generation step: u, delta_raw, z (batch, D); B, C (batch, N); state (batch, D, N)
+    fp32 updated in place.  Returns out (batch, D)."""
+    if u.dim() != 2 or B.dim() != 2:
+        raise ValueError("u must be (batch, D) and B (batch, N)")
+    if u.dtype not in _IO_CODES:
+        raise TypeError(f"I/O tensors must be float32 or bfloat16, got {u.dtype}")
+    batch, D = u.shape
+    N = B.shape[1]
+    prob = make_problem(batch, 1, D, N, _IO_CODES[u.dtype], delta_softplus)
+    dev, io = u.device, u.dtype
+    if dev.type != "cuda":
+        raise ValueError("libsscan works on CUDA tensors only")
+    for t, name, shape in ((delta_raw, "delta_raw", (batch, D)), (z, "z", (batch, D)), (B, "B", (batch, N)),
+                           (C, "C", (batch, N))):
+        _expect(t, name, shape, io, dev)
+    _expect(A, "A", (D, N), torch.float32, dev)
+    _expect(delta_bias, "delta_bias", (D,), torch.float32, dev)
+    _expect(D_skip, "D_skip", (D,), torch.float32, dev)
+    _expect(state, "state", (batch, D, N), torch.float32, dev)
+    if out is None:
+        out = torch.empty_like(u)
+    _expect(out, "out", (batch, D), io, dev)
+    _check(load_library().sscan_step(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias), _ptr(A),
+                                     _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(state), _ptr(out),
+                                     _stream(stream)))
+    return out

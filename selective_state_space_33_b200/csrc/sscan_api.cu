@@ -16,6 +16,7 @@
 namespace {
 
 thread_local char g_err[256] = "";
+thread_local int g_launches = 0;  // kernels the most recent call on this thread enqueued
 
 sscan_status fail(sscan_status s, const char* fmt, ...) {
     va_list ap;
@@ -75,6 +76,7 @@ void dispatch_fwd_rows(const sscan::ScanArgs& a, int mode, cudaStream_t st) {
 }
 
 void fwd_rows(const sscan::ScanArgs& a, int io, int mode, cudaStream_t st) {
+    ++g_launches;
     if (io == SSCAN_BF16) dispatch_fwd_rows<__nv_bfloat16>(a, mode, st);
     else dispatch_fwd_rows<float>(a, mode, st);
 }
@@ -131,6 +133,7 @@ sscan_status run_rows(const sscan_problem* p, sscan::ScanArgs a, void* ws, cudaS
         sscan::ScanArgs c = a;
         if (want_out) c.h_last = nullptr;  // the output pass writes h_last itself
         sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate, 128), 128, 0, st>>>(c);
+        ++g_launches;
         if (sscan_status s = cuda_check("carry kernel")) return s;
         if (!want_out) return SSCAN_OK;
     }
@@ -149,8 +152,8 @@ bool tiled_ok(const sscan_problem* p, const sscan::ScanArgs& a) {
 }
 
 sscan_status run_tiled(const sscan_problem* p, const sscan::ScanArgs& a, void* ws, cudaStream_t st) {
-    const int64_t DC = sscan::tiled_channels_per_cta(p->dstate);
-    const sscan::FwdPlan plan = sscan::plan_tiled(p->batch, p->seqlen, p->dim, p->dstate, DC);
+    const sscan::TiledGeom geo = sscan::tiled_geometry(p->batch, p->seqlen, p->dim, p->dstate);
+    const sscan::FwdPlan plan = sscan::plan_tiled(p->batch, p->seqlen, p->dim, p->dstate, geo.DC);
     sscan::TiledArgs t{};
     t.batch = p->batch;
     t.L = p->seqlen;
@@ -174,7 +177,8 @@ sscan_status run_tiled(const sscan_problem* p, const sscan::ScanArgs& a, void* w
     if (plan.nchunks > 1) {
         t.ws_state = static_cast<float*>(ws);
         t.ws_dsum = t.ws_state + plan.state_floats;
-        e = sscan::launch_fwd_tiled(t, ptr, bf16, sscan::kTiledAgg, st);
+        e = sscan::launch_fwd_tiled(t, ptr, geo, bf16, sscan::kTiledAgg, st);
+        ++g_launches;
         if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "chunk aggregate kernel: %s", cudaGetErrorString(e));
         sscan::ScanArgs c = a;
         c.nchunks = plan.nchunks;
@@ -183,12 +187,24 @@ sscan_status run_tiled(const sscan_problem* p, const sscan::ScanArgs& a, void* w
         c.ws_dsum = t.ws_dsum;
         if (want_out) c.h_last = nullptr;
         sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate, 128), 128, 0, st>>>(c);
+        ++g_launches;
         if (sscan_status s = cuda_check("carry kernel")) return s;
         if (!want_out) return SSCAN_OK;
     }
-    e = sscan::launch_fwd_tiled(t, ptr, bf16, want_out ? sscan::kTiledOut : sscan::kTiledLast, st);
+    ++g_launches;
+    e = sscan::launch_fwd_tiled(t, ptr, geo, bf16, want_out ? sscan::kTiledOut : sscan::kTiledLast, st);
     if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "tiled forward kernel: %s", cudaGetErrorString(e));
     return SSCAN_OK;
+}
+
+// The tiled backward reads and writes every (batch, L, D) tensor and the B, C rows
+// through TMA: 16-byte aligned bases, row pitches and B/C rows.
+bool bwd_tiled_ok(const sscan_problem* p, const void* u, const void* dr, const void* z, const void* dout,
+                  const void* B, const void* C, const void* du, const void* ddr, const void* dz) {
+    const int64_t es = p->io_dtype == SSCAN_BF16 ? 2 : 4;
+    return (p->dim * es) % 16 == 0 && (p->dstate * es) % 16 == 0 && aligned16(u) && aligned16(dr) &&
+           aligned16(z) && aligned16(dout) && aligned16(B) && aligned16(C) && aligned16(du) && aligned16(ddr) &&
+           aligned16(dz) && p->seqlen < (int64_t(1) << 31) && p->dim < (int64_t(1) << 31);
 }
 
 sscan_status run_fwd(const sscan_problem* p, const sscan::ScanArgs& a, void* ws, cudaStream_t st) {
@@ -198,6 +214,7 @@ sscan_status run_fwd(const sscan_problem* p, const sscan::ScanArgs& a, void* ws,
 
 template <typename T, int NMAX>
 void launch_bwd_rows(const sscan::BwdArgs& g, cudaStream_t st) {
+    ++g_launches;
     sscan::bwd_rows_kernel<T, NMAX><<<blocks_for(g.f.batch * g.f.D, 128), 128, 0, st>>>(g);
 }
 
@@ -210,7 +227,10 @@ void dispatch_bwd_rows(const sscan::BwdArgs& g, cudaStream_t st) {
 
 template <typename T>
 void cast_out(const float* src, void* dst, int64_t n, cudaStream_t st) {
-    if (n > 0) sscan::cast_kernel<T><<<blocks_for(n, 256), 256, 0, st>>>(src, static_cast<T*>(dst), n);
+    if (n > 0) {
+        sscan::cast_kernel<T><<<blocks_for(n, 256), 256, 0, st>>>(src, static_cast<T*>(dst), n);
+        ++g_launches;
+    }
 }
 
 // Fixed device scratch for sscan_fwd_noalloc.  Every GPU that loads this library
@@ -257,7 +277,7 @@ size_t sscan_workspace_size(const sscan_problem* p, int op) {
             // enough for either path (the choice also depends on pointer alignment)
             const size_t g = sscan::plan_fwd(p->batch, p->seqlen, p->dim, p->dstate).workspace_bytes;
             const size_t t = sscan::plan_tiled(p->batch, p->seqlen, p->dim, p->dstate,
-                                               sscan::tiled_channels_per_cta(p->dstate))
+                                               sscan::tiled_geometry(p->batch, p->seqlen, p->dim, p->dstate).DC)
                                  .workspace_bytes;
             return g > t ? g : t;
         }
@@ -273,6 +293,7 @@ sscan_status sscan_fwd(const sscan_problem* p, const void* u, const void* delta_
                        const float* D_skip, const void* z, const float* h0, void* out,
                        float* h_last, void* workspace, size_t workspace_bytes, void* stream) {
     g_err[0] = 0;
+    g_launches = 0;
     if (sscan_status s = check_problem(p)) return s;
     const bool any = p->batch * p->dim > 0;
     if (any && p->seqlen > 0) {
@@ -294,6 +315,7 @@ sscan_status sscan_last_state(const sscan_problem* p, const void* u, const void*
                               const float* h0, float* h_last, void* workspace,
                               size_t workspace_bytes, void* stream) {
     g_err[0] = 0;
+    g_launches = 0;
     if (sscan_status s = check_problem(p)) return s;
     const bool any = p->batch * p->dim > 0;
     if (any && !h_last) return fail(SSCAN_ERR_INVALID_ARG, "h_last is required");
@@ -315,6 +337,7 @@ sscan_status sscan_fwd_noalloc(const sscan_problem* p, const void* u, const void
                                const float* D_skip, const void* z, const float* h0, void* out,
                                float* h_last, void* stream) {
     g_err[0] = 0;
+    g_launches = 0;
     if (sscan_status s = check_problem(p)) return s;
     const bool any = p->batch * p->dim > 0;
     if (any && p->seqlen > 0) {
@@ -329,7 +352,7 @@ sscan_status sscan_fwd_noalloc(const sscan_problem* p, const void* u, const void
     // scratch of the path this call takes (run_fwd makes the same choice)
     const size_t need =
         tiled_ok(p, a) ? sscan::plan_tiled(p->batch, p->seqlen, p->dim, p->dstate,
-                                           sscan::tiled_channels_per_cta(p->dstate))
+                                           sscan::tiled_geometry(p->batch, p->seqlen, p->dim, p->dstate).DC)
                              .workspace_bytes
                        : sscan::plan_fwd(p->batch, p->seqlen, p->dim, p->dstate).workspace_bytes;
     if (need > kNoAllocScratchBytes)
@@ -349,6 +372,7 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
                        void* dC, float* dD, void* dz, float* dh0, void* workspace,
                        size_t workspace_bytes, void* stream) {
     g_err[0] = 0;
+    g_launches = 0;
     if (sscan_status s = check_problem(p)) return s;
     if ((z == nullptr) != (dz == nullptr)) return fail(SSCAN_ERR_INVALID_ARG, "dz must be given exactly when z is");
     if (dD && !D_skip) return fail(SSCAN_ERR_INVALID_ARG, "dD needs D_skip");
@@ -379,6 +403,63 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
         return SSCAN_OK;
     }
     const sscan::BwdPlan plan = sscan::plan_bwd(p->batch, p->seqlen, p->dim, p->dstate);
+    float* ws = static_cast<float*>(workspace);
+    e = cudaMemsetAsync(ws, 0, (size_t)(2 * BLN) * sizeof(float), st);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing workspace: %s", cudaGetErrorString(e));
+    if (bwd_tiled_ok(p, u, delta_raw, z, dout, B, C, du, ddelta_raw, dz)) {
+        // checkpoint pass: the state before every 8th step, by the tiled forward kernel
+        const sscan::TiledGeom geo = sscan::tiled_geometry(p->batch, p->seqlen, p->dim, p->dstate);
+        sscan::TiledArgs t{};
+        t.batch = p->batch;
+        t.L = p->seqlen;
+        t.D = p->dim;
+        t.N = (int)p->dstate;
+        t.softplus = (p->flags & SSCAN_DELTA_SOFTPLUS) ? 1 : 0;
+        t.has_z = 0;
+        t.bias = delta_bias;
+        t.A = A;
+        t.h0 = h0;
+        t.B = B;
+        t.chunk_len = p->seqlen;
+        t.nchunks = 1;
+        t.ws_ckpt = ws + 2 * BLN;
+        t.nck = (p->seqlen + sscan::kBwdTiledSeg - 1) / sscan::kBwdTiledSeg;
+        sscan::TiledPtrs tp{u, delta_raw, nullptr, nullptr};
+        const int bf16 = p->io_dtype == SSCAN_BF16;
+        ++g_launches;
+        e = sscan::launch_fwd_tiled(t, tp, geo, bf16, sscan::kTiledCkpt, st);
+        if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "checkpoint kernel: %s", cudaGetErrorString(e));
+        sscan::BwdTiledArgs ba{};
+        ba.batch = p->batch;
+        ba.L = p->seqlen;
+        ba.D = p->dim;
+        ba.N = (int)p->dstate;
+        ba.softplus = t.softplus;
+        ba.has_z = z != nullptr;
+        ba.bias = delta_bias;
+        ba.A = A;
+        ba.Dskip = D_skip;
+        ba.ws_ckpt = t.ws_ckpt;
+        ba.nck = t.nck;
+        ba.dB32 = ws;
+        ba.dC32 = ws + BLN;
+        ba.dA = dA;
+        ba.dD = dD;
+        ba.dbias = ddelta_bias;
+        ba.dh0 = dh0;
+        sscan::BwdTiledPtrs bp{u, delta_raw, z, dout, B, C, du, ddelta_raw, dz};
+        ++g_launches;
+        e = sscan::launch_bwd_tiled(ba, bp, bf16, st);
+        if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "backward kernel: %s", cudaGetErrorString(e));
+        if (bf16) {
+            cast_out<__nv_bfloat16>(ws, dB, BLN, st);
+            cast_out<__nv_bfloat16>(ws + BLN, dC, BLN, st);
+        } else {
+            cast_out<float>(ws, dB, BLN, st);
+            cast_out<float>(ws + BLN, dC, BLN, st);
+        }
+        return cuda_check("gradient cast kernel");
+    }
     sscan::BwdArgs g{};
     g.f = make_args(p, u, delta_raw, delta_bias, A, B, C, D_skip, z, h0, nullptr, nullptr);
     g.dout = dout;
@@ -390,12 +471,9 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
     g.dz = dz;
     g.dh0 = dh0;
     g.nseg = plan.nseg;
-    float* ws = static_cast<float*>(workspace);
     g.dB32 = ws;
     g.dC32 = ws + BLN;
     g.ckpt = ws + 2 * BLN;
-    e = cudaMemsetAsync(ws, 0, (size_t)(2 * BLN) * sizeof(float), st);
-    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing workspace: %s", cudaGetErrorString(e));
     if (p->io_dtype == SSCAN_BF16) dispatch_bwd_rows<__nv_bfloat16>(g, st);
     else dispatch_bwd_rows<float>(g, st);
     if (sscan_status s = cuda_check("backward kernel")) return s;
@@ -407,6 +485,37 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
         cast_out<float>(g.dC32, dC, BLN, st);
     }
     return cuda_check("gradient cast kernel");
+}
+
+sscan_status sscan_step(const sscan_problem* p, const void* u, const void* delta_raw, const float* delta_bias,
+                        const float* A, const void* B, const void* C, const float* D_skip, const void* z,
+                        float* state, void* out, void* stream) {
+    g_err[0] = 0;
+    g_launches = 0;
+    if (sscan_status s = check_problem(p)) return s;
+    if (p->seqlen != 1) return fail(SSCAN_ERR_INVALID_ARG, "sscan_step takes seqlen == 1, got %lld", (long long)p->seqlen);
+    if (p->batch * p->dim == 0) return SSCAN_OK;
+    if (!u || !delta_raw || !A || !B || !C || !state || !out)
+        return fail(SSCAN_ERR_INVALID_ARG, "u, delta_raw, A, B, C, state, out are required");
+    sscan::StepArgs a{};
+    a.batch = p->batch;
+    a.D = p->dim;
+    a.N = (int)p->dstate;
+    a.softplus = (p->flags & SSCAN_DELTA_SOFTPLUS) ? 1 : 0;
+    a.u = u;
+    a.delta_raw = delta_raw;
+    a.bias = delta_bias;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.Dskip = D_skip;
+    a.z = z;
+    a.state = state;
+    a.out = out;
+    ++g_launches;
+    const cudaError_t e = sscan::launch_step(a, p->io_dtype == SSCAN_BF16, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "step kernel: %s", cudaGetErrorString(e));
+    return SSCAN_OK;
 }
 
 const char* sscan_status_string(sscan_status s) {
@@ -422,11 +531,16 @@ const char* sscan_status_string(sscan_status s) {
 
 const char* sscan_last_error(void) { return g_err; }
 
+int sscan_last_launch_count(void) { return g_launches; }
+
 sscan_status sscan_device_status(int clear, unsigned int* flags) {
     g_err[0] = 0;
     if (!flags) return fail(SSCAN_ERR_INVALID_ARG, "flags is NULL");
-    const cudaError_t e = sscan::read_device_error(flags, clear);
+    unsigned int f1 = 0, f2 = 0;
+    cudaError_t e = sscan::read_device_error(&f1, clear);
+    if (e == cudaSuccess) e = sscan::read_device_error_bwd(&f2, clear);
     if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+    *flags = f1 | f2;
     return SSCAN_OK;
 }
 

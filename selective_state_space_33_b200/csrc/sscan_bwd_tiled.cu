@@ -1,0 +1,538 @@
+// sscan_bwd_tiled.cu -- backward of the selective scan for sm_100a, with the states
+// recomputed on chip (Mamba technical summary page, sec. 4.1 item 3).
+//
+// A forward pass in checkpoint mode (sscan_tiled.cu) first stores the state before
+// every 8th step.  This kernel then walks each (batch, 32-channel) block through
+// the sequence in reverse, 8 steps (one tile) at a time:
+//   TMA brings u, delta_raw, z, dout and the B, C rows of the tile into a 2-stage
+//   ring (bounded mbarrier waits);
+//   phase P turns them into fp32 (delta, x), (dy, dz factor, softplus') and the
+//   skip terms -- dy = dout SiLU(z), dz = dout y SiLU'(z), SiLU' = s (1 + z (1 - s));
+//   each lane recomputes its 4 states through the tile from the checkpoint,
+//   keeping h_t in shared memory, then runs the adjoint recurrence backwards:
+//     lam_t = C_t dy_t + Abar_{t+1} lam_{t+1}
+//     dx   += lam beta B,   dB += lam beta x,   dC += dy h_t        (beta = Bbar / B)
+//     d delta += lam Abar (A h_{t-1} + B x)
+//     dA   += delta lam Abar h_{t-1} + lam B x delta^2 psi(delta A)
+//   with psi(q) = (q e^q - expm1(q)) / q^2 (its Taylor series for |q| < 1/2, where the
+//   closed form would cancel) and beta = delta phi1(delta A) (series near 0);
+//   and the per-element sums over a channel's lanes, and the (t, n) sums over the
+//   channels of a warp, are formed with shuffles before anything touches memory.
+// dB and dC of a tile are summed across the CTA's warps in shared memory and then
+// added to fp32 accumulators in global memory; dA, dD and the bias gradient are
+// per-channel sums added once at the end.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+
+#include "sscan_launch.h"
+#include "sscan_math.cuh"
+#include "sscan_tma.cuh"
+
+namespace sscan {
+
+__device__ unsigned int g_device_error_bwd = 0;
+
+namespace {
+
+constexpr int kTB = 8;  // steps per tile (= checkpoint spacing of the forward kernel)
+constexpr int kWarpsB = 4;
+constexpr int kThreadsB = kWarpsB * 32;
+
+__device__ __forceinline__ float2 g2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 ex2p(float2 q) { return g2(ex2(q.x), ex2(q.y)); }
+
+template <typename T> struct BPair;
+template <> struct BPair<float> {
+    using type = float2;
+    static __device__ __forceinline__ float2 f(float2 v) { return v; }
+};
+template <> struct BPair<__nv_bfloat16> {
+    using type = __nv_bfloat162;
+    static __device__ __forceinline__ float2 f(__nv_bfloat162 v) { return __bfloat1622float2(v); }
+};
+
+template <typename T, int NG>
+struct BCfg {
+    static constexpr int CW = 32 / NG;                    // channels per warp
+    static constexpr int DC = CW * kWarpsB;               // channels per CTA
+    static constexpr int NS = NG * 4;                     // states covered
+    static constexpr int RAW = kTB * DC * (int)sizeof(T);
+    static constexpr int RAWBC = kTB * NS * (int)sizeof(T);
+    static constexpr int STAGE = 4 * RAW + 2 * RAWBC;     // u, delta_raw, z, dout, B, C
+    static constexpr int STAGES = 2;
+    static constexpr int PAIRS = kTB * DC / 2;
+    static constexpr int OFF_RAW = 0;
+    static constexpr int OFF_DX = OFF_RAW + STAGES * STAGE;     // float4 (d, d, x, x)      [kTB][DC]
+    static constexpr int OFF_DQ = OFF_DX + kTB * DC * 16;       // float4 (dy, dy, dzf, sr) [kTB][DC]
+    static constexpr int OFF_DD = OFF_DQ + kTB * DC * 16;       // float2 (D dy, D x)       [kTB][DC]
+    static constexpr int OFF_B = OFF_DD + kTB * DC * 8;         // float [kTB][NS]
+    static constexpr int OFF_C = OFF_B + kTB * NS * 4;          // float [kTB][NS]
+    static constexpr int OFF_HS = OFF_C + kTB * NS * 4;         // float4 [kTB][kThreadsB] recomputed states
+    static constexpr int OFF_ACC = OFF_HS + kTB * kThreadsB * 16;  // float [kTB][NS][2] dB, dC of the tile
+    static constexpr int OFF_OUT = OFF_ACC + kTB * NS * 2 * 4;  // [2 buffers][3 tensors][RAW]
+    static constexpr int OFF_BAR = OFF_OUT + 2 * 3 * RAW;
+    static constexpr int SMEM = OFF_BAR + STAGES * 8;
+};
+
+// Transposed butterfly over the NG lanes of a channel (lane bits at multiples of CW),
+// as in the forward kernel: lane g ends with the full sum for step g of the block.
+template <int NG, int CW>
+__device__ __forceinline__ float treduce_g(float (&p)[NG], int g) {
+    if constexpr (NG == 1) {
+        return p[0];
+    } else {
+        float cur[NG];
+#pragma unroll
+        for (int j = 0; j < NG; ++j) cur[j] = p[j];
+#pragma unroll
+        for (int m = NG / 2; m >= 1; m /= 2) {
+            const bool up = (g & m) != 0;
+#pragma unroll
+            for (int j = 0; j < m; ++j) {
+                const float keep = up ? cur[m + j] : cur[j];
+                const float send = up ? cur[j] : cur[m + j];
+                cur[j] = keep + __shfl_xor_sync(0xffffffffu, send, m * CW);
+            }
+        }
+        return cur[0];
+    }
+}
+
+// Sum 8 values over the CW channel lanes of a warp (the low lane bits): three
+// transposed rounds leave value (c & 7) in lane c summed over 8 lanes, then plain
+// rounds fold the remaining channel bits.
+template <int CW>
+__device__ __forceinline__ float treduce_c8(float (&v)[8], int c) {
+    float cur[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) cur[j] = v[j];
+#pragma unroll
+    for (int m = 4; m >= 1; m /= 2) {
+        const bool up = (c & m) != 0;
+#pragma unroll
+        for (int j = 0; j < m; ++j) {
+            const float keep = up ? cur[m + j] : cur[j];
+            const float send = up ? cur[j] : cur[m + j];
+            cur[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    float r = cur[0];
+#pragma unroll
+    for (int m = 8; m < CW; m *= 2) r += __shfl_xor_sync(0xffffffffu, r, m);
+    return r;
+}
+
+// beta = Bbar / B = expm1(delta A) / A for two states: delta phi1(q) by its series
+// for |q| < 1/16, (Abar - 1) / A otherwise (the same regions as sscan::bbar_coef).
+__device__ __forceinline__ float2 bbar2(float2 dd, float2 A2, float2 iA) {
+    const float2 q2 = __fmul2_rn(dd, A2);
+    const float2 q = __fmul2_rn(q2, g2(kLn2, kLn2));
+    const float2 bl = __fmul2_rn(__fadd2_rn(ex2p(q2), g2(-1.f, -1.f)), iA);
+    float2 ph = __ffma2_rn(q, g2(1.f / 120.f, 1.f / 120.f), g2(1.f / 24.f, 1.f / 24.f));
+    ph = __ffma2_rn(ph, q, g2(1.f / 6.f, 1.f / 6.f));
+    ph = __ffma2_rn(ph, q, g2(0.5f, 0.5f));
+    ph = __ffma2_rn(ph, q, g2(1.f, 1.f));
+    const float2 bs = __fmul2_rn(dd, ph);
+    return g2(fabsf(q.x) < 0.0625f ? bs.x : bl.x, fabsf(q.y) < 0.0625f ? bs.y : bl.y);
+}
+
+// softplus(r) and its derivative sigmoid(r) from one exponential (regions as in
+// sscan::softplus).
+__device__ __forceinline__ float2 softplus_dsig(float r) {
+    const float u = ex2(fminf(r, 30.f) * kLog2e);
+    const float ser = u * fmaf(u, fmaf(u, fmaf(u, fmaf(u, 0.2f, -0.25f), 1.f / 3.f), -0.5f), 1.f);
+    const float lg = kLn2 * lg2(1.f + u);
+    const float v = u < 0.03125f ? ser : lg;
+    const float sig = r > 20.f ? 1.f : u * rcp(1.f + u);
+    return g2(r > 20.f ? r : v, sig);
+}
+
+template <typename T, int NG>
+__global__ void __launch_bounds__(kThreadsB, 6)
+    bwd_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dr,
+                     const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_g,
+                     const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
+                     const __grid_constant__ CUtensorMap tm_du, const __grid_constant__ CUtensorMap tm_ddr,
+                     const __grid_constant__ CUtensorMap tm_dz, BwdTiledArgs a) {
+    using C = BCfg<T, NG>;
+    using P2 = typename BPair<T>::type;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t ncb = (a.D + C::DC - 1) / C::DC;
+    const int cb = (int)(blockIdx.x % ncb);
+    const int b = (int)(blockIdx.x / ncb);
+    const int N = a.N;
+    const int d0 = cb * C::DC;
+    const int ntb = (int)((a.L + kTB - 1) / kTB);
+    const bool has_z = a.has_z != 0;
+    const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
+    const uint32_t stage_bytes = (has_z ? 4u : 3u) * C::RAW + 2u * (uint32_t)(kTB * N * (int)sizeof(T));
+
+    // tiles are taken in reverse: processing index k covers tile ntb - 1 - k
+    auto issue = [&](int k) {
+        const int st = k % C::STAGES;
+        const uint32_t bar = bar0 + 8 * st;
+        const uint32_t base = smem_u32(smem + C::OFF_RAW + st * C::STAGE);
+        const int t0 = (ntb - 1 - k) * kTB;
+        mbar_expect_tx(bar, stage_bytes);
+        tma_load_3d(base, &tm_u, d0, t0, b, bar);
+        tma_load_3d(base + C::RAW, &tm_dr, d0, t0, b, bar);
+        if (has_z) tma_load_3d(base + 2 * C::RAW, &tm_z, d0, t0, b, bar);
+        tma_load_3d(base + 3 * C::RAW, &tm_g, d0, t0, b, bar);
+        tma_load_3d(base + 4 * C::RAW, &tm_B, 0, t0, b, bar);
+        tma_load_3d(base + 4 * C::RAW + C::RAWBC, &tm_C, 0, t0, b, bar);
+    };
+
+    int bad = 0;
+    if (tid == 0) {
+        for (int st = 0; st < C::STAGES; ++st) mbar_init(bar0 + 8 * st, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int k = 0; k < C::STAGES && k < ntb; ++k) issue(k);
+    }
+    float* sacc = reinterpret_cast<float*>(smem + C::OFF_ACC);
+    for (int e = tid; e < kTB * C::NS * 2; e += kThreadsB) sacc[e] = 0.f;
+
+    // lane state: channel cw, states g*4 .. g*4+3
+    const int g = lane / C::CW, c = lane % C::CW, cw = warp * C::CW + c;
+    const int64_t d = d0 + cw;
+    const bool cvalid = d < a.D;
+    float2 A2[2], iA[2], lam[2], P1[2], P2v[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        float av[2], ia[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int n = g * 4 + 2 * k + j;
+            const bool ok = cvalid && n < N;
+            const float An = ok ? __ldg(a.A + d * N + n) : 0.f;
+            av[j] = An * kLog2e;
+            ia[j] = An != 0.f ? 1.f / An : 0.f;
+        }
+        A2[k] = g2(av[0], av[1]);
+        iA[k] = g2(ia[0], ia[1]);
+        lam[k] = P1[k] = P2v[k] = g2(0.f, 0.f);
+    }
+    const int nvalid = cvalid ? min(4, N - g * 4) : 0;
+    float dbias_acc = 0.f;
+    // phase-P channel pair of this thread
+    const int pc = 2 * (tid % (C::DC / 2));
+    const int64_t pd = d0 + pc;
+    float2 dD_acc = g2(0.f, 0.f);
+
+    if (tid == 0 && ntb > 0) bad = !mbar_wait(bar0, 0);
+    bool failed = __syncthreads_or(bad) != 0;
+
+    for (int k = 0; k < ntb && !failed; ++k) {
+        const int it = ntb - 1 - k;
+        const int st = k % C::STAGES;
+        const int t0 = it * kTB;
+        const int tile_len = (int)(a.L - t0 < kTB ? a.L - t0 : kTB);
+        const unsigned char* raw = smem + C::OFF_RAW + st * C::STAGE;
+        // ---- phase P
+        {
+            const P2* ru = reinterpret_cast<const P2*>(raw);
+            const P2* rd = reinterpret_cast<const P2*>(raw + C::RAW);
+            const P2* rz = reinterpret_cast<const P2*>(raw + 2 * C::RAW);
+            const P2* rg = reinterpret_cast<const P2*>(raw + 3 * C::RAW);
+            float4* sdx = reinterpret_cast<float4*>(smem + C::OFF_DX);
+            float4* sdq = reinterpret_cast<float4*>(smem + C::OFF_DQ);
+            float4* sdd = reinterpret_cast<float4*>(smem + C::OFF_DD);
+            const float pb0 = (a.bias && pd < a.D) ? __ldg(a.bias + pd) : 0.f;
+            const float pb1 = (a.bias && pd + 1 < a.D) ? __ldg(a.bias + pd + 1) : 0.f;
+            const float pk0 = (a.Dskip && pd < a.D) ? __ldg(a.Dskip + pd) : 0.f;
+            const float pk1 = (a.Dskip && pd + 1 < a.D) ? __ldg(a.Dskip + pd + 1) : 0.f;
+#pragma unroll
+            for (int q = tid; q < C::PAIRS; q += kThreadsB) {
+                const int t = q / (C::DC / 2);
+                const bool tv = t < tile_len;
+                const float2 x = BPair<T>::f(ru[q]);
+                const float2 r = BPair<T>::f(rd[q]);
+                const float2 go = BPair<T>::f(rg[q]);
+                float dl0 = r.x + pb0, dl1 = r.y + pb1, s0 = 1.f, s1 = 1.f;
+                if (a.softplus) {
+                    const float2 p0 = softplus_dsig(dl0), p1 = softplus_dsig(dl1);
+                    dl0 = p0.x;
+                    s0 = p0.y;
+                    dl1 = p1.x;
+                    s1 = p1.y;
+                }
+                float dy0 = go.x, dy1 = go.y, dz0 = 0.f, dz1 = 0.f;
+                if (has_z) {
+                    const float2 zz = BPair<T>::f(rz[q]);
+                    const float sz0 = sigmoid(zz.x), sz1 = sigmoid(zz.y);
+                    dy0 = go.x * zz.x * sz0;
+                    dy1 = go.y * zz.y * sz1;
+                    dz0 = go.x * sz0 * fmaf(zz.x, 1.f - sz0, 1.f);
+                    dz1 = go.y * sz1 * fmaf(zz.y, 1.f - sz1, 1.f);
+                }
+                if (!tv) dy0 = dy1 = dz0 = dz1 = 0.f;
+                sdx[t * C::DC + pc] = make_float4(dl0, dl0, x.x, x.x);
+                sdx[t * C::DC + pc + 1] = make_float4(dl1, dl1, x.y, x.y);
+                sdq[t * C::DC + pc] = make_float4(dy0, dy0, dz0, s0);
+                sdq[t * C::DC + pc + 1] = make_float4(dy1, dy1, dz1, s1);
+                sdd[(t * C::DC + pc) / 2] = make_float4(pk0 * dy0, pk0 * x.x, pk1 * dy1, pk1 * x.y);
+                if (tv) dD_acc = g2(fmaf(dy0, x.x, dD_acc.x), fmaf(dy1, x.y, dD_acc.y));
+            }
+            const T* rB = reinterpret_cast<const T*>(raw + 4 * C::RAW);
+            const T* rC = reinterpret_cast<const T*>(raw + 4 * C::RAW + C::RAWBC);
+            float* sBf = reinterpret_cast<float*>(smem + C::OFF_B);
+            float* sCf = reinterpret_cast<float*>(smem + C::OFF_C);
+            for (int e = tid; e < kTB * C::NS; e += kThreadsB) {
+                const int t = e / C::NS, n = e % C::NS;
+                sBf[e] = n < N ? to_f32<T>(rB[t * N + n]) : 0.f;
+                sCf[e] = n < N ? to_f32<T>(rC[t * N + n]) : 0.f;
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0 && k + C::STAGES < ntb) issue(k + C::STAGES);
+
+        // ---- recompute the tile's states from the checkpoint
+        const float4* sdx = reinterpret_cast<const float4*>(smem + C::OFF_DX) + cw;
+        const float4* sdq = reinterpret_cast<const float4*>(smem + C::OFF_DQ) + cw;
+        const float2* sdd = reinterpret_cast<const float2*>(smem + C::OFF_DD) + cw;
+        const float4* sB = reinterpret_cast<const float4*>(smem + C::OFF_B) + g;
+        const float4* sC = reinterpret_cast<const float4*>(smem + C::OFF_C) + g;
+        float4* shs = reinterpret_cast<float4*>(smem + C::OFF_HS) + tid;
+        float2 hk[2];
+        {
+            const float* ck = a.ws_ckpt + (((int64_t)b * a.nck + it) * a.D + d) * N + g * 4;
+            float hv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) hv[j] = j < nvalid ? ck[j] : 0.f;
+            hk[0] = g2(hv[0], hv[1]);
+            hk[1] = g2(hv[2], hv[3]);
+        }
+        {
+            float2 h0 = hk[0], h1 = hk[1];
+            for (int t = 0; t < tile_len; ++t) {
+                const float4 dx = sdx[t * C::DC];
+                const float4 Bv = sB[t * NG];
+                const float2 dd = g2(dx.x, dx.y), xx = g2(dx.z, dx.w);
+                const float2 Bx0 = __fmul2_rn(g2(Bv.x, Bv.y), xx), Bx1 = __fmul2_rn(g2(Bv.z, Bv.w), xx);
+                h0 = __ffma2_rn(ex2p(__fmul2_rn(dd, A2[0])), h0, __fmul2_rn(bbar2(dd, A2[0], iA[0]), Bx0));
+                h1 = __ffma2_rn(ex2p(__fmul2_rn(dd, A2[1])), h1, __fmul2_rn(bbar2(dd, A2[1], iA[1]), Bx1));
+                shs[t * kThreadsB] = make_float4(h0.x, h0.y, h1.x, h1.y);
+            }
+        }
+        // ---- reverse sweep in blocks of NG steps (last block first)
+        T* so = reinterpret_cast<T*>(smem + C::OFF_OUT + (k & 1) * 3 * C::RAW);
+        for (int tb = ((tile_len - 1) / NG) * NG; tb >= 0; tb -= NG) {
+            float pdu[NG], pdd[NG], py[NG];
+#pragma unroll
+            for (int kk = NG - 1; kk >= 0; --kk) {
+                const int t = tb + kk;
+                pdu[kk] = pdd[kk] = py[kk] = 0.f;
+                float vbc[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) vbc[j] = 0.f;
+                if (t < tile_len) {
+                    const float4 dx = sdx[t * C::DC];
+                    const float4 dq = sdq[t * C::DC];
+                    const float4 Bv = sB[t * NG], Cv = sC[t * NG];
+                    const float4 hc = shs[t * kThreadsB];
+                    float2 hp[2];
+                    if (t > 0) {
+                        const float4 v = shs[(t - 1) * kThreadsB];
+                        hp[0] = g2(v.x, v.y);
+                        hp[1] = g2(v.z, v.w);
+                    } else {
+                        hp[0] = hk[0];
+                        hp[1] = hk[1];
+                    }
+                    const float2 dd = g2(dx.x, dx.y), xx = g2(dx.z, dx.w), dyy = g2(dq.x, dq.y);
+                    const float2 hcv[2] = {g2(hc.x, hc.y), g2(hc.z, hc.w)};
+                    const float2 Bp[2] = {g2(Bv.x, Bv.y), g2(Bv.z, Bv.w)};
+                    const float2 Cp[2] = {g2(Cv.x, Cv.y), g2(Cv.z, Cv.w)};
+                    float2 du2 = g2(0.f, 0.f), S1 = g2(0.f, 0.f), S2 = g2(0.f, 0.f), y2 = g2(0.f, 0.f);
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const float2 q2 = __fmul2_rn(dd, A2[p]);
+                        const float2 q = __fmul2_rn(q2, g2(kLn2, kLn2));
+                        const float2 ab = ex2p(q2);
+                        const float2 l = __ffma2_rn(Cp[p], dyy, lam[p]);
+                        const float2 la = __fmul2_rn(l, ab);
+                        // beta = Bbar / B = expm1(q) / A: series delta phi1(q) near q = 0
+                        const float2 em1 = __fadd2_rn(ab, g2(-1.f, -1.f));
+                        const float2 bl = __fmul2_rn(em1, iA[p]);
+                        float2 ph = __ffma2_rn(q, g2(1.f / 120.f, 1.f / 120.f), g2(1.f / 24.f, 1.f / 24.f));
+                        ph = __ffma2_rn(ph, q, g2(1.f / 6.f, 1.f / 6.f));
+                        ph = __ffma2_rn(ph, q, g2(0.5f, 0.5f));
+                        ph = __ffma2_rn(ph, q, g2(1.f, 1.f));
+                        const float2 bs = __fmul2_rn(dd, ph);
+                        const float2 beta = g2(fabsf(q.x) < 0.0625f ? bs.x : bl.x, fabsf(q.y) < 0.0625f ? bs.y : bl.y);
+                        // (delta Abar - beta) / A = delta^2 psi(q): series for |q| < 1/2
+                        float2 ps = __ffma2_rn(q, g2(1.f / 840.f, 1.f / 840.f), g2(1.f / 144.f, 1.f / 144.f));
+                        ps = __ffma2_rn(ps, q, g2(1.f / 30.f, 1.f / 30.f));
+                        ps = __ffma2_rn(ps, q, g2(0.125f, 0.125f));
+                        ps = __ffma2_rn(ps, q, g2(1.f / 3.f, 1.f / 3.f));
+                        ps = __ffma2_rn(ps, q, g2(0.5f, 0.5f));
+                        const float2 t2s = __fmul2_rn(__fmul2_rn(dd, dd), ps);
+                        const float2 t2c = __fmul2_rn(__ffma2_rn(dd, ab, g2(-beta.x, -beta.y)), iA[p]);
+                        const float2 t2 = g2(fabsf(q.x) < 0.5f ? t2s.x : t2c.x, fabsf(q.y) < 0.5f ? t2s.y : t2c.y);
+                        const float2 lb = __fmul2_rn(l, beta);
+                        const float2 dBv = __fmul2_rn(lb, xx);
+                        const float2 dCv = __fmul2_rn(dyy, hcv[p]);
+                        vbc[2 * p] = dBv.x;
+                        vbc[2 * p + 1] = dBv.y;
+                        vbc[4 + 2 * p] = dCv.x;
+                        vbc[4 + 2 * p + 1] = dCv.y;
+                        du2 = __ffma2_rn(lb, Bp[p], du2);
+                        S1 = __ffma2_rn(la, __fmul2_rn(A2[p], hp[p]), S1);
+                        S2 = __ffma2_rn(la, Bp[p], S2);
+                        const float2 Bx = __fmul2_rn(Bp[p], xx);
+                        P1[p] = __ffma2_rn(dd, __fmul2_rn(la, hp[p]), P1[p]);
+                        P2v[p] = __ffma2_rn(__fmul2_rn(l, Bx), t2, P2v[p]);
+                        y2 = __ffma2_rn(Cp[p], hcv[p], y2);
+                        lam[p] = la;
+                    }
+                    pdu[kk] = du2.x + du2.y;
+                    pdd[kk] = fmaf(kLn2, S1.x + S1.y, dx.z * (S2.x + S2.y));
+                    py[kk] = y2.x + y2.y;
+                }
+                // dB, dC of step t summed over this warp's channels, then over the CTA in smem
+                const float v = treduce_c8<C::CW>(vbc, c);
+                if (c < 8 && t < tile_len) {
+                    const int which = c >> 2, j = c & 3;
+                    atomicAdd(sacc + (t * C::NS + g * 4 + j) * 2 + which, v);
+                }
+            }
+            const float sdu = treduce_g<NG, C::CW>(pdu, g);
+            const float sdd_ = treduce_g<NG, C::CW>(pdd, g);
+            const float sy = treduce_g<NG, C::CW>(py, g);
+            const int t = tb + g;
+            if (t < tile_len && g < NG) {
+                const float4 dq = sdq[t * C::DC];
+                const float2 ddv = sdd[t * C::DC];
+                const float du = sdu + ddv.x;
+                const float ddr = sdd_ * dq.w;
+                const float dz = dq.z * (sy + ddv.y);
+                so[t * C::DC + cw] = from_f32<T>(du);
+                so[C::RAW / (int)sizeof(T) + t * C::DC + cw] = from_f32<T>(ddr);
+                so[2 * C::RAW / (int)sizeof(T) + t * C::DC + cw] = from_f32<T>(dz);
+                if (cvalid) dbias_acc += ddr;
+            }
+        }
+        fence_proxy_async();
+        if (tid == 0 && k + 1 < ntb)
+            bad = !mbar_wait(bar0 + 8 * ((k + 1) % C::STAGES), ((k + 1) / C::STAGES) & 1);
+        failed = __syncthreads_or(bad) != 0;
+        if (tid == 0) {
+            const uint32_t o = smem_u32(so);
+            tma_store_3d_nocommit(&tm_du, d0, t0, b, o);
+            tma_store_3d_nocommit(&tm_ddr, d0, t0, b, o + C::RAW);
+            if (has_z) tma_store_3d_nocommit(&tm_dz, d0, t0, b, o + 2 * C::RAW);
+            tma_commit();
+            tma_store_wait_read_1();
+        }
+        // the tile's dB, dC into the fp32 accumulators, then clear the smem sums
+        for (int e = tid; e < tile_len * C::NS; e += kThreadsB) {
+            const int t = e / C::NS, n = e % C::NS;
+            if (n < N) {
+                const int64_t gi = ((int64_t)b * a.L + t0 + t) * N + n;
+                atomicAdd(a.dB32 + gi, sacc[e * 2]);
+                atomicAdd(a.dC32 + gi, sacc[e * 2 + 1]);
+            }
+            sacc[e * 2] = 0.f;
+            sacc[e * 2 + 1] = 0.f;
+        }
+    }
+    if (tid == 0) tma_store_wait_all();
+    if (failed) {
+        if (tid == 0) {
+            atomicOr(&g_device_error_bwd, 2u);
+            for (int st = 0; st < C::STAGES; ++st) (void)mbar_wait(bar0 + 8 * st, 0), (void)mbar_wait(bar0 + 8 * st, 1);
+        }
+        return;
+    }
+    // per-channel sums
+    const float lamv[4] = {lam[0].x, lam[0].y, lam[1].x, lam[1].y};
+    const float dAv[4] = {P1[0].x + P2v[0].x, P1[0].y + P2v[0].y, P1[1].x + P2v[1].x, P1[1].y + P2v[1].y};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (j >= nvalid) continue;
+        const int n = g * 4 + j;
+        if (a.dh0) a.dh0[((int64_t)b * a.D + d) * N + n] = lamv[j];
+        // dA = sum_t [delta lam Abar h_{t-1} + lam B x delta^2 psi(delta A)]
+        atomicAdd(a.dA + d * N + n, dAv[j]);
+    }
+    if (a.dbias && cvalid) atomicAdd(a.dbias + d, dbias_acc);
+    if (a.dD && pd < a.D) {
+        atomicAdd(a.dD + pd, dD_acc.x);
+        if (pd + 1 < a.D) atomicAdd(a.dD + pd + 1, dD_acc.y);
+    }
+}
+
+// 3-D map over a (batch, L, W) tensor, box [1][kTB][box_w].
+template <typename T>
+bool make_map_b(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int64_t W, int box_w) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)L, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)(W * sizeof(T)), (cuuint64_t)(L * W * sizeof(T))};
+    const cuuint32_t box[3] = {(cuuint32_t)box_w, (cuuint32_t)kTB, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapDataType ty =
+        sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    return fn(m, ty, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int NG>
+cudaError_t launch_bwd_t(const BwdTiledArgs& a, const BwdTiledPtrs& p, cudaStream_t st) {
+    using C = BCfg<T, NG>;
+    CUtensorMap mu, md, mz, mg, mb, mc, mdu, mdd, mdz;
+    const void* zsrc = p.z ? p.z : p.u;
+    void* dzdst = p.dz ? p.dz : p.du;
+    if (!make_map_b<T>(&mu, p.u, a.batch, a.L, a.D, C::DC) || !make_map_b<T>(&md, p.delta_raw, a.batch, a.L, a.D, C::DC) ||
+        !make_map_b<T>(&mz, zsrc, a.batch, a.L, a.D, C::DC) || !make_map_b<T>(&mg, p.dout, a.batch, a.L, a.D, C::DC) ||
+        !make_map_b<T>(&mb, p.B, a.batch, a.L, a.N, a.N) || !make_map_b<T>(&mc, p.C, a.batch, a.L, a.N, a.N) ||
+        !make_map_b<T>(&mdu, p.du, a.batch, a.L, a.D, C::DC) || !make_map_b<T>(&mdd, p.ddelta_raw, a.batch, a.L, a.D, C::DC) ||
+        !make_map_b<T>(&mdz, dzdst, a.batch, a.L, a.D, C::DC))
+        return cudaErrorInvalidValue;
+    auto kern = bwd_tiled_kernel<T, NG>;
+    static bool configured = false;
+    if (!configured) {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        configured = true;
+    }
+    const int64_t blocks = a.batch * ((a.D + C::DC - 1) / C::DC);
+    kern<<<(unsigned)blocks, kThreadsB, C::SMEM, st>>>(mu, md, mz, mg, mb, mc, mdu, mdd, mdz, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t read_device_error_bwd(unsigned int* value, int clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(value, g_device_error_bwd, sizeof(unsigned int));
+    if (e == cudaSuccess && clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error_bwd, &zero, sizeof(unsigned int));
+    }
+    return e;
+}
+
+cudaError_t launch_bwd_tiled(const BwdTiledArgs& a, const BwdTiledPtrs& p, int io_bf16, cudaStream_t st) {
+    if (io_bf16) {
+        if (a.N <= 4) return launch_bwd_t<__nv_bfloat16, 1>(a, p, st);
+        if (a.N <= 8) return launch_bwd_t<__nv_bfloat16, 2>(a, p, st);
+        return launch_bwd_t<__nv_bfloat16, 4>(a, p, st);
+    }
+    if (a.N <= 4) return launch_bwd_t<float, 1>(a, p, st);
+    if (a.N <= 8) return launch_bwd_t<float, 2>(a, p, st);
+    return launch_bwd_t<float, 4>(a, p, st);
+}
+
+}  // namespace sscan

@@ -13,6 +13,7 @@ struct TiledArgs {
     int N;
     int softplus;
     int has_z;
+    int bc_tma;           // set by the launcher: B and C tiles travel by TMA
     const float* bias;    // (D) or null
     const float* A;       // (D, N)
     const float* Dskip;   // (D) or null
@@ -24,6 +25,8 @@ struct TiledArgs {
     int64_t nchunks;
     float* ws_state;      // [batch][nchunks][D][N]
     float* ws_dsum;       // [batch][nchunks][D]
+    float* ws_ckpt;       // [batch][nck][D][N]: state before every 8th step (checkpoint mode)
+    int64_t nck;          // ceil(L / 8)
 };
 
 // The (batch, L, D) tensors, reached through TMA tensor maps built per call.
@@ -34,12 +37,70 @@ struct TiledPtrs {
     void* out;            // or null
 };
 
-enum { kTiledOut = 0, kTiledAgg = 1, kTiledLast = 2 };
+enum { kTiledOut = 0, kTiledAgg = 1, kTiledLast = 2, kTiledCkpt = 3 };
 
-// Channels one CTA covers for a given state count (its TMA box width).
-int tiled_channels_per_cta(int64_t N);
+// Lane geometry of the tiled kernel: NG lanes per channel, G states per lane,
+// DC channels per CTA (its TMA box width).  A pure function of the problem.
+struct TiledGeom {
+    int NG, G, DC;
+};
+TiledGeom tiled_geometry(int64_t batch, int64_t L, int64_t D, int64_t N);
 
-cudaError_t launch_fwd_tiled(const TiledArgs& a, const TiledPtrs& p, int io_bf16, int mode, cudaStream_t st);
+cudaError_t launch_fwd_tiled(const TiledArgs& a, const TiledPtrs& p, const TiledGeom& geo, int io_bf16, int mode,
+                             cudaStream_t st);
+
+// One recurrence step (autoregressive generation): tensors of one time step.
+struct StepArgs {
+    int64_t batch, D;
+    int N;
+    int softplus;
+    const void* u;          // (batch, D)
+    const void* delta_raw;  // (batch, D)
+    const float* bias;      // (D) or null
+    const float* A;         // (D, N)
+    const void* B;          // (batch, N)
+    const void* C;          // (batch, N)
+    const float* Dskip;     // (D) or null
+    const void* z;          // (batch, D) or null
+    float* state;           // (batch, D, N), updated in place
+    void* out;              // (batch, D)
+};
+
+cudaError_t launch_step(const StepArgs& a, int io_bf16, cudaStream_t st);
+
+// Backward of the tiled path: scalars, small tensors and gradient accumulators.
+struct BwdTiledArgs {
+    int64_t batch, L, D;
+    int N;
+    int softplus;
+    int has_z;
+    const float* bias;   // (D) or null
+    const float* A;      // (D, N)
+    const float* Dskip;  // (D) or null
+    const float* ws_ckpt;  // [batch][nck][D][N] from the forward checkpoint pass
+    int64_t nck;
+    float* dB32;         // (batch, L, N) fp32, pre-zeroed
+    float* dC32;         // (batch, L, N) fp32, pre-zeroed
+    float* dA;           // (D, N), pre-zeroed
+    float* dD;           // (D) or null, pre-zeroed
+    float* dbias;        // (D) or null, pre-zeroed
+    float* dh0;          // (batch, D, N) or null
+};
+
+struct BwdTiledPtrs {
+    const void* u;
+    const void* delta_raw;
+    const void* z;       // or null
+    const void* dout;
+    const void* B;
+    const void* C;
+    void* du;
+    void* ddelta_raw;
+    void* dz;            // or null
+};
+
+cudaError_t launch_bwd_tiled(const BwdTiledArgs& a, const BwdTiledPtrs& p, int io_bf16, cudaStream_t st);
+cudaError_t read_device_error_bwd(unsigned int* value, int clear);
 
 // Read (and optionally clear) the library's device error word; nonzero means a
 // bounded wait in a kernel gave up.  Synchronous.

@@ -74,13 +74,17 @@ struct BwdPlan {
     size_t workspace_bytes;
 };
 
-// fp32 accumulators for dB and dC (batch, L, N), then one checkpointed state
-// every kBwdSeg steps of every row.
+// fp32 accumulators for dB and dC (batch, L, N), then checkpointed states: one
+// every kBwdSeg steps of every row for the general kernel, one every
+// kBwdTiledSeg steps for the tiled kernel.  The workspace covers either.
+constexpr int kBwdTiledSeg = 8;
 inline BwdPlan plan_bwd(int64_t batch, int64_t L, int64_t D, int64_t N) {
     BwdPlan p{0, 0};
     if (batch * D <= 0 || L <= 0) return p;
     p.nseg = (L + kBwdSeg - 1) / kBwdSeg;
-    const size_t floats = (size_t)(2 * batch * L * N) + (size_t)(batch * D * p.nseg * N);
+    const int64_t nck = (L + kBwdTiledSeg - 1) / kBwdTiledSeg;
+    const int64_t ck = (batch * D * p.nseg * N > batch * nck * D * N) ? batch * D * p.nseg * N : batch * nck * D * N;
+    const size_t floats = (size_t)(2 * batch * L * N) + (size_t)ck;
     p.workspace_bytes = align256(floats * sizeof(float));
     return p;
 }

@@ -31,6 +31,7 @@
 
 #include "sscan_launch.h"
 #include "sscan_math.cuh"
+#include "sscan_tma.cuh"
 
 namespace sscan {
 
@@ -41,136 +42,104 @@ namespace {
 constexpr int kTT = 16;       // steps per tile
 constexpr int kWarps = 4;     // warps per CTA
 constexpr int kThreads = kWarps * 32;
-constexpr int kG = 4;         // states per lane
-constexpr int kStages = 2;    // raw-tile ring depth
-constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr float kSmallA = 9.765625e-4f;  // |A| below 2^-10 takes the series form of Bbar
 
-enum { kOut = 0, kAgg = 1, kLast = 2 };
+enum { kOut = 0, kAgg = 1, kLast = 2, kCkpt = 3 };
+constexpr int kCkStep = 8;  // steps between checkpoints written by kCkpt
 
-// --------------------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-// Bounded wait on an mbarrier phase; false when the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (done) return true;
-    }
-    return false;
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
-                                            uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int x, int y, int z, uint32_t src) {
-    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y), "r"(z), "r"(src)
-                 : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-__device__ __forceinline__ void tma_store_wait_read_1() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-template <typename T> __device__ __forceinline__ float to_f32(T v);
-template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
-template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
-template <typename T> __device__ __forceinline__ T from_f32(float v);
-template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
-template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
-
-__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
-
-template <typename T, int NG>
-struct Cfg {
-    static constexpr int CW = 32 / NG;          // channels per warp
-    static constexpr int DC = CW * kWarps;      // channels per CTA
-    static constexpr int NS = NG * kG;          // states covered (>= N)
-    static constexpr int RAW = kTT * DC * (int)sizeof(T);  // bytes of one raw tile
-    static constexpr int BC_ENTRIES = kTT * NS;
-    static constexpr int BC_PER_THREAD = (BC_ENTRIES + kThreads - 1) / kThreads;
-    // shared-memory layout (byte offsets, all 128-aligned)
-    static constexpr int OFF_RAW = 0;                                   // [kStages][3][RAW]
-    static constexpr int OFF_DX = OFF_RAW + kStages * 3 * RAW;          // float2 [kTT][DC]
-    static constexpr int OFF_G = OFF_DX + kTT * DC * 8;                 // float  [kTT][DC]
-    static constexpr int OFF_B = OFF_G + kTT * DC * 4;                  // float  [kTT][NS]
-    static constexpr int OFF_C = OFF_B + kTT * NS * 4;                  // float  [kTT][NS]
-    static constexpr int OFF_OUT = OFF_C + kTT * NS * 4;                // [2][RAW]
-    static constexpr int OFF_BAR = OFF_OUT + 2 * RAW;                   // uint64 [kStages]
-    static constexpr int SMEM = OFF_BAR + kStages * 8;
+template <typename T> struct Pair;
+template <> struct Pair<float> {
+    using type = float2;
+    static __device__ __forceinline__ float2 f(float2 v) { return v; }
+};
+template <> struct Pair<__nv_bfloat16> {
+    using type = __nv_bfloat162;
+    static __device__ __forceinline__ float2 f(__nv_bfloat162 v) { return __bfloat1622float2(v); }
 };
 
-// One step of NG-th of a channel: 4 states in two f32x2 pairs.  b-form of eq. (2):
-// Bbar x = (Abar - 1) * (B x / A), evaluated as fma(Abar, w, -w) with w = B x / A.
-struct Lane4 {
-    float2 h01, h23, A2_01, A2_23, iA01, iA23;
+// Tile geometry for NG lanes per channel, G states per lane.
+template <typename T, int NG, int G>
+struct Cfg {
+    static constexpr int CW = 32 / NG;                     // channels per warp
+    static constexpr int DC = CW * kWarps;                 // channels per CTA
+    static constexpr int NS = NG * G;                      // states covered (>= N)
+    static constexpr int STAGES = sizeof(T) == 2 ? 2 : 1;  // raw-tile ring depth
+    static constexpr int RAW = kTT * DC * (int)sizeof(T);  // bytes of one raw (batch, L, D) tile
+    static constexpr int RAWBC = kTT * NS * (int)sizeof(T);  // bytes reserved for one raw B or C tile
+    static constexpr int STAGE = 3 * RAW + 2 * RAWBC;      // u, delta_raw, z, B, C
+    static constexpr int GD_PITCH = DC + 8;                // float2 row pitch of the epilogue operands
+    static constexpr int BC_ENTRIES = kTT * NS;
+    static constexpr int PAIRS = kTT * DC / 2;             // channel pairs of phase P
+    // shared-memory layout (byte offsets, all 128-aligned)
+    static constexpr int OFF_RAW = 0;                                     // [STAGES][STAGE]
+    static constexpr int OFF_DX = OFF_RAW + STAGES * STAGE;               // float4 (d, d, x, x) [kTT][DC]
+    static constexpr int OFF_GD = OFF_DX + kTT * DC * 16;                 // float2 (gate, D x gate) [kTT][GD_PITCH]
+    static constexpr int OFF_B = OFF_GD + kTT * GD_PITCH * 8;             // float  [kTT][NS]
+    static constexpr int OFF_C = OFF_B + kTT * NS * 4;                    // float  [kTT][NS]
+    static constexpr int OFF_OUT = OFF_C + kTT * NS * 4;                  // [2][RAW]
+    static constexpr int OFF_BAR = OFF_OUT + 2 * RAW;                     // uint64 [STAGES]
+    static constexpr int SMEM = OFF_BAR + STAGES * 8;
+};
+
+// Per lane: G states of one channel as G/2 f32x2 pairs, with A log2(e) and 1/A.
+template <int G>
+struct LaneG {
+    float2 h[G / 2], A2[G / 2], iA[G / 2];
 };
 
 __device__ __forceinline__ float2 ex2x2(float2 q) { return f2(ex2(q.x), ex2(q.y)); }
 
-__device__ __forceinline__ float step_fast(Lane4& s, float delta, float x, float4 Bv, float4 Cv, bool want_y) {
-    const float2 dd = f2(delta, delta), xx = f2(x, x);
-    const float2 a01 = ex2x2(__fmul2_rn(dd, s.A2_01));
-    const float2 a23 = ex2x2(__fmul2_rn(dd, s.A2_23));
-    const float2 w01 = __fmul2_rn(f2(Bv.x, Bv.y), __fmul2_rn(xx, s.iA01));
-    const float2 w23 = __fmul2_rn(f2(Bv.z, Bv.w), __fmul2_rn(xx, s.iA23));
-    const float2 b01 = __ffma2_rn(a01, w01, f2(-w01.x, -w01.y));
-    const float2 b23 = __ffma2_rn(a23, w23, f2(-w23.x, -w23.y));
-    s.h01 = __ffma2_rn(a01, s.h01, b01);
-    s.h23 = __ffma2_rn(a23, s.h23, b23);
-    if (!want_y) return 0.f;
-    float2 y = __fmul2_rn(f2(Cv.x, Cv.y), s.h01);
-    y = __ffma2_rn(f2(Cv.z, Cv.w), s.h23, y);
-    return y.x + y.y;
+// One step for the lane's G states, eq. (2) and (3a), in the b-form
+// Bbar x = (Abar - 1) w with w = B x / A, evaluated as fma(Abar, w, -w) (one
+// rounding).  dx = (delta, delta, x, x); Bp, Cp point at the lane's G values of B_t,
+// C_t.  Returns the partial readout sum_j C_j h_j over these states (eq. (3b)).
+template <int G, bool WANT_Y>
+__device__ __forceinline__ float step_fast(LaneG<G>& s, float4 dx, const float4* Bp, const float4* Cp) {
+    const float2 dd = f2(dx.x, dx.y), xx = f2(dx.z, dx.w);
+    float2 y = f2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < G / 4; ++k) {
+        const float4 Bv = Bp[k];
+        const float2 a0 = ex2x2(__fmul2_rn(dd, s.A2[2 * k]));
+        const float2 a1 = ex2x2(__fmul2_rn(dd, s.A2[2 * k + 1]));
+        const float2 w0 = __fmul2_rn(f2(Bv.x, Bv.y), __fmul2_rn(xx, s.iA[2 * k]));
+        const float2 w1 = __fmul2_rn(f2(Bv.z, Bv.w), __fmul2_rn(xx, s.iA[2 * k + 1]));
+        s.h[2 * k] = __ffma2_rn(a0, s.h[2 * k], __ffma2_rn(a0, w0, f2(-w0.x, -w0.y)));
+        s.h[2 * k + 1] = __ffma2_rn(a1, s.h[2 * k + 1], __ffma2_rn(a1, w1, f2(-w1.x, -w1.y)));
+        if (WANT_Y) {
+            const float4 Cv = Cp[k];
+            y = __ffma2_rn(f2(Cv.x, Cv.y), s.h[2 * k], y);
+            y = __ffma2_rn(f2(Cv.z, Cv.w), s.h[2 * k + 1], y);
+        }
+    }
+    return WANT_Y ? y.x + y.y : 0.f;
 }
 
 // Accurate form for blocks with a small |A| (or A = 0): Bbar / B = delta phi1(delta A)
-// with the series near 0, as in the general kernels.
-__device__ __forceinline__ float step_acc(Lane4& s, float delta, float x, float4 Bv, float4 Cv, bool want_y) {
-    float hv[4] = {s.h01.x, s.h01.y, s.h23.x, s.h23.y};
-    const float A2v[4] = {s.A2_01.x, s.A2_01.y, s.A2_23.x, s.A2_23.y};
-    const float iAv[4] = {s.iA01.x, s.iA01.y, s.iA23.x, s.iA23.y};
-    const float Bb[4] = {Bv.x, Bv.y, Bv.z, Bv.w}, Cc[4] = {Cv.x, Cv.y, Cv.z, Cv.w};
+// with phi1's series near 0, as in the general kernels.
+template <int G, bool WANT_Y>
+__device__ __forceinline__ float step_acc(LaneG<G>& s, float4 dx, const float4* Bp, const float4* Cp) {
+    const float delta = dx.x, x = dx.z;
     float y = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float q2 = delta * A2v[j];
-        const float abar = ex2(q2);
-        const float beta = bbar_coef(delta, q2 * kLn2, abar, iAv[j]);
-        hv[j] = fmaf(abar, hv[j], beta * Bb[j] * x);
-        y = fmaf(Cc[j], hv[j], y);
+    for (int k = 0; k < G / 4; ++k) {
+        const float4 Bv = Bp[k];
+        const float4 Cv = WANT_Y ? Cp[k] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float Bb[4] = {Bv.x, Bv.y, Bv.z, Bv.w}, Cc[4] = {Cv.x, Cv.y, Cv.z, Cv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float2& hp = s.h[2 * k + j / 2];
+            const float A2 = (j & 1) ? s.A2[2 * k + j / 2].y : s.A2[2 * k + j / 2].x;
+            const float iA = (j & 1) ? s.iA[2 * k + j / 2].y : s.iA[2 * k + j / 2].x;
+            const float q2 = delta * A2;
+            const float abar = ex2(q2);
+            const float beta = bbar_coef(delta, q2 * kLn2, abar, iA);
+            float& hv = (j & 1) ? hp.y : hp.x;
+            hv = fmaf(abar, hv, beta * Bb[j] * x);
+            y = fmaf(Cc[j], hv, y);
+        }
     }
-    s.h01 = f2(hv[0], hv[1]);
-    s.h23 = f2(hv[2], hv[3]);
-    return want_y ? y : 0.f;
+    return WANT_Y ? y : 0.f;
 }
 
 // Sum the partial readouts of the NG lanes of a channel for NG consecutive steps
@@ -198,47 +167,92 @@ __device__ __forceinline__ float transpose_reduce(float (&p)[NG], int g) {
     }
 }
 
-template <typename T, int NG, int MODE, bool ACC>
-__device__ __forceinline__ void scan_tile(const Cfg<T, NG>&, Lane4& s, unsigned char* smem, int tile_len, int g,
-                                          int cw, float dsk, T* sout, float& dsum) {
-    using C = Cfg<T, NG>;
-    const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX);
-    const float* sg = reinterpret_cast<const float*>(smem + C::OFF_G);
-    const float4* sB = reinterpret_cast<const float4*>(smem + C::OFF_B);
-    const float4* sC = reinterpret_cast<const float4*>(smem + C::OFF_C);
-    constexpr bool want_y = MODE == kOut;
+// Phase S over one tile.  FULL tiles (kTT valid steps) run fully unrolled with no
+// per-step predicate; the last, partial tile of a chunk takes the predicated form.
+template <typename T, int NG, int G, int MODE, bool ACC, bool FULL>
+__device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
+                                          float& dsum, float* ck, int64_t ck_stride, int nvalid) {
+    using C = Cfg<T, NG, G>;
+    constexpr bool WANT_Y = MODE == kOut;
+    const float4* sdx = reinterpret_cast<const float4*>(smem + C::OFF_DX) + cw;
+    const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
+    const float4* sB = reinterpret_cast<const float4*>(smem + C::OFF_B) + g * (G / 4);
+    const float4* sC = reinterpret_cast<const float4*>(smem + C::OFF_C) + g * (G / 4);
 #pragma unroll 1
     for (int tb = 0; tb < kTT; tb += NG) {
+        if (MODE == kCkpt && tb % kCkStep == 0 && (FULL || tb < tile_len)) {
+            // state before step tb, the starting point of one backward recomputation
+            float* dst = ck + (tb / kCkStep) * ck_stride;
+#pragma unroll
+            for (int j = 0; j < G; ++j)
+                if (j < nvalid) dst[j] = (j & 1) ? s.h[j / 2].y : s.h[j / 2].x;
+        }
         float p[NG];
 #pragma unroll
         for (int k = 0; k < NG; ++k) {
             const int t = tb + k;
             p[k] = 0.f;
-            if (t < tile_len) {
-                const float2 dx = sdx[t * C::DC + cw];
-                const float4 Bv = sB[t * NG + g];
-                const float4 Cv = want_y ? sC[t * NG + g] : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (FULL || t < tile_len) {
+                const float4 dx = sdx[t * C::DC];
                 if (MODE == kAgg) dsum += dx.x;
-                p[k] = ACC ? step_acc(s, dx.x, dx.y, Bv, Cv, want_y) : step_fast(s, dx.x, dx.y, Bv, Cv, want_y);
+                p[k] = ACC ? step_acc<G, WANT_Y>(s, dx, sB + t * (C::NS / 4), sC + t * (C::NS / 4))
+                           : step_fast<G, WANT_Y>(s, dx, sB + t * (C::NS / 4), sC + t * (C::NS / 4));
             }
         }
-        if constexpr (want_y) {
+        if constexpr (WANT_Y) {
             const float y = transpose_reduce<NG, C::CW>(p, g);
             const int t = tb + g;
-            if (t < tile_len) {
-                const float2 dx = sdx[t * C::DC + cw];
-                sout[t * C::DC + cw] = from_f32<T>(fmaf(dsk, dx.y, y) * sg[t * C::DC + cw]);
+            if (FULL || t < tile_len) {
+                const float2 gd = sgd[t * C::GD_PITCH];
+                sout[t * C::DC + cw] = from_f32<T>(fmaf(y, gd.x, gd.y));
             }
         }
     }
 }
 
-template <typename T, int NG, int MODE>
-__global__ void __launch_bounds__(kThreads, 8)
+template <typename T, int NG, int G, int MODE, bool ACC>
+__device__ __forceinline__ void scan_tile_any(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
+                                              float& dsum, float* ck, int64_t ck_stride, int nvalid) {
+    if (tile_len == kTT)
+        scan_tile<T, NG, G, MODE, ACC, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid);
+    else
+        scan_tile<T, NG, G, MODE, ACC, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid);
+}
+
+// softplus and SiLU of two values at once: the exponentials, logarithm and
+// reciprocal stay on the MUFU pipe, the surrounding arithmetic is packed f32x2.
+// softplus(r) = log(1 + e^r) in the same three regions as sscan::softplus
+// (r > 20: r; e^r < 2^-5: the log1p series; else ln2 * log2(1 + e^r)).
+__device__ __forceinline__ float2 softplus_x2(float2 r) {
+    const float2 q = __fmul2_rn(r, f2(kLog2e, kLog2e));
+    const float2 u = f2(ex2(q.x), ex2(q.y));
+    float2 ser = __ffma2_rn(u, f2(0.2f, 0.2f), f2(-0.25f, -0.25f));
+    ser = __ffma2_rn(ser, u, f2(1.f / 3.f, 1.f / 3.f));
+    ser = __ffma2_rn(ser, u, f2(-0.5f, -0.5f));
+    ser = __ffma2_rn(ser, u, f2(1.f, 1.f));
+    ser = __fmul2_rn(ser, u);
+    const float2 w = __fadd2_rn(u, f2(1.f, 1.f));
+    const float2 lg = __fmul2_rn(f2(lg2(w.x), lg2(w.y)), f2(kLn2, kLn2));
+    const float vx = u.x < 0.03125f ? ser.x : lg.x, vy = u.y < 0.03125f ? ser.y : lg.y;
+    return f2(r.x > 20.f ? r.x : vx, r.y > 20.f ? r.y : vy);
+}
+
+__device__ __forceinline__ float2 silu_x2(float2 z) {
+    const float2 q = __fmul2_rn(z, f2(-kLog2e, -kLog2e));
+    const float2 d = __fadd2_rn(f2(ex2(q.x), ex2(q.y)), f2(1.f, 1.f));
+    return __fmul2_rn(z, f2(rcp(d.x), rcp(d.y)));
+}
+
+template <int G> struct Occupancy { static constexpr int kCtas = G == 4 ? 9 : 5; };
+
+template <typename T, int NG, int G, int MODE>
+__global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
     fwd_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dr,
                      const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_out,
+                     const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
                      TiledArgs a) {
-    using C = Cfg<T, NG>;
+    using C = Cfg<T, NG, G>;
+    using P2 = typename Pair<T>::type;
     extern __shared__ __align__(128) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t ncb = (a.D + C::DC - 1) / C::DC;
@@ -252,134 +266,151 @@ __global__ void __launch_bounds__(kThreads, 8)
     const int ntile = (int)((t_end - t_begin + kTT - 1) / kTT);
     const int N = a.N;
     const int d0 = cb * C::DC;
-    const bool want_out = MODE == kOut;
+    constexpr bool want_out = MODE == kOut;
     const bool has_z = want_out && a.has_z;
-    const uint32_t nload = has_z ? 3u : 2u;
+    const bool bc_tma = a.bc_tma != 0;
     const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
-    const CUtensorMap* maps[3] = {&tm_u, &tm_dr, &tm_z};
+    const uint32_t raw_bytes = (has_z ? 3u : 2u) * C::RAW;
+    const uint32_t bc_bytes = (uint32_t)(kTT * N * (int)sizeof(T));
+    const uint32_t stage_bytes = raw_bytes + (bc_tma ? (want_out ? 2u : 1u) * bc_bytes : 0u);
 
-    if (tid == 0) {
-        for (int st = 0; st < kStages; ++st) mbar_init(bar0 + 8 * st, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        for (int st = 0; st < kStages && st < ntile; ++st) {
-            const uint32_t bar = bar0 + 8 * st;
-            mbar_expect_tx(bar, nload * C::RAW);
-            for (uint32_t k = 0; k < nload; ++k)
-                tma_load_3d(smem_u32(smem + C::OFF_RAW + (st * 3 + k) * C::RAW), maps[k], d0,
-                            (int)(t_begin + st * kTT), b, bar);
+    // issue the TMA copies of tile `it` into its ring stage (elected thread only)
+    auto issue = [&](int it) {
+        const int st = it % C::STAGES;
+        const uint32_t bar = bar0 + 8 * st;
+        const uint32_t base = smem_u32(smem + C::OFF_RAW + st * C::STAGE);
+        const int tt = (int)(t_begin + (int64_t)it * kTT);
+        mbar_expect_tx(bar, stage_bytes);
+        tma_load_3d(base, &tm_u, d0, tt, b, bar);
+        tma_load_3d(base + C::RAW, &tm_dr, d0, tt, b, bar);
+        if (has_z) tma_load_3d(base + 2 * C::RAW, &tm_z, d0, tt, b, bar);
+        if (bc_tma) {
+            tma_load_3d(base + 3 * C::RAW, &tm_B, 0, tt, b, bar);
+            if (want_out) tma_load_3d(base + 3 * C::RAW + C::RAWBC, &tm_C, 0, tt, b, bar);
         }
+    };
+
+    int bad = 0;
+    if (tid == 0) {
+        for (int st = 0; st < C::STAGES; ++st) mbar_init(bar0 + 8 * st, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int it = 0; it < C::STAGES && it < ntile; ++it) issue(it);
     }
 
-    // per-lane state: channel cw of this CTA, states g*4 .. g*4+3
+    // per-lane state: channel cw of this CTA, states g*G .. g*G+G-1
     const int g = lane / C::CW, c = lane % C::CW, cw = warp * C::CW + c;
     const int64_t d = d0 + cw;
     const bool cvalid = d < a.D;
-    Lane4 s;
-    float hv[4], A2v[4], iAv[4];
+    LaneG<G> s;
     bool small_a = false;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int n = g * kG + j;
+    for (int j = 0; j < G; ++j) {
+        const int n = g * G + j;
         const bool ok = cvalid && n < N;
         const float An = ok ? __ldg(a.A + d * N + n) : -1.f;
         small_a |= ok && fabsf(An) < kSmallA;
-        A2v[j] = ok ? An * kLog2e : 0.f;
-        iAv[j] = ok && An != 0.f ? 1.f / An : 0.f;
         float h = 0.f;
         if (ok && MODE != kAgg) {
             if (a.nchunks > 1) h = a.ws_state[(((int64_t)b * a.nchunks + chunk) * a.D + d) * N + n];
             else if (a.h0) h = __ldg(a.h0 + ((int64_t)b * a.D + d) * N + n);
         }
-        hv[j] = h;
+        const float A2 = ok ? An * kLog2e : 0.f;
+        const float iA = ok && An != 0.f ? 1.f / An : 0.f;
+        if (j & 1) {
+            s.h[j / 2].y = h;
+            s.A2[j / 2].y = A2;
+            s.iA[j / 2].y = iA;
+        } else {
+            s.h[j / 2].x = h;
+            s.A2[j / 2].x = A2;
+            s.iA[j / 2].x = iA;
+        }
     }
-    s.h01 = f2(hv[0], hv[1]);
-    s.h23 = f2(hv[2], hv[3]);
-    s.A2_01 = f2(A2v[0], A2v[1]);
-    s.A2_23 = f2(A2v[2], A2v[3]);
-    s.iA01 = f2(iAv[0], iAv[1]);
-    s.iA23 = f2(iAv[2], iAv[3]);
-    const float dsk = (want_out && cvalid && a.Dskip) ? __ldg(a.Dskip + d) : 0.f;
+    // the first tile's data; one CTA-wide choice of the Bbar form (block-uniform branch)
+    if (tid == 0 && ntile > 0) bad = !mbar_wait(bar0, 0);
+    const int flags = __syncthreads_or((small_a ? 1 : 0) | (bad ? 2 : 0));
+    const bool acc = (flags & 1) != 0;
+    bool failed = (flags & 2) != 0;
 
-    // phase-P channel of this thread (fixed, since kThreads is a multiple of DC)
-    const int pc = tid % C::DC;
-    const bool pvalid = d0 + pc < a.D;
-    const float pbias = (pvalid && a.bias) ? __ldg(a.bias + d0 + pc) : 0.f;
+    // phase-P channel pair of this thread (fixed, since kThreads is a multiple of DC/2)
+    const int pc = 2 * (tid % (C::DC / 2));
+    const int64_t pd = d0 + pc;
     const T* Bg = static_cast<const T*>(a.B);
     const T* Cg = static_cast<const T*>(a.C);
-    float bpre[C::BC_PER_THREAD], cpre[C::BC_PER_THREAD];
-    auto fetch_bc = [&](int it) {
-        const int64_t tt = t_begin + (int64_t)it * kTT;
-#pragma unroll
-        for (int k = 0; k < C::BC_PER_THREAD; ++k) {
-            const int e = tid + k * kThreads;
-            const int t = e / C::NS, n = e % C::NS;
-            const bool ok = e < C::BC_ENTRIES && n < N && tt + t < t_end;
-            const int64_t gi = ((int64_t)b * a.L + tt + t) * N + n;
-            bpre[k] = ok ? to_f32<T>(Bg[gi]) : 0.f;
-            cpre[k] = (ok && want_out) ? to_f32<T>(Cg[gi]) : 0.f;
-        }
-    };
-    fetch_bc(0);
-    const bool acc = __syncthreads_or(small_a) != 0;
     float dsum = 0.f;
-    bool failed = false;
 
-    for (int it = 0; it < ntile; ++it) {
-        const int st = it % kStages;
-        const uint32_t parity = (it / kStages) & 1;
-        int bad = 0;
-        if (tid == 0) bad = !mbar_wait(bar0 + 8 * st, parity);
-        if (__syncthreads_or(bad)) {
-            failed = true;
-            break;
-        }
+    for (int it = 0; it < ntile && !failed; ++it) {
+        const int st = it % C::STAGES;
         const int64_t tt = t_begin + (int64_t)it * kTT;
         const int tile_len = (int)(t_end - tt < kTT ? t_end - tt : kTT);
-        // phase P: raw tile -> fp32 (delta, x), gate; B and C rows
+        // phase P: raw tile -> (delta, delta, x, x) and (gate, D x gate); B and C rows as fp32
         {
-            const T* ru = reinterpret_cast<const T*>(smem + C::OFF_RAW + (st * 3 + 0) * C::RAW);
-            const T* rd = reinterpret_cast<const T*>(smem + C::OFF_RAW + (st * 3 + 1) * C::RAW);
-            const T* rz = reinterpret_cast<const T*>(smem + C::OFF_RAW + (st * 3 + 2) * C::RAW);
-            float2* sdx = reinterpret_cast<float2*>(smem + C::OFF_DX);
-            float* sg = reinterpret_cast<float*>(smem + C::OFF_G);
+            const unsigned char* raw = smem + C::OFF_RAW + st * C::STAGE;
+            const P2* ru = reinterpret_cast<const P2*>(raw);
+            const P2* rd = reinterpret_cast<const P2*>(raw + C::RAW);
+            const P2* rz = reinterpret_cast<const P2*>(raw + 2 * C::RAW);
+            float4* sdx = reinterpret_cast<float4*>(smem + C::OFF_DX);
+            float4* sgd = reinterpret_cast<float4*>(smem + C::OFF_GD);
+            const float2 pbias = f2((a.bias && pd < a.D) ? __ldg(a.bias + pd) : 0.f,
+                                    (a.bias && pd + 1 < a.D) ? __ldg(a.bias + pd + 1) : 0.f);
 #pragma unroll
-            for (int e = tid; e < kTT * C::DC; e += kThreads) {
-                const int t = e / C::DC;
-                const float x = to_f32<T>(ru[e]);
-                const float r = to_f32<T>(rd[e]) + pbias;
-                const float delta = (t < tile_len) ? (a.softplus ? softplus(r) : r) : 0.f;
-                sdx[e] = f2(delta, x);
-                if (want_out) sg[e] = has_z ? silu(to_f32<T>(rz[e])) : 1.f;
+            for (int q = tid; q < C::PAIRS; q += kThreads) {
+                const int t = q / (C::DC / 2);
+                const float2 x = Pair<T>::f(ru[q]);
+                float2 dl = __fadd2_rn(Pair<T>::f(rd[q]), pbias);
+                if (a.softplus) dl = softplus_x2(dl);
+                sdx[t * C::DC + pc] = make_float4(dl.x, dl.x, x.x, x.x);
+                sdx[t * C::DC + pc + 1] = make_float4(dl.y, dl.y, x.y, x.y);
+                if (want_out) {
+                    const float2 pdsk = f2((a.Dskip && pd < a.D) ? __ldg(a.Dskip + pd) : 0.f,
+                                           (a.Dskip && pd + 1 < a.D) ? __ldg(a.Dskip + pd + 1) : 0.f);
+                    const float2 gt = has_z ? silu_x2(Pair<T>::f(rz[q])) : f2(1.f, 1.f);
+                    const float2 dxg = __fmul2_rn(__fmul2_rn(pdsk, x), gt);
+                    sgd[(t * C::GD_PITCH + pc) / 2] = make_float4(gt.x, dxg.x, gt.y, dxg.y);
+                }
             }
             float* sBf = reinterpret_cast<float*>(smem + C::OFF_B);
             float* sCf = reinterpret_cast<float*>(smem + C::OFF_C);
+            const T* rB = reinterpret_cast<const T*>(raw + 3 * C::RAW);
+            const T* rC = reinterpret_cast<const T*>(raw + 3 * C::RAW + C::RAWBC);
 #pragma unroll
-            for (int k = 0; k < C::BC_PER_THREAD; ++k) {
-                const int e = tid + k * kThreads;
-                if (e < C::BC_ENTRIES) {
-                    sBf[e] = bpre[k];
-                    sCf[e] = cpre[k];
+            for (int e = tid; e < C::BC_ENTRIES; e += kThreads) {
+                const int t = e / C::NS, n = e % C::NS;
+                float bv = 0.f, cv = 0.f;
+                if (n < N) {
+                    if (bc_tma) {
+                        bv = to_f32<T>(rB[t * N + n]);
+                        if (want_out) cv = to_f32<T>(rC[t * N + n]);
+                    } else if (tt + t < t_end) {
+                        const int64_t gi = ((int64_t)b * a.L + tt + t) * N + n;
+                        bv = to_f32<T>(Bg[gi]);
+                        if (want_out) cv = to_f32<T>(Cg[gi]);
+                    }
                 }
+                sBf[e] = bv;
+                if (want_out) sCf[e] = cv;
             }
-            if (it + 1 < ntile) fetch_bc(it + 1);
         }
         fence_proxy_async();
         __syncthreads();
-        if (tid == 0 && it + kStages < ntile) {
-            const uint32_t bar = bar0 + 8 * st;
-            mbar_expect_tx(bar, nload * C::RAW);
-            for (uint32_t k = 0; k < nload; ++k)
-                tma_load_3d(smem_u32(smem + C::OFF_RAW + (st * 3 + k) * C::RAW), maps[k], d0,
-                            (int)(tt + kStages * kTT), b, bar);
-        }
+        if (tid == 0 && it + C::STAGES < ntile) issue(it + C::STAGES);
         // phase S
         T* sout = reinterpret_cast<T*>(smem + C::OFF_OUT + (it & 1) * C::RAW);
+        float* ck = nullptr;
+        if (MODE == kCkpt)
+            ck = a.ws_ckpt + ((((int64_t)b * a.nck) + tt / kCkStep) * a.D + d) * N + g * G;
+        const int64_t ck_stride = (int64_t)a.D * N;
+        const int nvalid = cvalid ? min(G, N - g * G) : 0;
         if (acc)
-            scan_tile<T, NG, MODE, true>(C{}, s, smem, tile_len, g, cw, dsk, sout, dsum);
+            scan_tile_any<T, NG, G, MODE, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid);
         else
-            scan_tile<T, NG, MODE, false>(C{}, s, smem, tile_len, g, cw, dsk, sout, dsum);
+            scan_tile_any<T, NG, G, MODE, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid);
         if (want_out) fence_proxy_async();
-        __syncthreads();
+        // the next tile's data, then one barrier for: outputs complete, tile buffers free,
+        // next raw tile landed (or a wait that gave up)
+        if (tid == 0 && it + 1 < ntile)
+            bad = !mbar_wait(bar0 + 8 * ((it + 1) % C::STAGES), ((it + 1) / C::STAGES) & 1);
+        failed = __syncthreads_or(bad) != 0;
         if (want_out && tid == 0) {
             tma_store_3d(&tm_out, d0, (int)tt, b, smem_u32(sout));
             tma_store_wait_read_1();
@@ -390,20 +421,20 @@ __global__ void __launch_bounds__(kThreads, 8)
         if (tid == 0) {
             atomicOr(&g_device_error, 1u);
             // let the loads still in flight land before the CTA's shared memory is released
-            for (int st = 0; st < kStages; ++st) (void)mbar_wait(bar0 + 8 * st, 0), (void)mbar_wait(bar0 + 8 * st, 1);
+            for (int st = 0; st < C::STAGES; ++st) (void)mbar_wait(bar0 + 8 * st, 0), (void)mbar_wait(bar0 + 8 * st, 1);
         }
         return;
     }
     // final state of this chunk
-    const float hf[4] = {s.h01.x, s.h01.y, s.h23.x, s.h23.y};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int n = g * kG + j;
+    for (int j = 0; j < G; ++j) {
+        const int n = g * G + j;
         if (!cvalid || n >= N) continue;
+        const float hf = (j & 1) ? s.h[j / 2].y : s.h[j / 2].x;
         if (MODE == kAgg)
-            a.ws_state[(((int64_t)b * a.nchunks + chunk) * a.D + d) * N + n] = hf[j];
+            a.ws_state[(((int64_t)b * a.nchunks + chunk) * a.D + d) * N + n] = hf;
         else if (a.h_last && chunk == a.nchunks - 1)
-            a.h_last[((int64_t)b * a.D + d) * N + n] = hf[j];
+            a.h_last[((int64_t)b * a.D + d) * N + n] = hf;
     }
     if (MODE == kAgg && g == 0 && cvalid) a.ws_dsum[((int64_t)b * a.nchunks + chunk) * a.D + d] = dsum;
 }
@@ -438,16 +469,34 @@ bool make_map(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int64_
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int NG, int MODE>
-cudaError_t launch_mode(const TiledArgs& a, const TiledPtrs& p, cudaStream_t st) {
-    using C = Cfg<T, NG>;
-    CUtensorMap mu, md, mz, mo;
+// B and C (batch, L, N) travel by TMA when a row of N values is a whole number of
+// 16-byte units; otherwise phase P reads them with plain loads.
+template <typename T>
+bool bc_by_tma(const TiledArgs& a) {
+    return (a.N * sizeof(T)) % 16 == 0 && reinterpret_cast<uintptr_t>(a.B) % 16 == 0 &&
+           (a.C == nullptr || reinterpret_cast<uintptr_t>(a.C) % 16 == 0);
+}
+
+template <typename T, int NG, int G, int MODE>
+cudaError_t launch_mode(const TiledArgs& args, const TiledPtrs& p, cudaStream_t st) {
+    using C = Cfg<T, NG, G>;
+    TiledArgs a = args;
+    a.bc_tma = bc_by_tma<T>(a) ? 1 : 0;
+    CUtensorMap mu, md, mz, mo, mb, mc;
     const void* zsrc = p.z ? p.z : p.u;      // an unused map still needs a valid address
     const void* osrc = p.out ? p.out : p.u;
     if (!make_map<T>(&mu, p.u, a.batch, a.L, a.D, C::DC) || !make_map<T>(&md, p.delta_raw, a.batch, a.L, a.D, C::DC) ||
         !make_map<T>(&mz, zsrc, a.batch, a.L, a.D, C::DC) || !make_map<T>(&mo, osrc, a.batch, a.L, a.D, C::DC))
         return cudaErrorInvalidValue;
-    auto kern = fwd_tiled_kernel<T, NG, MODE>;
+    if (a.bc_tma) {
+        if (!make_map<T>(&mb, a.B, a.batch, a.L, a.N, a.N) ||
+            !make_map<T>(&mc, a.C ? a.C : a.B, a.batch, a.L, a.N, a.N))
+            return cudaErrorInvalidValue;
+    } else {
+        mb = mu;
+        mc = mu;
+    }
+    auto kern = fwd_tiled_kernel<T, NG, G, MODE>;
     static bool configured = false;
     if (!configured) {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -456,31 +505,43 @@ cudaError_t launch_mode(const TiledArgs& a, const TiledPtrs& p, cudaStream_t st)
     }
     const int64_t ncb = (a.D + C::DC - 1) / C::DC;
     const int64_t blocks = a.batch * a.nchunks * ncb;
-    kern<<<(unsigned)blocks, kThreads, C::SMEM, st>>>(mu, md, mz, mo, a);
+    kern<<<(unsigned)blocks, kThreads, C::SMEM, st>>>(mu, md, mz, mo, mb, mc, a);
     return cudaGetLastError();
 }
 
-template <typename T, int NG>
-cudaError_t launch_ng(const TiledArgs& a, const TiledPtrs& p, int mode, cudaStream_t st) {
-    if (mode == kTiledOut) return launch_mode<T, NG, kOut>(a, p, st);
-    if (mode == kTiledAgg) return launch_mode<T, NG, kAgg>(a, p, st);
-    return launch_mode<T, NG, kLast>(a, p, st);
+template <typename T, int NG, int G>
+cudaError_t launch_geom(const TiledArgs& a, const TiledPtrs& p, int mode, cudaStream_t st) {
+    if (mode == kTiledOut) return launch_mode<T, NG, G, kOut>(a, p, st);
+    if (mode == kTiledAgg) return launch_mode<T, NG, G, kAgg>(a, p, st);
+    if (mode == kTiledCkpt) return launch_mode<T, NG, G, kCkpt>(a, p, st);
+    return launch_mode<T, NG, G, kLast>(a, p, st);
+}
+
+template <typename T>
+cudaError_t launch_t(const TiledArgs& a, const TiledPtrs& p, const TiledGeom& geo, int mode, cudaStream_t st) {
+    if (geo.NG == 1) return launch_geom<T, 1, 4>(a, p, mode, st);
+    if (geo.NG == 2) return launch_geom<T, 2, 4>(a, p, mode, st);
+    return launch_geom<T, 4, 4>(a, p, mode, st);
 }
 
 }  // namespace
 
-int tiled_channels_per_cta(int64_t N) { return N <= 4 ? 128 : (N <= 8 ? 64 : 32); }
+// Lane geometry: four states per lane, NG = ceil(N / 4) lanes per channel.  (Eight
+// states per lane halve the per-step overheads but halve the warps; at the Mamba
+// layer shapes that left too few warps per sub-partition to hide latency, and it
+// measured slower.)
+TiledGeom tiled_geometry(int64_t batch, int64_t L, int64_t D, int64_t N) {
+    (void)batch;
+    (void)L;
+    (void)D;
+    const int ng = N <= 4 ? 1 : (N <= 8 ? 2 : 4);
+    return TiledGeom{ng, 4, 32 / ng * kWarps};
+}
 
-cudaError_t launch_fwd_tiled(const TiledArgs& a, const TiledPtrs& p, int io_bf16, int mode, cudaStream_t st) {
+cudaError_t launch_fwd_tiled(const TiledArgs& a, const TiledPtrs& p, const TiledGeom& geo, int io_bf16, int mode,
+                             cudaStream_t st) {
     if (!encode_fn()) return cudaErrorNotSupported;
-    if (io_bf16) {
-        if (a.N <= 4) return launch_ng<__nv_bfloat16, 1>(a, p, mode, st);
-        if (a.N <= 8) return launch_ng<__nv_bfloat16, 2>(a, p, mode, st);
-        return launch_ng<__nv_bfloat16, 4>(a, p, mode, st);
-    }
-    if (a.N <= 4) return launch_ng<float, 1>(a, p, mode, st);
-    if (a.N <= 8) return launch_ng<float, 2>(a, p, mode, st);
-    return launch_ng<float, 4>(a, p, mode, st);
+    return io_bf16 ? launch_t<__nv_bfloat16>(a, p, geo, mode, st) : launch_t<float>(a, p, geo, mode, st);
 }
 
 cudaError_t read_device_error(unsigned int* value, int clear) {

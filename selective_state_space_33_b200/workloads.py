@@ -42,6 +42,7 @@ class Workload:
     dskip: str                   # "ones" or "normal"
     seed: int
     backward: bool = False
+    decode: bool = False         # one-token generation steps (seqlen 1, carried state)
     gate: bool = True
     description: str = ""
 
@@ -66,6 +67,8 @@ WORKLOADS = {
                         description="million-step sequence, D 1536, bf16 I/O"),
     "bwd130m": Workload("bwd130m", 8, 2048, 1536, 16, "bf16", 1e-3, 1e-1, "ones", 4,
                         backward=True, description="backward at the Mamba-130M layer shape"),
+    "decode2.8b": Workload("decode2.8b", 64, 1, 5120, 16, "bf16", 1e-3, 1e-1, "normal", 5,
+                           decode=True, description="one generation step, 64 sequences, Mamba-2.8B layer width"),
 }
 
 
@@ -116,6 +119,8 @@ def make_inputs(w: Workload) -> dict:
     x["delta_bias"] = np.log(np.expm1(dt)).astype(np.float32)
     x["A"] = np.ascontiguousarray(
         np.broadcast_to(-(np.arange(w.dstate, dtype=np.float32) + 1.0), (w.dim, w.dstate)))
+    if w.decode:
+        x["state"] = rng.standard_normal((w.batch, w.dim, w.dstate), dtype=np.float32)
     if not w.gate:
         del x["z"]
     return x

@@ -110,3 +110,14 @@ def test_binding_refuses_cpu_tensors(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(sb.SscanError):
         sb.load_library(str(tmp_path / "nope.so"))
+
+
+def test_step_requires_single_token(lib):
+    fake = ctypes.c_void_p(0x10000)
+    p = _p(L=2)
+    assert lib.sscan_step(ctypes.byref(p), *([fake] * 10), None) == 1
+    assert b"seqlen" in lib.sscan_last_error()
+    p = _p(L=1)
+    args = [fake] * 10
+    args[8] = None  # state
+    assert lib.sscan_step(ctypes.byref(p), *args, None) == 1

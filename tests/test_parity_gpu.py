@@ -230,7 +230,8 @@ def _check_bwd(x, io, dev, h0=None):
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
-@pytest.mark.parametrize("shape", [(1, 64, 4, 4), (2, 100, 37, 16), (1, 33, 5, 1), (2, 70, 9, 7)])
+@pytest.mark.parametrize("shape", [(1, 64, 4, 4), (2, 100, 37, 16), (1, 33, 5, 1), (2, 70, 9, 7),
+                                   (2, 100, 64, 16), (1, 37, 32, 8), (3, 50, 24, 4), (1, 300, 96, 16)])
 def test_backward_small(cuda_device, io, shape):
     x = W.small_case(*shape, io=io, seed=sum(shape) + 1, backward=True)
     h0 = np.random.default_rng(5).standard_normal((shape[0], shape[2], shape[3])) * 0.3
@@ -280,3 +281,24 @@ def test_device_status_is_clear(cuda_device):
     flags = ctypes.c_uint(123)
     assert lib.sscan_device_status(1, ctypes.byref(flags)) == 0
     assert flags.value == 0
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_backward_general_path_matches_tiled_path(cuda_device, io):
+    """Misaligned copies of the inputs send the call down the general row kernel; both
+    paths must agree with the oracle and with each other."""
+    x = W.small_case(2, 120, 64, 16, io=io, seed=91, backward=True)
+    t = to_torch(x, cuda_device)
+    args = lambda tt: (tt["u"], tt["delta_raw"], tt["A"], tt["B"], tt["C"], tt["dout"], tt["delta_bias"],
+                       tt["D_skip"], tt["z"])
+    fast = sb.sscan_bwd(*args(t))
+    m = dict(t)
+    for k in ("u", "delta_raw", "z", "dout"):
+        m[k] = _misaligned_copy(t[k])
+    slow = sb.sscan_bwd(*args(m))
+    torch.cuda.synchronize()
+    ref = oracle.bwd(x["u"], x["delta_raw"], x["A"], x["B"], x["C"], x["dout"], delta_bias=x["delta_bias"],
+                     D_skip=x["D_skip"], z=x["z"])
+    for k in ref:
+        assert normwise(to_f64(fast[k]), ref[k]) <= TOL[io], k
+        assert normwise(to_f64(slow[k]), ref[k]) <= TOL[io], k
