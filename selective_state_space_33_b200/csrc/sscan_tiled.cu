@@ -67,7 +67,7 @@ struct Cfg {
     static constexpr int RAW = kTT * DC * (int)sizeof(T);  // bytes of one raw (batch, L, D) tile
     static constexpr int RAWBC = kTT * NS * (int)sizeof(T);  // bytes reserved for one raw B or C tile
     static constexpr int STAGE = 3 * RAW + 2 * RAWBC;      // u, delta_raw, z, B, C
-    static constexpr int GD_PITCH = DC + 8;                // float2 row pitch of the epilogue operands
+    static constexpr int GD_PITCH = DC;                    // float2 row pitch of the epilogue operands
     static constexpr int BC_ENTRIES = kTT * NS;
     static constexpr int PAIRS = kTT * DC / 2;             // channel pairs of phase P
     // shared-memory layout (byte offsets, all 128-aligned)
@@ -76,8 +76,8 @@ struct Cfg {
     static constexpr int OFF_GD = OFF_DX + kTT * DC * 16;                 // float2 (gate, D x gate) [kTT][GD_PITCH]
     static constexpr int OFF_B = OFF_GD + kTT * GD_PITCH * 8;             // float  [kTT][NS]
     static constexpr int OFF_C = OFF_B + kTT * NS * 4;                    // float  [kTT][NS]
-    static constexpr int OFF_OUT = OFF_C + kTT * NS * 4;                  // [2][RAW]
-    static constexpr int OFF_BAR = OFF_OUT + 2 * RAW;                     // uint64 [STAGES]
+    static constexpr int OFF_OUT = OFF_C + kTT * NS * 4;                  // [RAW] output tile
+    static constexpr int OFF_BAR = OFF_OUT + RAW;                         // uint64 [STAGES]
     static constexpr int SMEM = OFF_BAR + STAGES * 8;
 };
 
@@ -353,6 +353,8 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
             float4* sgd = reinterpret_cast<float4*>(smem + C::OFF_GD);
             const float2 pbias = f2((a.bias && pd < a.D) ? __ldg(a.bias + pd) : 0.f,
                                     (a.bias && pd + 1 < a.D) ? __ldg(a.bias + pd + 1) : 0.f);
+            const float2 pdsk = f2((want_out && a.Dskip && pd < a.D) ? __ldg(a.Dskip + pd) : 0.f,
+                                   (want_out && a.Dskip && pd + 1 < a.D) ? __ldg(a.Dskip + pd + 1) : 0.f);
 #pragma unroll
             for (int q = tid; q < C::PAIRS; q += kThreads) {
                 const int t = q / (C::DC / 2);
@@ -362,8 +364,6 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
                 sdx[t * C::DC + pc] = make_float4(dl.x, dl.x, x.x, x.x);
                 sdx[t * C::DC + pc + 1] = make_float4(dl.y, dl.y, x.y, x.y);
                 if (want_out) {
-                    const float2 pdsk = f2((a.Dskip && pd < a.D) ? __ldg(a.Dskip + pd) : 0.f,
-                                           (a.Dskip && pd + 1 < a.D) ? __ldg(a.Dskip + pd + 1) : 0.f);
                     const float2 gt = has_z ? silu_x2(Pair<T>::f(rz[q])) : f2(1.f, 1.f);
                     const float2 dxg = __fmul2_rn(__fmul2_rn(pdsk, x), gt);
                     sgd[(t * C::GD_PITCH + pc) / 2] = make_float4(gt.x, dxg.x, gt.y, dxg.y);
@@ -392,10 +392,12 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
             }
         }
         fence_proxy_async();
+        // the previous tile's output store must have read the one output tile
+        if (want_out && tid == 0) tma_store_wait_read_0();
         __syncthreads();
         if (tid == 0 && it + C::STAGES < ntile) issue(it + C::STAGES);
         // phase S
-        T* sout = reinterpret_cast<T*>(smem + C::OFF_OUT + (it & 1) * C::RAW);
+        T* sout = reinterpret_cast<T*>(smem + C::OFF_OUT);
         float* ck = nullptr;
         if (MODE == kCkpt)
             ck = a.ws_ckpt + ((((int64_t)b * a.nck) + tt / kCkStep) * a.D + d) * N + g * G;
@@ -411,10 +413,7 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
         if (tid == 0 && it + 1 < ntile)
             bad = !mbar_wait(bar0 + 8 * ((it + 1) % C::STAGES), ((it + 1) / C::STAGES) & 1);
         failed = __syncthreads_or(bad) != 0;
-        if (want_out && tid == 0) {
-            tma_store_3d(&tm_out, d0, (int)tt, b, smem_u32(sout));
-            tma_store_wait_read_1();
-        }
+        if (want_out && tid == 0) tma_store_3d(&tm_out, d0, (int)tt, b, smem_u32(sout));
     }
     if (tid == 0 && want_out) tma_store_wait_all();
     if (failed) {

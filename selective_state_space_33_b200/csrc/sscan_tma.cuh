@@ -66,6 +66,10 @@ __device__ __forceinline__ void tma_store_3d_nocommit(const CUtensorMap* map, in
 
 __device__ __forceinline__ void tma_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
+__device__ __forceinline__ void tma_store_wait_read_0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_store_wait_read_1() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
