@@ -76,7 +76,12 @@ typedef struct sscan_problem {
     uint32_t flags;   /* SSCAN_DELTA_SOFTPLUS or 0 */
 } sscan_problem;
 
-typedef enum sscan_op { SSCAN_OP_FWD = 0, SSCAN_OP_LAST_STATE = 1, SSCAN_OP_BWD = 2 } sscan_op;
+typedef enum sscan_op {
+    SSCAN_OP_FWD = 0,
+    SSCAN_OP_LAST_STATE = 1,
+    SSCAN_OP_BWD = 2,
+    SSCAN_OP_SUMMARY = 3
+} sscan_op;
 
 /* Bytes of device workspace the operation needs for this problem (0 when none).
  * The size depends only on the problem and the op.  Returns 0 for an invalid
@@ -164,6 +169,30 @@ SSCAN_API sscan_status sscan_bwd(const sscan_problem* problem, const void* u, co
 SSCAN_API sscan_status sscan_step(const sscan_problem* problem, const void* u, const void* delta_raw,
                                   const float* delta_bias, const float* A, const void* B, const void* C,
                                   const float* D_skip, const void* z, float* state, void* out, void* stream);
+
+/*
+ * Summary of one stretch of the sequence, for splitting a long sequence across
+ * devices (sec. 4.1 / sec. 5: the recurrence is linear in the state, so a stretch
+ * acts on its initial state as the affine map h -> P h + H):
+ *   P = prod_t Abar_t = exp(A * sum_t delta_t)   (batch, D, N) fp32
+ *   H = the final state of the stretch started from zero   (batch, D, N) fp32
+ * C, z and D_skip are not needed.  Workspace: sscan_workspace_size(problem,
+ * SSCAN_OP_SUMMARY) bytes.  seqlen 0 gives the identity (P = 1, H = 0).
+ */
+SSCAN_API sscan_status sscan_chunk_summary(const sscan_problem* problem, const void* u, const void* delta_raw,
+                                           const float* delta_bias, const float* A, const void* B, float* P,
+                                           float* H, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Compose the summaries of nchunks consecutive stretches, in order, starting from
+ * h0 (NULL = zero): carry_in[k] = the state entering stretch k, h_final = the state
+ * after the last.  P, H, carry_in: (nchunks, batch, D, N) fp32, chunk-major;
+ * h0, h_final: (batch, D, N).  Running sscan_fwd on stretch k with
+ * h0 = carry_in[k] reproduces the unsplit scan.  carry_in or h_final may be NULL.
+ * Only problem->batch, dim, dstate are read.
+ */
+SSCAN_API sscan_status sscan_carry(const sscan_problem* problem, int64_t nchunks, const float* P, const float* H,
+                                   const float* h0, float* carry_in, float* h_final, void* stream);
 
 /* Static, human-readable name of a status code. */
 SSCAN_API const char* sscan_status_string(sscan_status status);

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libsscan.so")
 
 SSCAN_F32, SSCAN_BF16 = 0, 1
 SSCAN_DELTA_SOFTPLUS = 1
-SSCAN_OP_FWD, SSCAN_OP_LAST_STATE, SSCAN_OP_BWD = 0, 1, 2
+SSCAN_OP_FWD, SSCAN_OP_LAST_STATE, SSCAN_OP_BWD, SSCAN_OP_SUMMARY = 0, 1, 2, 3
 
 _IO_CODES = {torch.float32: SSCAN_F32, torch.bfloat16: SSCAN_BF16}
 _lib = None
@@ -57,6 +57,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sscan_last_state.restype = ctypes.c_int
     lib.sscan_bwd.argtypes = [pp] + [vp] * 20 + [sz, vp]
     lib.sscan_bwd.restype = ctypes.c_int
+    lib.sscan_chunk_summary.argtypes = [pp] + [vp] * 8 + [sz, vp]
+    lib.sscan_chunk_summary.restype = ctypes.c_int
+    lib.sscan_carry.argtypes = [pp, ctypes.c_int64] + [vp] * 5 + [vp]
+    lib.sscan_carry.restype = ctypes.c_int
     lib.sscan_step.argtypes = [pp] + [vp] * 10 + [vp]
     lib.sscan_step.restype = ctypes.c_int
     lib.sscan_status_string.argtypes = [ctypes.c_int]
@@ -246,3 +250,37 @@ def sscan_step(u, delta_raw, A, B, C, state, delta_bias=None, D_skip=None, z=Non
                                      _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(state), _ptr(out),
                                      _stream(stream)))
     return out
+
+
+def sscan_chunk_summary(u, delta_raw, A, B, delta_bias=None, *, delta_softplus=True, workspace=None,
+                        stream=None):
+    """(P, H), each (batch, D, N) fp32: the stretch u[:, 0:L] acts on its initial state as
+    h -> P h + H (P = exp(A * sum of delta), H = final state from zero)."""
+    prob = _io_problem(u, B, delta_softplus)
+    _check_inputs(prob, u, delta_raw, A, B, None, delta_bias, None, None, None)
+    f32 = dict(dtype=torch.float32, device=u.device)
+    P = torch.empty((prob.batch, prob.dim, prob.dstate), **f32)
+    H = torch.empty((prob.batch, prob.dim, prob.dstate), **f32)
+    ws, nbytes = _workspace(prob, SSCAN_OP_SUMMARY, workspace, u.device)
+    _check(load_library().sscan_chunk_summary(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias),
+                                              _ptr(A), _ptr(B), _ptr(P), _ptr(H), _ptr(ws), nbytes,
+                                              _stream(stream)))
+    return P, H
+
+
+def sscan_carry(P, H, h0=None, *, stream=None):
+    """Compose K stretch summaries P, H (K, batch, D, N) in order from h0 (batch, D, N):
+    returns (carry_in (K, batch, D, N), h_final (batch, D, N))."""
+    if P.dim() != 4 or P.shape != H.shape:
+        raise ValueError("P and H must both be (K, batch, D, N)")
+    K, batch, D, N = P.shape
+    dev = P.device
+    _expect(P, "P", P.shape, torch.float32, dev)
+    _expect(H, "H", P.shape, torch.float32, dev)
+    _expect(h0, "h0", (batch, D, N), torch.float32, dev)
+    prob = make_problem(batch, 0, D, N, SSCAN_F32)
+    carry = torch.empty_like(P)
+    h_final = torch.empty((batch, D, N), dtype=torch.float32, device=dev)
+    _check(load_library().sscan_carry(ctypes.byref(prob), int(K), _ptr(P), _ptr(H), _ptr(h0), _ptr(carry),
+                                      _ptr(h_final), _stream(stream)))
+    return carry, h_final

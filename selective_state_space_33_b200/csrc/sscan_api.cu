@@ -283,6 +283,10 @@ size_t sscan_workspace_size(const sscan_problem* p, int op) {
         }
         case SSCAN_OP_BWD:
             return sscan::plan_bwd(p->batch, p->seqlen, p->dim, p->dstate).workspace_bytes;
+        case SSCAN_OP_SUMMARY:
+            return (p->batch * p->dim > 0 && p->seqlen > 0)
+                       ? sscan::align256((size_t)(p->batch * p->dim) * sizeof(float))
+                       : 0;
         default:
             return 0;
     }
@@ -516,6 +520,76 @@ sscan_status sscan_step(const sscan_problem* p, const void* u, const void* delta
     const cudaError_t e = sscan::launch_step(a, p->io_dtype == SSCAN_BF16, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "step kernel: %s", cudaGetErrorString(e));
     return SSCAN_OK;
+}
+
+sscan_status sscan_chunk_summary(const sscan_problem* p, const void* u, const void* delta_raw,
+                                 const float* delta_bias, const float* A, const void* B, float* P, float* H,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    g_err[0] = 0;
+    g_launches = 0;
+    if (sscan_status s = check_problem(p)) return s;
+    const int64_t BD = p->batch * p->dim, BDN = BD * p->dstate;
+    if (BD == 0) return SSCAN_OK;
+    if (!P || !H) return fail(SSCAN_ERR_INVALID_ARG, "P and H are required");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (p->seqlen == 0) {  // the identity map
+        cudaError_t e = cudaMemsetAsync(H, 0, (size_t)BDN * sizeof(float), st);
+        if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing H: %s", cudaGetErrorString(e));
+        sscan::fill_kernel<<<blocks_for(BDN, 256), 256, 0, st>>>(P, 1.f, BDN);
+        ++g_launches;
+        return cuda_check("fill kernel");
+    }
+    if (!u || !delta_raw || !A || !B) return fail(SSCAN_ERR_INVALID_ARG, "u, delta_raw, A, B are required");
+    if (sscan_status s = check_workspace(sscan_workspace_size(p, SSCAN_OP_SUMMARY), workspace, workspace_bytes))
+        return s;
+    // one aggregate pass over the whole sequence: H = end state from zero, dsum = sum of delta
+    sscan::ScanArgs a = make_args(p, u, delta_raw, delta_bias, A, B, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                  nullptr);
+    a.nchunks = 1;
+    a.chunk_len = p->seqlen;
+    a.ws_state = H;
+    a.ws_dsum = static_cast<float*>(workspace);
+    if (tiled_ok(p, a)) {
+        const sscan::TiledGeom geo = sscan::tiled_geometry(p->batch, p->seqlen, p->dim, p->dstate);
+        sscan::TiledArgs t{};
+        t.batch = p->batch;
+        t.L = p->seqlen;
+        t.D = p->dim;
+        t.N = (int)p->dstate;
+        t.softplus = a.softplus;
+        t.bias = delta_bias;
+        t.A = A;
+        t.B = B;
+        t.chunk_len = p->seqlen;
+        t.nchunks = 1;
+        t.ws_state = H;
+        t.ws_dsum = a.ws_dsum;
+        sscan::TiledPtrs tp{u, delta_raw, nullptr, nullptr};
+        ++g_launches;
+        const cudaError_t e = sscan::launch_fwd_tiled(t, tp, geo, p->io_dtype == SSCAN_BF16, sscan::kTiledAgg, st);
+        if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "aggregate kernel: %s", cudaGetErrorString(e));
+    } else {
+        fwd_rows(a, p->io_dtype, sscan::kModeAggregate, st);
+        if (sscan_status s = cuda_check("aggregate kernel")) return s;
+    }
+    sscan::decay_kernel<<<blocks_for(BDN, 128), 128, 0, st>>>(a.ws_dsum, A, P, p->batch, p->dim, p->dstate);
+    ++g_launches;
+    return cuda_check("decay kernel");
+}
+
+sscan_status sscan_carry(const sscan_problem* p, int64_t nchunks, const float* P, const float* H, const float* h0,
+                         float* carry_in, float* h_final, void* stream) {
+    g_err[0] = 0;
+    g_launches = 0;
+    if (sscan_status s = check_problem(p)) return s;
+    if (nchunks < 0) return fail(SSCAN_ERR_INVALID_ARG, "nchunks must be >= 0");
+    const int64_t BDN = p->batch * p->dim * p->dstate;
+    if (BDN == 0 || (!carry_in && !h_final)) return SSCAN_OK;
+    if (nchunks > 0 && (!P || !H)) return fail(SSCAN_ERR_INVALID_ARG, "P and H are required");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    sscan::compose_kernel<<<blocks_for(BDN, 128), 128, 0, st>>>(P, H, h0, carry_in, h_final, nchunks, BDN);
+    ++g_launches;
+    return cuda_check("compose kernel");
 }
 
 const char* sscan_status_string(sscan_status s) {

@@ -151,7 +151,7 @@ __device__ __forceinline__ float2 softplus_dsig(float r) {
 }
 
 template <typename T, int NG>
-__global__ void __launch_bounds__(kThreadsB, 6)
+__global__ void __launch_bounds__(kThreadsB, 5)
     bwd_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dr,
                      const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_g,
                      const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -318,8 +318,10 @@ __global__ void __launch_bounds__(kThreadsB, 6)
                 shs[t * kThreadsB] = make_float4(h0.x, h0.y, h1.x, h1.y);
             }
         }
-        // ---- reverse sweep in blocks of NG steps (last block first)
+        // ---- reverse sweep in blocks of NG steps (last block first); the state loaded as
+        // h_{t-1} at step t is the h_t of step t-1, so it is carried in registers
         T* so = reinterpret_cast<T*>(smem + C::OFF_OUT + (k & 1) * 3 * C::RAW);
+        float4 hnext = tile_len > 0 ? shs[(tile_len - 1) * kThreadsB] : make_float4(0.f, 0.f, 0.f, 0.f);
         for (int tb = ((tile_len - 1) / NG) * NG; tb >= 0; tb -= NG) {
             float pdu[NG], pdd[NG], py[NG];
 #pragma unroll
@@ -333,12 +335,12 @@ __global__ void __launch_bounds__(kThreadsB, 6)
                     const float4 dx = sdx[t * C::DC];
                     const float4 dq = sdq[t * C::DC];
                     const float4 Bv = sB[t * NG], Cv = sC[t * NG];
-                    const float4 hc = shs[t * kThreadsB];
+                    const float4 hc = hnext;
                     float2 hp[2];
                     if (t > 0) {
-                        const float4 v = shs[(t - 1) * kThreadsB];
-                        hp[0] = g2(v.x, v.y);
-                        hp[1] = g2(v.z, v.w);
+                        hnext = shs[(t - 1) * kThreadsB];
+                        hp[0] = g2(hnext.x, hnext.y);
+                        hp[1] = g2(hnext.z, hnext.w);
                     } else {
                         hp[0] = hk[0];
                         hp[1] = hk[1];

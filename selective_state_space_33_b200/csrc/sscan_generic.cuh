@@ -135,4 +135,29 @@ __global__ void __launch_bounds__(128) carry_kernel(ScanArgs a) {
     if (a.h_last) a.h_last[gid] = h;
 }
 
+// P = exp(A_n * sum of delta): the decay of a chunk summary, from the per-row sums
+// that the aggregate pass leaves in dsum (batch, D).  One thread per (b, d, n).
+__global__ void __launch_bounds__(128) decay_kernel(const float* dsum, const float* A, float* P, int64_t batch,
+                                                    int64_t D, int64_t N) {
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= batch * D * N) return;
+    const int64_t n = gid % N, bd = gid / N, d = bd % D;
+    P[gid] = ex2(__ldg(A + d * N + n) * kLog2e * dsum[bd]);
+}
+
+// Compose K chunk maps h -> P_k h + H_k (each (batch, D, N), chunk-major) in order,
+// starting from h0: carry_in[k] is the state entering chunk k, h_final the state
+// after the last.  One thread per (b, d, n).
+__global__ void __launch_bounds__(128) compose_kernel(const float* P, const float* H, const float* h0,
+                                                      float* carry_in, float* h_final, int64_t K, int64_t BDN) {
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= BDN) return;
+    float h = h0 ? __ldg(h0 + gid) : 0.f;
+    for (int64_t k = 0; k < K; ++k) {
+        if (carry_in) carry_in[k * BDN + gid] = h;
+        h = fmaf(__ldg(P + k * BDN + gid), h, __ldg(H + k * BDN + gid));
+    }
+    if (h_final) h_final[gid] = h;
+}
+
 }  // namespace sscan

@@ -185,6 +185,11 @@ __global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
     if (g.dbias) atomicAdd(g.dbias + d, dbacc);
 }
 
+__global__ void fill_kernel(float* dst, float v, int64_t n) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) dst[i] = v;
+}
+
 // fp32 accumulator -> I/O type (dB, dC)
 template <typename T>
 __global__ void cast_kernel(const float* src, T* dst, int64_t n) {
