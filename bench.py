@@ -104,6 +104,40 @@ def roofline_units(w: W.Workload) -> dict:
     return {"elements": E, "bytes": bytes_, "exps": E * (w.dstate + 2)}
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of each
+# workload's dominant kernel, read from one ncu capture of that workload (summaries
+# under profiles/).  A figure holds only for the kernel source it was taken on: it is
+# keyed by the SHA-256 of those source files and reported as null once they change.
+NCU_TRAFFIC = {
+    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 506368768 + 151190272,
+                  "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "5a5b29414ed43428",
+                  "profile": "profiles/fwd_tiled_kernel_mamba2.8b_bf16.md"},
+    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 406294784 + 133817088,
+                "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "2178d0fd962a137f",
+                "profile": "profiles/bwd_tiled_kernel_bwd130m_fp32.md"},
+    "decode2.8b": {"kernel": "step_kernel", "bytes": 23327232 + 2048,
+                   "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "b358a00da4e6ff0b",
+                   "profile": "profiles/step_kernel_decode2.8b_bf16.md"},
+}
+
+
+def ncu_traffic(workload: str):
+    """The recorded per-launch DRAM traffic of the workload's dominant kernel, or None
+    when none was recorded or the kernel's sources changed since the capture."""
+    import hashlib
+    rec = NCU_TRAFFIC.get(workload)
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    for name in rec["sources"]:
+        path = os.path.join(ROOT, "selective_state_space_33_b200", "csrc", name)
+        if not os.path.exists(path):
+            return None
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return rec["bytes"] if h.hexdigest()[:16] == rec["sha256"] else None
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -421,9 +455,9 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
         "e2e": None if e2e_value is None else {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                                                "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
-        "roofline": hbm_roofline(units, launch_s, hbm_peak, hbm_src) if w.decode else {
+        "roofline": hbm_roofline(units, launch_s, hbm_peak, hbm_src, ncu_traffic(args.workload)) if w.decode else {
             "bound": "alu", "pipe": "MUFU ex2", "achieved": exps_rate / 1e9, "peak": mufu_nominal / 1e9,
-            "unit": "Gexp/s", "frac": exps_rate / mufu_nominal, "traffic": None,
+            "unit": "Gexp/s", "frac": exps_rate / mufu_nominal, "traffic": ncu_traffic(args.workload),
             "peak_source": f"derived: {SM_COUNT} SMs x {MUFU_PER_SM_CLK} ex2/clk x {sm_max:.0f} MHz",
             "peak_probe_gexps": None if mufu_probe is None else mufu_probe / 1e9,
             "frac_of_probe": None if mufu_probe is None else exps_rate / mufu_probe,
@@ -438,10 +472,10 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
     print(json.dumps(line), flush=True)
 
 
-def hbm_roofline(units, launch_s, hbm_peak, hbm_src):
+def hbm_roofline(units, launch_s, hbm_peak, hbm_src, traffic=None):
     gbs = units["bytes"] / launch_s / 1e9
     return {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
-            "traffic": None, "source": hbm_src, "per_launch_ms": launch_s * 1e3,
+            "traffic": traffic, "source": hbm_src, "per_launch_ms": launch_s * 1e3,
             "alg_bytes_per_launch": units["bytes"]}
 
 
