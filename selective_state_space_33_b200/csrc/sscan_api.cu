@@ -451,9 +451,22 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
         ba.dD = dD;
         ba.dbias = ddelta_bias;
         ba.dh0 = dh0;
+        ba.seg_len = plan.seg_len;
+        ba.nseg = plan.nsegs;
+        ba.ws_lam = ws + 2 * BLN + plan.ck_floats;
+        ba.ws_dsum = ba.ws_lam + p->batch * plan.nsegs * p->dim * p->dstate;
         sscan::BwdTiledPtrs bp{u, delta_raw, z, dout, B, C, du, ddelta_raw, dz};
+        if (plan.nsegs > 1) {
+            // the reverse sweep split in time: segment summaries, then their carry
+            ++g_launches;
+            e = sscan::launch_bwd_tiled(ba, bp, bf16, sscan::kBwdSummary, st);
+            if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "backward summary kernel: %s", cudaGetErrorString(e));
+            ++g_launches;
+            e = sscan::launch_bwd_carry(ba, st);
+            if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "backward carry kernel: %s", cudaGetErrorString(e));
+        }
         ++g_launches;
-        e = sscan::launch_bwd_tiled(ba, bp, bf16, st);
+        e = sscan::launch_bwd_tiled(ba, bp, bf16, sscan::kBwdFull, st);
         if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "backward kernel: %s", cudaGetErrorString(e));
         if (bf16) {
             cast_out<__nv_bfloat16>(ws, dB, BLN, st);

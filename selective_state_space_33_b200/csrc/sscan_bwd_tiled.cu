@@ -150,7 +150,7 @@ __device__ __forceinline__ float2 softplus_dsig(float r) {
     return g2(r > 20.f ? r : v, sig);
 }
 
-template <typename T, int NG>
+template <typename T, int NG, int MODE>
 __global__ void __launch_bounds__(kThreadsB, 5)
     bwd_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dr,
                      const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_g,
@@ -163,20 +163,28 @@ __global__ void __launch_bounds__(kThreadsB, 5)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t ncb = (a.D + C::DC - 1) / C::DC;
     const int cb = (int)(blockIdx.x % ncb);
-    const int b = (int)(blockIdx.x / ncb);
+    // segment of the sequence (the summary pass skips segment 0, whose summary no
+    // segment needs)
+    const int64_t nsl = MODE == kBwdSummary ? a.nseg - 1 : a.nseg;
+    const int64_t rest = blockIdx.x / ncb;
+    const int seg = (int)(rest % nsl) + (MODE == kBwdSummary ? 1 : 0);
+    const int b = (int)(rest / nsl);
     const int N = a.N;
     const int d0 = cb * C::DC;
-    const int ntb = (int)((a.L + kTB - 1) / kTB);
+    const int tiles_all = (int)((a.L + kTB - 1) / kTB);
+    const int tile_lo = seg * (int)(a.seg_len / kTB);
+    const int tile_hi = min(tiles_all, tile_lo + (int)((a.seg_len + kTB - 1) / kTB));
+    const int ntb = tile_hi - tile_lo;  // tiles of this segment
     const bool has_z = a.has_z != 0;
     const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
     const uint32_t stage_bytes = (has_z ? 4u : 3u) * C::RAW + 2u * (uint32_t)(kTB * N * (int)sizeof(T));
 
-    // tiles are taken in reverse: processing index k covers tile ntb - 1 - k
+    // tiles are taken in reverse: processing index k covers tile tile_hi - 1 - k
     auto issue = [&](int k) {
         const int st = k % C::STAGES;
         const uint32_t bar = bar0 + 8 * st;
         const uint32_t base = smem_u32(smem + C::OFF_RAW + st * C::STAGE);
-        const int t0 = (ntb - 1 - k) * kTB;
+        const int t0 = (tile_hi - 1 - k) * kTB;
         mbar_expect_tx(bar, stage_bytes);
         tma_load_3d(base, &tm_u, d0, t0, b, bar);
         tma_load_3d(base + C::RAW, &tm_dr, d0, t0, b, bar);
@@ -215,6 +223,18 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         iA[k] = g2(ia[0], ia[1]);
         lam[k] = P1[k] = P2v[k] = g2(0.f, 0.f);
     }
+    if (MODE == kBwdFull && a.nseg > 1) {
+        // the adjoint state the segments to the right pass in
+        float lv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = g * 4 + j;
+            lv[j] = cvalid && n < N ? a.ws_lam[(((int64_t)b * a.nseg + seg) * a.D + d) * N + n] : 0.f;
+        }
+        lam[0] = g2(lv[0], lv[1]);
+        lam[1] = g2(lv[2], lv[3]);
+    }
+    float dsum = 0.f;
     const int nvalid = cvalid ? min(4, N - g * 4) : 0;
     float dbias_acc = 0.f;
     // phase-P channel pair of this thread
@@ -226,7 +246,7 @@ __global__ void __launch_bounds__(kThreadsB, 5)
     bool failed = __syncthreads_or(bad) != 0;
 
     for (int k = 0; k < ntb && !failed; ++k) {
-        const int it = ntb - 1 - k;
+        const int it = tile_hi - 1 - k;
         const int st = k % C::STAGES;
         const int t0 = it * kTB;
         const int tile_len = (int)(a.L - t0 < kTB ? a.L - t0 : kTB);
@@ -289,6 +309,28 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         fence_proxy_async();
         __syncthreads();
         if (tid == 0 && k + C::STAGES < ntb) issue(k + C::STAGES);
+
+        if constexpr (MODE == kBwdSummary) {
+            // adjoint only: lam <- Abar_t (C_t dy_t + lam), from the right end of the segment
+            const float4* sdx = reinterpret_cast<const float4*>(smem + C::OFF_DX) + cw;
+            const float4* sdq = reinterpret_cast<const float4*>(smem + C::OFF_DQ) + cw;
+            const float4* sC = reinterpret_cast<const float4*>(smem + C::OFF_C) + g;
+            for (int t = tile_len - 1; t >= 0; --t) {
+                const float4 dx = sdx[t * C::DC];
+                const float4 dq = sdq[t * C::DC];
+                const float4 Cv = sC[t * NG];
+                const float2 dd = g2(dx.x, dx.y), dyy = g2(dq.x, dq.y);
+                const float2 Cp[2] = {g2(Cv.x, Cv.y), g2(Cv.z, Cv.w)};
+#pragma unroll
+                for (int p = 0; p < 2; ++p)
+                    lam[p] = __fmul2_rn(__ffma2_rn(Cp[p], dyy, lam[p]), ex2p(__fmul2_rn(dd, A2[p])));
+                dsum += dx.x;
+            }
+            if (tid == 0 && k + 1 < ntb)
+                bad = !mbar_wait(bar0 + 8 * ((k + 1) % C::STAGES), ((k + 1) / C::STAGES) & 1);
+            failed = __syncthreads_or(bad) != 0;
+            continue;
+        }
 
         // ---- recompute the tile's states from the checkpoint
         const float4* sdx = reinterpret_cast<const float4*>(smem + C::OFF_DX) + cw;
@@ -450,14 +492,22 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         }
         return;
     }
-    // per-channel sums
     const float lamv[4] = {lam[0].x, lam[0].y, lam[1].x, lam[1].y};
+    if constexpr (MODE == kBwdSummary) {
+        // the segment's summary: adjoint state passed on from zero, and its sum of delta
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (j < nvalid) a.ws_lam[(((int64_t)b * a.nseg + seg) * a.D + d) * N + g * 4 + j] = lamv[j];
+        if (g == 0 && cvalid) a.ws_dsum[((int64_t)b * a.nseg + seg) * a.D + d] = dsum;
+        return;
+    }
+    // per-channel sums
     const float dAv[4] = {P1[0].x + P2v[0].x, P1[0].y + P2v[0].y, P1[1].x + P2v[1].x, P1[1].y + P2v[1].y};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         if (j >= nvalid) continue;
         const int n = g * 4 + j;
-        if (a.dh0) a.dh0[((int64_t)b * a.D + d) * N + n] = lamv[j];
+        if (a.dh0 && seg == 0) a.dh0[((int64_t)b * a.D + d) * N + n] = lamv[j];
         // dA = sum_t [delta lam Abar h_{t-1} + lam B x delta^2 psi(delta A)]
         atomicAdd(a.dA + d * N + n, dAv[j]);
     }
@@ -491,28 +541,57 @@ bool make_map_b(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int6
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int NG>
-cudaError_t launch_bwd_t(const BwdTiledArgs& a, const BwdTiledPtrs& p, cudaStream_t st) {
+template <typename T, int NG, int MODE>
+void launch_bwd_kernel(const CUtensorMap (&m)[9], const BwdTiledArgs& a, cudaStream_t st) {
     using C = BCfg<T, NG>;
-    CUtensorMap mu, md, mz, mg, mb, mc, mdu, mdd, mdz;
-    const void* zsrc = p.z ? p.z : p.u;
-    void* dzdst = p.dz ? p.dz : p.du;
-    if (!make_map_b<T>(&mu, p.u, a.batch, a.L, a.D, C::DC) || !make_map_b<T>(&md, p.delta_raw, a.batch, a.L, a.D, C::DC) ||
-        !make_map_b<T>(&mz, zsrc, a.batch, a.L, a.D, C::DC) || !make_map_b<T>(&mg, p.dout, a.batch, a.L, a.D, C::DC) ||
-        !make_map_b<T>(&mb, p.B, a.batch, a.L, a.N, a.N) || !make_map_b<T>(&mc, p.C, a.batch, a.L, a.N, a.N) ||
-        !make_map_b<T>(&mdu, p.du, a.batch, a.L, a.D, C::DC) || !make_map_b<T>(&mdd, p.ddelta_raw, a.batch, a.L, a.D, C::DC) ||
-        !make_map_b<T>(&mdz, dzdst, a.batch, a.L, a.D, C::DC))
-        return cudaErrorInvalidValue;
-    auto kern = bwd_tiled_kernel<T, NG>;
+    auto kern = bwd_tiled_kernel<T, NG, MODE>;
     static bool configured = false;
     if (!configured) {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         configured = true;
     }
-    const int64_t blocks = a.batch * ((a.D + C::DC - 1) / C::DC);
-    kern<<<(unsigned)blocks, kThreadsB, C::SMEM, st>>>(mu, md, mz, mg, mb, mc, mdu, mdd, mdz, a);
+    const int64_t segs = MODE == kBwdSummary ? a.nseg - 1 : a.nseg;
+    const int64_t blocks = a.batch * segs * ((a.D + C::DC - 1) / C::DC);
+    if (blocks > 0)
+        kern<<<(unsigned)blocks, kThreadsB, C::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], m[8], a);
+}
+
+template <typename T, int NG>
+cudaError_t launch_bwd_t(const BwdTiledArgs& a, const BwdTiledPtrs& p, int mode, cudaStream_t st) {
+    using C = BCfg<T, NG>;
+    CUtensorMap m[9];
+    const void* zsrc = p.z ? p.z : p.u;
+    void* dzdst = p.dz ? p.dz : p.du;
+    if (!make_map_b<T>(&m[0], p.u, a.batch, a.L, a.D, C::DC) || !make_map_b<T>(&m[1], p.delta_raw, a.batch, a.L, a.D, C::DC) ||
+        !make_map_b<T>(&m[2], zsrc, a.batch, a.L, a.D, C::DC) || !make_map_b<T>(&m[3], p.dout, a.batch, a.L, a.D, C::DC) ||
+        !make_map_b<T>(&m[4], p.B, a.batch, a.L, a.N, a.N) || !make_map_b<T>(&m[5], p.C, a.batch, a.L, a.N, a.N) ||
+        !make_map_b<T>(&m[6], p.du, a.batch, a.L, a.D, C::DC) || !make_map_b<T>(&m[7], p.ddelta_raw, a.batch, a.L, a.D, C::DC) ||
+        !make_map_b<T>(&m[8], dzdst, a.batch, a.L, a.D, C::DC))
+        return cudaErrorInvalidValue;
+    if (mode == kBwdSummary) launch_bwd_kernel<T, NG, kBwdSummary>(m, a, st);
+    else launch_bwd_kernel<T, NG, kBwdFull>(m, a, st);
     return cudaGetLastError();
+}
+
+// One thread per (batch, channel, state): walk the segments right to left, leaving
+// in ws_lam the adjoint state that enters each segment from its right.  A segment
+// maps an entering adjoint state lam to P lam + H, with P = exp(A * its sum of delta)
+// (the product of its Abar) and H its summary.
+__global__ void __launch_bounds__(128) bwd_carry_kernel(BwdTiledArgs a) {
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= a.batch * a.D * a.N) return;
+    const int64_t n = gid % a.N, bd = gid / a.N;
+    const int64_t d = bd % a.D, b = bd / a.D;
+    const float A2 = __ldg(a.A + d * a.N + n) * kLog2e;
+    float lam = 0.f;
+    for (int64_t s = a.nseg - 1; s >= 1; --s) {
+        const int64_t i = ((b * a.nseg + s) * a.D + d) * a.N + n;
+        const float H = a.ws_lam[i];
+        a.ws_lam[i] = lam;
+        lam = fmaf(ex2(A2 * a.ws_dsum[(b * a.nseg + s) * a.D + d]), lam, H);
+    }
+    a.ws_lam[((b * a.nseg) * a.D + d) * a.N + n] = lam;
 }
 
 }  // namespace
@@ -526,15 +605,21 @@ cudaError_t read_device_error_bwd(unsigned int* value, int clear) {
     return e;
 }
 
-cudaError_t launch_bwd_tiled(const BwdTiledArgs& a, const BwdTiledPtrs& p, int io_bf16, cudaStream_t st) {
+cudaError_t launch_bwd_tiled(const BwdTiledArgs& a, const BwdTiledPtrs& p, int io_bf16, int mode, cudaStream_t st) {
     if (io_bf16) {
-        if (a.N <= 4) return launch_bwd_t<__nv_bfloat16, 1>(a, p, st);
-        if (a.N <= 8) return launch_bwd_t<__nv_bfloat16, 2>(a, p, st);
-        return launch_bwd_t<__nv_bfloat16, 4>(a, p, st);
+        if (a.N <= 4) return launch_bwd_t<__nv_bfloat16, 1>(a, p, mode, st);
+        if (a.N <= 8) return launch_bwd_t<__nv_bfloat16, 2>(a, p, mode, st);
+        return launch_bwd_t<__nv_bfloat16, 4>(a, p, mode, st);
     }
-    if (a.N <= 4) return launch_bwd_t<float, 1>(a, p, st);
-    if (a.N <= 8) return launch_bwd_t<float, 2>(a, p, st);
-    return launch_bwd_t<float, 4>(a, p, st);
+    if (a.N <= 4) return launch_bwd_t<float, 1>(a, p, mode, st);
+    if (a.N <= 8) return launch_bwd_t<float, 2>(a, p, mode, st);
+    return launch_bwd_t<float, 4>(a, p, mode, st);
+}
+
+cudaError_t launch_bwd_carry(const BwdTiledArgs& a, cudaStream_t st) {
+    const int64_t n = a.batch * a.D * a.N;
+    if (n > 0) bwd_carry_kernel<<<(unsigned)((n + 127) / 128), 128, 0, st>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace sscan

@@ -85,7 +85,14 @@ struct BwdTiledArgs {
     float* dD;           // (D) or null, pre-zeroed
     float* dbias;        // (D) or null, pre-zeroed
     float* dh0;          // (batch, D, N) or null
+    // sequence split of the reverse sweep: segment s covers steps
+    // [s * seg_len, min(L, (s + 1) * seg_len)), seg_len a multiple of 8
+    int64_t seg_len, nseg;
+    float* ws_lam;       // [batch][nseg][D][N]: segment adjoint summaries, then carry-ins
+    float* ws_dsum;      // [batch][nseg][D]: sum of delta over each segment
 };
+
+enum { kBwdFull = 0, kBwdSummary = 1 };
 
 struct BwdTiledPtrs {
     const void* u;
@@ -99,7 +106,12 @@ struct BwdTiledPtrs {
     void* dz;            // or null
 };
 
-cudaError_t launch_bwd_tiled(const BwdTiledArgs& a, const BwdTiledPtrs& p, int io_bf16, cudaStream_t st);
+// kBwdFull: the gradients of every segment (adjoint state entering each segment from
+// ws_lam when nseg > 1).  kBwdSummary: for segments 1 .. nseg-1 only, the adjoint
+// state a segment passes to its left from zero and its sum of delta.
+cudaError_t launch_bwd_tiled(const BwdTiledArgs& a, const BwdTiledPtrs& p, int io_bf16, int mode, cudaStream_t st);
+// Turn the segment summaries in ws_lam into each segment's entering adjoint state.
+cudaError_t launch_bwd_carry(const BwdTiledArgs& a, cudaStream_t st);
 cudaError_t read_device_error_bwd(unsigned int* value, int clear);
 
 // Read (and optionally clear) the library's device error word; nonzero means a

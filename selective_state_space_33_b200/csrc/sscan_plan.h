@@ -70,21 +70,65 @@ inline FwdPlan plan_tiled(int64_t batch, int64_t L, int64_t D, int64_t N, int64_
 }
 
 struct BwdPlan {
-    int64_t nseg;
+    int64_t nseg;           // general kernel: checkpoint segments per row
+    int64_t ck_floats;      // checkpoint floats (general or tiled layout, the larger)
+    int64_t seg_len;        // tiled kernel: steps per reverse-sweep segment
+    int64_t nsegs;          // tiled kernel: reverse-sweep segments
     size_t workspace_bytes;
 };
 
-// fp32 accumulators for dB and dC (batch, L, N), then checkpointed states: one
-// every kBwdSeg steps of every row for the general kernel, one every
-// kBwdTiledSeg steps for the tiled kernel.  The workspace covers either.
+// The tiled backward gives every channel 1, 2 or 4 lanes (4 states each), so a CTA
+// of 4 warps holds 128, 64 or 32 channels of one batch, and 5 CTAs fit an SM.
+// When batch x channel blocks leave the GPU short of that, the reverse sweep is
+// split in time into segments, each started from the adjoint state its right
+// neighbours pass in (one summary pass over all but the first segment, plus a
+// carry).  The segment count fills the resident slots best over whole waves (up to
+// kBwdMaxSegs); segments are whole checkpoint tiles of at least kBwdMinSeg steps.
 constexpr int kBwdTiledSeg = 8;
+constexpr int64_t kBwdSlots = 5 * kSmCount;
+constexpr int64_t kBwdMinSeg = 128;
+constexpr int64_t kBwdMaxSegs = 8;
+
+inline int64_t bwd_tiled_channels(int64_t N) {
+    const int64_t ng = N <= 4 ? 1 : (N <= 8 ? 2 : 4);
+    return 4 * (32 / ng);
+}
+
+// fp32 accumulators for dB and dC (batch, L, N); checkpointed states (one every
+// kBwdSeg steps of every row for the general kernel, one every kBwdTiledSeg steps
+// for the tiled kernel; the workspace covers either); then, for the tiled kernel's
+// segments, their adjoint summaries [batch][nsegs][D][N] and delta sums
+// [batch][nsegs][D].
 inline BwdPlan plan_bwd(int64_t batch, int64_t L, int64_t D, int64_t N) {
-    BwdPlan p{0, 0};
+    BwdPlan p{0, 0, 0, 1, 0};
     if (batch * D <= 0 || L <= 0) return p;
     p.nseg = (L + kBwdSeg - 1) / kBwdSeg;
     const int64_t nck = (L + kBwdTiledSeg - 1) / kBwdTiledSeg;
-    const int64_t ck = (batch * D * p.nseg * N > batch * nck * D * N) ? batch * D * p.nseg * N : batch * nck * D * N;
-    const size_t floats = (size_t)(2 * batch * L * N) + (size_t)ck;
+    p.ck_floats = (batch * D * p.nseg * N > batch * nck * D * N) ? batch * D * p.nseg * N : batch * nck * D * N;
+    p.seg_len = L;
+    const int64_t cols = batch * ((D + bwd_tiled_channels(N) - 1) / bwd_tiled_channels(N));
+    int64_t want = 1;
+    if (cols < kBwdSlots) {
+        // fraction of slot-time used over whole waves: cols n / (waves * slots)
+        double best = (double)cols / (double)kBwdSlots;
+        const int64_t most = L / kBwdMinSeg < kBwdMaxSegs ? L / kBwdMinSeg : kBwdMaxSegs;
+        for (int64_t n = 2; n <= most; ++n) {
+            const int64_t ctas = cols * n, waves = (ctas + kBwdSlots - 1) / kBwdSlots;
+            const double eff = (double)ctas / (double)(waves * kBwdSlots);
+            if (eff > best * 1.05) {
+                best = eff;
+                want = n;
+            }
+        }
+    }
+    if (want > 1) {
+        int64_t len = (L + want - 1) / want;
+        len = (len + kBwdTiledSeg - 1) / kBwdTiledSeg * kBwdTiledSeg;
+        p.seg_len = len;
+        p.nsegs = (L + len - 1) / len;
+    }
+    const int64_t seg_floats = p.nsegs > 1 ? batch * p.nsegs * D * (N + 1) : 0;
+    const size_t floats = (size_t)(2 * batch * L * N) + (size_t)p.ck_floats + (size_t)seg_floats;
     p.workspace_bytes = align256(floats * sizeof(float));
     return p;
 }

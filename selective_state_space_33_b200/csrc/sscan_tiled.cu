@@ -81,18 +81,27 @@ struct Cfg {
     static constexpr int SMEM = OFF_BAR + STAGES * 8;
 };
 
-// Per lane: G states of one channel as G/2 f32x2 pairs, with A log2(e) and 1/A.
+// Per lane: G states of one channel as G/2 f32x2 pairs, with A log2(e) and -1/A.
 template <int G>
 struct LaneG {
-    float2 h[G / 2], A2[G / 2], iA[G / 2];
+    float2 h[G / 2], A2[G / 2], niA[G / 2];
 };
 
 __device__ __forceinline__ float2 ex2x2(float2 q) { return f2(ex2(q.x), ex2(q.y)); }
 
-// One step for the lane's G states, eq. (2) and (3a), in the b-form
-// Bbar x = (Abar - 1) w with w = B x / A, evaluated as fma(Abar, w, -w) (one
-// rounding).  dx = (delta, delta, x, x); Bp, Cp point at the lane's G values of B_t,
-// C_t.  Returns the partial readout sum_j C_j h_j over these states (eq. (3b)).
+// a - b on both halves (one packed f32x2 instruction).
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+    unsigned long long ra = *reinterpret_cast<unsigned long long*>(&a), rb = *reinterpret_cast<unsigned long long*>(&b),
+                       rd;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+    return *reinterpret_cast<float2*>(&rd);
+}
+
+// One step for the lane's G states, eq. (2) and (3a).  With v = -B x / A the update
+// h' = Abar h + (Abar - 1) B x / A is Abar (h - v) + v: one packed subtract and one
+// packed fma per pair, no negation.  dx = (delta, delta, x, x); Bp, Cp point at the
+// lane's G values of B_t, C_t.  Returns the partial readout sum_j C_j h_j over these
+// states (eq. (3b)).
 template <int G, bool WANT_Y>
 __device__ __forceinline__ float step_fast(LaneG<G>& s, float4 dx, const float4* Bp, const float4* Cp) {
     const float2 dd = f2(dx.x, dx.y), xx = f2(dx.z, dx.w);
@@ -102,10 +111,10 @@ __device__ __forceinline__ float step_fast(LaneG<G>& s, float4 dx, const float4*
         const float4 Bv = Bp[k];
         const float2 a0 = ex2x2(__fmul2_rn(dd, s.A2[2 * k]));
         const float2 a1 = ex2x2(__fmul2_rn(dd, s.A2[2 * k + 1]));
-        const float2 w0 = __fmul2_rn(f2(Bv.x, Bv.y), __fmul2_rn(xx, s.iA[2 * k]));
-        const float2 w1 = __fmul2_rn(f2(Bv.z, Bv.w), __fmul2_rn(xx, s.iA[2 * k + 1]));
-        s.h[2 * k] = __ffma2_rn(a0, s.h[2 * k], __ffma2_rn(a0, w0, f2(-w0.x, -w0.y)));
-        s.h[2 * k + 1] = __ffma2_rn(a1, s.h[2 * k + 1], __ffma2_rn(a1, w1, f2(-w1.x, -w1.y)));
+        const float2 v0 = __fmul2_rn(f2(Bv.x, Bv.y), __fmul2_rn(xx, s.niA[2 * k]));
+        const float2 v1 = __fmul2_rn(f2(Bv.z, Bv.w), __fmul2_rn(xx, s.niA[2 * k + 1]));
+        s.h[2 * k] = __ffma2_rn(a0, fsub2(s.h[2 * k], v0), v0);
+        s.h[2 * k + 1] = __ffma2_rn(a1, fsub2(s.h[2 * k + 1], v1), v1);
         if (WANT_Y) {
             const float4 Cv = Cp[k];
             y = __ffma2_rn(f2(Cv.x, Cv.y), s.h[2 * k], y);
@@ -130,7 +139,7 @@ __device__ __forceinline__ float step_acc(LaneG<G>& s, float4 dx, const float4* 
         for (int j = 0; j < 4; ++j) {
             float2& hp = s.h[2 * k + j / 2];
             const float A2 = (j & 1) ? s.A2[2 * k + j / 2].y : s.A2[2 * k + j / 2].x;
-            const float iA = (j & 1) ? s.iA[2 * k + j / 2].y : s.iA[2 * k + j / 2].x;
+            const float iA = -((j & 1) ? s.niA[2 * k + j / 2].y : s.niA[2 * k + j / 2].x);
             const float q2 = delta * A2;
             const float abar = ex2(q2);
             const float beta = bbar_coef(delta, q2 * kLn2, abar, iA);
@@ -167,8 +176,10 @@ __device__ __forceinline__ float transpose_reduce(float (&p)[NG], int g) {
     }
 }
 
-// Phase S over one tile.  FULL tiles (kTT valid steps) run fully unrolled with no
-// per-step predicate; the last, partial tile of a chunk takes the predicated form.
+// Phase S over one tile, NG steps per block (the readouts of a block are reduced
+// together); with outputs, two blocks per loop iteration so that one block's
+// reduction overlaps the next block's steps.  FULL tiles (kTT valid steps) need no per-step predicate;
+// the last, partial tile of a chunk takes the predicated form.
 template <typename T, int NG, int G, int MODE, bool ACC, bool FULL>
 __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
                                           float& dsum, float* ck, int64_t ck_stride, int nvalid) {
@@ -178,7 +189,7 @@ __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int 
     const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
     const float4* sB = reinterpret_cast<const float4*>(smem + C::OFF_B) + g * (G / 4);
     const float4* sC = reinterpret_cast<const float4*>(smem + C::OFF_C) + g * (G / 4);
-#pragma unroll 1
+#pragma unroll(MODE == kOut ? 2 : 1)
     for (int tb = 0; tb < kTT; tb += NG) {
         if (MODE == kCkpt && tb % kCkStep == 0 && (FULL || tb < tile_len)) {
             // state before step tb, the starting point of one backward recomputation
@@ -315,15 +326,15 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
             else if (a.h0) h = __ldg(a.h0 + ((int64_t)b * a.D + d) * N + n);
         }
         const float A2 = ok ? An * kLog2e : 0.f;
-        const float iA = ok && An != 0.f ? 1.f / An : 0.f;
+        const float niA = ok && An != 0.f ? -1.f / An : 0.f;
         if (j & 1) {
             s.h[j / 2].y = h;
             s.A2[j / 2].y = A2;
-            s.iA[j / 2].y = iA;
+            s.niA[j / 2].y = niA;
         } else {
             s.h[j / 2].x = h;
             s.A2[j / 2].x = A2;
-            s.iA[j / 2].x = iA;
+            s.niA[j / 2].x = niA;
         }
     }
     // the first tile's data; one CTA-wide choice of the Bbar form (block-uniform branch)

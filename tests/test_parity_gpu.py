@@ -231,8 +231,11 @@ def _check_bwd(x, io, dev, h0=None):
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("shape", [(1, 64, 4, 4), (2, 100, 37, 16), (1, 33, 5, 1), (2, 70, 9, 7),
-                                   (2, 100, 64, 16), (1, 37, 32, 8), (3, 50, 24, 4), (1, 300, 96, 16)])
+                                   (2, 100, 64, 16), (1, 37, 32, 8), (3, 50, 24, 4), (1, 300, 96, 16),
+                                   (1, 1000, 64, 16), (2, 777, 40, 8), (1, 1100, 8, 4)])
 def test_backward_small(cuda_device, io, shape):
+    """Includes shapes whose reverse sweep the library splits into sequence segments
+    (L >= 256 with few channel blocks), with a ragged last segment."""
     x = W.small_case(*shape, io=io, seed=sum(shape) + 1, backward=True)
     h0 = np.random.default_rng(5).standard_normal((shape[0], shape[2], shape[3])) * 0.3
     _check_bwd(x, io, cuda_device, h0=h0)
