@@ -109,15 +109,15 @@ def roofline_units(w: W.Workload) -> dict:
 # under profiles/).  A figure holds only for the kernel source it was taken on: it is
 # keyed by the SHA-256 of those source files and reported as null once they change.
 NCU_TRAFFIC = {
-    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 506368768 + 151190272,
-                  "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "5a5b29414ed43428",
+    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 505175808 + 151315712,
+                  "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "f3865566659428ee",
                   "profile": "profiles/fwd_tiled_kernel_mamba2.8b_bf16.md"},
     "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 406294784 + 133817088,
                 "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "2178d0fd962a137f",
-                "profile": "profiles/bwd_tiled_kernel_bwd130m_fp32.md"},
+                "profile": "profiles/bwd_tiled_kernel_bwd130m_bf16.md"},
     "decode2.8b": {"kernel": "step_kernel", "bytes": 23327232 + 2048,
                    "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "b358a00da4e6ff0b",
-                   "profile": "profiles/step_kernel_decode2.8b_bf16.md"},
+                   "profile": "profiles/step_quad_kernel_decode2.8b_bf16.md"},
 }
 
 

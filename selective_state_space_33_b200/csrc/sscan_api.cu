@@ -207,6 +207,34 @@ bool bwd_tiled_ok(const sscan_problem* p, const void* u, const void* dr, const v
            aligned16(dz) && p->seqlen < (int64_t(1) << 31) && p->dim < (int64_t(1) << 31);
 }
 
+// A second stream per device on which the backward runs its segment summaries while
+// the caller's stream runs the checkpoint pass (the two read the same inputs and
+// write disjoint workspace).  Created on first use and kept for the process; the
+// fork / join events are recorded under a mutex so that concurrent callers do not
+// interleave them.  The fork and join are event record / wait pairs, which stream
+// capture turns into graph edges.
+struct AuxStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_aux_mutex;
+AuxStream g_aux[64];
+
+cudaError_t aux_stream(AuxStream** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    AuxStream& a = g_aux[dev];
+    if (!a.stream) {
+        if ((e = cudaStreamCreateWithFlags(&a.stream, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
+    *out = &a;
+    return cudaSuccess;
+}
+
 sscan_status run_fwd(const sscan_problem* p, const sscan::ScanArgs& a, void* ws, cudaStream_t st) {
     if (tiled_ok(p, a)) return run_tiled(p, a, ws, st);
     return run_rows(p, a, ws, st);
@@ -430,9 +458,6 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
         t.nck = (p->seqlen + sscan::kBwdTiledSeg - 1) / sscan::kBwdTiledSeg;
         sscan::TiledPtrs tp{u, delta_raw, nullptr, nullptr};
         const int bf16 = p->io_dtype == SSCAN_BF16;
-        ++g_launches;
-        e = sscan::launch_fwd_tiled(t, tp, geo, bf16, sscan::kTiledCkpt, st);
-        if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "checkpoint kernel: %s", cudaGetErrorString(e));
         sscan::BwdTiledArgs ba{};
         ba.batch = p->batch;
         ba.L = p->seqlen;
@@ -457,13 +482,30 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
         ba.ws_dsum = ba.ws_lam + p->batch * plan.nsegs * p->dim * p->dstate;
         sscan::BwdTiledPtrs bp{u, delta_raw, z, dout, B, C, du, ddelta_raw, dz};
         if (plan.nsegs > 1) {
-            // the reverse sweep split in time: segment summaries, then their carry
+            // the reverse sweep split in time: segment summaries and their carry on the
+            // second stream, the checkpoint pass on the caller's, joined before the
+            // reverse kernel
+            std::lock_guard<std::mutex> lock(g_aux_mutex);
+            AuxStream* ax = nullptr;
+            if ((e = aux_stream(&ax)) != cudaSuccess || (e = cudaEventRecord(ax->fork, st)) != cudaSuccess ||
+                (e = cudaStreamWaitEvent(ax->stream, ax->fork, 0)) != cudaSuccess)
+                return fail(SSCAN_ERR_CUDA, "backward stream fork: %s", cudaGetErrorString(e));
             ++g_launches;
-            e = sscan::launch_bwd_tiled(ba, bp, bf16, sscan::kBwdSummary, st);
+            e = sscan::launch_bwd_tiled(ba, bp, bf16, sscan::kBwdSummary, ax->stream);
             if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "backward summary kernel: %s", cudaGetErrorString(e));
             ++g_launches;
-            e = sscan::launch_bwd_carry(ba, st);
+            e = sscan::launch_bwd_carry(ba, ax->stream);
             if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "backward carry kernel: %s", cudaGetErrorString(e));
+            ++g_launches;
+            e = sscan::launch_fwd_tiled(t, tp, geo, bf16, sscan::kTiledCkpt, st);
+            if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "checkpoint kernel: %s", cudaGetErrorString(e));
+            if ((e = cudaEventRecord(ax->join, ax->stream)) != cudaSuccess ||
+                (e = cudaStreamWaitEvent(st, ax->join, 0)) != cudaSuccess)
+                return fail(SSCAN_ERR_CUDA, "backward stream join: %s", cudaGetErrorString(e));
+        } else {
+            ++g_launches;
+            e = sscan::launch_fwd_tiled(t, tp, geo, bf16, sscan::kTiledCkpt, st);
+            if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "checkpoint kernel: %s", cudaGetErrorString(e));
         }
         ++g_launches;
         e = sscan::launch_bwd_tiled(ba, bp, bf16, sscan::kBwdFull, st);

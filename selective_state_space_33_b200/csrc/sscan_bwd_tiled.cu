@@ -18,8 +18,8 @@
 //   closed form would cancel) and beta = delta phi1(delta A) (series near 0);
 //   and the per-element sums over a channel's lanes, and the (t, n) sums over the
 //   channels of a warp, are formed with shuffles before anything touches memory.
-// dB and dC of a tile are summed across the CTA's warps in shared memory and then
-// added to fp32 accumulators in global memory; dA, dD and the bias gradient are
+// dB and dC of a tile are stored per warp in shared memory, summed across the CTA's
+// warps and then added to fp32 accumulators in global memory; dA, dD and the bias gradient are
 // per-channel sums added once at the end.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -71,8 +71,8 @@ struct BCfg {
     static constexpr int OFF_B = OFF_DD + kTB * DC * 8;         // float [kTB][NS]
     static constexpr int OFF_C = OFF_B + kTB * NS * 4;          // float [kTB][NS]
     static constexpr int OFF_HS = OFF_C + kTB * NS * 4;         // float4 [kTB][kThreadsB] recomputed states
-    static constexpr int OFF_ACC = OFF_HS + kTB * kThreadsB * 16;  // float [kTB][NS][2] dB, dC of the tile
-    static constexpr int OFF_OUT = OFF_ACC + kTB * NS * 2 * 4;  // [2 buffers][3 tensors][RAW]
+    static constexpr int OFF_ACC = OFF_HS + kTB * kThreadsB * 16;  // float [warp][kTB][NS][2] dB, dC of the tile
+    static constexpr int OFF_OUT = OFF_ACC + kWarpsB * kTB * NS * 2 * 4;  // [2 buffers][3 tensors][RAW]
     static constexpr int OFF_BAR = OFF_OUT + 2 * 3 * RAW;
     static constexpr int SMEM = OFF_BAR + STAGES * 8;
 };
@@ -200,8 +200,9 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         for (int k = 0; k < C::STAGES && k < ntb; ++k) issue(k);
     }
+    // per-warp tile sums of dB and dC: every slot a tile reads was written in that tile
     float* sacc = reinterpret_cast<float*>(smem + C::OFF_ACC);
-    for (int e = tid; e < kTB * C::NS * 2; e += kThreadsB) sacc[e] = 0.f;
+    constexpr int kAccWarp = kTB * C::NS * 2;
 
     // lane state: channel cw, states g*4 .. g*4+3
     const int g = lane / C::CW, c = lane % C::CW, cw = warp * C::CW + c;
@@ -441,7 +442,7 @@ __global__ void __launch_bounds__(kThreadsB, 5)
                 const float v = treduce_c8<C::CW>(vbc, c);
                 if (c < 8 && t < tile_len) {
                     const int which = c >> 2, j = c & 3;
-                    atomicAdd(sacc + (t * C::NS + g * 4 + j) * 2 + which, v);
+                    sacc[warp * kAccWarp + (t * C::NS + g * 4 + j) * 2 + which] = v;
                 }
             }
             const float sdu = treduce_g<NG, C::CW>(pdu, g);
@@ -472,16 +473,21 @@ __global__ void __launch_bounds__(kThreadsB, 5)
             tma_commit();
             tma_store_wait_read_1();
         }
-        // the tile's dB, dC into the fp32 accumulators, then clear the smem sums
+        // the tile's dB, dC: the warps' sums into the fp32 accumulators
         for (int e = tid; e < tile_len * C::NS; e += kThreadsB) {
             const int t = e / C::NS, n = e % C::NS;
             if (n < N) {
+                float2 v = reinterpret_cast<const float2*>(sacc)[e];
+#pragma unroll
+                for (int w = 1; w < kWarpsB; ++w) {
+                    const float2 u = reinterpret_cast<const float2*>(sacc + w * kAccWarp)[e];
+                    v.x += u.x;
+                    v.y += u.y;
+                }
                 const int64_t gi = ((int64_t)b * a.L + t0 + t) * N + n;
-                atomicAdd(a.dB32 + gi, sacc[e * 2]);
-                atomicAdd(a.dC32 + gi, sacc[e * 2 + 1]);
+                atomicAdd(a.dB32 + gi, v.x);
+                atomicAdd(a.dC32 + gi, v.y);
             }
-            sacc[e * 2] = 0.f;
-            sacc[e * 2 + 1] = 0.f;
         }
     }
     if (tid == 0) tma_store_wait_all();

@@ -78,16 +78,18 @@ __device__ __forceinline__ float4 load4(const T* p) {
     }
 }
 
+// Grid: (lane blocks over one batch's D x LPR lanes, batch); no integer division
+// by a runtime size anywhere.
 template <typename T, int LPR>
 __global__ void __launch_bounds__(256) step_quad_kernel(StepArgs a) {
     constexpr int N = 4 * LPR;
-    const int64_t rows = a.batch * a.D;
-    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    // lanes past the last row still take part in the row shuffles, on the last row
-    const bool valid = gt / LPR < rows;
-    const int64_t row = valid ? gt / LPR : rows - 1;
-    const int q = (int)(gt % LPR);
-    const int64_t b = row / a.D, d = row - b * a.D;
+    const int64_t b = blockIdx.y;
+    const int64_t gl = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // lanes past the last channel still take part in the row shuffles, on the last channel
+    const bool valid = gl / LPR < a.D;
+    const int64_t d = valid ? gl / LPR : a.D - 1;
+    const int q = (int)(gl % LPR);
+    const int64_t row = b * a.D + d;
     float4* hp = reinterpret_cast<float4*>(a.state + row * N) + q;
 
     const float4 h = *hp;
@@ -129,12 +131,11 @@ cudaError_t launch_t(const StepArgs& a, cudaStream_t st) {
                       reinterpret_cast<uintptr_t>(a.A) % 16 == 0 &&
                       reinterpret_cast<uintptr_t>(a.B) % (4 * sizeof(T)) == 0 &&
                       reinterpret_cast<uintptr_t>(a.C) % (4 * sizeof(T)) == 0;
-    if (quad) {
-        const int64_t lanes = rows * (a.N / 4);
-        const unsigned qb = (unsigned)((lanes + 255) / 256);
-        if (a.N == 16) step_quad_kernel<T, 4><<<qb, 256, 0, st>>>(a);
-        else if (a.N == 8) step_quad_kernel<T, 2><<<qb, 256, 0, st>>>(a);
-        else step_quad_kernel<T, 1><<<qb, 256, 0, st>>>(a);
+    if (quad && a.batch <= 65535) {
+        const dim3 grid((unsigned)((a.D * (a.N / 4) + 255) / 256), (unsigned)a.batch);
+        if (a.N == 16) step_quad_kernel<T, 4><<<grid, 256, 0, st>>>(a);
+        else if (a.N == 8) step_quad_kernel<T, 2><<<grid, 256, 0, st>>>(a);
+        else step_quad_kernel<T, 1><<<grid, 256, 0, st>>>(a);
         return cudaGetLastError();
     }
     if (a.N <= 4) step_kernel<T, 4><<<blocks, 128, 0, st>>>(a);
