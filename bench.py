@@ -115,8 +115,8 @@ NCU_TRAFFIC = {
     "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 406294784 + 133817088,
                 "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "2178d0fd962a137f",
                 "profile": "profiles/bwd_tiled_kernel_bwd130m_bf16.md"},
-    "decode2.8b": {"kernel": "step_kernel", "bytes": 23327232 + 2048,
-                   "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "b358a00da4e6ff0b",
+    "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23315968 + 0,
+                   "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "5144163678ece024",
                    "profile": "profiles/step_quad_kernel_decode2.8b_bf16.md"},
 }
 

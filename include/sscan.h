@@ -59,7 +59,8 @@ typedef enum sscan_status {
     SSCAN_ERR_INVALID_ARG = 1, /* NULL required pointer, negative size, unknown dtype or flag */
     SSCAN_ERR_UNSUPPORTED = 2, /* a well-formed problem this build does not handle (dstate > 16) */
     SSCAN_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than sscan_workspace_size() */
-    SSCAN_ERR_CUDA = 4         /* a CUDA runtime call or kernel launch failed */
+    SSCAN_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+    SSCAN_ERR_TIMEOUT = 5      /* sscan_device_status: a kernel's bounded wait gave up */
 } sscan_status;
 
 typedef enum sscan_dtype { SSCAN_F32 = 0, SSCAN_BF16 = 1 } sscan_dtype;
@@ -210,8 +211,11 @@ SSCAN_API int sscan_last_launch_count(void);
  * receives the OR of every error bit raised since the last clear (bit 0: in a
  * forward kernel, bit 1: in the backward kernel, a bounded wait for an
  * asynchronous tile copy gave up, so that kernel stopped early and its outputs
- * are incomplete).  clear != 0 resets the word after
- * reading.  Synchronous: it waits for work already submitted to the device.
+ * are incomplete; bit 2: sscan_probe_wait_timeout's wait ran out, as it is meant
+ * to).  Returns SSCAN_ERR_TIMEOUT when any bit is set, SSCAN_OK when none is.
+ * clear != 0 resets the word after reading.  Synchronous: it waits for work
+ * already submitted to the device.  Every wait in the library's kernels is
+ * bounded, so a failed copy surfaces here instead of hanging the device.
  */
 SSCAN_API sscan_status sscan_device_status(int clear, unsigned int* flags);
 

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libsscan.so")
 SSCAN_F32, SSCAN_BF16 = 0, 1
 SSCAN_DELTA_SOFTPLUS = 1
 SSCAN_OP_FWD, SSCAN_OP_LAST_STATE, SSCAN_OP_BWD, SSCAN_OP_SUMMARY = 0, 1, 2, 3
+SSCAN_ERR_TIMEOUT = 5
 
 _IO_CODES = {torch.float32: SSCAN_F32, torch.bfloat16: SSCAN_BF16}
 _lib = None
@@ -69,6 +70,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sscan_last_error.restype = ctypes.c_char_p
     lib.sscan_version.argtypes = []
     lib.sscan_version.restype = ctypes.c_int
+    lib.sscan_device_status.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_uint)]
+    lib.sscan_device_status.restype = ctypes.c_int
+    lib.sscan_probe_wait_timeout.argtypes = [ctypes.c_uint, vp]
+    lib.sscan_probe_wait_timeout.restype = ctypes.c_int
     if path is None:
         _lib = lib
     return lib
@@ -284,3 +289,21 @@ def sscan_carry(P, H, h0=None, *, stream=None):
     _check(load_library().sscan_carry(ctypes.byref(prob), int(K), _ptr(P), _ptr(H), _ptr(h0), _ptr(carry),
                                       _ptr(h_final), _stream(stream)))
     return carry, h_final
+
+
+def device_status(clear: bool = False) -> int:
+    """Error bits the library's kernels raised on the current device since the last
+    clear (0: none; bit 0 forward, bit 1 backward: a bounded wait for a tile copy gave
+    up; bit 2: the wait-timeout probe).  Synchronous."""
+    lib = load_library()
+    flags = ctypes.c_uint(0)
+    st = lib.sscan_device_status(int(clear), ctypes.byref(flags))
+    if st not in (0, SSCAN_ERR_TIMEOUT):
+        _check(st)
+    return flags.value
+
+
+def probe_wait_timeout(polls: int = 4096, *, stream=None):
+    """Enqueue the bounded-wait self-test: one thread waits on a barrier nothing
+    arrives on, gives up after ``polls`` polls and raises bit 2 of the device status."""
+    _check(load_library().sscan_probe_wait_timeout(polls, _stream(stream)))

@@ -132,7 +132,7 @@ sscan_status run_rows(const sscan_problem* p, sscan::ScanArgs a, void* ws, cudaS
         if (sscan_status s = cuda_check("chunk aggregate kernel")) return s;
         sscan::ScanArgs c = a;
         if (want_out) c.h_last = nullptr;  // the output pass writes h_last itself
-        sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate, 128), 128, 0, st>>>(c);
+        sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate * 32, 128), 128, 0, st>>>(c);
         ++g_launches;
         if (sscan_status s = cuda_check("carry kernel")) return s;
         if (!want_out) return SSCAN_OK;
@@ -186,7 +186,7 @@ sscan_status run_tiled(const sscan_problem* p, const sscan::ScanArgs& a, void* w
         c.ws_state = t.ws_state;
         c.ws_dsum = t.ws_dsum;
         if (want_out) c.h_last = nullptr;
-        sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate, 128), 128, 0, st>>>(c);
+        sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate * 32, 128), 128, 0, st>>>(c);
         ++g_launches;
         if (sscan_status s = cuda_check("carry kernel")) return s;
         if (!want_out) return SSCAN_OK;
@@ -642,7 +642,7 @@ sscan_status sscan_carry(const sscan_problem* p, int64_t nchunks, const float* P
     if (BDN == 0 || (!carry_in && !h_final)) return SSCAN_OK;
     if (nchunks > 0 && (!P || !H)) return fail(SSCAN_ERR_INVALID_ARG, "P and H are required");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    sscan::compose_kernel<<<blocks_for(BDN, 128), 128, 0, st>>>(P, H, h0, carry_in, h_final, nchunks, BDN);
+    sscan::compose_kernel<<<blocks_for(BDN * 32, 128), 128, 0, st>>>(P, H, h0, carry_in, h_final, nchunks, BDN);
     ++g_launches;
     return cuda_check("compose kernel");
 }
@@ -654,6 +654,7 @@ const char* sscan_status_string(sscan_status s) {
         case SSCAN_ERR_UNSUPPORTED: return "SSCAN_ERR_UNSUPPORTED";
         case SSCAN_ERR_WORKSPACE: return "SSCAN_ERR_WORKSPACE";
         case SSCAN_ERR_CUDA: return "SSCAN_ERR_CUDA";
+        case SSCAN_ERR_TIMEOUT: return "SSCAN_ERR_TIMEOUT";
         default: return "SSCAN_ERR_UNKNOWN";
     }
 }
@@ -670,7 +671,7 @@ sscan_status sscan_device_status(int clear, unsigned int* flags) {
     if (e == cudaSuccess) e = sscan::read_device_error_bwd(&f2, clear);
     if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
     *flags = f1 | f2;
-    return SSCAN_OK;
+    return *flags ? SSCAN_ERR_TIMEOUT : SSCAN_OK;
 }
 
 int sscan_version(void) { return 100; }

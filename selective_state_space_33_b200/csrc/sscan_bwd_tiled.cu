@@ -28,6 +28,7 @@
 #include <cstdint>
 
 #include "sscan_launch.h"
+#include "sscan_affine.cuh"
 #include "sscan_math.cuh"
 #include "sscan_tma.cuh"
 
@@ -580,24 +581,28 @@ cudaError_t launch_bwd_t(const BwdTiledArgs& a, const BwdTiledPtrs& p, int mode,
     return cudaGetLastError();
 }
 
-// One thread per (batch, channel, state): walk the segments right to left, leaving
-// in ws_lam the adjoint state that enters each segment from its right.  A segment
-// maps an entering adjoint state lam to P lam + H, with P = exp(A * its sum of delta)
-// (the product of its Abar) and H its summary.
+// One warp per (batch, channel, state): compose the segments right to left with
+// the warp's affine-pair scan, leaving in ws_lam the adjoint state that enters each
+// segment from its right.  A segment maps an entering adjoint state lam to
+// P lam + H, with P = exp(A * its sum of delta) (the product of its Abar) and H its
+// summary; segment nseg-1 is entered with zero, and segment 0's own map is never
+// needed.
 __global__ void __launch_bounds__(128) bwd_carry_kernel(BwdTiledArgs a) {
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= a.batch * a.D * a.N) return;
-    const int64_t n = gid % a.N, bd = gid / a.N;
+    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (w >= a.batch * a.D * a.N) return;  // warp-uniform
+    const int64_t n = w % a.N, bd = w / a.N;
     const int64_t d = bd % a.D, b = bd / a.D;
     const float A2 = __ldg(a.A + d * a.N + n) * kLog2e;
-    float lam = 0.f;
-    for (int64_t s = a.nseg - 1; s >= 1; --s) {
-        const int64_t i = ((b * a.nseg + s) * a.D + d) * a.N + n;
-        const float H = a.ws_lam[i];
-        a.ws_lam[i] = lam;
-        lam = fmaf(ex2(A2 * a.ws_dsum[(b * a.nseg + s) * a.D + d]), lam, H);
-    }
-    a.ws_lam[((b * a.nseg) * a.D + d) * a.N + n] = lam;
+    // map j (j = 0 .. nseg-2) is segment s = nseg-1-j
+    const float lam0 = affine_carry_warp(
+        a.nseg - 1, 0.f,
+        [&](int64_t j, float& p, float& q) {
+            const int64_t s = a.nseg - 1 - j;
+            p = ex2(A2 * a.ws_dsum[(b * a.nseg + s) * a.D + d]);
+            q = a.ws_lam[((b * a.nseg + s) * a.D + d) * a.N + n];
+        },
+        [&](int64_t j, float v) { a.ws_lam[((b * a.nseg + (a.nseg - 1 - j)) * a.D + d) * a.N + n] = v; });
+    if ((threadIdx.x & 31) == 0) a.ws_lam[((b * a.nseg) * a.D + d) * a.N + n] = lam0;
 }
 
 }  // namespace
@@ -623,7 +628,7 @@ cudaError_t launch_bwd_tiled(const BwdTiledArgs& a, const BwdTiledPtrs& p, int i
 }
 
 cudaError_t launch_bwd_carry(const BwdTiledArgs& a, cudaStream_t st) {
-    const int64_t n = a.batch * a.D * a.N;
+    const int64_t n = a.batch * a.D * a.N * 32;  // one warp per (batch, channel, state)
     if (n > 0) bwd_carry_kernel<<<(unsigned)((n + 127) / 128), 128, 0, st>>>(a);
     return cudaGetLastError();
 }

@@ -7,6 +7,7 @@
 // Fig. 3 (Mamba technical summary page, kb.agiseed.tech).
 #pragma once
 
+#include "sscan_affine.cuh"
 #include "sscan_math.cuh"
 
 namespace sscan {
@@ -116,23 +117,23 @@ __global__ void __launch_bounds__(128) fwd_rows_kernel(ScanArgs a) {
 // P_c = exp(A_n * sum of delta over the chunk) (the product of its Abar) and H_c the
 // chunk's end state from zero.  Composing the maps in order gives every chunk's
 // carry-in; the composition of all of them applied to h0 is h_last.
-// One thread per (batch, channel, state); the carry-ins overwrite H in place.
+// One warp per (batch, channel, state); the carry-ins overwrite H in place.
 __global__ void __launch_bounds__(128) carry_kernel(ScanArgs a) {
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t total = a.batch * a.D * a.N;
-    if (gid >= total) return;
-    const int64_t n = gid % a.N, bd = gid / a.N;
+    if (w >= total) return;  // warp-uniform
+    const int64_t n = w % a.N, bd = w / a.N;
     const int64_t d = bd % a.D, b = bd / a.D;
     const float A2 = __ldg(a.A + d * a.N + n) * kLog2e;
-    float h = a.h0 ? __ldg(a.h0 + gid) : 0.f;
-    for (int64_t c = 0; c < a.nchunks; ++c) {
-        const int64_t i = ((b * a.nchunks + c) * a.D + d) * a.N + n;
-        const float H = a.ws_state[i];
-        const float S = a.ws_dsum[(b * a.nchunks + c) * a.D + d];
-        a.ws_state[i] = h;
-        h = fmaf(ex2(A2 * S), h, H);
-    }
-    if (a.h_last) a.h_last[gid] = h;
+    const float h0 = a.h0 ? __ldg(a.h0 + w) : 0.f;
+    const float h = affine_carry_warp(
+        a.nchunks, h0,
+        [&](int64_t c, float& p, float& q) {
+            p = ex2(A2 * a.ws_dsum[(b * a.nchunks + c) * a.D + d]);
+            q = a.ws_state[((b * a.nchunks + c) * a.D + d) * a.N + n];
+        },
+        [&](int64_t c, float v) { a.ws_state[((b * a.nchunks + c) * a.D + d) * a.N + n] = v; });
+    if (a.h_last && (threadIdx.x & 31) == 0) a.h_last[w] = h;
 }
 
 // P = exp(A_n * sum of delta): the decay of a chunk summary, from the per-row sums
@@ -147,17 +148,21 @@ __global__ void __launch_bounds__(128) decay_kernel(const float* dsum, const flo
 
 // Compose K chunk maps h -> P_k h + H_k (each (batch, D, N), chunk-major) in order,
 // starting from h0: carry_in[k] is the state entering chunk k, h_final the state
-// after the last.  One thread per (b, d, n).
+// after the last.  One warp per (b, d, n).
 __global__ void __launch_bounds__(128) compose_kernel(const float* P, const float* H, const float* h0,
                                                       float* carry_in, float* h_final, int64_t K, int64_t BDN) {
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= BDN) return;
-    float h = h0 ? __ldg(h0 + gid) : 0.f;
-    for (int64_t k = 0; k < K; ++k) {
-        if (carry_in) carry_in[k * BDN + gid] = h;
-        h = fmaf(__ldg(P + k * BDN + gid), h, __ldg(H + k * BDN + gid));
-    }
-    if (h_final) h_final[gid] = h;
+    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (w >= BDN) return;  // warp-uniform
+    const float h = affine_carry_warp(
+        K, h0 ? __ldg(h0 + w) : 0.f,
+        [&](int64_t k, float& p, float& q) {
+            p = __ldg(P + k * BDN + w);
+            q = __ldg(H + k * BDN + w);
+        },
+        [&](int64_t k, float v) {
+            if (carry_in) carry_in[k * BDN + w] = v;
+        });
+    if (h_final && (threadIdx.x & 31) == 0) h_final[w] = h;
 }
 
 }  // namespace sscan

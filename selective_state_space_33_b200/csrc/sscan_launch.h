@@ -118,4 +118,8 @@ cudaError_t read_device_error_bwd(unsigned int* value, int clear);
 // bounded wait in a kernel gave up.  Synchronous.
 cudaError_t read_device_error(unsigned int* value, int clear);
 
+// One thread waits, with the kernels' bounded wait cut to `polls` polls, on an
+// mbarrier that nothing arrives on, then raises bit 2 of the device error word.
+cudaError_t launch_wait_probe(unsigned int polls, cudaStream_t st);
+
 }  // namespace sscan

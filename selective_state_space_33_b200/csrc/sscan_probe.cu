@@ -1,6 +1,7 @@
 // sscan_probe.cu -- MUFU ex2 throughput probe (include/sscan_probe.h).
 #include <cuda_runtime.h>
 
+#include "sscan_launch.h"
 #include "sscan_math.cuh"
 #include "sscan_probe.h"
 
@@ -28,4 +29,10 @@ extern "C" sscan_status sscan_probe_ex2(float* sink, int64_t iters, int blocks, 
     if (!sink || iters <= 0 || blocks <= 0 || threads <= 0 || threads > 1024) return SSCAN_ERR_INVALID_ARG;
     ex2_probe_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(sink, iters);
     return cudaGetLastError() == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
+}
+
+extern "C" sscan_status sscan_probe_wait_timeout(unsigned int polls, void* stream) {
+    if (polls == 0 || polls > (1u << 20)) return SSCAN_ERR_INVALID_ARG;
+    return sscan::launch_wait_probe(polls, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SSCAN_OK
+                                                                                            : SSCAN_ERR_CUDA;
 }

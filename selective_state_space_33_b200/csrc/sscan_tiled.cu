@@ -70,6 +70,7 @@ struct Cfg {
     static constexpr int GD_PITCH = DC;                    // float2 row pitch of the epilogue operands
     static constexpr int BC_ENTRIES = kTT * NS;
     static constexpr int PAIRS = kTT * DC / 2;             // channel pairs of phase P
+    static_assert(PAIRS % kThreads == 0, "phase P runs a fixed number of pairs per thread");
     // shared-memory layout (byte offsets, all 128-aligned)
     static constexpr int OFF_RAW = 0;                                     // [STAGES][STAGE]
     static constexpr int OFF_DX = OFF_RAW + STAGES * STAGE;               // float4 (d, d, x, x) [kTT][DC]
@@ -89,17 +90,9 @@ struct LaneG {
 
 __device__ __forceinline__ float2 ex2x2(float2 q) { return f2(ex2(q.x), ex2(q.y)); }
 
-// a - b on both halves (one packed f32x2 instruction).
-__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
-    unsigned long long ra = *reinterpret_cast<unsigned long long*>(&a), rb = *reinterpret_cast<unsigned long long*>(&b),
-                       rd;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
-    return *reinterpret_cast<float2*>(&rd);
-}
-
 // One step for the lane's G states, eq. (2) and (3a).  With v = -B x / A the update
-// h' = Abar h + (Abar - 1) B x / A is Abar (h - v) + v: one packed subtract and one
-// packed fma per pair, no negation.  dx = (delta, delta, x, x); Bp, Cp point at the
+// h' = Abar h + (Abar - 1) B x / A is Abar (h - v) + v: two packed fmas per pair
+// (h - v as fma(v, -1, h), exact), no negated operand.  dx = (delta, delta, x, x); Bp, Cp point at the
 // lane's G values of B_t, C_t.  Returns the partial readout sum_j C_j h_j over these
 // states (eq. (3b)).
 template <int G, bool WANT_Y>
@@ -113,8 +106,8 @@ __device__ __forceinline__ float step_fast(LaneG<G>& s, float4 dx, const float4*
         const float2 a1 = ex2x2(__fmul2_rn(dd, s.A2[2 * k + 1]));
         const float2 v0 = __fmul2_rn(f2(Bv.x, Bv.y), __fmul2_rn(xx, s.niA[2 * k]));
         const float2 v1 = __fmul2_rn(f2(Bv.z, Bv.w), __fmul2_rn(xx, s.niA[2 * k + 1]));
-        s.h[2 * k] = __ffma2_rn(a0, fsub2(s.h[2 * k], v0), v0);
-        s.h[2 * k + 1] = __ffma2_rn(a1, fsub2(s.h[2 * k + 1], v1), v1);
+        s.h[2 * k] = __ffma2_rn(a0, __ffma2_rn(v0, f2(-1.f, -1.f), s.h[2 * k]), v0);
+        s.h[2 * k + 1] = __ffma2_rn(a1, __ffma2_rn(v1, f2(-1.f, -1.f), s.h[2 * k + 1]), v1);
         if (WANT_Y) {
             const float4 Cv = Cp[k];
             y = __ffma2_rn(f2(Cv.x, Cv.y), s.h[2 * k], y);
@@ -349,6 +342,10 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
     const T* Bg = static_cast<const T*>(a.B);
     const T* Cg = static_cast<const T*>(a.C);
     float dsum = 0.f;
+    const float2 pbias = f2((a.bias && pd < a.D) ? __ldg(a.bias + pd) : 0.f,
+                            (a.bias && pd + 1 < a.D) ? __ldg(a.bias + pd + 1) : 0.f);
+    const float2 pdsk = f2((want_out && a.Dskip && pd < a.D) ? __ldg(a.Dskip + pd) : 0.f,
+                           (want_out && a.Dskip && pd + 1 < a.D) ? __ldg(a.Dskip + pd + 1) : 0.f);
 
     for (int it = 0; it < ntile && !failed; ++it) {
         const int st = it % C::STAGES;
@@ -362,12 +359,10 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
             const P2* rz = reinterpret_cast<const P2*>(raw + 2 * C::RAW);
             float4* sdx = reinterpret_cast<float4*>(smem + C::OFF_DX);
             float4* sgd = reinterpret_cast<float4*>(smem + C::OFF_GD);
-            const float2 pbias = f2((a.bias && pd < a.D) ? __ldg(a.bias + pd) : 0.f,
-                                    (a.bias && pd + 1 < a.D) ? __ldg(a.bias + pd + 1) : 0.f);
-            const float2 pdsk = f2((want_out && a.Dskip && pd < a.D) ? __ldg(a.Dskip + pd) : 0.f,
-                                   (want_out && a.Dskip && pd + 1 < a.D) ? __ldg(a.Dskip + pd + 1) : 0.f);
+            // a fixed trip count (PAIRS is a multiple of kThreads for every geometry)
 #pragma unroll
-            for (int q = tid; q < C::PAIRS; q += kThreads) {
+            for (int qi = 0; qi < C::PAIRS / kThreads; ++qi) {
+                const int q = tid + qi * kThreads;
                 const int t = q / (C::DC / 2);
                 const float2 x = Pair<T>::f(ru[q]);
                 float2 dl = __fadd2_rn(Pair<T>::f(rd[q]), pbias);
@@ -385,7 +380,9 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
             const T* rB = reinterpret_cast<const T*>(raw + 3 * C::RAW);
             const T* rC = reinterpret_cast<const T*>(raw + 3 * C::RAW + C::RAWBC);
 #pragma unroll
-            for (int e = tid; e < C::BC_ENTRIES; e += kThreads) {
+            for (int ei = 0; ei < (C::BC_ENTRIES + kThreads - 1) / kThreads; ++ei) {
+                const int e = tid + ei * kThreads;
+                if (C::BC_ENTRIES % kThreads != 0 && e >= C::BC_ENTRIES) break;
                 const int t = e / C::NS, n = e % C::NS;
                 float bv = 0.f, cv = 0.f;
                 if (n < N) {
@@ -552,6 +549,25 @@ cudaError_t launch_fwd_tiled(const TiledArgs& a, const TiledPtrs& p, const Tiled
                              cudaStream_t st) {
     if (!encode_fn()) return cudaErrorNotSupported;
     return io_bf16 ? launch_t<__nv_bfloat16>(a, p, geo, mode, st) : launch_t<float>(a, p, geo, mode, st);
+}
+
+namespace {
+// The failure path of a bounded wait, exercised on purpose: an mbarrier with one
+// expected arrival that never comes.  Nothing is in flight on it, so giving up
+// leaves nothing behind.
+__global__ void wait_probe_kernel(unsigned int polls) {
+    __shared__ __align__(8) unsigned long long bar;
+    if (threadIdx.x != 0) return;
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (!mbar_wait(b, 0, polls)) atomicOr(&g_device_error, 4u);
+}
+}  // namespace
+
+cudaError_t launch_wait_probe(unsigned int polls, cudaStream_t st) {
+    wait_probe_kernel<<<1, 32, 0, st>>>(polls);
+    return cudaGetLastError();
 }
 
 cudaError_t read_device_error(unsigned int* value, int clear) {
