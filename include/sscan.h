@@ -149,6 +149,13 @@ SSCAN_API sscan_status sscan_fwd_noalloc(const sscan_problem* problem, const voi
  * dh0 are fp32.  ddelta_bias, dD, dz and dh0 may be NULL when not wanted; dz must
  * be given exactly when z is, dD only when D_skip is.  The argument list of the
  * forward pass must be repeated exactly as it was given to sscan_fwd.
+ * Streams: when the reverse sweep is split into sequence segments (few batch x
+ * channel blocks, long L), the segment summaries run on a second stream while the
+ * checkpoint pass runs on `stream`; the call forks to it and joins back with an
+ * event record / wait pair, so all work is still ordered after earlier work on
+ * `stream` and before later work on it (and stream capture records the fork as
+ * graph edges).  That stream and its two events are created once per device on
+ * first use and kept for the process (no device memory is allocated).
  */
 SSCAN_API sscan_status sscan_bwd(const sscan_problem* problem, const void* u, const void* delta_raw,
                        const float* delta_bias, const float* A, const void* B, const void* C,
@@ -187,7 +194,7 @@ SSCAN_API sscan_status sscan_chunk_summary(const sscan_problem* problem, const v
 /*
  * Compose the summaries of nchunks consecutive stretches, in order, starting from
  * h0 (NULL = zero): carry_in[k] = the state entering stretch k, h_final = the state
- * after the last.  P, H, carry_in: (nchunks, batch, D, N) fp32, chunk-major;
+ * after the last (a warp-shuffle scan of the affine pairs, 32 stretches at a time).  P, H, carry_in: (nchunks, batch, D, N) fp32, chunk-major;
  * h0, h_final: (batch, D, N).  Running sscan_fwd on stretch k with
  * h0 = carry_in[k] reproduces the unsplit scan.  carry_in or h_final may be NULL.
  * Only problem->batch, dim, dstate are read.

@@ -132,7 +132,8 @@ sscan_status run_rows(const sscan_problem* p, sscan::ScanArgs a, void* ws, cudaS
         if (sscan_status s = cuda_check("chunk aggregate kernel")) return s;
         sscan::ScanArgs c = a;
         if (want_out) c.h_last = nullptr;  // the output pass writes h_last itself
-        sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate * 32, 128), 128, 0, st>>>(c);
+        const int W = sscan::affine_lanes(c.nchunks);
+        sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate * W, 128), 128, 0, st>>>(c, W);
         ++g_launches;
         if (sscan_status s = cuda_check("carry kernel")) return s;
         if (!want_out) return SSCAN_OK;
@@ -186,7 +187,8 @@ sscan_status run_tiled(const sscan_problem* p, const sscan::ScanArgs& a, void* w
         c.ws_state = t.ws_state;
         c.ws_dsum = t.ws_dsum;
         if (want_out) c.h_last = nullptr;
-        sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate * 32, 128), 128, 0, st>>>(c);
+        const int W = sscan::affine_lanes(c.nchunks);
+        sscan::carry_kernel<<<blocks_for(p->batch * p->dim * p->dstate * W, 128), 128, 0, st>>>(c, W);
         ++g_launches;
         if (sscan_status s = cuda_check("carry kernel")) return s;
         if (!want_out) return SSCAN_OK;
@@ -642,7 +644,8 @@ sscan_status sscan_carry(const sscan_problem* p, int64_t nchunks, const float* P
     if (BDN == 0 || (!carry_in && !h_final)) return SSCAN_OK;
     if (nchunks > 0 && (!P || !H)) return fail(SSCAN_ERR_INVALID_ARG, "P and H are required");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    sscan::compose_kernel<<<blocks_for(BDN * 32, 128), 128, 0, st>>>(P, H, h0, carry_in, h_final, nchunks, BDN);
+    const int W = sscan::affine_lanes(nchunks);
+    sscan::compose_kernel<<<blocks_for(BDN * W, 128), 128, 0, st>>>(P, H, h0, carry_in, h_final, nchunks, BDN, W);
     ++g_launches;
     return cuda_check("compose kernel");
 }

@@ -581,28 +581,30 @@ cudaError_t launch_bwd_t(const BwdTiledArgs& a, const BwdTiledPtrs& p, int mode,
     return cudaGetLastError();
 }
 
-// One warp per (batch, channel, state): compose the segments right to left with
-// the warp's affine-pair scan, leaving in ws_lam the adjoint state that enters each
+// W lanes per (batch, channel, state): compose the segments right to left with
+// the warp-shuffle affine-pair scan, leaving in ws_lam the adjoint state that enters each
 // segment from its right.  A segment maps an entering adjoint state lam to
 // P lam + H, with P = exp(A * its sum of delta) (the product of its Abar) and H its
 // summary; segment nseg-1 is entered with zero, and segment 0's own map is never
 // needed.
-__global__ void __launch_bounds__(128) bwd_carry_kernel(BwdTiledArgs a) {
-    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (w >= a.batch * a.D * a.N) return;  // warp-uniform
+__global__ void __launch_bounds__(128) bwd_carry_kernel(BwdTiledArgs a, int W) {
+    const int64_t total = a.batch * a.D * a.N;
+    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / W;
+    const bool valid = r < total;
+    const int64_t w = valid ? r : total - 1;
     const int64_t n = w % a.N, bd = w / a.N;
     const int64_t d = bd % a.D, b = bd / a.D;
     const float A2 = __ldg(a.A + d * a.N + n) * kLog2e;
     // map j (j = 0 .. nseg-2) is segment s = nseg-1-j
     const float lam0 = affine_carry_warp(
-        a.nseg - 1, 0.f,
+        a.nseg - 1, 0.f, W, valid,
         [&](int64_t j, float& p, float& q) {
             const int64_t s = a.nseg - 1 - j;
             p = ex2(A2 * a.ws_dsum[(b * a.nseg + s) * a.D + d]);
             q = a.ws_lam[((b * a.nseg + s) * a.D + d) * a.N + n];
         },
         [&](int64_t j, float v) { a.ws_lam[((b * a.nseg + (a.nseg - 1 - j)) * a.D + d) * a.N + n] = v; });
-    if ((threadIdx.x & 31) == 0) a.ws_lam[((b * a.nseg) * a.D + d) * a.N + n] = lam0;
+    if (valid && (threadIdx.x & (W - 1)) == 0) a.ws_lam[((b * a.nseg) * a.D + d) * a.N + n] = lam0;
 }
 
 }  // namespace
@@ -628,8 +630,9 @@ cudaError_t launch_bwd_tiled(const BwdTiledArgs& a, const BwdTiledPtrs& p, int i
 }
 
 cudaError_t launch_bwd_carry(const BwdTiledArgs& a, cudaStream_t st) {
-    const int64_t n = a.batch * a.D * a.N * 32;  // one warp per (batch, channel, state)
-    if (n > 0) bwd_carry_kernel<<<(unsigned)((n + 127) / 128), 128, 0, st>>>(a);
+    const int W = affine_lanes(a.nseg - 1);
+    const int64_t n = a.batch * a.D * a.N * W;  // W lanes per (batch, channel, state)
+    if (n > 0) bwd_carry_kernel<<<(unsigned)((n + 127) / 128), 128, 0, st>>>(a, W);
     return cudaGetLastError();
 }
 

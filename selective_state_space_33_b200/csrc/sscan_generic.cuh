@@ -117,23 +117,25 @@ __global__ void __launch_bounds__(128) fwd_rows_kernel(ScanArgs a) {
 // P_c = exp(A_n * sum of delta over the chunk) (the product of its Abar) and H_c the
 // chunk's end state from zero.  Composing the maps in order gives every chunk's
 // carry-in; the composition of all of them applied to h0 is h_last.
-// One warp per (batch, channel, state); the carry-ins overwrite H in place.
-__global__ void __launch_bounds__(128) carry_kernel(ScanArgs a) {
-    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+// W lanes (affine_lanes(nchunks)) per (batch, channel, state); the carry-ins
+// overwrite H in place.
+__global__ void __launch_bounds__(128) carry_kernel(ScanArgs a, int W) {
     const int64_t total = a.batch * a.D * a.N;
-    if (w >= total) return;  // warp-uniform
+    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / W;
+    const bool valid = r < total;
+    const int64_t w = valid ? r : total - 1;
     const int64_t n = w % a.N, bd = w / a.N;
     const int64_t d = bd % a.D, b = bd / a.D;
     const float A2 = __ldg(a.A + d * a.N + n) * kLog2e;
     const float h0 = a.h0 ? __ldg(a.h0 + w) : 0.f;
     const float h = affine_carry_warp(
-        a.nchunks, h0,
+        a.nchunks, h0, W, valid,
         [&](int64_t c, float& p, float& q) {
             p = ex2(A2 * a.ws_dsum[(b * a.nchunks + c) * a.D + d]);
             q = a.ws_state[((b * a.nchunks + c) * a.D + d) * a.N + n];
         },
         [&](int64_t c, float v) { a.ws_state[((b * a.nchunks + c) * a.D + d) * a.N + n] = v; });
-    if (a.h_last && (threadIdx.x & 31) == 0) a.h_last[w] = h;
+    if (valid && a.h_last && (threadIdx.x & (W - 1)) == 0) a.h_last[w] = h;
 }
 
 // P = exp(A_n * sum of delta): the decay of a chunk summary, from the per-row sums
@@ -148,13 +150,15 @@ __global__ void __launch_bounds__(128) decay_kernel(const float* dsum, const flo
 
 // Compose K chunk maps h -> P_k h + H_k (each (batch, D, N), chunk-major) in order,
 // starting from h0: carry_in[k] is the state entering chunk k, h_final the state
-// after the last.  One warp per (b, d, n).
+// after the last.  W lanes (affine_lanes(K)) per (b, d, n).
 __global__ void __launch_bounds__(128) compose_kernel(const float* P, const float* H, const float* h0,
-                                                      float* carry_in, float* h_final, int64_t K, int64_t BDN) {
-    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (w >= BDN) return;  // warp-uniform
+                                                      float* carry_in, float* h_final, int64_t K, int64_t BDN,
+                                                      int W) {
+    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / W;
+    const bool valid = r < BDN;
+    const int64_t w = valid ? r : BDN - 1;
     const float h = affine_carry_warp(
-        K, h0 ? __ldg(h0 + w) : 0.f,
+        K, h0 ? __ldg(h0 + w) : 0.f, W, valid,
         [&](int64_t k, float& p, float& q) {
             p = __ldg(P + k * BDN + w);
             q = __ldg(H + k * BDN + w);
@@ -162,7 +166,7 @@ __global__ void __launch_bounds__(128) compose_kernel(const float* P, const floa
         [&](int64_t k, float v) {
             if (carry_in) carry_in[k * BDN + w] = v;
         });
-    if (h_final && (threadIdx.x & 31) == 0) h_final[w] = h;
+    if (valid && h_final && (threadIdx.x & (W - 1)) == 0) h_final[w] = h;
 }
 
 }  // namespace sscan
