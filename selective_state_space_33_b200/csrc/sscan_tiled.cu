@@ -379,24 +379,44 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
             float* sCf = reinterpret_cast<float*>(smem + C::OFF_C);
             const T* rB = reinterpret_cast<const T*>(raw + 3 * C::RAW);
             const T* rC = reinterpret_cast<const T*>(raw + 3 * C::RAW + C::RAWBC);
-#pragma unroll
-            for (int ei = 0; ei < (C::BC_ENTRIES + kThreads - 1) / kThreads; ++ei) {
-                const int e = tid + ei * kThreads;
-                if (C::BC_ENTRIES % kThreads != 0 && e >= C::BC_ENTRIES) break;
-                const int t = e / C::NS, n = e % C::NS;
-                float bv = 0.f, cv = 0.f;
-                if (n < N) {
-                    if (bc_tma) {
-                        bv = to_f32<T>(rB[t * N + n]);
-                        if (want_out) cv = to_f32<T>(rC[t * N + n]);
-                    } else if (tt + t < t_end) {
-                        const int64_t gi = ((int64_t)b * a.L + tt + t) * N + n;
-                        bv = to_f32<T>(Bg[gi]);
-                        if (want_out) cv = to_f32<T>(Cg[gi]);
+            if (bc_tma && N == C::NS) {
+                // dense [kTT][N] tiles: one thread converts 4 consecutive values of B
+                // (threads 0 .. V-1) or of C (V .. 2V-1)
+                constexpr int V = C::BC_ENTRIES / 4;
+                static_assert(2 * V <= kThreads, "one 4-value group per thread");
+                const int which = tid / V, v = tid % V;
+                if (which == 0 || (which == 1 && want_out)) {
+                    const T* src = which ? rC : rB;
+                    float4 f;
+                    if constexpr (sizeof(T) == 4) {
+                        f = reinterpret_cast<const float4*>(src)[v];
+                    } else {
+                        const uint2 w = reinterpret_cast<const uint2*>(src)[v];
+                        f = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                                        __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
                     }
+                    reinterpret_cast<float4*>(which ? sCf : sBf)[v] = f;
                 }
-                sBf[e] = bv;
-                if (want_out) sCf[e] = cv;
+            } else {
+#pragma unroll
+                for (int ei = 0; ei < (C::BC_ENTRIES + kThreads - 1) / kThreads; ++ei) {
+                    const int e = tid + ei * kThreads;
+                    if (C::BC_ENTRIES % kThreads != 0 && e >= C::BC_ENTRIES) break;
+                    const int t = e / C::NS, n = e % C::NS;
+                    float bv = 0.f, cv = 0.f;
+                    if (n < N) {
+                        if (bc_tma) {
+                            bv = to_f32<T>(rB[t * N + n]);
+                            if (want_out) cv = to_f32<T>(rC[t * N + n]);
+                        } else if (tt + t < t_end) {
+                            const int64_t gi = ((int64_t)b * a.L + tt + t) * N + n;
+                            bv = to_f32<T>(Bg[gi]);
+                            if (want_out) cv = to_f32<T>(Cg[gi]);
+                        }
+                    }
+                    sBf[e] = bv;
+                    if (want_out) sCf[e] = cv;
+                }
             }
         }
         fence_proxy_async();

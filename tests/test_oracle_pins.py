@@ -315,6 +315,19 @@ def test_backward_skip_gradient_closed_form():
     np.testing.assert_allclose(g["dD"], np.sum(dout * s * p["u"], axis=(0, 1)), rtol=1e-12)
 
 
+def test_backward_gate_gradient_closed_form():
+    """dz = dout * y * sigma(z) * (1 + z (1 - sigma(z))), y the ungated output (the
+    derivative of SiLU(z) = z sigma(z); the gate of Fig. 3)."""
+    p, dout = _fd_case(seed=3)
+    g = oracle.bwd(p["u"], p["delta_raw"], p["A"], p["B"], p["C"], dout, delta_bias=p["delta_bias"],
+                   D_skip=p["D_skip"], z=p["z"], h0=p["h0"])
+    y, _ = oracle.fwd(p["u"], p["delta_raw"], p["A"], p["B"], p["C"], delta_bias=p["delta_bias"],
+                      D_skip=p["D_skip"], h0=p["h0"])
+    from scipy.special import expit
+    sg = expit(p["z"])
+    np.testing.assert_allclose(g["dz"], dout * y * sg * (1.0 + p["z"] * (1.0 - sg)), rtol=1e-12, atol=1e-14)
+
+
 # ---------------------------------------------------------------- one step, high precision
 def _dec_expm1_over(q_str, a_str, digits=60):
     """expm1(q)/a and the A-derivative delta^2 (q e^q - expm1(q))/q^2 in 60-digit decimals."""
