@@ -96,23 +96,16 @@ __device__ __forceinline__ float2 ex2x2(float2 q) { return f2(ex2(q.x), ex2(q.y)
 // lane's G values of B_t, C_t.  Returns the partial readout sum_j C_j h_j over these
 // states (eq. (3b)).
 template <int G, bool WANT_Y>
-__device__ __forceinline__ float step_fast(LaneG<G>& s, float4 dx, const float4* Bp, const float4* Cp) {
+__device__ __forceinline__ float step_fast(LaneG<G>& s, float4 dx, const float* Bp, const float* Cp) {
     const float2 dd = f2(dx.x, dx.y), xx = f2(dx.z, dx.w);
     float2 y = f2(0.f, 0.f);
 #pragma unroll
-    for (int k = 0; k < G / 4; ++k) {
-        const float4 Bv = Bp[k];
-        const float2 a0 = ex2x2(__fmul2_rn(dd, s.A2[2 * k]));
-        const float2 a1 = ex2x2(__fmul2_rn(dd, s.A2[2 * k + 1]));
-        const float2 v0 = __fmul2_rn(f2(Bv.x, Bv.y), __fmul2_rn(xx, s.niA[2 * k]));
-        const float2 v1 = __fmul2_rn(f2(Bv.z, Bv.w), __fmul2_rn(xx, s.niA[2 * k + 1]));
-        s.h[2 * k] = __ffma2_rn(a0, __ffma2_rn(v0, f2(-1.f, -1.f), s.h[2 * k]), v0);
-        s.h[2 * k + 1] = __ffma2_rn(a1, __ffma2_rn(v1, f2(-1.f, -1.f), s.h[2 * k + 1]), v1);
-        if (WANT_Y) {
-            const float4 Cv = Cp[k];
-            y = __ffma2_rn(f2(Cv.x, Cv.y), s.h[2 * k], y);
-            y = __ffma2_rn(f2(Cv.z, Cv.w), s.h[2 * k + 1], y);
-        }
+    for (int k = 0; k < G / 2; ++k) {
+        const float2 Bv = reinterpret_cast<const float2*>(Bp)[k];
+        const float2 a = ex2x2(__fmul2_rn(dd, s.A2[k]));
+        const float2 v = __fmul2_rn(Bv, __fmul2_rn(xx, s.niA[k]));
+        s.h[k] = __ffma2_rn(a, __ffma2_rn(v, f2(-1.f, -1.f), s.h[k]), v);
+        if (WANT_Y) y = __ffma2_rn(reinterpret_cast<const float2*>(Cp)[k], s.h[k], y);
     }
     return WANT_Y ? y.x + y.y : 0.f;
 }
@@ -120,26 +113,20 @@ __device__ __forceinline__ float step_fast(LaneG<G>& s, float4 dx, const float4*
 // Accurate form for blocks with a small |A| (or A = 0): Bbar / B = delta phi1(delta A)
 // with phi1's series near 0, as in the general kernels.
 template <int G, bool WANT_Y>
-__device__ __forceinline__ float step_acc(LaneG<G>& s, float4 dx, const float4* Bp, const float4* Cp) {
+__device__ __forceinline__ float step_acc(LaneG<G>& s, float4 dx, const float* Bp, const float* Cp) {
     const float delta = dx.x, x = dx.z;
     float y = 0.f;
 #pragma unroll
-    for (int k = 0; k < G / 4; ++k) {
-        const float4 Bv = Bp[k];
-        const float4 Cv = WANT_Y ? Cp[k] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float Bb[4] = {Bv.x, Bv.y, Bv.z, Bv.w}, Cc[4] = {Cv.x, Cv.y, Cv.z, Cv.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float2& hp = s.h[2 * k + j / 2];
-            const float A2 = (j & 1) ? s.A2[2 * k + j / 2].y : s.A2[2 * k + j / 2].x;
-            const float iA = -((j & 1) ? s.niA[2 * k + j / 2].y : s.niA[2 * k + j / 2].x);
-            const float q2 = delta * A2;
-            const float abar = ex2(q2);
-            const float beta = bbar_coef(delta, q2 * kLn2, abar, iA);
-            float& hv = (j & 1) ? hp.y : hp.x;
-            hv = fmaf(abar, hv, beta * Bb[j] * x);
-            y = fmaf(Cc[j], hv, y);
-        }
+    for (int j = 0; j < G; ++j) {
+        float2& hp = s.h[j / 2];
+        const float A2 = (j & 1) ? s.A2[j / 2].y : s.A2[j / 2].x;
+        const float iA = -((j & 1) ? s.niA[j / 2].y : s.niA[j / 2].x);
+        const float q2 = delta * A2;
+        const float abar = ex2(q2);
+        const float beta = bbar_coef(delta, q2 * kLn2, abar, iA);
+        float& hv = (j & 1) ? hp.y : hp.x;
+        hv = fmaf(abar, hv, beta * Bp[j] * x);
+        if (WANT_Y) y = fmaf(Cp[j], hv, y);
     }
     return WANT_Y ? y : 0.f;
 }
@@ -180,8 +167,8 @@ __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int 
     constexpr bool WANT_Y = MODE == kOut;
     const float4* sdx = reinterpret_cast<const float4*>(smem + C::OFF_DX) + cw;
     const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
-    const float4* sB = reinterpret_cast<const float4*>(smem + C::OFF_B) + g * (G / 4);
-    const float4* sC = reinterpret_cast<const float4*>(smem + C::OFF_C) + g * (G / 4);
+    const float* sB = reinterpret_cast<const float*>(smem + C::OFF_B) + g * G;
+    const float* sC = reinterpret_cast<const float*>(smem + C::OFF_C) + g * G;
 #pragma unroll(MODE == kOut ? 2 : 1)
     for (int tb = 0; tb < kTT; tb += NG) {
         if (MODE == kCkpt && tb % kCkStep == 0 && (FULL || tb < tile_len)) {
@@ -199,8 +186,8 @@ __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int 
             if (FULL || t < tile_len) {
                 const float4 dx = sdx[t * C::DC];
                 if (MODE == kAgg) dsum += dx.x;
-                p[k] = ACC ? step_acc<G, WANT_Y>(s, dx, sB + t * (C::NS / 4), sC + t * (C::NS / 4))
-                           : step_fast<G, WANT_Y>(s, dx, sB + t * (C::NS / 4), sC + t * (C::NS / 4));
+                p[k] = ACC ? step_acc<G, WANT_Y>(s, dx, sB + t * C::NS, sC + t * C::NS)
+                           : step_fast<G, WANT_Y>(s, dx, sB + t * C::NS, sC + t * C::NS);
             }
         }
         if constexpr (WANT_Y) {
@@ -556,7 +543,8 @@ cudaError_t launch_t(const TiledArgs& a, const TiledPtrs& p, const TiledGeom& ge
 // Lane geometry: four states per lane, NG = ceil(N / 4) lanes per channel.  (Eight
 // states per lane halve the per-step overheads but halve the warps; at the Mamba
 // layer shapes that left too few warps per sub-partition to hide latency, and it
-// measured slower.)
+// measured slower.  Two states per lane double the warps, more than the 2.8B-layer
+// grid can hold in one wave, and measured slower at both layer shapes.)
 TiledGeom tiled_geometry(int64_t batch, int64_t L, int64_t D, int64_t N) {
     (void)batch;
     (void)L;
