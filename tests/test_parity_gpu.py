@@ -241,6 +241,21 @@ def test_backward_small(cuda_device, io, shape):
     _check_bwd(x, io, cuda_device, h0=h0)
 
 
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_backward_general_A_values(cuda_device, io):
+    """A with zeros (the delta B limit), tiny and large magnitudes: the channel block
+    holding them recomputes states with phi1's series, the other block with the
+    forward kernel's form; both must match the oracle."""
+    x = W.small_case(2, 90, 64, 16, io=io, seed=43, backward=True)
+    rng = np.random.default_rng(43)
+    A = -np.exp(rng.uniform(-6, 3, size=(64, 16))).astype(np.float32)
+    A[0, :4] = 0.0
+    A[2, 7] = -1e-7
+    A[5, 3] = -3e-4
+    x["A"] = A
+    _check_bwd(x, io, cuda_device)
+
+
 def test_backward_mamba130m_full(cuda_device):
     x = W.make_inputs(W.WORKLOADS["bwd130m"])
     _check_bwd(x, "bf16", cuda_device)
