@@ -35,6 +35,7 @@ DEFAULT_WORKLOAD = "mamba2.8b"
 SM_COUNT = 148
 MUFU_PER_SM_CLK = 16          # ex2 results per SM per clock (4 per sub-partition)
 HBM_FALLBACK_GBS = 6650.0     # used only when MEASURED_PEAKS.json is absent
+HBM_NOMINAL_GBS = 7700.0      # B200 HBM3e nominal (HGX figure), for context
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -109,14 +110,14 @@ def roofline_units(w: W.Workload) -> dict:
 # under profiles/).  A figure holds only for the kernel source it was taken on: it is
 # keyed by the SHA-256 of those source files and reported as null once they change.
 NCU_TRAFFIC = {
-    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 505149440 + 152071680,
-                  "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "c0b8a6386a3feae3",
+    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 504947968 + 151214848,
+                  "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "70a9ef22462fd8b3",
                   "profile": "profiles/fwd_tiled_kernel_mamba2.8b_bf16.md"},
-    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 406294784 + 133817088,
-                "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "2178d0fd962a137f",
+    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410339840 + 134322688,
+                "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "fcc0aaaa58a1c74e",
                 "profile": "profiles/bwd_tiled_kernel_bwd130m_bf16.md"},
-    "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23315968 + 0,
-                   "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "5144163678ece024",
+    "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317504 + 0,
+                   "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "3f0237a88da992b3",
                    "profile": "profiles/step_quad_kernel_decode2.8b_bf16.md"},
 }
 
@@ -514,6 +515,8 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
     hbm_src = "measured" if "hbm_gbs" in peaks else "fallback"
     sm_max = float(peaks.get("sm_max_mhz", 1965.0))
     mufu_nominal = SM_COUNT * MUFU_PER_SM_CLK * sm_max * 1e6
+    # the same unit count at the SM clock sampled during the timed region
+    mufu_at_clock = SM_COUNT * MUFU_PER_SM_CLK * float(clk["sm_mhz"]) * 1e6 if clk.get("sm_mhz") else None
     mufu_probe = ex2_probe(torch, lib, dev)
     launch_s = statistics.mean(per_launch_ms) * 1e-3
     exps_rate = units["exps"] / launch_s
@@ -543,8 +546,10 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
             "peak_source": f"derived: {SM_COUNT} SMs x {MUFU_PER_SM_CLK} ex2/clk x {sm_max:.0f} MHz",
             "peak_probe_gexps": None if mufu_probe is None else mufu_probe / 1e9,
             "frac_of_probe": None if mufu_probe is None else exps_rate / mufu_probe,
+            "peak_at_sampled_clock_gexps": mufu_at_clock / 1e9 if mufu_at_clock else None,
+            "frac_at_sampled_clock": exps_rate / mufu_at_clock if mufu_at_clock else None,
             "hbm": {"achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
-                    "source": hbm_src},
+                    "source": hbm_src, "nominal": HBM_NOMINAL_GBS, "frac_nominal": gbs / HBM_NOMINAL_GBS},
             "roofline_frac": t_roof / launch_s,
             "per_launch_ms": launch_s * 1e3,
             "alg_bytes_per_launch": units["bytes"], "alg_exps_per_launch": units["exps"],
