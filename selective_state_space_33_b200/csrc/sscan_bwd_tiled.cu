@@ -569,19 +569,23 @@ bool make_map_b(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int6
 }
 
 template <typename T, int NG, int MODE>
-void launch_bwd_kernel(const CUtensorMap (&m)[9], const BwdTiledArgs& a, cudaStream_t st) {
+cudaError_t launch_bwd_kernel(const CUtensorMap (&m)[9], const BwdTiledArgs& a, cudaStream_t st) {
     using C = BCfg<T, NG>;
     auto kern = bwd_tiled_kernel<T, NG, MODE>;
-    static bool configured = false;
-    if (!configured) {
+    // function attributes are per device: set them once on each device used
+    static bool configured[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        configured = true;
+        configured[dev] = true;
     }
     const int64_t segs = MODE == kBwdSummary ? a.nseg - 1 : a.nseg;
     const int64_t blocks = a.batch * segs * ((a.D + C::DC - 1) / C::DC);
     if (blocks > 0)
         kern<<<(unsigned)blocks, kThreadsB, C::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], m[8], a);
+    return cudaGetLastError();
 }
 
 template <typename T, int NG>
@@ -596,9 +600,8 @@ cudaError_t launch_bwd_t(const BwdTiledArgs& a, const BwdTiledPtrs& p, int mode,
         !make_map_b<T>(&m[6], p.du, a.batch, a.L, a.D, C::DC) || !make_map_b<T>(&m[7], p.ddelta_raw, a.batch, a.L, a.D, C::DC) ||
         !make_map_b<T>(&m[8], dzdst, a.batch, a.L, a.D, C::DC))
         return cudaErrorInvalidValue;
-    if (mode == kBwdSummary) launch_bwd_kernel<T, NG, kBwdSummary>(m, a, st);
-    else launch_bwd_kernel<T, NG, kBwdFull>(m, a, st);
-    return cudaGetLastError();
+    return mode == kBwdSummary ? launch_bwd_kernel<T, NG, kBwdSummary>(m, a, st)
+                               : launch_bwd_kernel<T, NG, kBwdFull>(m, a, st);
 }
 
 // W lanes per (batch, channel, state): compose the segments right to left with

@@ -41,6 +41,8 @@ enum { kTiledOut = 0, kTiledAgg = 1, kTiledLast = 2, kTiledCkpt = 3 };
 
 // Lane geometry of the tiled kernel: NG lanes per channel, G states per lane,
 // DC channels per CTA (its TMA box width).  A pure function of the problem.
+constexpr int kMaxDevices = 64;  // per-device caches of the host code
+
 struct TiledGeom {
     int NG, G, DC;
 };

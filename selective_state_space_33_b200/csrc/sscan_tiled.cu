@@ -511,11 +511,14 @@ cudaError_t launch_mode(const TiledArgs& args, const TiledPtrs& p, cudaStream_t 
         mc = mu;
     }
     auto kern = fwd_tiled_kernel<T, NG, G, MODE>;
-    static bool configured = false;
-    if (!configured) {
+    // function attributes are per device: set them once on each device used
+    static bool configured[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        configured = true;
+        configured[dev] = true;
     }
     const int64_t ncb = (a.D + C::DC - 1) / C::DC;
     const int64_t blocks = a.batch * a.nchunks * ncb;
