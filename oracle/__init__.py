@@ -39,6 +39,8 @@ def _load():
         lib.orc_fwd.restype = ctypes.c_int
         lib.orc_bwd.argtypes = [ctypes.POINTER(_Problem)] + [vp] * 19
         lib.orc_bwd.restype = ctypes.c_int
+        lib.orc_fwd_complex.argtypes = [ctypes.POINTER(_Problem)] + [vp] * 11
+        lib.orc_fwd_complex.restype = ctypes.c_int
         lib.orc_set_threads.argtypes = [ctypes.c_int]
         lib.orc_set_threads.restype = ctypes.c_int
         _lib = lib
@@ -147,4 +149,37 @@ def bwd(u, delta_raw, A, B, C, dout, *, delta_bias=None, D_skip=None, z=None, h0
     return {k: v for k, v in g.items() if v is not None}
 
 
-__all__ = ["fwd", "bwd", "set_threads"]
+def _interleave(c, shape):
+    """complex (…) or real (…, 2) -> contiguous float64 (…, 2) pairs (re, im)."""
+    if c is None:
+        return None
+    c = np.asarray(c)
+    if np.iscomplexobj(c):
+        c = np.stack([c.real, c.imag], axis=-1)
+    c = np.ascontiguousarray(c, dtype=np.float64)
+    assert c.shape == tuple(shape) + (2,), (c.shape, shape)
+    return c
+
+
+def fwd_complex(u, delta_raw, A, B, C, *, delta_bias=None, D_skip=None, z=None, h0=None,
+                delta_softplus=True, want_out=True):
+    """Forward scan with a complex diagonal A in fp64.  A: (D, N) complex (or (D, N, 2)
+    real pairs); h0: (batch, D, N) complex or None.  B, C real (batch, L, N).
+    Returns (out (batch, L, D) real, h_last (batch, D, N) complex128)."""
+    (u, delta_raw, B, C, z), code = _ios(u, delta_raw, B, C, z)
+    batch, L, D = u.shape
+    N = B.shape[-1]
+    A2 = _interleave(A, (D, N))
+    h02 = _interleave(h0, (batch, D, N))
+    delta_bias, D_skip = _f64(delta_bias), _f64(D_skip)
+    out = np.empty((batch, L, D), np.float64) if want_out else None
+    h_last = np.empty((batch, D, N, 2), np.float64)
+    prob = _Problem(batch, L, D, N, code, 1 if delta_softplus else 0)
+    rc = _load().orc_fwd_complex(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias), _ptr(A2),
+                                 _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h02), _ptr(out), _ptr(h_last))
+    if rc != 0:
+        raise ValueError("orc_fwd_complex rejected its arguments")
+    return out, h_last[..., 0] + 1j * h_last[..., 1]
+
+
+__all__ = ["fwd", "bwd", "fwd_complex", "set_threads"]

@@ -293,6 +293,96 @@ int orc_bwd(const orc_problem* p, const void* u, const void* delta_raw,
 }
 
 /* Thread control for the CPU-baseline timing (0 = leave OpenMP's default). */
+/*
+ * Forward scan with a complex diagonal A -- the complex initialisation
+ * A_n = -1/2 + n i named in the sec. 6.5 A-init ablation table -- i.e. eqs. (2)
+ * and (3) in complex arithmetic.  Readings where the pages are silent:
+ *   - A is (D, N) complex, stored interleaved as (re, im) pairs: A[(d*N + n)*2 + k];
+ *   - B and C stay the real (batch, L, N) input-dependent projections of sec. 3.2;
+ *     the state is complex: h_t = Abar h_{t-1} + Bbar x_t with
+ *     Abar = exp(delta a) and Bbar = (exp(delta a) - 1)/a * B (eq. 2; limit
+ *     delta*B at a = 0);
+ *   - the output is the real part of the readout eq. (3b):
+ *     y_t = Re(sum_n C_tn h_tn) + D_skip x_t, then the SiLU gate;
+ *   - h0 / h_last are (batch, D, N) complex, interleaved like A.
+ * exp(q) - 1 for complex q = x + iy is formed as
+ *   (expm1(x) cos y - 2 sin^2(y/2)) + i exp(x) sin y,
+ * the same value without the cancellation of e^x cos y - 1 near q = 0.
+ * Same argument conventions as orc_fwd (all rows; out, h_last may be NULL).
+ */
+int orc_fwd_complex(const orc_problem* p, const void* u, const void* delta_raw,
+                    const double* delta_bias, const double* A, const void* B,
+                    const void* C, const double* D_skip, const void* z,
+                    const double* h0, double* out, double* h_last)
+{
+    if (check(p) || !u || !delta_raw || !A || !B || (out && !C)) return 1;
+    const int64_t Bt = p->batch, L = p->seqlen, D = p->dim, N = p->dstate;
+    const int32_t dt = p->io_dtype;
+
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t row = 0; row < Bt * D; ++row) {
+        const int64_t b = row / D, d = row % D;
+        double* hr = (double*)malloc((size_t)N * 2 * sizeof(double));
+        if (!hr) {
+#pragma omp atomic write
+            bad = 1;
+            continue;
+        }
+        double* hi = hr + N;
+        for (int64_t n = 0; n < N; ++n) {
+            hr[n] = h0 ? h0[(row * N + n) * 2] : 0.0;
+            hi[n] = h0 ? h0[(row * N + n) * 2 + 1] : 0.0;
+        }
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t e = (b * L + t) * D + d;
+            const int64_t s = (b * L + t) * N;
+            const double x = ld(u, dt, e);
+            const double r = ld(delta_raw, dt, e) + (delta_bias ? delta_bias[d] : 0.0);
+            const double delta = p->delta_softplus ? softplus(r) : r;
+            double y = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                const double ar = A[(d * N + n) * 2], ai = A[(d * N + n) * 2 + 1];
+                const double qr = delta * ar, qi = delta * ai;
+                /* Abar = exp(q), eq. (2) */
+                const double ex = exp(qr);
+                const double abr = ex * cos(qi), abi = ex * sin(qi);
+                /* Bbar / B = (exp(q) - 1) / a, or delta at a = 0 */
+                double cr, ci;
+                if (ar == 0.0 && ai == 0.0) {
+                    cr = delta;
+                    ci = 0.0;
+                } else {
+                    const double sh = sin(0.5 * qi);
+                    const double em1r = expm1(qr) * cos(qi) - 2.0 * sh * sh, em1i = ex * sin(qi);
+                    const double den = ar * ar + ai * ai;
+                    cr = (em1r * ar + em1i * ai) / den;
+                    ci = (em1i * ar - em1r * ai) / den;
+                }
+                const double bx = ld(B, dt, s + n) * x;
+                /* eq. (3a) in complex arithmetic */
+                const double nr = abr * hr[n] - abi * hi[n] + cr * bx;
+                const double ni = abr * hi[n] + abi * hr[n] + ci * bx;
+                hr[n] = nr;
+                hi[n] = ni;
+                if (out) y += ld(C, dt, s + n) * hr[n]; /* Re of eq. (3b) */
+            }
+            if (out) {
+                if (D_skip) y += D_skip[d] * x;
+                if (z) y *= silu(ld(z, dt, e));
+                out[e] = y;
+            }
+        }
+        if (h_last)
+            for (int64_t n = 0; n < N; ++n) {
+                h_last[(row * N + n) * 2] = hr[n];
+                h_last[(row * N + n) * 2 + 1] = hi[n];
+            }
+        free(hr);
+    }
+    return bad;
+}
+
 int orc_set_threads(int n)
 {
 #ifdef _OPENMP

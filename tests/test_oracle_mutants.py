@@ -37,7 +37,15 @@ MUTANTS = {
     "bwd_dz_formula": ("(1.0 + zz * (1.0 - sg))", "(1.0 + (1.0 - sg))"),
     "bwd_no_softplus_chain": ("ddelta * sigmoid(r) : ddelta;", "ddelta : ddelta;"),
     "psi_series_term": ("q * (1.0 / 8.0 + q * (1.0 / 30.0", "q * (1.0 / 6.0 + q * (1.0 / 30.0"),
+    "complex_rotation_sign": ("const double abr = ex * cos(qi), abi = ex * sin(qi);",
+                              "const double abr = ex * cos(qi), abi = -ex * sin(qi);"),
+    "complex_readout_imag": ("if (out) y += ld(C, dt, s + n) * hr[n];", "if (out) y += ld(C, dt, s + n) * hi[n];"),
+    "complex_division_sign": ("ci = (em1i * ar - em1r * ai) / den;", "ci = (em1i * ar + em1r * ai) / den;"),
+    "complex_state_mix": ("const double ni = abr * hi[n] + abi * hr[n] + ci * bx;",
+                          "const double ni = abr * hi[n] - abi * hr[n] + ci * bx;"),
+    "complex_half_angle": ("- 2.0 * sh * sh, em1i", "- sh * sh, em1i"),
 }
+PIN_FILES = ["test_oracle_pins.py", "test_oracle_complex_pins.py"]
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
@@ -51,7 +59,7 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp", str(mutated),
                     "-o", str(lib), "-lm"], check=True)
     env = dict(os.environ, SSCAN_ORACLE_LIB=str(lib))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider"]
+                       + [os.path.join(ROOT, "tests", f) for f in PIN_FILES],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
