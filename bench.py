@@ -30,6 +30,7 @@ from selective_state_space_33_b200 import workloads as W  # noqa: E402
 METRIC = "selective-scan fwd Gelem/s (B·L·D) & % of HBM/MUFU roofline at 2.8B-layer shape"
 METRIC_BWD = "selective-scan bwd Gelem/s (B·L·D), states recomputed on chip"
 METRIC_STEP = "selective-scan generation step Gelem/s (batch·D per token), state read and written in HBM"
+METRIC_COMPLEX = "selective-scan fwd with complex diagonal A, Gelem/s (B·L·D)"
 UNIT = "Gelem/s"
 DEFAULT_WORKLOAD = "mamba2.8b"
 SM_COUNT = 148
@@ -90,6 +91,11 @@ def roofline_units(w: W.Workload) -> dict:
     s = 2 if w.io == "bf16" else 4
     E = w.batch * w.seqlen * w.dim
     BLN = w.batch * w.seqlen * w.dstate
+    if w.complex_a:
+        # complex A: the same bytes (A is (D, N, 2) fp32); per state the MUFU computes
+        # 2^(delta Re a), cos and sin of delta Im a: 3 N + 2 MUFU operations per element.
+        bytes_ = 4 * E * s + 2 * BLN * s + (2 * w.dim * w.dstate + 2 * w.dim) * 4
+        return {"elements": E, "bytes": bytes_, "exps": E * (3 * w.dstate + 2)}
     if w.decode:
         # one token: read and write the fp32 state (the dominant term), read u, delta_raw,
         # z and write out (batch, D), read B, C (batch, N) and the parameters.
@@ -359,7 +365,10 @@ def gpu_arm(args, w: W.Workload):
     nstep = [0]
 
     def step(stream=st):
-        if w.decode:
+        if w.complex_a:
+            sb.sscan_fwd_complex(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["delta_bias"], t["D_skip"],
+                                 t.get("z"), out=out, stream=stream)
+        elif w.decode:
             i = nstep[0] % nsets
             nstep[0] += 1
             sq = sets[i]
@@ -438,7 +447,7 @@ def gpu_arm(args, w: W.Workload):
             print(json.dumps({"profile_run": True, "workload": w.name, "value": value, "unit": UNIT,
                               "per_launch_ms": statistics.mean(per_launch_ms)}), flush=True)
         return
-    if w.backward or w.decode:
+    if w.backward or w.decode or w.complex_a:
         e2e_value, h2d, d2h = None, 0, 0
     else:
         e2e_value, h2d, d2h = e2e_leg(args, t, out, ws, st, units, world, dev)
@@ -523,7 +532,7 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
     gbs = units["bytes"] / launch_s / 1e9
     t_roof = max(units["bytes"] / (hbm_peak * 1e9), units["exps"] / mufu_nominal)
     cpu = None
-    if world == 1 and not args.no_cpu_baseline and not w.backward and not w.decode:
+    if world == 1 and not args.no_cpu_baseline and not w.backward and not w.decode and not w.complex_a:
         rate, cores, rows, secs = cpu_oracle_rate(x, w, args.cpu_seconds)
         rate1, rows1, secs1 = cpu_oracle_rate_1thread(x, w)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -532,7 +541,8 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
                "single_thread": {"value": rate1, "unit": UNIT,
                                  "sample": f"{rows1} random rows x L={w.seqlen}, {secs1:.1f} s on 1 thread"}}
     line = {
-        "metric": METRIC_BWD if w.backward else (METRIC_STEP if w.decode else METRIC), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": (METRIC_BWD if w.backward else METRIC_STEP if w.decode else METRIC_COMPLEX if w.complex_a
+                   else METRIC), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": max_s / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(w, world, l2_note),
@@ -541,7 +551,8 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
                                                "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "roofline": hbm_roofline(units, launch_s, hbm_peak, hbm_src, ncu_traffic(args.workload)) if w.decode else {
-            "bound": "alu", "pipe": "MUFU ex2", "achieved": exps_rate / 1e9, "peak": mufu_nominal / 1e9,
+            "bound": "alu", "pipe": "MUFU (ex2, sin, cos)" if w.complex_a else "MUFU ex2",
+            "achieved": exps_rate / 1e9, "peak": mufu_nominal / 1e9,
             "unit": "Gexp/s", "frac": exps_rate / mufu_nominal, "traffic": ncu_traffic(args.workload),
             "peak_source": f"derived: {SM_COUNT} SMs x {MUFU_PER_SM_CLK} ex2/clk x {sm_max:.0f} MHz",
             "peak_probe_gexps": None if mufu_probe is None else mufu_probe / 1e9,

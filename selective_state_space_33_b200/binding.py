@@ -53,6 +53,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sscan_workspace_size.argtypes = [pp, ctypes.c_int]
     lib.sscan_workspace_size.restype = sz
     lib.sscan_fwd.argtypes = [pp] + [vp] * 12 + [sz, vp]
+    lib.sscan_fwd_complex.argtypes = [pp] + [vp] * 12
+    lib.sscan_fwd_complex.restype = ctypes.c_int
     lib.sscan_fwd.restype = ctypes.c_int
     lib.sscan_last_state.argtypes = [pp] + [vp] * 8 + [sz, vp]
     lib.sscan_last_state.restype = ctypes.c_int
@@ -170,6 +172,39 @@ def sscan_fwd(u, delta_raw, A, B, C, delta_bias=None, D_skip=None, z=None, h0=No
                                     _ptr(A), _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h0),
                                     _ptr(out), _ptr(h_last), _ptr(ws), nbytes, _stream(stream)))
     return (out, h_last) if (return_last_state or h_last is not None) else out
+
+
+def _as_pairs(t, name, shape, dev):
+    """complex64 (...) -> float32 (..., 2) view of (re, im) pairs; float32 (..., 2) as is."""
+    if t is None:
+        return None
+    if t.is_complex():
+        if t.dtype != torch.complex64:
+            raise ValueError(f"{name}: complex64 expected, got {t.dtype}")
+        t = torch.view_as_real(t)
+    _expect(t, name, tuple(shape) + (2,), torch.float32, dev)
+    return t
+
+
+def sscan_fwd_complex(u, delta_raw, A, B, C, delta_bias=None, D_skip=None, z=None, h0=None, *,
+                      delta_softplus=True, out=None, return_last_state=False, stream=None):
+    """Forward scan with a complex diagonal A: (D, N) complex64 or (D, N, 2) float32
+    (re, im) pairs; h0 likewise (batch, D, N).  B, C real.  Returns ``out`` or
+    ``(out, h_last)`` with h_last (batch, D, N) complex64."""
+    prob = _io_problem(u, B, delta_softplus)
+    dev = u.device
+    _check_inputs(prob, u, delta_raw, None, B, C, delta_bias, D_skip, z, None)
+    A2 = _as_pairs(A, "A", (prob.dim, prob.dstate), dev)
+    h02 = _as_pairs(h0, "h0", (prob.batch, prob.dim, prob.dstate), dev)
+    if out is None:
+        out = torch.empty_like(u)
+    _expect(out, "out", u.shape, u.dtype, dev)
+    h_last = (torch.empty((prob.batch, prob.dim, prob.dstate, 2), dtype=torch.float32, device=dev)
+              if return_last_state else None)
+    _check(load_library().sscan_fwd_complex(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias),
+                                            _ptr(A2), _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h02),
+                                            _ptr(out), _ptr(h_last), _stream(stream)))
+    return (out, torch.view_as_complex(h_last)) if return_last_state else out
 
 
 def sscan_last_state(u, delta_raw, A, B, delta_bias=None, h0=None, *, delta_softplus=True,

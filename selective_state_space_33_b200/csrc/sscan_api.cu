@@ -548,6 +548,48 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
     return cuda_check("gradient cast kernel");
 }
 
+sscan_status sscan_fwd_complex(const sscan_problem* p, const void* u, const void* delta_raw,
+                               const float* delta_bias, const float* A, const void* B, const void* C,
+                               const float* D_skip, const void* z, const float* h0, void* out, float* h_last,
+                               void* stream) {
+    g_err[0] = 0;
+    g_launches = 0;
+    if (sscan_status s = check_problem(p)) return s;
+    const int64_t rows = p->batch * p->dim;
+    if (rows == 0) return SSCAN_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t state_bytes = (size_t)(rows * p->dstate * 2) * sizeof(float);
+    if (p->seqlen == 0) {
+        if (!h_last) return SSCAN_OK;
+        const cudaError_t e = h0 ? cudaMemcpyAsync(h_last, h0, state_bytes, cudaMemcpyDeviceToDevice, st)
+                                 : cudaMemsetAsync(h_last, 0, state_bytes, st);
+        return e == cudaSuccess ? SSCAN_OK : fail(SSCAN_ERR_CUDA, "empty sequence: %s", cudaGetErrorString(e));
+    }
+    if (!u || !delta_raw || !A || !B || !C || !out)
+        return fail(SSCAN_ERR_INVALID_ARG, "u, delta_raw, A, B, C and out are required");
+    sscan::ComplexArgs a{};
+    a.batch = p->batch;
+    a.L = p->seqlen;
+    a.D = p->dim;
+    a.N = (int)p->dstate;
+    a.softplus = (p->flags & SSCAN_DELTA_SOFTPLUS) ? 1 : 0;
+    a.u = u;
+    a.delta_raw = delta_raw;
+    a.bias = delta_bias;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.Dskip = D_skip;
+    a.z = z;
+    a.h0 = h0;
+    a.out = out;
+    a.h_last = h_last;
+    ++g_launches;
+    const cudaError_t e = sscan::launch_fwd_complex(a, p->io_dtype == SSCAN_BF16, st);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "complex forward kernel: %s", cudaGetErrorString(e));
+    return SSCAN_OK;
+}
+
 sscan_status sscan_step(const sscan_problem* p, const void* u, const void* delta_raw, const float* delta_bias,
                         const float* A, const void* B, const void* C, const float* D_skip, const void* z,
                         float* state, void* out, void* stream) {

@@ -1,0 +1,239 @@
+// sscan_complex.cu -- forward selective scan with a complex diagonal A (the complex
+// initialisation A_n = -1/2 + n i of the A-init ablation table, sec. 6.5 of the
+// Mamba technical summary page): eqs. (2) and (3) of sec. 2.1 in complex
+// arithmetic, with B and C the real input projections of sec. 3.2 and the output
+// the real part of the readout, y_t = Re(sum_n C_tn h_tn) + D_skip x_t, gated by
+// SiLU(z) (Fig. 3).
+//
+// Work decomposition (as the real tiled kernel): a CTA of 4 warps owns one batch
+// and DC channels for the whole sequence; the NG = ceil(N/4) lanes of a channel
+// each hold 4 complex states (8 fp32) in registers.  Per 16-step tile all threads
+// stage (delta, x) and (gate, D x gate) for the tile's channels and the tile's B
+// and C rows in shared memory with coalesced loads (phase P), then every lane
+// advances its states through the tile (phase S) and the NG lanes of a channel
+// sum their partial readouts with a butterfly; lane 0 of the channel writes out.
+//
+// One step of one complex state a = ar + i ai, with v = -B x / a:
+//   Abar = 2^(delta ar log2 e) (cos(delta ai) + i sin(delta ai))       (eq. 2)
+//   h'   = Abar (h - v) + v  = Abar h + (Abar - 1) B x / a             (eq. 3a)
+// (the update form of the real kernels).  The angle is reduced to [-pi, pi] with a
+// two-part 2 pi before the MUFU sine and cosine.  A CTA whose block holds an
+// |a| < 2^-10 (a = 0 included) takes Bbar / B = delta phi1(delta a) with phi1's
+// Taylor series in complex arithmetic where |delta a| < 1/16 instead.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "sscan_launch.h"
+#include "sscan_math.cuh"
+
+namespace sscan {
+namespace {
+
+constexpr int kCTT = 16;           // steps per tile
+constexpr int kCWarps = 4;
+constexpr int kCThreads = kCWarps * 32;
+constexpr int kCG = 4;             // complex states per lane
+constexpr float kCSmallA = 9.765625e-4f;
+constexpr float kTwoPiHi = 6.28318548202514648f;   // fp32 nearest to 2 pi
+constexpr float kTwoPiLo = -1.7484556e-7f;         // 2 pi - kTwoPiHi
+constexpr float kInvTwoPi = 0.159154943091895336f;
+
+__device__ __forceinline__ float sin_approx(float x) {
+    float y;
+    asm("sin.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float cos_approx(float x) {
+    float y;
+    asm("cos.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// cos and sin of an angle of any size: reduce by a multiple of 2 pi first.
+__device__ __forceinline__ float2 cis(float th) {
+    const float k = rintf(th * kInvTwoPi);
+    float r = fmaf(-k, kTwoPiHi, th);
+    r = fmaf(-k, kTwoPiLo, r);
+    return make_float2(cos_approx(r), sin_approx(r));
+}
+
+template <int NG>
+struct CCfg {
+    static constexpr int CW = 32 / NG;       // channels per warp
+    static constexpr int DC = CW * kCWarps;  // channels per CTA
+    static constexpr int NS = NG * kCG;      // states covered (>= N)
+};
+
+template <typename T, int NG, bool ACC>
+__device__ __forceinline__ void scan_tile_c(float2 (&h)[kCG], const float2 (&aq)[kCG], const float2 (&nia)[kCG],
+                                            const float2 (&ia)[kCG], const float2* sdx, const float2* sgd,
+                                            const float* sB, const float* sC, int tl, int g, int cw, bool write,
+                                            T* out, int64_t out_stride) {
+    using C = CCfg<NG>;
+    for (int t = 0; t < tl; ++t) {
+        const float2 dx = sdx[t * C::DC + cw];  // (delta, x)
+        const float delta = dx.x, x = dx.y;
+        const float* Bt = sB + t * C::NS + g * kCG;
+        const float* Ct = sC + t * C::NS + g * kCG;
+        float y = 0.f;
+#pragma unroll
+        for (int j = 0; j < kCG; ++j) {
+            const float e = ex2(delta * aq[j].x);
+            const float2 cs = cis(delta * aq[j].y);
+            const float abr = e * cs.x, abi = e * cs.y;
+            const float bx = Bt[j] * x;
+            float nr, ni;
+            if (!ACC) {
+                const float vr = bx * nia[j].x, vi = bx * nia[j].y;
+                const float tr = h[j].x - vr, ti = h[j].y - vi;
+                nr = fmaf(abr, tr, fmaf(-abi, ti, vr));
+                ni = fmaf(abr, ti, fmaf(abi, tr, vi));
+            } else {
+                // Bbar / B = delta phi1(q), q = delta a: series for |q| < 1/16, else (Abar - 1) / a
+                const float qr = delta * aq[j].x * kLn2, qi = delta * aq[j].y;
+                float cr, ci;
+                if (qr * qr + qi * qi < 0.00390625f) {
+                    // phi1(q) = 1 + q/2 + q^2/6 + q^3/24 + q^4/120, Horner in complex arithmetic
+                    float pr = 1.f / 120.f, pi = 0.f;
+                    const float cf[4] = {1.f / 24.f, 1.f / 6.f, 0.5f, 1.f};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float r2 = fmaf(pr, qr, fmaf(-pi, qi, cf[k]));
+                        pi = fmaf(pr, qi, pi * qr);
+                        pr = r2;
+                    }
+                    cr = delta * pr;
+                    ci = delta * pi;
+                } else {
+                    const float er = abr - 1.f;
+                    cr = fmaf(er, ia[j].x, -abi * ia[j].y);
+                    ci = fmaf(er, ia[j].y, abi * ia[j].x);
+                }
+                nr = fmaf(abr, h[j].x, fmaf(-abi, h[j].y, cr * bx));
+                ni = fmaf(abr, h[j].y, fmaf(abi, h[j].x, ci * bx));
+            }
+            h[j] = make_float2(nr, ni);
+            y = fmaf(Ct[j], nr, y);  // Re of eq. (3b)
+        }
+        // the NG lanes of a channel (lane bits at multiples of CW) sum their readouts
+#pragma unroll
+        for (int m = 1; m < NG; m <<= 1) y += __shfl_xor_sync(0xffffffffu, y, m * C::CW);
+        if (write && g == 0) {
+            const float2 gd = sgd[t * C::DC + cw];
+            IO<T>::store(out, (int64_t)t * out_stride, fmaf(y, gd.x, gd.y));
+        }
+    }
+}
+
+template <typename T, int NG>
+__global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a) {
+    using C = CCfg<NG>;
+    __shared__ float2 sdx[kCTT * C::DC];  // (delta, x)
+    __shared__ float2 sgd[kCTT * C::DC];  // (gate, D x gate)
+    __shared__ float sB[kCTT * C::NS], sC[kCTT * C::NS];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t ncb = (a.D + C::DC - 1) / C::DC;
+    const int64_t b = blockIdx.x / ncb;
+    const int64_t d0 = (blockIdx.x % ncb) * C::DC;
+    const int N = a.N;
+    const T* u = static_cast<const T*>(a.u);
+    const T* dr = static_cast<const T*>(a.delta_raw);
+    const T* zz = static_cast<const T*>(a.z);
+    const T* Bg = static_cast<const T*>(a.B);
+    const T* Cg = static_cast<const T*>(a.C);
+
+    const int g = lane / C::CW, c = lane % C::CW, cw = warp * C::CW + c;
+    const int64_t d = d0 + cw;
+    const bool cvalid = d < a.D;
+    float2 h[kCG], aq[kCG], nia[kCG], ia[kCG];
+    bool small_a = false;
+#pragma unroll
+    for (int j = 0; j < kCG; ++j) {
+        const int n = g * kCG + j;
+        const bool ok = cvalid && n < N;
+        const float ar = ok ? __ldg(a.A + (d * N + n) * 2) : -1.f;
+        const float ai = ok ? __ldg(a.A + (d * N + n) * 2 + 1) : 0.f;
+        const float m2 = ar * ar + ai * ai;
+        small_a |= ok && m2 < kCSmallA * kCSmallA;
+        aq[j] = make_float2(ar * kLog2e, ai);
+        const float inv = ok && m2 > 0.f ? 1.f / m2 : 0.f;
+        ia[j] = make_float2(ar * inv, -ai * inv);      // 1 / a
+        nia[j] = make_float2(-ia[j].x, -ia[j].y);      // -1 / a
+        h[j] = make_float2(0.f, 0.f);
+        if (ok && a.h0) h[j] = make_float2(__ldg(a.h0 + ((b * a.D + d) * N + n) * 2),
+                                           __ldg(a.h0 + ((b * a.D + d) * N + n) * 2 + 1));
+    }
+    const bool acc = __syncthreads_or(small_a ? 1 : 0) != 0;
+
+    for (int64_t t0 = 0; t0 < a.L; t0 += kCTT) {
+        const int tl = (int)(a.L - t0 < kCTT ? a.L - t0 : kCTT);
+        // phase P: (delta, x), (gate, D x gate), and the tile's B and C rows
+        for (int e = tid; e < kCTT * C::DC; e += kCThreads) {
+            const int t = e / C::DC, cc = e % C::DC;
+            const int64_t dd = d0 + cc;
+            float2 dx = make_float2(0.f, 0.f), gd = make_float2(0.f, 0.f);
+            if (t < tl && dd < a.D) {
+                const int64_t gi = (b * a.L + t0 + t) * a.D + dd;
+                const float x = IO<T>::load(u, gi);
+                const float r = IO<T>::load(dr, gi) + (a.bias ? __ldg(a.bias + dd) : 0.f);
+                const float gate = zz ? silu(IO<T>::load(zz, gi)) : 1.f;
+                const float dsk = a.Dskip ? __ldg(a.Dskip + dd) : 0.f;
+                dx = make_float2(a.softplus ? softplus(r) : r, x);
+                gd = make_float2(gate, dsk * x * gate);
+            }
+            sdx[e] = dx;
+            sgd[e] = gd;
+        }
+        for (int e = tid; e < kCTT * C::NS; e += kCThreads) {
+            const int t = e / C::NS, n = e % C::NS;
+            float bv = 0.f, cv = 0.f;
+            if (t < tl && n < N) {
+                const int64_t gi = (b * a.L + t0 + t) * N + n;
+                bv = IO<T>::load(Bg, gi);
+                cv = IO<T>::load(Cg, gi);
+            }
+            sB[e] = bv;
+            sC[e] = cv;
+        }
+        __syncthreads();
+        T* out = static_cast<T*>(a.out) + (b * a.L + t0) * a.D + d;
+        if (acc)
+            scan_tile_c<T, NG, true>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, cvalid, out, a.D);
+        else
+            scan_tile_c<T, NG, false>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, cvalid, out, a.D);
+        __syncthreads();
+    }
+    if (a.h_last && cvalid) {
+#pragma unroll
+        for (int j = 0; j < kCG; ++j) {
+            const int n = g * kCG + j;
+            if (n < N) {
+                a.h_last[((b * a.D + d) * N + n) * 2] = h[j].x;
+                a.h_last[((b * a.D + d) * N + n) * 2 + 1] = h[j].y;
+            }
+        }
+    }
+}
+
+template <typename T, int NG>
+cudaError_t launch_c(const ComplexArgs& a, cudaStream_t st) {
+    const int64_t blocks = a.batch * ((a.D + CCfg<NG>::DC - 1) / CCfg<NG>::DC);
+    if (blocks > 0) fwd_complex_kernel<T, NG><<<(unsigned)blocks, kCThreads, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_ct(const ComplexArgs& a, cudaStream_t st) {
+    if (a.N <= 4) return launch_c<T, 1>(a, st);
+    if (a.N <= 8) return launch_c<T, 2>(a, st);
+    return launch_c<T, 4>(a, st);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_complex(const ComplexArgs& a, int io_bf16, cudaStream_t st) {
+    return io_bf16 ? launch_ct<__nv_bfloat16>(a, st) : launch_ct<float>(a, st);
+}
+
+}  // namespace sscan

@@ -70,6 +70,26 @@ struct StepArgs {
 
 cudaError_t launch_step(const StepArgs& a, int io_bf16, cudaStream_t st);
 
+// Forward scan with a complex diagonal A (sscan_complex.cu).
+struct ComplexArgs {
+    int64_t batch, L, D;
+    int N;
+    int softplus;
+    const void* u;          // (batch, L, D)
+    const void* delta_raw;  // (batch, L, D)
+    const float* bias;      // (D) or null
+    const float* A;         // (D, N, 2): (re, im) pairs
+    const void* B;          // (batch, L, N), real
+    const void* C;          // (batch, L, N), real
+    const float* Dskip;     // (D) or null
+    const void* z;          // (batch, L, D) or null
+    const float* h0;        // (batch, D, N, 2) or null
+    void* out;              // (batch, L, D)
+    float* h_last;          // (batch, D, N, 2) or null
+};
+
+cudaError_t launch_fwd_complex(const ComplexArgs& a, int io_bf16, cudaStream_t st);
+
 // Backward of the tiled path: scalars, small tensors and gradient accumulators.
 struct BwdTiledArgs {
     int64_t batch, L, D;

@@ -12,7 +12,8 @@ chunks of ``_CHUNK`` elements so the stream does not depend on memory limits):
   log_dt          ~ U[ln dt_min, ln dt_max], shape (D,)
   D_skip          = 1, or ~ N(0, 1) when the workload says so, shape (D,)
   dout            ~ N(0, 1), shape (batch, L, D), only for backward workloads
-  A[d, n]         = -(n + 1)                      (S4D-real initialisation)
+  A[d, n]         = -(n + 1)                      (S4D-real initialisation), or,
+                    for complex-A workloads, -1/2 + n i (complex64)
   delta_bias[d]   = log(expm1(dt_d)), the value whose softplus is dt_d, so that
                     softplus(delta_raw + bias) centres log-uniformly in
                     [dt_min, dt_max] before the N(0,1) draw spreads it.
@@ -44,6 +45,7 @@ class Workload:
     backward: bool = False
     decode: bool = False         # one-token generation steps (seqlen 1, carried state)
     gate: bool = True
+    complex_a: bool = False      # A_n = -1/2 + n i (complex diagonal A)
     description: str = ""
 
     @property
@@ -69,6 +71,8 @@ WORKLOADS = {
                         backward=True, description="backward at the Mamba-130M layer shape"),
     "decode2.8b": Workload("decode2.8b", 64, 1, 5120, 16, "bf16", 1e-3, 1e-1, "normal", 5,
                            decode=True, description="one generation step, 64 sequences, Mamba-2.8B layer width"),
+    "complex130m": Workload("complex130m", 8, 2048, 1536, 16, "bf16", 1e-3, 1e-1, "ones", 6, complex_a=True,
+                            description="complex A = -1/2 + n i at the Mamba-130M layer shape, bf16 I/O"),
 }
 
 
@@ -117,8 +121,12 @@ def make_inputs(w: Workload) -> dict:
         x["dout"] = _normal(rng, big, w.io)
     dt = np.exp(log_dt)
     x["delta_bias"] = np.log(np.expm1(dt)).astype(np.float32)
-    x["A"] = np.ascontiguousarray(
-        np.broadcast_to(-(np.arange(w.dstate, dtype=np.float32) + 1.0), (w.dim, w.dstate)))
+    if w.complex_a:
+        x["A"] = np.ascontiguousarray(np.broadcast_to(
+            (-0.5 + 1j * np.arange(w.dstate)).astype(np.complex64), (w.dim, w.dstate)))
+    else:
+        x["A"] = np.ascontiguousarray(
+            np.broadcast_to(-(np.arange(w.dstate, dtype=np.float32) + 1.0), (w.dim, w.dstate)))
     if w.decode:
         x["state"] = rng.standard_normal((w.batch, w.dim, w.dstate), dtype=np.float32)
     if not w.gate:
@@ -128,10 +136,10 @@ def make_inputs(w: Workload) -> dict:
 
 def small_case(batch: int, seqlen: int, dim: int, dstate: int, io: str = "f32", seed: int = 0,
                dt_min: float = 1e-3, dt_max: float = 1e-1, dskip: str = "normal",
-               backward: bool = False) -> dict:
+               backward: bool = False, complex_a: bool = False) -> dict:
     """Inputs of any shape drawn with the same recipe (for tails and edge cases)."""
     return make_inputs(Workload("custom", batch, seqlen, dim, dstate, io, dt_min, dt_max,
-                                dskip, seed, backward=backward))
+                                dskip, seed, backward=backward, complex_a=complex_a))
 
 
 def to_device(x: dict, device) -> dict:

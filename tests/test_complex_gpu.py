@@ -1,0 +1,94 @@
+"""sscan_fwd_complex (complex diagonal A, the -1/2 + n i initialisation of the A-init
+ablation table) against the fp64 oracle's complex scan, on the GPU."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_33_b200 import binding as sb
+from selective_state_space_33_b200 import workloads as W
+
+from .helpers import TOL, normwise, to_f64, to_torch
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(x, io, dev, h0=None, A=None):
+    t = to_torch(x, dev)
+    A_np = x["A"] if A is None else A
+    A_t = torch.from_numpy(np.ascontiguousarray(A_np.astype(np.complex64))).to(dev)
+    h0_t = None if h0 is None else torch.from_numpy(h0.astype(np.complex64)).to(dev)
+    out, h_last = sb.sscan_fwd_complex(t["u"], t["delta_raw"], A_t, t["B"], t["C"], t["delta_bias"], t["D_skip"],
+                                       t.get("z"), h0_t, return_last_state=True)
+    torch.cuda.synchronize()
+    ref, ref_h = oracle.fwd_complex(x["u"], x["delta_raw"], A_np.astype(np.complex64).astype(np.complex128),
+                                    x["B"], x["C"], delta_bias=x["delta_bias"], D_skip=x["D_skip"], z=x.get("z"),
+                                    h0=None if h0 is None else h0.astype(np.complex64).astype(np.complex128))
+    e_out = normwise(to_f64(out), ref)
+    hl = h_last.detach().cpu().numpy().astype(np.complex128)
+    e_h = float(np.max(np.abs(hl - ref_h)) / max(np.max(np.abs(ref_h)), 1e-300))
+    return e_out, e_h
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 100, 37, 16), (1, 257, 8, 4), (3, 33, 5, 1), (2, 64, 40, 7),
+                                   (1, 40, 130, 16)])
+def test_complex_shapes_and_tails(cuda_device, io, shape):
+    x = W.small_case(*shape, io=io, seed=sum(shape) + 5, complex_a=True)
+    h0 = np.random.default_rng(3).standard_normal((shape[0], shape[2], shape[3], 2)) @ np.array([1.0, 1j]) * 0.5
+    e_out, e_h = _run(x, io, cuda_device, h0=h0)
+    assert e_out <= TOL[io], e_out
+    assert e_h <= 1e-4, e_h
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_complex_general_A_values(cuda_device, io):
+    """Random complex A with large angles, a zero and tiny entries: the channel block holding
+    the small ones takes the series form, the others the fast form."""
+    x = W.small_case(2, 80, 64, 16, io=io, seed=71, complex_a=True)
+    rng = np.random.default_rng(71)
+    A = (-np.exp(rng.uniform(-3, 2, size=(64, 16))) + 1j * rng.uniform(-40, 40, size=(64, 16)))
+    A[0, 0] = 0.0
+    A[1, 3] = 1e-5 - 2e-5j
+    A[40, 2] = -3e-2 + 1e-2j  # small delta*a, but the block takes the fast form
+    e_out, e_h = _run(x, io, cuda_device, A=A)
+    assert e_out <= TOL[io], e_out
+    assert e_h <= 1e-4, e_h
+
+
+def test_complex_with_zero_imaginary_part_matches_the_real_kernel(cuda_device):
+    x = W.small_case(2, 300, 64, 16, io="f32", seed=72)
+    t = to_torch(x, cuda_device)
+    real_out = sb.sscan_fwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["delta_bias"], t["D_skip"], t["z"])
+    A_c = torch.complex(t["A"], torch.zeros_like(t["A"]))
+    cplx_out = sb.sscan_fwd_complex(t["u"], t["delta_raw"], A_c, t["B"], t["C"], t["delta_bias"], t["D_skip"],
+                                    t["z"])
+    torch.cuda.synchronize()
+    assert normwise(to_f64(cplx_out), to_f64(real_out)) <= 1e-5
+
+
+def test_complex130m_sampled(cuda_device):
+    """The benchmark's workload (batch 8, L 2048, D 1536, N 16) in one launch; the first
+    batch element is checked against the oracle."""
+    w = W.WORKLOADS["complex130m"]
+    x = W.make_inputs(w)
+    t = to_torch(x, cuda_device)
+    out, h_last = sb.sscan_fwd_complex(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["delta_bias"],
+                                       t["D_skip"], t["z"], return_last_state=True)
+    torch.cuda.synchronize()
+    one = {k: (v[:1] if k in ("u", "delta_raw", "z", "B", "C") else v) for k, v in x.items()}
+    ref, ref_h = oracle.fwd_complex(one["u"], one["delta_raw"], x["A"].astype(np.complex128), one["B"], one["C"],
+                                    delta_bias=x["delta_bias"], D_skip=x["D_skip"], z=one["z"])
+    assert normwise(to_f64(out[:1]), ref) <= TOL["bf16"]
+    hl = h_last[:1].cpu().numpy().astype(np.complex128)
+    assert np.max(np.abs(hl - ref_h)) / np.max(np.abs(ref_h)) <= 1e-4
+
+
+def test_complex_rejects_bad_A(cuda_device):
+    x = W.small_case(1, 16, 8, 4, io="f32", seed=73, complex_a=True)
+    t = to_torch(x, cuda_device)
+    with pytest.raises((TypeError, ValueError)):
+        sb.sscan_fwd_complex(t["u"], t["delta_raw"], torch.zeros(8, 4, device=cuda_device), t["B"], t["C"])
+    with pytest.raises((TypeError, ValueError)):
+        sb.sscan_fwd_complex(t["u"], t["delta_raw"], torch.zeros(8, 5, dtype=torch.complex64, device=cuda_device),
+                             t["B"], t["C"])
