@@ -6,8 +6,8 @@
 // SiLU(z) (Fig. 3).
 //
 // Work decomposition (as the real tiled kernel): a CTA of 4 warps owns one batch
-// and DC channels for the whole sequence; the NG = ceil(N/4) lanes of a channel
-// each hold 4 complex states (8 fp32) in registers.  Per 16-step tile all threads
+// and DC channels for the whole sequence; the NG lanes of a channel each hold CG
+// complex states (CG = 4, or 2 when the grid is small) in registers.  Per 16-step tile all threads
 // stage (delta, x) and (gate, D x gate) for the tile's channels and the tile's B
 // and C rows in shared memory with coalesced loads (phase P), then every lane
 // advances its states through the tile (phase S) and the NG lanes of a channel
@@ -26,6 +26,7 @@
 
 #include "sscan_launch.h"
 #include "sscan_math.cuh"
+#include "sscan_plan.h"
 
 namespace sscan {
 namespace {
@@ -33,7 +34,6 @@ namespace {
 constexpr int kCTT = 16;           // steps per tile
 constexpr int kCWarps = 4;
 constexpr int kCThreads = kCWarps * 32;
-constexpr int kCG = 4;             // complex states per lane
 constexpr float kCSmallA = 9.765625e-4f;
 constexpr float kTwoPiHi = 6.28318548202514648f;   // fp32 nearest to 2 pi
 constexpr float kTwoPiLo = -1.7484556e-7f;         // 2 pi - kTwoPiHi
@@ -58,27 +58,27 @@ __device__ __forceinline__ float2 cis(float th) {
     return make_float2(cos_approx(r), sin_approx(r));
 }
 
-template <int NG>
+template <int NG, int CG>
 struct CCfg {
     static constexpr int CW = 32 / NG;       // channels per warp
     static constexpr int DC = CW * kCWarps;  // channels per CTA
-    static constexpr int NS = NG * kCG;      // states covered (>= N)
+    static constexpr int NS = NG * CG;       // states covered (>= N)
 };
 
-template <typename T, int NG, bool ACC>
-__device__ __forceinline__ void scan_tile_c(float2 (&h)[kCG], const float2 (&aq)[kCG], const float2 (&nia)[kCG],
-                                            const float2 (&ia)[kCG], const float2* sdx, const float2* sgd,
+template <typename T, int NG, int CG, bool ACC>
+__device__ __forceinline__ void scan_tile_c(float2 (&h)[CG], const float2 (&aq)[CG], const float2 (&nia)[CG],
+                                            const float2 (&ia)[CG], const float2* sdx, const float2* sgd,
                                             const float* sB, const float* sC, int tl, int g, int cw, bool write,
                                             T* out, int64_t out_stride) {
-    using C = CCfg<NG>;
+    using C = CCfg<NG, CG>;
     for (int t = 0; t < tl; ++t) {
         const float2 dx = sdx[t * C::DC + cw];  // (delta, x)
         const float delta = dx.x, x = dx.y;
-        const float* Bt = sB + t * C::NS + g * kCG;
-        const float* Ct = sC + t * C::NS + g * kCG;
+        const float* Bt = sB + t * C::NS + g * CG;
+        const float* Ct = sC + t * C::NS + g * CG;
         float y = 0.f;
 #pragma unroll
-        for (int j = 0; j < kCG; ++j) {
+        for (int j = 0; j < CG; ++j) {
             const float e = ex2(delta * aq[j].x);
             const float2 cs = cis(delta * aq[j].y);
             const float abr = e * cs.x, abi = e * cs.y;
@@ -126,9 +126,9 @@ __device__ __forceinline__ void scan_tile_c(float2 (&h)[kCG], const float2 (&aq)
     }
 }
 
-template <typename T, int NG>
+template <typename T, int NG, int CG>
 __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a) {
-    using C = CCfg<NG>;
+    using C = CCfg<NG, CG>;
     __shared__ float2 sdx[kCTT * C::DC];  // (delta, x)
     __shared__ float2 sgd[kCTT * C::DC];  // (gate, D x gate)
     __shared__ float sB[kCTT * C::NS], sC[kCTT * C::NS];
@@ -146,11 +146,11 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a) {
     const int g = lane / C::CW, c = lane % C::CW, cw = warp * C::CW + c;
     const int64_t d = d0 + cw;
     const bool cvalid = d < a.D;
-    float2 h[kCG], aq[kCG], nia[kCG], ia[kCG];
+    float2 h[CG], aq[CG], nia[CG], ia[CG];
     bool small_a = false;
 #pragma unroll
-    for (int j = 0; j < kCG; ++j) {
-        const int n = g * kCG + j;
+    for (int j = 0; j < CG; ++j) {
+        const int n = g * CG + j;
         const bool ok = cvalid && n < N;
         const float ar = ok ? __ldg(a.A + (d * N + n) * 2) : -1.f;
         const float ai = ok ? __ldg(a.A + (d * N + n) * 2 + 1) : 0.f;
@@ -199,15 +199,15 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a) {
         __syncthreads();
         T* out = static_cast<T*>(a.out) + (b * a.L + t0) * a.D + d;
         if (acc)
-            scan_tile_c<T, NG, true>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, cvalid, out, a.D);
+            scan_tile_c<T, NG, CG, true>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, cvalid, out, a.D);
         else
-            scan_tile_c<T, NG, false>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, cvalid, out, a.D);
+            scan_tile_c<T, NG, CG, false>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, cvalid, out, a.D);
         __syncthreads();
     }
     if (a.h_last && cvalid) {
 #pragma unroll
-        for (int j = 0; j < kCG; ++j) {
-            const int n = g * kCG + j;
+        for (int j = 0; j < CG; ++j) {
+            const int n = g * CG + j;
             if (n < N) {
                 a.h_last[((b * a.D + d) * N + n) * 2] = h[j].x;
                 a.h_last[((b * a.D + d) * N + n) * 2 + 1] = h[j].y;
@@ -216,18 +216,30 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a) {
     }
 }
 
-template <typename T, int NG>
+template <typename T, int NG, int CG>
 cudaError_t launch_c(const ComplexArgs& a, cudaStream_t st) {
-    const int64_t blocks = a.batch * ((a.D + CCfg<NG>::DC - 1) / CCfg<NG>::DC);
-    if (blocks > 0) fwd_complex_kernel<T, NG><<<(unsigned)blocks, kCThreads, 0, st>>>(a);
+    const int64_t blocks = a.batch * ((a.D + CCfg<NG, CG>::DC - 1) / CCfg<NG, CG>::DC);
+    if (blocks > 0) fwd_complex_kernel<T, NG, CG><<<(unsigned)blocks, kCThreads, 0, st>>>(a);
     return cudaGetLastError();
 }
 
+// Four complex states per lane, or two (twice the lanes per channel, half the
+// channels per CTA) when the four-state grid would leave the GPU short of CTAs:
+// measured at batch 8, L 2048, N 16: D 1536 0.90 ms with two states against 1.08 ms
+// with four; D 5120 2.34 ms with four against 2.37 ms with two.
 template <typename T>
 cudaError_t launch_ct(const ComplexArgs& a, cudaStream_t st) {
-    if (a.N <= 4) return launch_c<T, 1>(a, st);
-    if (a.N <= 8) return launch_c<T, 2>(a, st);
-    return launch_c<T, 4>(a, st);
+    const int64_t ng4 = a.N <= 4 ? 1 : (a.N <= 8 ? 2 : 4);
+    const int64_t ctas4 = a.batch * ((a.D + 4 * (32 / ng4) - 1) / (4 * (32 / ng4)));
+    if (ctas4 < 4 * (int64_t)kSmCount) {
+        if (a.N <= 2) return launch_c<T, 1, 2>(a, st);
+        if (a.N <= 4) return launch_c<T, 2, 2>(a, st);
+        if (a.N <= 8) return launch_c<T, 4, 2>(a, st);
+        return launch_c<T, 8, 2>(a, st);
+    }
+    if (a.N <= 4) return launch_c<T, 1, 4>(a, st);
+    if (a.N <= 8) return launch_c<T, 2, 4>(a, st);
+    return launch_c<T, 4, 4>(a, st);
 }
 
 }  // namespace

@@ -201,9 +201,70 @@ __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int 
     }
 }
 
+// Full tiles of the fast form with outputs, software-pipelined: the exponentials and
+// the v terms of step t+1 are issued before the state update of step t, so the MUFU
+// latency of one step overlaps the dependent fmas of the previous one (measured
+// 0.633 -> 0.620 ms at the 2.8B-layer shape, bf16; identical results).
+template <int G>
+struct Prep { float2 a[G / 2]; float2 v[G / 2]; };
+
+template <int G>
+__device__ __forceinline__ Prep<G> prep_step(const LaneG<G>& s, float4 dx, const float* Bp) {
+    Prep<G> P;
+    const float2 dd = f2(dx.x, dx.y), xx = f2(dx.z, dx.w);
+#pragma unroll
+    for (int k = 0; k < G / 2; ++k) {
+        P.a[k] = ex2x2(__fmul2_rn(dd, s.A2[k]));
+        P.v[k] = __fmul2_rn(reinterpret_cast<const float2*>(Bp)[k], __fmul2_rn(xx, s.niA[k]));
+    }
+    return P;
+}
+
+template <int G>
+__device__ __forceinline__ float upd_step(LaneG<G>& s, const Prep<G>& P, const float* Cp) {
+    float2 y = f2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < G / 2; ++k) {
+        s.h[k] = __ffma2_rn(P.a[k], __ffma2_rn(P.v[k], f2(-1.f, -1.f), s.h[k]), P.v[k]);
+        y = __ffma2_rn(reinterpret_cast<const float2*>(Cp)[k], s.h[k], y);
+    }
+    return y.x + y.y;
+}
+
+template <typename T, int NG, int G>
+__device__ __forceinline__ void scan_tile_pipe(LaneG<G>& s, unsigned char* smem, int g, int cw, T* sout) {
+    using C = Cfg<T, NG, G>;
+    const float4* sdx = reinterpret_cast<const float4*>(smem + C::OFF_DX) + cw;
+    const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
+    const float* sB = reinterpret_cast<const float*>(smem + C::OFF_B) + g * G;
+    const float* sC = reinterpret_cast<const float*>(smem + C::OFF_C) + g * G;
+    Prep<G> P = prep_step<G>(s, sdx[0], sB);
+#pragma unroll
+    for (int tb = 0; tb < kTT; tb += NG) {
+        float p[NG];
+#pragma unroll
+        for (int k = 0; k < NG; ++k) {
+            const int t = tb + k;
+            Prep<G> Pn = P;
+            if (t + 1 < kTT) Pn = prep_step<G>(s, sdx[(t + 1) * C::DC], sB + (t + 1) * C::NS);
+            p[k] = upd_step<G>(s, P, sC + t * C::NS);
+            P = Pn;
+        }
+        const float y = transpose_reduce<NG, C::CW>(p, g);
+        const int t = tb + g;
+        const float2 gd = sgd[t * C::GD_PITCH];
+        sout[t * C::DC + cw] = from_f32<T>(fmaf(y, gd.x, gd.y));
+    }
+}
 template <typename T, int NG, int G, int MODE, bool ACC>
 __device__ __forceinline__ void scan_tile_any(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
                                               float& dsum, float* ck, int64_t ck_stride, int nvalid) {
+    if constexpr (MODE == kOut && !ACC) {
+        if (tile_len == kTT) {
+            scan_tile_pipe<T, NG, G>(s, smem, g, cw, sout);
+            return;
+        }
+    }
     if (tile_len == kTT)
         scan_tile<T, NG, G, MODE, ACC, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid);
     else

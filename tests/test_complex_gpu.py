@@ -42,6 +42,16 @@ def test_complex_shapes_and_tails(cuda_device, io, shape):
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_complex_large_grid_geometry(cuda_device, io):
+    """Enough (batch, channel-block) CTAs that the kernel keeps four complex states per
+    lane (small grids take two): both geometries must match the oracle."""
+    x = W.small_case(20, 40, 1024, 16, io=io, seed=74, complex_a=True)
+    e_out, e_h = _run(x, io, cuda_device)
+    assert e_out <= TOL[io], e_out
+    assert e_h <= 1e-4, e_h
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_complex_general_A_values(cuda_device, io):
     """Random complex A with large angles, a zero and tiny entries: the channel block holding
     the small ones takes the series form, the others the fast form."""
