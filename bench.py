@@ -114,17 +114,21 @@ def roofline_units(w: W.Workload) -> dict:
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of each
 # workload's dominant kernel, read from one ncu capture of that workload (summaries
 # under profiles/).  A figure holds only for the kernel source it was taken on: it is
-# keyed by the SHA-256 of those source files and reported as null once they change.
+# keyed by the SHA-256 of those source files (with comments and blank lines removed,
+# so that only code counts) and reported as null once the code changes.
 NCU_TRAFFIC = {
-    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 504947968 + 151214848,
-                  "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "70a9ef22462fd8b3",
+    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 505026048 + 150930176,
+                  "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "0bc36e87ea5e1afc",
                   "profile": "profiles/fwd_tiled_kernel_mamba2.8b_bf16.md"},
-    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410339840 + 134322688,
-                "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "fcc0aaaa58a1c74e",
+    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410256640 + 133296640,
+                "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "9d2486f634d56827",
                 "profile": "profiles/bwd_tiled_kernel_bwd130m_bf16.md"},
     "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317504 + 0,
-                   "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "3f0237a88da992b3",
+                   "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "b7c6e53d71a0bd30",
                    "profile": "profiles/step_quad_kernel_decode2.8b_bf16.md"},
+    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152287488 + 32752640,
+                    "sources": ("sscan_complex.cu", "sscan_math.cuh"), "sha256": "4a792ca9083060f5",
+                    "profile": "profiles/fwd_complex_kernel_complex130m_bf16.md"},
 }
 
 
@@ -140,9 +144,22 @@ def ncu_traffic(workload: str):
         path = os.path.join(ROOT, "selective_state_space_33_b200", "csrc", name)
         if not os.path.exists(path):
             return None
-        with open(path, "rb") as f:
-            h.update(f.read())
+        with open(path) as f:
+            h.update(code_only(f.read()).encode())
     return rec["bytes"] if h.hexdigest()[:16] == rec["sha256"] else None
+
+
+def code_only(src: str) -> str:
+    """C++/CUDA source without // comments, trailing spaces and blank lines."""
+    lines = []
+    for line in src.splitlines():
+        cut = line.find("//")
+        if cut >= 0 and line.count('"', 0, cut) % 2 == 0:
+            line = line[:cut]
+        line = line.rstrip()
+        if line:
+            lines.append(line)
+    return "\n".join(lines)
 
 
 def measured_peaks() -> dict:

@@ -21,7 +21,8 @@
 //
 // Modes: kOut writes out (and h_last from the last chunk), kAgg writes each
 // chunk's end state from zero plus its sum of delta (for the cross-chunk carry),
-// kLast writes only h_last.
+// kLast writes only h_last, kCkpt writes the state before every 8th step (the
+// backward pass's recomputation starting points).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -92,9 +93,9 @@ __device__ __forceinline__ float2 ex2x2(float2 q) { return f2(ex2(q.x), ex2(q.y)
 
 // One step for the lane's G states, eq. (2) and (3a).  With v = -B x / A the update
 // h' = Abar h + (Abar - 1) B x / A is Abar (h - v) + v: two packed fmas per pair
-// (h - v as fma(v, -1, h), exact), no negated operand.  dx = (delta, delta, x, x); Bp, Cp point at the
-// lane's G values of B_t, C_t.  Returns the partial readout sum_j C_j h_j over these
-// states (eq. (3b)).
+// (h - v as fma(v, -1, h), exact), no negated operand.  dx = (delta, delta, x, x);
+// Bp, Cp point at the lane's G values of B_t, C_t.  Returns the partial readout
+// sum_j C_j h_j over these states (eq. (3b)).
 template <int G, bool WANT_Y>
 __device__ __forceinline__ float step_fast(LaneG<G>& s, float4 dx, const float* Bp, const float* Cp) {
     const float2 dd = f2(dx.x, dx.y), xx = f2(dx.z, dx.w);
