@@ -29,8 +29,10 @@
  *
  * Ownership and execution: every pointer is a device pointer owned by the caller
  * (except `problem`, a host pointer read during the call).  The library never
- * allocates, frees or synchronises; it enqueues its kernels on `stream` (a
- * cudaStream_t, NULL = legacy default stream) and returns.  Outputs are
+ * allocates device memory, frees or synchronises; it enqueues its kernels on
+ * `stream` (a cudaStream_t, NULL = legacy default stream) and returns.  (The only
+ * CUDA objects it creates -- once per device, kept for the process -- are the
+ * auxiliary stream and two events of sscan_bwd, described there.)  Outputs are
  * overwritten, never accumulated into.  Inputs must not alias outputs.
  *
  * Errors: arguments are checked on the host before anything is launched; a
