@@ -41,6 +41,8 @@ def _load():
         lib.orc_bwd.restype = ctypes.c_int
         lib.orc_fwd_complex.argtypes = [ctypes.POINTER(_Problem)] + [vp] * 11
         lib.orc_fwd_complex.restype = ctypes.c_int
+        lib.orc_bwd_complex.argtypes = [ctypes.POINTER(_Problem)] + [vp] * 19
+        lib.orc_bwd_complex.restype = ctypes.c_int
         lib.orc_set_threads.argtypes = [ctypes.c_int]
         lib.orc_set_threads.restype = ctypes.c_int
         _lib = lib
@@ -182,4 +184,34 @@ def fwd_complex(u, delta_raw, A, B, C, *, delta_bias=None, D_skip=None, z=None, 
     return out, h_last[..., 0] + 1j * h_last[..., 1]
 
 
-__all__ = ["fwd", "bwd", "fwd_complex", "set_threads"]
+def bwd_complex(u, delta_raw, A, B, C, dout, *, delta_bias=None, D_skip=None, z=None, h0=None,
+                delta_softplus=True):
+    """Reverse-mode gradients of sum(out * dout) for the complex-A scan, fp64.
+    dA (D, N) and dh0 (batch, D, N) are complex128 (dL/dRe + i dL/dIm); the rest real,
+    keyed as in ``bwd``."""
+    (u, delta_raw, B, C, dout, z), code = _ios(u, delta_raw, B, C, dout, z)
+    batch, L, D = u.shape
+    N = B.shape[-1]
+    A2 = _interleave(A, (D, N))
+    h02 = _interleave(h0, (batch, D, N))
+    delta_bias, D_skip = _f64(delta_bias), _f64(D_skip)
+    g = {"du": np.empty((batch, L, D)), "ddelta_raw": np.empty((batch, L, D)),
+         "dA": np.empty((D, N, 2)), "dB": np.empty((batch, L, N)), "dC": np.empty((batch, L, N)),
+         "dh0": np.empty((batch, D, N, 2))}
+    g["ddelta_bias"] = np.empty(D) if delta_bias is not None else None
+    g["dD"] = np.empty(D) if D_skip is not None else None
+    g["dz"] = np.empty((batch, L, D)) if z is not None else None
+    prob = _Problem(batch, L, D, N, code, 1 if delta_softplus else 0)
+    rc = _load().orc_bwd_complex(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias), _ptr(A2),
+                                 _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h02), _ptr(dout),
+                                 _ptr(g["du"]), _ptr(g["ddelta_raw"]), _ptr(g["ddelta_bias"]),
+                                 _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]),
+                                 _ptr(g["dz"]), _ptr(g["dh0"]))
+    if rc != 0:
+        raise ValueError("orc_bwd_complex rejected its arguments")
+    g["dA"] = g["dA"][..., 0] + 1j * g["dA"][..., 1]
+    g["dh0"] = g["dh0"][..., 0] + 1j * g["dh0"][..., 1]
+    return {k: v for k, v in g.items() if v is not None}
+
+
+__all__ = ["fwd", "bwd", "fwd_complex", "bwd_complex", "set_threads"]

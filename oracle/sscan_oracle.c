@@ -34,6 +34,7 @@
  * float32 or bfloat16 are widened exactly.  No blocking, fusion or reordering:
  * each (batch, channel) row is a plain loop over t and n.
  */
+#include <complex.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -379,6 +380,136 @@ int orc_fwd_complex(const orc_problem* p, const void* u, const void* delta_raw,
                 h_last[(row * N + n) * 2 + 1] = hi[n];
             }
         free(hr);
+    }
+    return bad;
+}
+
+/* exp(q) - 1 for complex q without the cancellation of e^x cos y - 1 near 0. */
+static double complex cexpm1_(double complex q)
+{
+    const double x = creal(q), y = cimag(q), sh = sin(0.5 * y);
+    return (expm1(x) * cos(y) - 2.0 * sh * sh) + I * (exp(x) * sin(y));
+}
+
+/* psi(q) = (q e^q - (e^q - 1)) / q^2 for complex q (the derivative of (e^q - 1)/q);
+ * its Taylor series 1/2 + q/3 + q^2/8 + q^3/30 + q^4/144 near 0. */
+static double complex cpsi(double complex q)
+{
+    if (cabs(q) < 1e-3)
+        return 0.5 + q * (1.0 / 3.0 + q * (1.0 / 8.0 + q * (1.0 / 30.0 + q * (1.0 / 144.0))));
+    return (q * cexp(q) - cexpm1_(q)) / (q * q);
+}
+
+/*
+ * Reverse-mode gradient of orc_fwd_complex's `out` (all rows), by hand.  The
+ * complex state is a pair of real variables, so the adjoint lam = dL/dRe h +
+ * i dL/dIm h; multiplying h by Abar maps the adjoint by conj(Abar):
+ *   lam_t = C_t dy_t + conj(Abar_{t+1}) lam_{t+1}        (C dy is real)
+ * and for any real parameter p entering h_t through dh/dp, dL/dp += Re(conj(lam) dh/dp):
+ *   dx    += Re(conj(lam) beta) B,   dB += Re(conj(lam) beta) x,   dC += dy Re(h_t)
+ *   d delta += Re(conj(lam) (a Abar h_{t-1} + Abar B x))     (d beta/d delta = Abar)
+ *   dA   : h is holomorphic in a, so with g = conj(lam) (delta Abar h_{t-1} + delta^2
+ *          psi(delta a) B x):  dA_re += Re(g),  dA_im += -Im(g)
+ *   dh0 = conj(Abar_0) lam_0.
+ * A, dA, h0, dh0 are (re, im) interleaved like orc_fwd_complex; the other outputs
+ * as orc_bwd (ddelta_bias, dD, dz, dh0 may be NULL).
+ */
+int orc_bwd_complex(const orc_problem* p, const void* u, const void* delta_raw,
+                    const double* delta_bias, const double* A, const void* B,
+                    const void* C, const double* D_skip, const void* z,
+                    const double* h0, const void* dout, double* du,
+                    double* ddelta_raw, double* ddelta_bias, double* dA, double* dB,
+                    double* dC, double* dD, double* dz, double* dh0)
+{
+    if (check(p) || !u || !delta_raw || !A || !B || !C || !dout || !du || !ddelta_raw || !dA || !dB || !dC)
+        return 1;
+    const int64_t Bt = p->batch, L = p->seqlen, D = p->dim, N = p->dstate;
+    const int32_t dt = p->io_dtype;
+    memset(dA, 0, (size_t)(D * N * 2) * sizeof(double));
+    memset(dB, 0, (size_t)(Bt * L * N) * sizeof(double));
+    memset(dC, 0, (size_t)(Bt * L * N) * sizeof(double));
+    if (ddelta_bias) memset(ddelta_bias, 0, (size_t)D * sizeof(double));
+    if (dD) memset(dD, 0, (size_t)D * sizeof(double));
+    int bad = 0;
+    /* rows are independent except for the sums over (batch, channel) -- dA, dB, dC,
+     * dbias, dD -- so rows run sequentially here (plain, not fast) */
+    for (int64_t row = 0; row < Bt * D && !bad; ++row) {
+        const int64_t b = row / D, d = row % D;
+        double complex* h = (double complex*)malloc((size_t)((L + 1) * N) * sizeof(double complex));
+        double complex* lam = (double complex*)malloc((size_t)N * sizeof(double complex));
+        if (!h || !lam) {
+            free(h);
+            free(lam);
+            bad = 1;
+            break;
+        }
+        /* forward, keeping every state: h[(t+1)*N + n] = h_t, h[n] = h_{-1} = h0 */
+        for (int64_t n = 0; n < N; ++n)
+            h[n] = h0 ? h0[(row * N + n) * 2] + I * h0[(row * N + n) * 2 + 1] : 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t e = (b * L + t) * D + d, s = (b * L + t) * N;
+            const double x = ld(u, dt, e);
+            const double r = ld(delta_raw, dt, e) + (delta_bias ? delta_bias[d] : 0.0);
+            const double delta = p->delta_softplus ? softplus(r) : r;
+            for (int64_t n = 0; n < N; ++n) {
+                const double complex a = A[(d * N + n) * 2] + I * A[(d * N + n) * 2 + 1];
+                const double complex abar = cexp(delta * a);
+                const double complex beta = (a == 0.0) ? delta : cexpm1_(delta * a) / a;
+                h[(t + 1) * N + n] = abar * h[t * N + n] + beta * ld(B, dt, s + n) * x;
+            }
+        }
+        /* reverse */
+        for (int64_t n = 0; n < N; ++n) lam[n] = 0.0;
+        double dDacc = 0.0, dbacc = 0.0;
+        for (int64_t t = L - 1; t >= 0; --t) {
+            const int64_t e = (b * L + t) * D + d, s = (b * L + t) * N;
+            const double x = ld(u, dt, e);
+            const double r = ld(delta_raw, dt, e) + (delta_bias ? delta_bias[d] : 0.0);
+            const double delta = p->delta_softplus ? softplus(r) : r;
+            const double go = ld(dout, dt, e);
+            double dy = go;
+            if (z) {
+                double y = D_skip ? D_skip[d] * x : 0.0;
+                for (int64_t n = 0; n < N; ++n) y += ld(C, dt, s + n) * creal(h[(t + 1) * N + n]);
+                const double zz = ld(z, dt, e), sg = sigmoid(zz);
+                dy = go * zz * sg;
+                if (dz) dz[e] = go * y * sg * (1.0 + zz * (1.0 - sg));
+            }
+            double dx = D_skip ? D_skip[d] * dy : 0.0;
+            dDacc += dy * x;
+            double ddelta = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                const double complex a = A[(d * N + n) * 2] + I * A[(d * N + n) * 2 + 1];
+                const double complex q = delta * a;
+                const double complex abar = cexp(q);
+                const double complex beta = (a == 0.0) ? delta : cexpm1_(q) / a;
+                const double Bn = ld(B, dt, s + n), Cn = ld(C, dt, s + n);
+                const double complex l = Cn * dy + lam[n];
+                const double complex hp = h[t * N + n];
+                dC[s + n] += dy * creal(h[(t + 1) * N + n]);
+                const double lb = creal(conj(l) * beta);
+                dB[s + n] += lb * x;
+                dx += lb * Bn;
+                ddelta += creal(conj(l) * (a * abar * hp + abar * Bn * x));
+                const double complex g = conj(l) * (delta * abar * hp + delta * delta * cpsi(q) * Bn * x);
+                dA[(d * N + n) * 2] += creal(g);
+                dA[(d * N + n) * 2 + 1] -= cimag(g);
+                lam[n] = conj(abar) * l;
+            }
+            const double drr = p->delta_softplus ? ddelta * sigmoid(r) : ddelta;
+            du[e] = dx;
+            ddelta_raw[e] = drr;
+            dbacc += drr;
+        }
+        for (int64_t n = 0; n < N; ++n)
+            if (dh0) {
+                dh0[(row * N + n) * 2] = creal(lam[n]);
+                dh0[(row * N + n) * 2 + 1] = cimag(lam[n]);
+            }
+        if (dD) dD[d] += dDacc;
+        if (ddelta_bias) ddelta_bias[d] += dbacc;
+        free(h);
+        free(lam);
     }
     return bad;
 }

@@ -4,7 +4,9 @@ summary page), each against something other than the oracle itself: the real
 oracle in the Im(A) = 0 special case, a brute-force convolution with complex powers
 (eq. 4), a numerical integration of the continuous system (eq. 1, which pins the
 discretisation eq. 2), the continuous step response, exact splitting with a carried
-state, linearity and causality.  CPU only.
+state, linearity and causality; and for its backward, central finite differences of
+every input (real and imaginary parts of A and h0 separately), the real backward in
+the Im(A) = 0 case, and the adjoint identity.  CPU only.
 """
 import numpy as np
 import pytest
@@ -134,3 +136,99 @@ def test_linearity_and_causality():
     up[:, 20, :] += 4.0
     op, _ = f(up, g1)
     assert np.array_equal(op[:, :20], o1[:, :20]) and not np.allclose(op[:, 20:], o1[:, 20:])
+
+
+# ---------------------------------------------------------------- backward
+def _bwd_case(seed):
+    """Small case with every optional input, complex A and h0, in float64."""
+    x = W.small_case(1, 24, 3, 3, io="f32", seed=seed, backward=True, complex_a=True)
+    rng = np.random.default_rng(200 + seed)
+    p = {k: x[k].astype(np.float64) for k in ("u", "delta_raw", "z", "B", "C", "delta_bias", "D_skip")}
+    p["A"] = _complex_A(3, 3, 300 + seed)
+    p["h0"] = (rng.standard_normal((1, 3, 3)) + 1j * rng.standard_normal((1, 3, 3))) * 0.5
+    dout = rng.standard_normal((1, 24, 3))
+    return p, dout
+
+
+def _closs(p, dout):
+    out, _ = oracle.fwd_complex(p["u"], p["delta_raw"], p["A"], p["B"], p["C"], delta_bias=p["delta_bias"],
+                                D_skip=p["D_skip"], z=p["z"], h0=p["h0"])
+    return float(np.sum(out * dout))
+
+
+def _cgrads(p, dout):
+    return oracle.bwd_complex(p["u"], p["delta_raw"], p["A"], p["B"], p["C"], dout, delta_bias=p["delta_bias"],
+                              D_skip=p["D_skip"], z=p["z"], h0=p["h0"])
+
+
+def test_complex_backward_matches_central_differences():
+    p, dout = _bwd_case(0)
+    g = _cgrads(p, dout)
+    names = {"u": "du", "delta_raw": "ddelta_raw", "z": "dz", "B": "dB", "C": "dC", "delta_bias": "ddelta_bias",
+             "D_skip": "dD", "A": "dA", "h0": "dh0"}
+    for pn, gn in names.items():
+        arr = p[pn]
+        parts = [(1.0, np.real)] + ([(1j, np.imag)] if np.iscomplexobj(arr) else [])
+        for unit, take in parts:
+            fd = np.empty(arr.shape)
+            for idx in np.ndindex(arr.shape):
+                v = arr[idx]
+                step = 1e-6 * max(1.0, abs(v))
+                arr[idx] = v + unit * step
+                lp = _closs(p, dout)
+                arr[idx] = v - unit * step
+                lm = _closs(p, dout)
+                arr[idx] = v
+                fd[idx] = (lp - lm) / (2 * step)
+            ref = take(g[gn]) if np.iscomplexobj(g[gn]) else g[gn]
+            err = np.max(np.abs(fd - ref)) / max(np.max(np.abs(ref)), 1e-300)
+            assert err < 1e-6, (pn, take.__name__, err)
+
+
+def test_complex_backward_with_zero_imaginary_part_is_the_real_backward():
+    x = W.small_case(2, 30, 4, 3, io="f32", seed=31, backward=True)
+    A = x["A"].astype(np.float64)
+    A[1, 1] = 0.0
+    h0 = np.random.default_rng(32).standard_normal((2, 4, 3))
+    kw = dict(delta_bias=x["delta_bias"], D_skip=x["D_skip"], z=x["z"])
+    gr = oracle.bwd(x["u"], x["delta_raw"], A, x["B"], x["C"], x["dout"], h0=h0, **kw)
+    gc = oracle.bwd_complex(x["u"], x["delta_raw"], A + 0j, x["B"], x["C"], x["dout"], h0=h0 + 0j, **kw)
+    for k in gr:
+        got = gc[k].real if np.iscomplexobj(gc[k]) else gc[k]
+        np.testing.assert_allclose(got, gr[k], rtol=1e-9, atol=1e-11, err_msg=k)
+
+
+def test_complex_backward_adjoint_identity():
+    p, dout = _bwd_case(1)
+    g = _cgrads(p, dout)
+    rng = np.random.default_rng(9)
+    names = {"u": "du", "delta_raw": "ddelta_raw", "z": "dz", "B": "dB", "C": "dC", "delta_bias": "ddelta_bias",
+             "D_skip": "dD", "A": "dA", "h0": "dh0"}
+    v = {k: (rng.standard_normal(p[k].shape) + (1j * rng.standard_normal(p[k].shape) if np.iscomplexobj(p[k])
+                                                else 0.0)) for k in names}
+    eps = 1e-6
+    plus = {k: p[k] + eps * v[k] for k in p}
+    minus = {k: p[k] - eps * v[k] for k in p}
+    jvp = (_closs(plus, dout) - _closs(minus, dout)) / (2 * eps)
+    # for complex parameters, <grad, v> pairs the real parts and the imaginary parts
+    vjp = sum(float(np.sum(np.real(g[gn]) * np.real(v[pn]) + np.imag(g[gn]) * np.imag(v[pn])))
+              for pn, gn in names.items())
+    assert abs(jvp - vjp) <= 1e-7 * max(1.0, abs(vjp))
+
+
+@pytest.mark.parametrize("delta,a", [(1e-3, -0.5 + 0.3j), (2e-4, -0.5 + 2.0j), (0.05, -0.01 + 0.01j),
+                                     (0.7, -0.5 + 4.0j), (1e-6, -3.0 + 1.0j)])
+def test_complex_single_step_gradient_against_mpmath(delta, a):
+    """L = 1, N = 1, h0 = 0, no skip, no gate, softplus off: the A-gradient of one step is
+    dout C B x delta^2 conj(psi(delta a)) with psi(q) = (q e^q - (e^q - 1)) / q^2, here
+    evaluated in 50-digit arithmetic (mpmath), small q included."""
+    import mpmath
+    mpmath.mp.dps = 50
+    q = mpmath.mpc(delta) * mpmath.mpc(a.real, a.imag)
+    psi = (q * mpmath.exp(q) - mpmath.expm1(q)) / (q * q)
+    B, C, x, go = 0.7, -1.3, 0.9, 1.1
+    g = oracle.bwd_complex(np.full((1, 1, 1), x), np.full((1, 1, 1), delta), np.array([[a]]),
+                           np.full((1, 1, 1), B), np.full((1, 1, 1), C), np.full((1, 1, 1), go),
+                           delta_softplus=False)
+    ref = go * C * B * x * delta * delta * complex(mpmath.conj(psi))
+    assert abs(g["dA"][0, 0] - ref) <= 1e-12 * abs(ref)

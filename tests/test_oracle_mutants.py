@@ -44,6 +44,12 @@ MUTANTS = {
     "complex_state_mix": ("const double ni = abr * hi[n] + abi * hr[n] + ci * bx;",
                           "const double ni = abr * hi[n] - abi * hr[n] + ci * bx;"),
     "complex_half_angle": ("- 2.0 * sh * sh, em1i", "- sh * sh, em1i"),
+    "complex_bwd_no_conj": ("lam[n] = conj(abar) * l;", "lam[n] = abar * l;"),
+    "complex_bwd_dA_imag_sign": ("dA[(d * N + n) * 2 + 1] -= cimag(g);", "dA[(d * N + n) * 2 + 1] += cimag(g);"),
+    "complex_bwd_psi_term": ("q * (1.0 / 8.0 + q * (1.0 / 30.0 + q * (1.0 / 144.0))));\n    return (q * cexp(q)",
+                             "q * (1.0 / 6.0 + q * (1.0 / 30.0 + q * (1.0 / 144.0))));\n    return (q * cexp(q)"),
+    "complex_bwd_ddelta_drop": ("ddelta += creal(conj(l) * (a * abar * hp + abar * Bn * x));",
+                                "ddelta += creal(conj(l) * (abar * Bn * x));"),
 }
 PIN_FILES = ["test_oracle_pins.py", "test_oracle_complex_pins.py"]
 
