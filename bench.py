@@ -31,6 +31,7 @@ METRIC = "selective-scan fwd Gelem/s (B·L·D) & % of HBM/MUFU roofline at 2.8B-
 METRIC_BWD = "selective-scan bwd Gelem/s (B·L·D), states recomputed on chip"
 METRIC_STEP = "selective-scan generation step Gelem/s (batch·D per token), state read and written in HBM"
 METRIC_COMPLEX = "selective-scan fwd with complex diagonal A, Gelem/s (B·L·D)"
+METRIC_COMPLEX_BWD = "selective-scan bwd with complex diagonal A, Gelem/s (B·L·D), states recomputed on chip"
 UNIT = "Gelem/s"
 DEFAULT_WORKLOAD = "mamba2.8b"
 SM_COUNT = 148
@@ -91,6 +92,12 @@ def roofline_units(w: W.Workload) -> dict:
     s = 2 if w.io == "bf16" else 4
     E = w.batch * w.seqlen * w.dim
     BLN = w.batch * w.seqlen * w.dstate
+    if w.complex_a and w.backward:
+        # complex backward: read u, delta_raw, z, dout, B, C; write du, ddelta_raw, dz and
+        # dB, dC; the checkpoint pass and the reverse kernel each take 2^x, cos and sin
+        # per state (the recomputation and the reverse step): 2 x 3 N + 4 MUFU operations.
+        bytes_ = 7 * E * s + 4 * BLN * s + 2 * (2 * w.dim * w.dstate + 2 * w.dim) * 4
+        return {"elements": E, "bytes": bytes_, "exps": E * (6 * w.dstate + 4)}
     if w.complex_a:
         # complex A: the same bytes (A is (D, N, 2) fp32); per state the MUFU computes
         # 2^(delta Re a), cos and sin of delta Im a: 3 N + 2 MUFU operations per element.
@@ -355,12 +362,13 @@ def gpu_arm(args, w: W.Workload):
     t = W.to_device(x, dev)
     out = torch.empty_like(t["u"])
     prob = sb.make_problem(w.batch, w.seqlen, w.dim, w.dstate, sb.SSCAN_BF16 if w.io == "bf16" else sb.SSCAN_F32)
-    op = sb.SSCAN_OP_BWD if w.backward else sb.SSCAN_OP_FWD
+    op = (sb.SSCAN_OP_BWD_COMPLEX if w.backward and w.complex_a else sb.SSCAN_OP_BWD if w.backward
+          else sb.SSCAN_OP_FWD)
     ws_bytes = sb.sscan_workspace_size(prob, op)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream()
     grads = None
-    if w.backward:
+    if w.backward and not w.complex_a:
         grads = sb.sscan_bwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t["delta_bias"],
                              t["D_skip"], t.get("z"), workspace=ws)
 
@@ -382,7 +390,10 @@ def gpu_arm(args, w: W.Workload):
     nstep = [0]
 
     def step(stream=st):
-        if w.complex_a:
+        if w.complex_a and w.backward:
+            sb.sscan_bwd_complex(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t["delta_bias"],
+                                 t["D_skip"], t.get("z"), workspace=ws, stream=stream)
+        elif w.complex_a:
             sb.sscan_fwd_complex(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["delta_bias"], t["D_skip"],
                                  t.get("z"), out=out, stream=stream)
         elif w.decode:
@@ -558,8 +569,8 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
                "single_thread": {"value": rate1, "unit": UNIT,
                                  "sample": f"{rows1} random rows x L={w.seqlen}, {secs1:.1f} s on 1 thread"}}
     line = {
-        "metric": (METRIC_BWD if w.backward else METRIC_STEP if w.decode else METRIC_COMPLEX if w.complex_a
-                   else METRIC), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": (METRIC_COMPLEX_BWD if w.backward and w.complex_a else METRIC_BWD if w.backward
+                   else METRIC_STEP if w.decode else METRIC_COMPLEX if w.complex_a else METRIC), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": max_s / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(w, world, l2_note),

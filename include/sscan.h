@@ -83,7 +83,8 @@ typedef enum sscan_op {
     SSCAN_OP_FWD = 0,
     SSCAN_OP_LAST_STATE = 1,
     SSCAN_OP_BWD = 2,
-    SSCAN_OP_SUMMARY = 3
+    SSCAN_OP_SUMMARY = 3,
+    SSCAN_OP_BWD_COMPLEX = 4
 } sscan_op;
 
 /* Bytes of device workspace the operation needs for this problem (0 when none).
@@ -221,6 +222,22 @@ SSCAN_API sscan_status sscan_fwd_complex(const sscan_problem* problem, const voi
                                          const float* delta_bias, const float* A, const void* B, const void* C,
                                          const float* D_skip, const void* z, const float* h0, void* out,
                                          float* h_last, void* stream);
+
+/*
+ * Backward of sscan_fwd_complex: gradients of sum(out * dout), the states
+ * recomputed on chip from checkpoints of every 8th step (sec. 4.1 item 3).  The
+ * gradient with respect to a complex quantity (dA, dh0) is the pair
+ * (dL/dRe, dL/dIm) in the same (re, im) layout as the quantity.  du, ddelta_raw, dB,
+ * dC, dz in io_dtype; dA (D, N, 2), ddelta_bias, dD, dh0 (batch, D, N, 2) fp32.
+ * NULL rules as sscan_bwd.  Workspace: sscan_workspace_size(problem,
+ * SSCAN_OP_BWD_COMPLEX) bytes (fp32 dB, dC accumulators and the checkpoints).
+ */
+SSCAN_API sscan_status sscan_bwd_complex(const sscan_problem* problem, const void* u, const void* delta_raw,
+                                         const float* delta_bias, const float* A, const void* B, const void* C,
+                                         const float* D_skip, const void* z, const float* h0, const void* dout,
+                                         void* du, void* ddelta_raw, float* ddelta_bias, float* dA, void* dB,
+                                         void* dC, float* dD, void* dz, float* dh0, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 
 /* Static, human-readable name of a status code. */
 SSCAN_API const char* sscan_status_string(sscan_status status);

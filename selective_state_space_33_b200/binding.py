@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libsscan.so")
 
 SSCAN_F32, SSCAN_BF16 = 0, 1
 SSCAN_DELTA_SOFTPLUS = 1
-SSCAN_OP_FWD, SSCAN_OP_LAST_STATE, SSCAN_OP_BWD, SSCAN_OP_SUMMARY = 0, 1, 2, 3
+SSCAN_OP_FWD, SSCAN_OP_LAST_STATE, SSCAN_OP_BWD, SSCAN_OP_SUMMARY, SSCAN_OP_BWD_COMPLEX = 0, 1, 2, 3, 4
 SSCAN_ERR_TIMEOUT = 5
 
 _IO_CODES = {torch.float32: SSCAN_F32, torch.bfloat16: SSCAN_BF16}
@@ -55,6 +55,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sscan_fwd.argtypes = [pp] + [vp] * 12 + [sz, vp]
     lib.sscan_fwd_complex.argtypes = [pp] + [vp] * 12
     lib.sscan_fwd_complex.restype = ctypes.c_int
+    lib.sscan_bwd_complex.argtypes = [pp] + [vp] * 20 + [sz, vp]
+    lib.sscan_bwd_complex.restype = ctypes.c_int
     lib.sscan_fwd.restype = ctypes.c_int
     lib.sscan_last_state.argtypes = [pp] + [vp] * 8 + [sz, vp]
     lib.sscan_last_state.restype = ctypes.c_int
@@ -205,6 +207,40 @@ def sscan_fwd_complex(u, delta_raw, A, B, C, delta_bias=None, D_skip=None, z=Non
                                             _ptr(A2), _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h02),
                                             _ptr(out), _ptr(h_last), _stream(stream)))
     return (out, torch.view_as_complex(h_last)) if return_last_state else out
+
+
+def sscan_bwd_complex(u, delta_raw, A, B, C, dout, delta_bias=None, D_skip=None, z=None, h0=None, *,
+                      delta_softplus=True, want_dh0=True, workspace=None, stream=None):
+    """Gradients of sum(out * dout) for the complex-A scan.  Returns a dict keyed du,
+    ddelta_raw, dA (D, N) complex64, dB, dC and, when the matching input is given,
+    ddelta_bias, dD, dz; dh0 (batch, D, N) complex64 when ``want_dh0``."""
+    prob = _io_problem(u, B, delta_softplus)
+    dev = u.device
+    _check_inputs(prob, u, delta_raw, None, B, C, delta_bias, D_skip, z, None)
+    _expect(dout, "dout", u.shape, u.dtype, dev)
+    A2 = _as_pairs(A, "A", (prob.dim, prob.dstate), dev)
+    h02 = _as_pairs(h0, "h0", (prob.batch, prob.dim, prob.dstate), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"du": torch.empty_like(u), "ddelta_raw": torch.empty_like(u),
+         "dA": torch.empty((prob.dim, prob.dstate, 2), **f32), "dB": torch.empty_like(B), "dC": torch.empty_like(C)}
+    if delta_bias is not None:
+        g["ddelta_bias"] = torch.empty((prob.dim,), **f32)
+    if D_skip is not None:
+        g["dD"] = torch.empty((prob.dim,), **f32)
+    if z is not None:
+        g["dz"] = torch.empty_like(z)
+    if want_dh0:
+        g["dh0"] = torch.empty((prob.batch, prob.dim, prob.dstate, 2), **f32)
+    ws, nbytes = _workspace(prob, SSCAN_OP_BWD_COMPLEX, workspace, dev)
+    _check(load_library().sscan_bwd_complex(
+        ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias), _ptr(A2), _ptr(B), _ptr(C), _ptr(D_skip),
+        _ptr(z), _ptr(h02), _ptr(dout), _ptr(g["du"]), _ptr(g["ddelta_raw"]), _ptr(g.get("ddelta_bias")),
+        _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g.get("dD")), _ptr(g.get("dz")), _ptr(g.get("dh0")),
+        _ptr(ws), nbytes, _stream(stream)))
+    g["dA"] = torch.view_as_complex(g["dA"])
+    if want_dh0:
+        g["dh0"] = torch.view_as_complex(g["dh0"])
+    return g
 
 
 def sscan_last_state(u, delta_raw, A, B, delta_bias=None, h0=None, *, delta_softplus=True,

@@ -317,6 +317,14 @@ size_t sscan_workspace_size(const sscan_problem* p, int op) {
             return (p->batch * p->dim > 0 && p->seqlen > 0)
                        ? sscan::align256((size_t)(p->batch * p->dim) * sizeof(float))
                        : 0;
+        case SSCAN_OP_BWD_COMPLEX: {
+            // fp32 dB, dC accumulators, then the complex state before every 8th step
+            if (p->batch * p->dim <= 0 || p->seqlen <= 0) return 0;
+            const int64_t nck = (p->seqlen + 7) / 8;
+            const size_t floats = (size_t)(2 * p->batch * p->seqlen * p->dstate) +
+                                  (size_t)(p->batch * nck * p->dim * p->dstate * 2);
+            return sscan::align256(floats * sizeof(float));
+        }
         default:
             return 0;
     }
@@ -588,6 +596,85 @@ sscan_status sscan_fwd_complex(const sscan_problem* p, const void* u, const void
     const cudaError_t e = sscan::launch_fwd_complex(a, p->io_dtype == SSCAN_BF16, st);
     if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "complex forward kernel: %s", cudaGetErrorString(e));
     return SSCAN_OK;
+}
+
+sscan_status sscan_bwd_complex(const sscan_problem* p, const void* u, const void* delta_raw,
+                               const float* delta_bias, const float* A, const void* B, const void* C,
+                               const float* D_skip, const void* z, const float* h0, const void* dout, void* du,
+                               void* ddelta_raw, float* ddelta_bias, float* dA, void* dB, void* dC, float* dD,
+                               void* dz, float* dh0, void* workspace, size_t workspace_bytes, void* stream) {
+    g_err[0] = 0;
+    g_launches = 0;
+    if (sscan_status s = check_problem(p)) return s;
+    if ((z == nullptr) != (dz == nullptr)) return fail(SSCAN_ERR_INVALID_ARG, "dz must be given exactly when z is");
+    if (dD && !D_skip) return fail(SSCAN_ERR_INVALID_ARG, "dD needs D_skip");
+    const int64_t rows = p->batch * p->dim;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (rows > 0 && p->seqlen > 0 &&
+        (!u || !delta_raw || !A || !B || !C || !dout || !du || !ddelta_raw || !dB || !dC))
+        return fail(SSCAN_ERR_INVALID_ARG, "u, delta_raw, A, B, C, dout, du, ddelta_raw, dB, dC are required");
+    if (p->dim > 0 && !dA) return fail(SSCAN_ERR_INVALID_ARG, "dA is required");
+    if (sscan_status s = check_workspace(sscan_workspace_size(p, SSCAN_OP_BWD_COMPLEX), workspace, workspace_bytes))
+        return s;
+    const int64_t DN = p->dim * p->dstate, BLN = p->batch * p->seqlen * p->dstate;
+    cudaError_t e = cudaSuccess;
+    if (DN > 0) e = cudaMemsetAsync(dA, 0, (size_t)(2 * DN) * sizeof(float), st);
+    if (e == cudaSuccess && dD && p->dim > 0) e = cudaMemsetAsync(dD, 0, (size_t)p->dim * sizeof(float), st);
+    if (e == cudaSuccess && ddelta_bias && p->dim > 0)
+        e = cudaMemsetAsync(ddelta_bias, 0, (size_t)p->dim * sizeof(float), st);
+    if (e == cudaSuccess && rows > 0 && p->seqlen == 0 && dh0)
+        e = cudaMemsetAsync(dh0, 0, (size_t)(2 * rows * p->dstate) * sizeof(float), st);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing gradients: %s", cudaGetErrorString(e));
+    if (rows == 0 || p->seqlen == 0) return SSCAN_OK;
+    float* ws = static_cast<float*>(workspace);
+    e = cudaMemsetAsync(ws, 0, (size_t)(2 * BLN) * sizeof(float), st);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing workspace: %s", cudaGetErrorString(e));
+    sscan::ComplexBwdArgs g{};
+    sscan::ComplexArgs& a = g.f;
+    a.batch = p->batch;
+    a.L = p->seqlen;
+    a.D = p->dim;
+    a.N = (int)p->dstate;
+    a.softplus = (p->flags & SSCAN_DELTA_SOFTPLUS) ? 1 : 0;
+    a.u = u;
+    a.delta_raw = delta_raw;
+    a.bias = delta_bias;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.Dskip = D_skip;
+    a.z = z;
+    a.h0 = h0;
+    a.out = nullptr;
+    a.h_last = nullptr;
+    a.ckpt = ws + 2 * BLN;
+    a.nck = (p->seqlen + 7) / 8;
+    const int bf16 = p->io_dtype == SSCAN_BF16;
+    // checkpoint pass: the complex forward kernel storing the state before every 8th step
+    ++g_launches;
+    e = sscan::launch_fwd_complex(a, bf16, st);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "complex checkpoint kernel: %s", cudaGetErrorString(e));
+    g.dout = dout;
+    g.du = du;
+    g.ddelta_raw = ddelta_raw;
+    g.dz = dz;
+    g.dA = dA;
+    g.dB32 = ws;
+    g.dC32 = ws + BLN;
+    g.dD = dD;
+    g.dbias = ddelta_bias;
+    g.dh0 = dh0;
+    ++g_launches;
+    e = sscan::launch_bwd_complex(g, bf16, st);
+    if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "complex backward kernel: %s", cudaGetErrorString(e));
+    if (bf16) {
+        cast_out<__nv_bfloat16>(ws, dB, BLN, st);
+        cast_out<__nv_bfloat16>(ws + BLN, dC, BLN, st);
+    } else {
+        cast_out<float>(ws, dB, BLN, st);
+        cast_out<float>(ws + BLN, dC, BLN, st);
+    }
+    return cuda_check("gradient cast kernel");
 }
 
 sscan_status sscan_step(const sscan_problem* p, const void* u, const void* delta_raw, const float* delta_bias,

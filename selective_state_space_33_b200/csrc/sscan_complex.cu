@@ -25,6 +25,7 @@
 #include <cstdint>
 
 #include "sscan_launch.h"
+#include "sscan_complex_math.cuh"
 #include "sscan_math.cuh"
 #include "sscan_plan.h"
 
@@ -35,29 +36,6 @@ constexpr int kCTT = 16;           // steps per tile
 constexpr int kCWarps = 4;
 constexpr int kCThreads = kCWarps * 32;
 constexpr float kCSmallA = 9.765625e-4f;
-constexpr float kTwoPiHi = 6.28318548202514648f;   // fp32 nearest to 2 pi
-constexpr float kTwoPiLo = -1.7484556e-7f;         // 2 pi - kTwoPiHi
-constexpr float kInvTwoPi = 0.159154943091895336f;
-
-__device__ __forceinline__ float sin_approx(float x) {
-    float y;
-    asm("sin.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ float cos_approx(float x) {
-    float y;
-    asm("cos.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// cos and sin of an angle of any size: reduce by a multiple of 2 pi first.
-__device__ __forceinline__ float2 cis(float th) {
-    const float k = rintf(th * kInvTwoPi);
-    float r = fmaf(-k, kTwoPiHi, th);
-    r = fmaf(-k, kTwoPiLo, r);
-    return make_float2(cos_approx(r), sin_approx(r));
-}
-
 template <int NG, int CG>
 struct CCfg {
     static constexpr int CW = 32 / NG;       // channels per warp
@@ -69,9 +47,18 @@ template <typename T, int NG, int CG, bool ACC>
 __device__ __forceinline__ void scan_tile_c(float2 (&h)[CG], const float2 (&aq)[CG], const float2 (&nia)[CG],
                                             const float2 (&ia)[CG], const float2* sdx, const float2* sgd,
                                             const float* sB, const float* sC, int tl, int g, int cw, bool write,
-                                            T* out, int64_t out_stride) {
+                                            T* out, int64_t out_stride, float* ck, int64_t ck_stride, int nvalid) {
     using C = CCfg<NG, CG>;
     for (int t = 0; t < tl; ++t) {
+        if (ck && t % 8 == 0) {
+            // the state before step t: a starting point of the backward's recomputation
+#pragma unroll
+            for (int j = 0; j < CG; ++j)
+                if (j < nvalid) {
+                    ck[(t / 8) * ck_stride + 2 * j] = h[j].x;
+                    ck[(t / 8) * ck_stride + 2 * j + 1] = h[j].y;
+                }
+        }
         const float2 dx = sdx[t * C::DC + cw];  // (delta, x)
         const float delta = dx.x, x = dx.y;
         const float* Bt = sB + t * C::NS + g * CG;
@@ -80,7 +67,7 @@ __device__ __forceinline__ void scan_tile_c(float2 (&h)[CG], const float2 (&aq)[
 #pragma unroll
         for (int j = 0; j < CG; ++j) {
             const float e = ex2(delta * aq[j].x);
-            const float2 cs = cis(delta * aq[j].y);
+            const float2 cs = cplx::cis(delta * aq[j].y);
             const float abr = e * cs.x, abi = e * cs.y;
             const float bx = Bt[j] * x;
             float nr, ni;
@@ -165,6 +152,7 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a) {
                                            __ldg(a.h0 + ((b * a.D + d) * N + n) * 2 + 1));
     }
     const bool acc = __syncthreads_or(small_a ? 1 : 0) != 0;
+    const int nvalid = cvalid ? (N - g * CG < CG ? N - g * CG : CG) : 0;
 
     for (int64_t t0 = 0; t0 < a.L; t0 += kCTT) {
         const int tl = (int)(a.L - t0 < kCTT ? a.L - t0 : kCTT);
@@ -197,11 +185,16 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a) {
             sC[e] = cv;
         }
         __syncthreads();
-        T* out = static_cast<T*>(a.out) + (b * a.L + t0) * a.D + d;
+        T* out = a.out ? static_cast<T*>(a.out) + (b * a.L + t0) * a.D + d : nullptr;
+        float* ck = a.ckpt ? a.ckpt + (((b * a.nck + t0 / 8) * a.D + d) * N + g * CG) * 2 : nullptr;
+        const int64_t ck_stride = a.D * N * 2;
+        const bool wr = cvalid && out != nullptr;
         if (acc)
-            scan_tile_c<T, NG, CG, true>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, cvalid, out, a.D);
+            scan_tile_c<T, NG, CG, true>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
+                                         nvalid);
         else
-            scan_tile_c<T, NG, CG, false>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, cvalid, out, a.D);
+            scan_tile_c<T, NG, CG, false>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
+                                          nvalid);
         __syncthreads();
     }
     if (a.h_last && cvalid) {

@@ -84,11 +84,30 @@ struct ComplexArgs {
     const float* Dskip;     // (D) or null
     const void* z;          // (batch, L, D) or null
     const float* h0;        // (batch, D, N, 2) or null
-    void* out;              // (batch, L, D)
+    void* out;              // (batch, L, D), or null when only checkpoints are wanted
     float* h_last;          // (batch, D, N, 2) or null
+    float* ckpt;            // [batch][nck][D][N][2]: the state before every 8th step, or null
+    int64_t nck;
 };
 
 cudaError_t launch_fwd_complex(const ComplexArgs& a, int io_bf16, cudaStream_t st);
+
+// Backward of the complex-A scan (sscan_complex_bwd.cu).
+struct ComplexBwdArgs {
+    ComplexArgs f;          // forward inputs; f.ckpt / f.nck hold the checkpoints
+    const void* dout;       // (batch, L, D)
+    void* du;               // (batch, L, D)
+    void* ddelta_raw;       // (batch, L, D)
+    void* dz;               // (batch, L, D) or null
+    float* dA;              // (D, N, 2), pre-zeroed
+    float* dB32;            // (batch, L, N) fp32, pre-zeroed
+    float* dC32;            // (batch, L, N) fp32, pre-zeroed
+    float* dD;              // (D) or null, pre-zeroed
+    float* dbias;           // (D) or null, pre-zeroed
+    float* dh0;             // (batch, D, N, 2) or null
+};
+
+cudaError_t launch_bwd_complex(const ComplexBwdArgs& a, int io_bf16, cudaStream_t st);
 
 // Backward of the tiled path: scalars, small tensors and gradient accumulators.
 struct BwdTiledArgs {

@@ -73,6 +73,9 @@ WORKLOADS = {
                            decode=True, description="one generation step, 64 sequences, Mamba-2.8B layer width"),
     "complex130m": Workload("complex130m", 8, 2048, 1536, 16, "bf16", 1e-3, 1e-1, "ones", 6, complex_a=True,
                             description="complex A = -1/2 + n i at the Mamba-130M layer shape, bf16 I/O"),
+    "complexbwd130m": Workload("complexbwd130m", 8, 2048, 1536, 16, "bf16", 1e-3, 1e-1, "ones", 7,
+                               backward=True, complex_a=True,
+                               description="backward with complex A = -1/2 + n i at the Mamba-130M layer shape"),
 }
 
 

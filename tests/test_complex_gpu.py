@@ -102,3 +102,50 @@ def test_complex_rejects_bad_A(cuda_device):
     with pytest.raises((TypeError, ValueError)):
         sb.sscan_fwd_complex(t["u"], t["delta_raw"], torch.zeros(8, 5, dtype=torch.complex64, device=cuda_device),
                              t["B"], t["C"])
+
+
+# ---------------------------------------------------------------- backward
+def _check_complex_bwd(x, io, dev, A=None, h0=None):
+    t = to_torch(x, dev)
+    A_np = (x["A"] if A is None else A).astype(np.complex64)
+    A_t = torch.from_numpy(np.ascontiguousarray(A_np)).to(dev)
+    h0_t = None if h0 is None else torch.from_numpy(h0.astype(np.complex64)).to(dev)
+    g = sb.sscan_bwd_complex(t["u"], t["delta_raw"], A_t, t["B"], t["C"], t["dout"], t["delta_bias"], t["D_skip"],
+                             t.get("z"), h0_t)
+    torch.cuda.synchronize()
+    ref = oracle.bwd_complex(x["u"], x["delta_raw"], A_np.astype(np.complex128), x["B"], x["C"], x["dout"],
+                             delta_bias=x["delta_bias"], D_skip=x["D_skip"], z=x.get("z"),
+                             h0=None if h0 is None else h0.astype(np.complex64).astype(np.complex128))
+    errs = {}
+    for k, r in ref.items():
+        got = g[k].detach().cpu()
+        got = got.numpy().astype(np.complex128) if got.is_complex() else to_f64(g[k])
+        errs[k] = float(np.max(np.abs(got - r)) / max(np.max(np.abs(r)), 1e-300))
+    bad = {k: e for k, e in errs.items() if not e <= TOL[io]}
+    assert not bad, errs
+    return errs
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 100, 37, 16), (1, 70, 8, 4), (3, 33, 5, 1), (2, 64, 40, 7), (1, 45, 130, 16)])
+def test_complex_backward_small(cuda_device, io, shape):
+    x = W.small_case(*shape, io=io, seed=sum(shape) + 9, backward=True, complex_a=True)
+    h0 = np.random.default_rng(4).standard_normal((shape[0], shape[2], shape[3], 2)) @ np.array([1.0, 1j]) * 0.5
+    _check_complex_bwd(x, io, cuda_device, h0=h0)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_complex_backward_general_A_values(cuda_device, io):
+    x = W.small_case(2, 60, 32, 16, io=io, seed=75, backward=True, complex_a=True)
+    rng = np.random.default_rng(75)
+    A = (-np.exp(rng.uniform(-3, 2, size=(32, 16))) + 1j * rng.uniform(-40, 40, size=(32, 16)))
+    A[0, 0] = 0.0
+    A[1, 3] = 1e-5 - 2e-5j
+    A[5, 2] = -3e-2 + 1e-2j
+    _check_complex_bwd(x, io, cuda_device, A=A)
+
+
+def test_complex_backward_long_sequence(cuda_device):
+    """L 2048 at the layer's state size (batch 1, D 256, N 16, bf16): 256 checkpoint tiles."""
+    x = W.small_case(1, 2048, 256, 16, io="bf16", seed=76, backward=True, complex_a=True)
+    _check_complex_bwd(x, "bf16", cuda_device)
