@@ -15,7 +15,8 @@
 //     d delta += lam Abar (A h_{t-1} + B x)
 //     dA   += delta lam Abar h_{t-1} + lam B x delta^2 psi(delta A)
 //   with psi(q) = (q e^q - expm1(q)) / q^2 (its Taylor series for |q| < 1/2, where the
-//   closed form would cancel) and beta = delta phi1(delta A) (series near 0);
+//   closed form would cancel) and beta = delta phi1(delta A), phi1 = Abar - q psi there
+//   (no cancellation) and (Abar - 1) / A elsewhere;
 //   and the per-element sums over a channel's lanes, and the (t, n) sums over the
 //   channels of a warp, are formed with shuffles before anything touches memory.
 // dB and dC of a tile are stored per warp in shared memory, summed across the CTA's
@@ -422,23 +423,22 @@ __global__ void __launch_bounds__(kThreadsB, 5)
                         const float2 l = __ffma2_rn(Cp[p], dyy, lam[p]);
                         const float2 la = __fmul2_rn(l, ab);
                         // beta = Bbar / B = expm1(q) / A: series delta phi1(q) near q = 0
-                        const float2 em1 = __fadd2_rn(ab, g2(-1.f, -1.f));
-                        const float2 bl = __fmul2_rn(em1, iA[p]);
-                        float2 ph = __ffma2_rn(q, g2(1.f / 120.f, 1.f / 120.f), g2(1.f / 24.f, 1.f / 24.f));
-                        ph = __ffma2_rn(ph, q, g2(1.f / 6.f, 1.f / 6.f));
-                        ph = __ffma2_rn(ph, q, g2(0.5f, 0.5f));
-                        ph = __ffma2_rn(ph, q, g2(1.f, 1.f));
-                        const float2 bs = __fmul2_rn(dd, ph);
-                        const float2 beta = g2(fabsf(q.x) < 0.0625f ? bs.x : bl.x, fabsf(q.y) < 0.0625f ? bs.y : bl.y);
-                        // (delta Abar - beta) / A = delta^2 psi(q): series for |q| < 1/2
-                        float2 ps = __ffma2_rn(q, g2(1.f / 840.f, 1.f / 840.f), g2(1.f / 144.f, 1.f / 144.f));
-                        ps = __ffma2_rn(ps, q, g2(1.f / 30.f, 1.f / 30.f));
-                        ps = __ffma2_rn(ps, q, g2(0.125f, 0.125f));
-                        ps = __ffma2_rn(ps, q, g2(1.f / 3.f, 1.f / 3.f));
-                        ps = __ffma2_rn(ps, q, g2(0.5f, 0.5f));
-                        const float2 t2s = __fmul2_rn(__fmul2_rn(dd, dd), ps);
-                        const float2 t2c = __fmul2_rn(__ffma2_rn(dd, ab, g2(-beta.x, -beta.y)), iA[p]);
-                        const float2 t2 = g2(fabsf(q.x) < 0.5f ? t2s.x : t2c.x, fabsf(q.y) < 0.5f ? t2s.y : t2c.y);
+                        // -psi(q), psi(q) = (q e^q - expm1(q)) / q^2, by its series (|q| < 1/2 uses it)
+                        float2 nps = __ffma2_rn(q, g2(-1.f / 840.f, -1.f / 840.f), g2(-1.f / 144.f, -1.f / 144.f));
+                        nps = __ffma2_rn(nps, q, g2(-1.f / 30.f, -1.f / 30.f));
+                        nps = __ffma2_rn(nps, q, g2(-0.125f, -0.125f));
+                        nps = __ffma2_rn(nps, q, g2(-1.f / 3.f, -1.f / 3.f));
+                        nps = __ffma2_rn(nps, q, g2(-0.5f, -0.5f));
+                        // beta = Bbar / B: for |q| < 1/2, delta phi1(q) with phi1 = Abar - q psi (no
+                        // cancellation); else (Abar - 1) / A
+                        const float2 bs = __fmul2_rn(dd, __ffma2_rn(q, nps, ab));
+                        const float2 bl = __fmul2_rn(__fadd2_rn(ab, g2(-1.f, -1.f)), iA[p]);
+                        const bool sx = fabsf(q.x) < 0.5f, sy = fabsf(q.y) < 0.5f;
+                        const float2 beta = g2(sx ? bs.x : bl.x, sy ? bs.y : bl.y);
+                        // -(delta Abar - beta) / A = -delta^2 psi(q): the series where |q| < 1/2
+                        const float2 nt2s = __fmul2_rn(__fmul2_rn(dd, dd), nps);
+                        const float2 nt2c = __fmul2_rn(__ffma2_rn(dd, g2(-ab.x, -ab.y), beta), iA[p]);
+                        const float2 nt2 = g2(sx ? nt2s.x : nt2c.x, sy ? nt2s.y : nt2c.y);
                         const float2 lb = __fmul2_rn(l, beta);
                         const float2 dBv = __fmul2_rn(lb, xx);
                         const float2 dCv = __fmul2_rn(dyy, hcv[p]);
@@ -447,11 +447,12 @@ __global__ void __launch_bounds__(kThreadsB, 5)
                         vbc[4 + 2 * p] = dCv.x;
                         vbc[4 + 2 * p + 1] = dCv.y;
                         du2 = __ffma2_rn(lb, Bp[p], du2);
-                        S1 = __ffma2_rn(la, __fmul2_rn(A2[p], hp[p]), S1);
+                        const float2 lah = __fmul2_rn(la, hp[p]);
+                        S1 = __ffma2_rn(A2[p], lah, S1);
                         S2 = __ffma2_rn(la, Bp[p], S2);
                         const float2 Bx = __fmul2_rn(Bp[p], xx);
-                        P1[p] = __ffma2_rn(dd, __fmul2_rn(la, hp[p]), P1[p]);
-                        P2v[p] = __ffma2_rn(__fmul2_rn(l, Bx), t2, P2v[p]);
+                        P1[p] = __ffma2_rn(dd, lah, P1[p]);
+                        P2v[p] = __ffma2_rn(__fmul2_rn(l, Bx), nt2, P2v[p]);  // minus the psi term
                         y2 = __ffma2_rn(Cp[p], hcv[p], y2);
                         lam[p] = la;
                     }
@@ -529,7 +530,7 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         return;
     }
     // per-channel sums
-    const float dAv[4] = {P1[0].x + P2v[0].x, P1[0].y + P2v[0].y, P1[1].x + P2v[1].x, P1[1].y + P2v[1].y};
+    const float dAv[4] = {P1[0].x - P2v[0].x, P1[0].y - P2v[0].y, P1[1].x - P2v[1].x, P1[1].y - P2v[1].y};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         if (j >= nvalid) continue;
