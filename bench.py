@@ -127,8 +127,8 @@ NCU_TRAFFIC = {
     "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 505026048 + 150930176,
                   "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "0bc36e87ea5e1afc",
                   "profile": "profiles/fwd_tiled_kernel_mamba2.8b_bf16.md"},
-    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410256640 + 133296640,
-                "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "9d2486f634d56827",
+    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410381824 + 133053184,
+                "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "aef87df5fae5e9de",
                 "profile": "profiles/bwd_tiled_kernel_bwd130m_bf16.md"},
     "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317504 + 0,
                    "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "b7c6e53d71a0bd30",
@@ -136,6 +136,9 @@ NCU_TRAFFIC = {
     "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152287488 + 32752640,
                     "sources": ("sscan_complex.cu", "sscan_math.cuh"), "sha256": "4a792ca9083060f5",
                     "profile": "profiles/fwd_complex_kernel_complex130m_bf16.md"},
+    "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 612191744 + 138920448,
+                       "sources": ("sscan_complex_bwd.cu", "sscan_complex_math.cuh", "sscan_math.cuh"),
+                       "sha256": "70ea3be94b22aacc", "profile": "profiles/bwd_complex_kernel_complexbwd130m_bf16.md"},
 }
 
 
@@ -294,7 +297,7 @@ def reference_arm(args, w: W.Workload):
     total_rows = w.batch * w.dim
     rng = np.random.default_rng(1234)
     rate0, _, _, _ = cpu_oracle_rate(x, w, 2.0)
-    per_step_rows = int(min(total_rows, max(threads, rate0 * 1e9 * 4.0 / w.seqlen)))  # ~4 s per step
+    per_step_rows = int(min(total_rows, max(threads, rate0 * 1e9 * 2.0 / w.seqlen)))  # ~2 s per step
 
     def step():
         rows = np.sort(rng.choice(total_rows, size=per_step_rows, replace=False))
