@@ -124,8 +124,8 @@ def roofline_units(w: W.Workload) -> dict:
 # keyed by the SHA-256 of those source files (with comments and blank lines removed,
 # so that only code counts) and reported as null once the code changes.
 NCU_TRAFFIC = {
-    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 505026048 + 150930176,
-                  "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "0bc36e87ea5e1afc",
+    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 505560576 + 150813184,
+                  "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "8645152b11aa39aa",
                   "profile": "profiles/fwd_tiled_kernel_mamba2.8b_bf16.md"},
     "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410381824 + 133053184,
                 "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "aef87df5fae5e9de",
@@ -133,8 +133,9 @@ NCU_TRAFFIC = {
     "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317504 + 0,
                    "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "b7c6e53d71a0bd30",
                    "profile": "profiles/step_quad_kernel_decode2.8b_bf16.md"},
-    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152287488 + 32752640,
-                    "sources": ("sscan_complex.cu", "sscan_math.cuh"), "sha256": "4a792ca9083060f5",
+    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152277248 + 32187392,
+                    "sources": ("sscan_complex.cu", "sscan_complex_math.cuh", "sscan_math.cuh"),
+                    "sha256": "9aff9384dc9ba9aa",
                     "profile": "profiles/fwd_complex_kernel_complex130m_bf16.md"},
     "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 612191744 + 138920448,
                        "sources": ("sscan_complex_bwd.cu", "sscan_complex_math.cuh", "sscan_math.cuh"),

@@ -593,7 +593,7 @@ sscan_status sscan_fwd_complex(const sscan_problem* p, const void* u, const void
     a.out = out;
     a.h_last = h_last;
     ++g_launches;
-    const cudaError_t e = sscan::launch_fwd_complex(a, p->io_dtype == SSCAN_BF16, st);
+    const cudaError_t e = sscan::launch_fwd_complex(a, nullptr, 0, p->io_dtype == SSCAN_BF16, st);
     if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "complex forward kernel: %s", cudaGetErrorString(e));
     return SSCAN_OK;
 }
@@ -647,12 +647,13 @@ sscan_status sscan_bwd_complex(const sscan_problem* p, const void* u, const void
     a.h0 = h0;
     a.out = nullptr;
     a.h_last = nullptr;
-    a.ckpt = ws + 2 * BLN;
-    a.nck = (p->seqlen + 7) / 8;
+    float* ckpt = ws + 2 * BLN;
+    g.ckpt = ckpt;
+    g.nck = (p->seqlen + 7) / 8;
     const int bf16 = p->io_dtype == SSCAN_BF16;
     // checkpoint pass: the complex forward kernel storing the state before every 8th step
     ++g_launches;
-    e = sscan::launch_fwd_complex(a, bf16, st);
+    e = sscan::launch_fwd_complex(a, ckpt, g.nck, bf16, st);
     if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "complex checkpoint kernel: %s", cudaGetErrorString(e));
     g.dout = dout;
     g.du = du;

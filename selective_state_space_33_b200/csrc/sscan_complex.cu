@@ -43,14 +43,14 @@ struct CCfg {
     static constexpr int NS = NG * CG;       // states covered (>= N)
 };
 
-template <typename T, int NG, int CG, bool ACC>
+template <typename T, int NG, int CG, bool ACC, bool CKPT>
 __device__ __forceinline__ void scan_tile_c(float2 (&h)[CG], const float2 (&aq)[CG], const float2 (&nia)[CG],
                                             const float2 (&ia)[CG], const float2* sdx, const float2* sgd,
                                             const float* sB, const float* sC, int tl, int g, int cw, bool write,
                                             T* out, int64_t out_stride, float* ck, int64_t ck_stride, int nvalid) {
     using C = CCfg<NG, CG>;
     for (int t = 0; t < tl; ++t) {
-        if (ck && t % 8 == 0) {
+        if (CKPT && t % 8 == 0) {
             // the state before step t: a starting point of the backward's recomputation
 #pragma unroll
             for (int j = 0; j < CG; ++j)
@@ -106,15 +106,18 @@ __device__ __forceinline__ void scan_tile_c(float2 (&h)[CG], const float2 (&aq)[
         // the NG lanes of a channel (lane bits at multiples of CW) sum their readouts
 #pragma unroll
         for (int m = 1; m < NG; m <<= 1) y += __shfl_xor_sync(0xffffffffu, y, m * C::CW);
-        if (write && g == 0) {
+        if (!CKPT && write && g == 0) {
             const float2 gd = sgd[t * C::DC + cw];
             IO<T>::store(out, (int64_t)t * out_stride, fmaf(y, gd.x, gd.y));
         }
     }
 }
 
-template <typename T, int NG, int CG>
-__global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a) {
+// CKPT: the checkpoint pass of the backward (states before every 8th step, no output);
+// otherwise the forward with outputs.  Separate instantiations keep the per-step
+// checkpoint test out of the output kernel's loop.
+template <typename T, int NG, int CG, bool CKPT>
+__global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, float* ckpt, int64_t nck) {
     using C = CCfg<NG, CG>;
     __shared__ float2 sdx[kCTT * C::DC];  // (delta, x)
     __shared__ float2 sgd[kCTT * C::DC];  // (gate, D x gate)
@@ -185,15 +188,15 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a) {
             sC[e] = cv;
         }
         __syncthreads();
-        T* out = a.out ? static_cast<T*>(a.out) + (b * a.L + t0) * a.D + d : nullptr;
-        float* ck = a.ckpt ? a.ckpt + (((b * a.nck + t0 / 8) * a.D + d) * N + g * CG) * 2 : nullptr;
+        T* out = CKPT ? nullptr : static_cast<T*>(a.out) + (b * a.L + t0) * a.D + d;
+        float* ck = CKPT ? ckpt + (((b * nck + t0 / 8) * a.D + d) * N + g * CG) * 2 : nullptr;
         const int64_t ck_stride = a.D * N * 2;
-        const bool wr = cvalid && out != nullptr;
+        const bool wr = cvalid;
         if (acc)
-            scan_tile_c<T, NG, CG, true>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
+            scan_tile_c<T, NG, CG, true, CKPT>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
                                          nvalid);
         else
-            scan_tile_c<T, NG, CG, false>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
+            scan_tile_c<T, NG, CG, false, CKPT>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
                                           nvalid);
         __syncthreads();
     }
@@ -210,9 +213,13 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a) {
 }
 
 template <typename T, int NG, int CG>
-cudaError_t launch_c(const ComplexArgs& a, cudaStream_t st) {
+cudaError_t launch_c(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream_t st) {
     const int64_t blocks = a.batch * ((a.D + CCfg<NG, CG>::DC - 1) / CCfg<NG, CG>::DC);
-    if (blocks > 0) fwd_complex_kernel<T, NG, CG><<<(unsigned)blocks, kCThreads, 0, st>>>(a);
+    if (blocks <= 0) return cudaGetLastError();
+    if (ckpt)
+        fwd_complex_kernel<T, NG, CG, true><<<(unsigned)blocks, kCThreads, 0, st>>>(a, ckpt, nck);
+    else
+        fwd_complex_kernel<T, NG, CG, false><<<(unsigned)blocks, kCThreads, 0, st>>>(a, nullptr, 0);
     return cudaGetLastError();
 }
 
@@ -221,24 +228,24 @@ cudaError_t launch_c(const ComplexArgs& a, cudaStream_t st) {
 // measured at batch 8, L 2048, N 16: D 1536 0.90 ms with two states against 1.08 ms
 // with four; D 5120 2.34 ms with four against 2.37 ms with two.
 template <typename T>
-cudaError_t launch_ct(const ComplexArgs& a, cudaStream_t st) {
+cudaError_t launch_ct(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream_t st) {
     const int64_t ng4 = a.N <= 4 ? 1 : (a.N <= 8 ? 2 : 4);
     const int64_t ctas4 = a.batch * ((a.D + 4 * (32 / ng4) - 1) / (4 * (32 / ng4)));
     if (ctas4 < 4 * (int64_t)kSmCount) {
-        if (a.N <= 2) return launch_c<T, 1, 2>(a, st);
-        if (a.N <= 4) return launch_c<T, 2, 2>(a, st);
-        if (a.N <= 8) return launch_c<T, 4, 2>(a, st);
-        return launch_c<T, 8, 2>(a, st);
+        if (a.N <= 2) return launch_c<T, 1, 2>(a, ckpt, nck, st);
+        if (a.N <= 4) return launch_c<T, 2, 2>(a, ckpt, nck, st);
+        if (a.N <= 8) return launch_c<T, 4, 2>(a, ckpt, nck, st);
+        return launch_c<T, 8, 2>(a, ckpt, nck, st);
     }
-    if (a.N <= 4) return launch_c<T, 1, 4>(a, st);
-    if (a.N <= 8) return launch_c<T, 2, 4>(a, st);
-    return launch_c<T, 4, 4>(a, st);
+    if (a.N <= 4) return launch_c<T, 1, 4>(a, ckpt, nck, st);
+    if (a.N <= 8) return launch_c<T, 2, 4>(a, ckpt, nck, st);
+    return launch_c<T, 4, 4>(a, ckpt, nck, st);
 }
 
 }  // namespace
 
-cudaError_t launch_fwd_complex(const ComplexArgs& a, int io_bf16, cudaStream_t st) {
-    return io_bf16 ? launch_ct<__nv_bfloat16>(a, st) : launch_ct<float>(a, st);
+cudaError_t launch_fwd_complex(const ComplexArgs& a, float* ckpt, int64_t nck, int io_bf16, cudaStream_t st) {
+    return io_bf16 ? launch_ct<__nv_bfloat16>(a, ckpt, nck, st) : launch_ct<float>(a, ckpt, nck, st);
 }
 
 }  // namespace sscan

@@ -133,8 +133,8 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
 #pragma unroll
         for (int j = 0; j < kXCG; ++j) {
             const int n = gq * kXCG + j;
-            hk[j] = j < nvalid ? make_float2(a.ckpt[(((b * a.nck + it) * a.D + d) * N + n) * 2],
-                                             a.ckpt[(((b * a.nck + it) * a.D + d) * N + n) * 2 + 1])
+            hk[j] = j < nvalid ? make_float2(g.ckpt[(((b * g.nck + it) * a.D + d) * N + n) * 2],
+                                             g.ckpt[(((b * g.nck + it) * a.D + d) * N + n) * 2 + 1])
                                : make_float2(0.f, 0.f);
         }
         {

@@ -86,15 +86,18 @@ struct ComplexArgs {
     const float* h0;        // (batch, D, N, 2) or null
     void* out;              // (batch, L, D), or null when only checkpoints are wanted
     float* h_last;          // (batch, D, N, 2) or null
-    float* ckpt;            // [batch][nck][D][N][2]: the state before every 8th step, or null
-    int64_t nck;
 };
 
-cudaError_t launch_fwd_complex(const ComplexArgs& a, int io_bf16, cudaStream_t st);
+// ckpt: null for the forward with outputs; else [batch][nck][D][N][2] receives the
+// state before every 8th step (the backward's checkpoint pass, a.out unused).  Kept
+// out of ComplexArgs: the kernel's parameter block stays as small as the forward needs.
+cudaError_t launch_fwd_complex(const ComplexArgs& a, float* ckpt, int64_t nck, int io_bf16, cudaStream_t st);
 
 // Backward of the complex-A scan (sscan_complex_bwd.cu).
 struct ComplexBwdArgs {
-    ComplexArgs f;          // forward inputs; f.ckpt / f.nck hold the checkpoints
+    ComplexArgs f;          // forward inputs
+    const float* ckpt;      // [batch][nck][D][N][2], written by the checkpoint pass
+    int64_t nck;
     const void* dout;       // (batch, L, D)
     void* du;               // (batch, L, D)
     void* ddelta_raw;       // (batch, L, D)

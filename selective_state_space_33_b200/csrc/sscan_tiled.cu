@@ -74,8 +74,8 @@ struct Cfg {
     static_assert(PAIRS % kThreads == 0, "phase P runs a fixed number of pairs per thread");
     // shared-memory layout (byte offsets, all 128-aligned)
     static constexpr int OFF_RAW = 0;                                     // [STAGES][STAGE]
-    static constexpr int OFF_DX = OFF_RAW + STAGES * STAGE;               // float4 (d, d, x, x) [kTT][DC]
-    static constexpr int OFF_GD = OFF_DX + kTT * DC * 16;                 // float2 (gate, D x gate) [kTT][GD_PITCH]
+    static constexpr int OFF_DX = OFF_RAW + STAGES * STAGE;               // float2 (delta, x) [kTT][DC]
+    static constexpr int OFF_GD = OFF_DX + kTT * DC * 8;                  // float2 (gate, D x gate) [kTT][GD_PITCH]
     static constexpr int OFF_B = OFF_GD + kTT * GD_PITCH * 8;             // float  [kTT][NS]
     static constexpr int OFF_C = OFF_B + kTT * NS * 4;                    // float  [kTT][NS]
     static constexpr int OFF_OUT = OFF_C + kTT * NS * 4;                  // [RAW] output tile
@@ -93,12 +93,12 @@ __device__ __forceinline__ float2 ex2x2(float2 q) { return f2(ex2(q.x), ex2(q.y)
 
 // One step for the lane's G states, eq. (2) and (3a).  With v = -B x / A the update
 // h' = Abar h + (Abar - 1) B x / A is Abar (h - v) + v: two packed fmas per pair
-// (h - v as fma(v, -1, h), exact), no negated operand.  dx = (delta, delta, x, x);
+// (h - v as fma(v, -1, h), exact), no negated operand.  dx = (delta, x);
 // Bp, Cp point at the lane's G values of B_t, C_t.  Returns the partial readout
 // sum_j C_j h_j over these states (eq. (3b)).
 template <int G, bool WANT_Y>
-__device__ __forceinline__ float step_fast(LaneG<G>& s, float4 dx, const float* Bp, const float* Cp) {
-    const float2 dd = f2(dx.x, dx.y), xx = f2(dx.z, dx.w);
+__device__ __forceinline__ float step_fast(LaneG<G>& s, float2 dx, const float* Bp, const float* Cp) {
+    const float2 dd = f2(dx.x, dx.x), xx = f2(dx.y, dx.y);
     float2 y = f2(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < G / 2; ++k) {
@@ -114,8 +114,8 @@ __device__ __forceinline__ float step_fast(LaneG<G>& s, float4 dx, const float* 
 // Accurate form for blocks with a small |A| (or A = 0): Bbar / B = delta phi1(delta A)
 // with phi1's series near 0, as in the general kernels.
 template <int G, bool WANT_Y>
-__device__ __forceinline__ float step_acc(LaneG<G>& s, float4 dx, const float* Bp, const float* Cp) {
-    const float delta = dx.x, x = dx.z;
+__device__ __forceinline__ float step_acc(LaneG<G>& s, float2 dx, const float* Bp, const float* Cp) {
+    const float delta = dx.x, x = dx.y;
     float y = 0.f;
 #pragma unroll
     for (int j = 0; j < G; ++j) {
@@ -166,7 +166,7 @@ __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int 
                                           float& dsum, float* ck, int64_t ck_stride, int nvalid) {
     using C = Cfg<T, NG, G>;
     constexpr bool WANT_Y = MODE == kOut;
-    const float4* sdx = reinterpret_cast<const float4*>(smem + C::OFF_DX) + cw;
+    const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
     const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
     const float* sB = reinterpret_cast<const float*>(smem + C::OFF_B) + g * G;
     const float* sC = reinterpret_cast<const float*>(smem + C::OFF_C) + g * G;
@@ -185,7 +185,7 @@ __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int 
             const int t = tb + k;
             p[k] = 0.f;
             if (FULL || t < tile_len) {
-                const float4 dx = sdx[t * C::DC];
+                const float2 dx = sdx[t * C::DC];
                 if (MODE == kAgg) dsum += dx.x;
                 p[k] = ACC ? step_acc<G, WANT_Y>(s, dx, sB + t * C::NS, sC + t * C::NS)
                            : step_fast<G, WANT_Y>(s, dx, sB + t * C::NS, sC + t * C::NS);
@@ -210,9 +210,9 @@ template <int G>
 struct Prep { float2 a[G / 2]; float2 v[G / 2]; };
 
 template <int G>
-__device__ __forceinline__ Prep<G> prep_step(const LaneG<G>& s, float4 dx, const float* Bp) {
+__device__ __forceinline__ Prep<G> prep_step(const LaneG<G>& s, float2 dx, const float* Bp) {
     Prep<G> P;
-    const float2 dd = f2(dx.x, dx.y), xx = f2(dx.z, dx.w);
+    const float2 dd = f2(dx.x, dx.x), xx = f2(dx.y, dx.y);
 #pragma unroll
     for (int k = 0; k < G / 2; ++k) {
         P.a[k] = ex2x2(__fmul2_rn(dd, s.A2[k]));
@@ -235,7 +235,7 @@ __device__ __forceinline__ float upd_step(LaneG<G>& s, const Prep<G>& P, const f
 template <typename T, int NG, int G>
 __device__ __forceinline__ void scan_tile_pipe(LaneG<G>& s, unsigned char* smem, int g, int cw, T* sout) {
     using C = Cfg<T, NG, G>;
-    const float4* sdx = reinterpret_cast<const float4*>(smem + C::OFF_DX) + cw;
+    const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
     const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
     const float* sB = reinterpret_cast<const float*>(smem + C::OFF_B) + g * G;
     const float* sC = reinterpret_cast<const float*>(smem + C::OFF_C) + g * G;
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
         const int st = it % C::STAGES;
         const int64_t tt = t_begin + (int64_t)it * kTT;
         const int tile_len = (int)(t_end - tt < kTT ? t_end - tt : kTT);
-        // phase P: raw tile -> (delta, delta, x, x) and (gate, D x gate); B and C rows as fp32
+        // phase P: raw tile -> (delta, x) pairs and (gate, D x gate); B and C rows as fp32
         {
             const unsigned char* raw = smem + C::OFF_RAW + st * C::STAGE;
             const P2* ru = reinterpret_cast<const P2*>(raw);
@@ -416,8 +416,7 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
                 const float2 x = Pair<T>::f(ru[q]);
                 float2 dl = __fadd2_rn(Pair<T>::f(rd[q]), pbias);
                 if (a.softplus) dl = softplus_x2(dl);
-                sdx[t * C::DC + pc] = make_float4(dl.x, dl.x, x.x, x.x);
-                sdx[t * C::DC + pc + 1] = make_float4(dl.y, dl.y, x.y, x.y);
+                sdx[(t * C::DC + pc) / 2] = make_float4(dl.x, x.x, dl.y, x.y);
                 if (want_out) {
                     const float2 gt = has_z ? silu_x2(Pair<T>::f(rz[q])) : f2(1.f, 1.f);
                     const float2 dxg = __fmul2_rn(__fmul2_rn(pdsk, x), gt);
