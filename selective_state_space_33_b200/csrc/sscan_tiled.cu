@@ -58,13 +58,18 @@ template <> struct Pair<__nv_bfloat16> {
     static __device__ __forceinline__ float2 f(__nv_bfloat162 v) { return __bfloat1622float2(v); }
 };
 
-// Tile geometry for NG lanes per channel, G states per lane.
-template <typename T, int NG, int G>
+// Tile geometry for NG lanes per channel, G states per lane.  Raw-tile ring depth:
+// one stage (the next tile's copy is issued once phase P has consumed the stage and
+// lands during phase S), except for the backward's bf16 checkpoint pass, which runs
+// beside other kernels and keeps two.  Measured, bf16: one stage 0.583 against
+// 0.592 ms at the 2.8B-layer shape and 0.254 against 0.259 ms at the 130M shape;
+// two stages for the checkpoint pass 1.374 against 1.386 ms per backward call.
+template <typename T, int NG, int G, int MODE>
 struct Cfg {
     static constexpr int CW = 32 / NG;                     // channels per warp
     static constexpr int DC = CW * kWarps;                 // channels per CTA
     static constexpr int NS = NG * G;                      // states covered (>= N)
-    static constexpr int STAGES = sizeof(T) == 2 ? 2 : 1;  // raw-tile ring depth
+    static constexpr int STAGES = (sizeof(T) == 2 && MODE == kCkpt) ? 2 : 1;
     static constexpr int RAW = kTT * DC * (int)sizeof(T);  // bytes of one raw (batch, L, D) tile
     static constexpr int RAWBC = kTT * NS * (int)sizeof(T);  // bytes reserved for one raw B or C tile
     static constexpr int STAGE = 3 * RAW + 2 * RAWBC;      // u, delta_raw, z, B, C
@@ -164,7 +169,7 @@ __device__ __forceinline__ float transpose_reduce(float (&p)[NG], int g) {
 template <typename T, int NG, int G, int MODE, bool ACC, bool FULL>
 __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
                                           float& dsum, float* ck, int64_t ck_stride, int nvalid) {
-    using C = Cfg<T, NG, G>;
+    using C = Cfg<T, NG, G, MODE>;
     constexpr bool WANT_Y = MODE == kOut;
     const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
     const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
@@ -234,7 +239,7 @@ __device__ __forceinline__ float upd_step(LaneG<G>& s, const Prep<G>& P, const f
 
 template <typename T, int NG, int G>
 __device__ __forceinline__ void scan_tile_pipe(LaneG<G>& s, unsigned char* smem, int g, int cw, T* sout) {
-    using C = Cfg<T, NG, G>;
+    using C = Cfg<T, NG, G, kOut>;
     const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
     const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
     const float* sB = reinterpret_cast<const float*>(smem + C::OFF_B) + g * G;
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
                      const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_out,
                      const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
                      TiledArgs a) {
-    using C = Cfg<T, NG, G>;
+    using C = Cfg<T, NG, G, MODE>;
     using P2 = typename Pair<T>::type;
     extern __shared__ __align__(128) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -554,7 +559,7 @@ bool bc_by_tma(const TiledArgs& a) {
 
 template <typename T, int NG, int G, int MODE>
 cudaError_t launch_mode(const TiledArgs& args, const TiledPtrs& p, cudaStream_t st) {
-    using C = Cfg<T, NG, G>;
+    using C = Cfg<T, NG, G, MODE>;
     TiledArgs a = args;
     a.bc_tma = bc_by_tma<T>(a) ? 1 : 0;
     CUtensorMap mu, md, mz, mo, mb, mc;
