@@ -43,72 +43,123 @@ struct CCfg {
     static constexpr int NS = NG * CG;       // states covered (>= N)
 };
 
-template <typename T, int NG, int CG, bool ACC, bool CKPT>
+// One step of the lane's CG complex states (eq. (2) and (3a) with complex a; B, x
+// real): fast form h' = Abar (h - v) + v with v = -B x / a, or for a block with a
+// small |a| Bbar / B = delta phi1(delta a) by its series.  Returns the partial readout
+// Re(sum_j C_j h_j) over these states (eq. (3b)).
+template <int CG, bool ACC>
+__device__ __forceinline__ float cstep(float2 (&h)[CG], const float2 (&aq)[CG], const float2 (&nia)[CG],
+                                       const float2 (&ia)[CG], float delta, float x, const float* Bt,
+                                       const float* Ct) {
+    float y = 0.f;
+#pragma unroll
+    for (int j = 0; j < CG; ++j) {
+        const float e = ex2(delta * aq[j].x);
+        const float2 cs = cplx::cis(delta * aq[j].y);
+        const float abr = e * cs.x, abi = e * cs.y;
+        const float bx = Bt[j] * x;
+        float nr, ni;
+        if (!ACC) {
+            const float vr = bx * nia[j].x, vi = bx * nia[j].y;
+            const float tr = h[j].x - vr, ti = h[j].y - vi;
+            nr = fmaf(abr, tr, fmaf(-abi, ti, vr));
+            ni = fmaf(abr, ti, fmaf(abi, tr, vi));
+        } else {
+            // Bbar / B = delta phi1(q), q = delta a: series for |q| < 1/16, else (Abar - 1) / a
+            const float qr = delta * aq[j].x * kLn2, qi = delta * aq[j].y;
+            float cr, ci;
+            if (qr * qr + qi * qi < 0.00390625f) {
+                // phi1(q) = 1 + q/2 + q^2/6 + q^3/24 + q^4/120, Horner in complex arithmetic
+                float pr = 1.f / 120.f, pi = 0.f;
+                const float cf[4] = {1.f / 24.f, 1.f / 6.f, 0.5f, 1.f};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float r2 = fmaf(pr, qr, fmaf(-pi, qi, cf[k]));
+                    pi = fmaf(pr, qi, pi * qr);
+                    pr = r2;
+                }
+                cr = delta * pr;
+                ci = delta * pi;
+            } else {
+                const float er = abr - 1.f;
+                cr = fmaf(er, ia[j].x, -abi * ia[j].y);
+                ci = fmaf(er, ia[j].y, abi * ia[j].x);
+            }
+            nr = fmaf(abr, h[j].x, fmaf(-abi, h[j].y, cr * bx));
+            ni = fmaf(abr, h[j].y, fmaf(abi, h[j].x, ci * bx));
+        }
+        h[j] = make_float2(nr, ni);
+        y = fmaf(Ct[j], nr, y);
+    }
+    return y;
+}
+
+// Sum the partial readouts of a channel's NG lanes (lane bits at multiples of CW)
+// for NG consecutive steps so that lane g ends with the sum for step g: a transposed
+// butterfly, NG - 1 shuffles per NG steps instead of log2(NG) per step.
+template <int NG, int CW>
+__device__ __forceinline__ float creduce(float (&p)[NG], int g) {
+    if constexpr (NG == 1) {
+        return p[0];
+    } else {
+#pragma unroll
+        for (int m = NG / 2; m >= 1; m /= 2) {
+            const bool up = (g & m) != 0;
+#pragma unroll
+            for (int j = 0; j < m; ++j) {
+                const float keep = up ? p[m + j] : p[j];
+                const float send = up ? p[j] : p[m + j];
+                p[j] = keep + __shfl_xor_sync(0xffffffffu, send, m * CW);
+            }
+        }
+        return p[0];
+    }
+}
+
+// Phase S over one tile.  Checkpoint pass: the state before every 8th step, no
+// readout.  Output pass: blocks of NG steps whose readouts are reduced together, lane
+// g finishing step tb + g; FULL tiles (kCTT steps) are unrolled with no step predicate.
+template <typename T, int NG, int CG, bool ACC, bool CKPT, bool FULL>
 __device__ __forceinline__ void scan_tile_c(float2 (&h)[CG], const float2 (&aq)[CG], const float2 (&nia)[CG],
                                             const float2 (&ia)[CG], const float2* sdx, const float2* sgd,
                                             const float* sB, const float* sC, int tl, int g, int cw, bool write,
                                             T* out, int64_t out_stride, float* ck, int64_t ck_stride, int nvalid) {
     using C = CCfg<NG, CG>;
-    for (int t = 0; t < tl; ++t) {
-        if (CKPT && t % 8 == 0) {
-            // the state before step t: a starting point of the backward's recomputation
+    const float* Bg = sB + g * CG;
+    const float* Cg = sC + g * CG;
+    if constexpr (CKPT) {
+        for (int t = 0; t < tl; ++t) {
+            if (t % 8 == 0) {
+                // the state before step t: a starting point of the backward's recomputation
 #pragma unroll
-            for (int j = 0; j < CG; ++j)
-                if (j < nvalid) {
-                    ck[(t / 8) * ck_stride + 2 * j] = h[j].x;
-                    ck[(t / 8) * ck_stride + 2 * j + 1] = h[j].y;
-                }
-        }
-        const float2 dx = sdx[t * C::DC + cw];  // (delta, x)
-        const float delta = dx.x, x = dx.y;
-        const float* Bt = sB + t * C::NS + g * CG;
-        const float* Ct = sC + t * C::NS + g * CG;
-        float y = 0.f;
-#pragma unroll
-        for (int j = 0; j < CG; ++j) {
-            const float e = ex2(delta * aq[j].x);
-            const float2 cs = cplx::cis(delta * aq[j].y);
-            const float abr = e * cs.x, abi = e * cs.y;
-            const float bx = Bt[j] * x;
-            float nr, ni;
-            if (!ACC) {
-                const float vr = bx * nia[j].x, vi = bx * nia[j].y;
-                const float tr = h[j].x - vr, ti = h[j].y - vi;
-                nr = fmaf(abr, tr, fmaf(-abi, ti, vr));
-                ni = fmaf(abr, ti, fmaf(abi, tr, vi));
-            } else {
-                // Bbar / B = delta phi1(q), q = delta a: series for |q| < 1/16, else (Abar - 1) / a
-                const float qr = delta * aq[j].x * kLn2, qi = delta * aq[j].y;
-                float cr, ci;
-                if (qr * qr + qi * qi < 0.00390625f) {
-                    // phi1(q) = 1 + q/2 + q^2/6 + q^3/24 + q^4/120, Horner in complex arithmetic
-                    float pr = 1.f / 120.f, pi = 0.f;
-                    const float cf[4] = {1.f / 24.f, 1.f / 6.f, 0.5f, 1.f};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float r2 = fmaf(pr, qr, fmaf(-pi, qi, cf[k]));
-                        pi = fmaf(pr, qi, pi * qr);
-                        pr = r2;
+                for (int j = 0; j < CG; ++j)
+                    if (j < nvalid) {
+                        ck[(t / 8) * ck_stride + 2 * j] = h[j].x;
+                        ck[(t / 8) * ck_stride + 2 * j + 1] = h[j].y;
                     }
-                    cr = delta * pr;
-                    ci = delta * pi;
-                } else {
-                    const float er = abr - 1.f;
-                    cr = fmaf(er, ia[j].x, -abi * ia[j].y);
-                    ci = fmaf(er, ia[j].y, abi * ia[j].x);
-                }
-                nr = fmaf(abr, h[j].x, fmaf(-abi, h[j].y, cr * bx));
-                ni = fmaf(abr, h[j].y, fmaf(abi, h[j].x, ci * bx));
             }
-            h[j] = make_float2(nr, ni);
-            y = fmaf(Ct[j], nr, y);  // Re of eq. (3b)
+            const float2 dx = sdx[t * C::DC + cw];  // (delta, x)
+            (void)cstep<CG, ACC>(h, aq, nia, ia, dx.x, dx.y, Bg + t * C::NS, Cg + t * C::NS);
         }
-        // the NG lanes of a channel (lane bits at multiples of CW) sum their readouts
+    } else {
+#pragma unroll(FULL ? kCTT / NG : 1)
+        for (int tb = 0; tb < (FULL ? kCTT : tl); tb += NG) {
+            float p[NG];
 #pragma unroll
-        for (int m = 1; m < NG; m <<= 1) y += __shfl_xor_sync(0xffffffffu, y, m * C::CW);
-        if (!CKPT && write && g == 0) {
-            const float2 gd = sgd[t * C::DC + cw];
-            IO<T>::store(out, (int64_t)t * out_stride, fmaf(y, gd.x, gd.y));
+            for (int k = 0; k < NG; ++k) {
+                const int t = tb + k;
+                p[k] = 0.f;
+                if (FULL || t < tl) {
+                    const float2 dx = sdx[t * C::DC + cw];  // (delta, x)
+                    p[k] = cstep<CG, ACC>(h, aq, nia, ia, dx.x, dx.y, Bg + t * C::NS, Cg + t * C::NS);
+                }
+            }
+            const float y = creduce<NG, C::CW>(p, g);
+            const int t = tb + g;
+            if (write && (FULL || t < tl)) {
+                const float2 gd = sgd[t * C::DC + cw];
+                IO<T>::store(out, (int64_t)t * out_stride, fmaf(y, gd.x, gd.y));
+            }
         }
     }
 }
@@ -193,11 +244,14 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
         const int64_t ck_stride = a.D * N * 2;
         const bool wr = cvalid;
         if (acc)
-            scan_tile_c<T, NG, CG, true, CKPT>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
-                                         nvalid);
+            scan_tile_c<T, NG, CG, true, CKPT, false>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck,
+                                                      ck_stride, nvalid);
+        else if (tl == kCTT)
+            scan_tile_c<T, NG, CG, false, CKPT, true>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck,
+                                                      ck_stride, nvalid);
         else
-            scan_tile_c<T, NG, CG, false, CKPT>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
-                                          nvalid);
+            scan_tile_c<T, NG, CG, false, CKPT, false>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck,
+                                                       ck_stride, nvalid);
         __syncthreads();
     }
     if (a.h_last && cvalid) {
