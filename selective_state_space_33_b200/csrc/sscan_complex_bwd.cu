@@ -12,8 +12,9 @@
 //   dx      += Re(conj(lam) beta) B,   dB += Re(conj(lam) beta) x,   dC += dy Re(h_t)
 //   d delta += Re(conj(lam) Abar (a h_{t-1} + B x))
 //   dA      += conj(conj(lam) (delta Abar h_{t-1} + delta^2 psi(delta a) B x))
-// with beta = (Abar - 1)/a (phi1's series delta phi1(delta a) for |delta a| < 1/16)
-// and psi(q) = (q e^q - (e^q - 1)) / q^2 (its series for |q| < 1/2).  Per-element
+// with beta = (Abar - 1)/a and psi(q) = (q e^q - (e^q - 1)) / q^2; for |delta a| < 1/2 the
+// reverse step takes psi's series and beta = delta (Abar - delta a psi), the
+// recomputation phi1's series for |delta a| < 1/16.  Per-element
 // sums over a channel's lanes use shuffles; dB and dC (t, n) are summed over the
 // warp's channels with shuffles, over the CTA's warps in shared memory, and added to
 // fp32 accumulators in global memory.
@@ -186,21 +187,11 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
                 const float2 ab = make_float2(e * cs.x, e * cs.y);
                 const float2 q = make_float2(delta * av[j].x, delta * av[j].y);
                 const float qq = q.x * q.x + q.y * q.y;
-                float2 beta;
-                if (qq < 0.00390625f) {
-                    float2 p = make_float2(1.f / 120.f, 0.f);
-                    const float cf[4] = {1.f / 24.f, 1.f / 6.f, 0.5f, 1.f};
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        p = cmul(p, q);
-                        p.x += cf[m];
-                    }
-                    beta = make_float2(delta * p.x, delta * p.y);
-                } else {
-                    beta = cmul(make_float2(ab.x - 1.f, ab.y), ia[j]);
-                }
-                // psi(q) = (q e^q - (e^q - 1)) / q^2: series for |q| < 1/2
-                float2 psi;
+                // beta = Bbar / B and the dA term delta^2 psi(q), psi(q) = (q e^q - (e^q - 1)) / q^2.
+                // |q| < 1/2: psi by its series, beta = delta phi1(q) = delta (Abar - q psi) (no
+                // cancellation); else beta = (Abar - 1) / a and delta^2 psi = (delta Abar - beta) / a,
+                // whose cancellation costs at most a few 1e-6 relative there.  One branch per state.
+                float2 beta, d2psi;
                 if (qq < 0.25f) {
                     float2 p = make_float2(1.f / 840.f, 0.f);
                     const float cf[5] = {1.f / 144.f, 1.f / 30.f, 0.125f, 1.f / 3.f, 0.5f};
@@ -209,13 +200,13 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
                         p = cmul(p, q);
                         p.x += cf[m];
                     }
-                    psi = p;
+                    const float2 qp = cmul(q, p);
+                    beta = make_float2(delta * (ab.x - qp.x), delta * (ab.y - qp.y));
+                    const float dd2 = delta * delta;
+                    d2psi = make_float2(dd2 * p.x, dd2 * p.y);
                 } else {
-                    const float2 qa = cmul(q, ab);
-                    const float2 num = make_float2(qa.x - ab.x + 1.f, qa.y - ab.y);
-                    const float2 q2 = cmul(q, q);
-                    const float inv = 1.f / (q2.x * q2.x + q2.y * q2.y);
-                    psi = cmul(num, make_float2(q2.x * inv, -q2.y * inv));
+                    beta = cmul(make_float2(ab.x - 1.f, ab.y), ia[j]);
+                    d2psi = cmul(make_float2(fmaf(delta, ab.x, -beta.x), fmaf(delta, ab.y, -beta.y)), ia[j]);
                 }
                 const float2 l = make_float2(fmaf(Cn, dy, lam[j].x), lam[j].y);
                 const float lb = fmaf(l.x, beta.x, l.y * beta.y);  // Re(conj(l) beta)
@@ -228,8 +219,7 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
                 ddp = fmaf(l.x, dhd.x, fmaf(l.y, dhd.y, ddp));
                 // dh/da = delta Abar h_{t-1} + delta^2 psi B x
                 const float2 abh = cmul(ab, hp[j]);
-                const float d2 = delta * delta * bx;
-                const float2 dha = make_float2(fmaf(delta, abh.x, d2 * psi.x), fmaf(delta, abh.y, d2 * psi.y));
+                const float2 dha = make_float2(fmaf(delta, abh.x, bx * d2psi.x), fmaf(delta, abh.y, bx * d2psi.y));
                 // conj(conj(l) dha): (Re, -Im) of conj(l) dha
                 gA[j].x = fmaf(l.x, dha.x, fmaf(l.y, dha.y, gA[j].x));
                 gA[j].y = fmaf(-l.x, dha.y, fmaf(l.y, dha.x, gA[j].y));
