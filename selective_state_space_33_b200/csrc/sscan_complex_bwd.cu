@@ -13,9 +13,11 @@
 //   d delta += Re(conj(lam) Abar (a h_{t-1} + B x))
 //   dA      += conj(conj(lam) (delta Abar h_{t-1} + delta^2 psi(delta a) B x))
 // with beta = (Abar - 1)/a and psi(q) = (q e^q - (e^q - 1)) / q^2; for |delta a| < 1/2 the
-// reverse step takes psi's series and beta = delta (Abar - delta a psi), the
-// recomputation phi1's series for |delta a| < 1/16.  Per-element
-// sums over a channel's lanes use shuffles; dB and dC (t, n) are summed over the
+// reverse step takes psi's series and beta = delta (Abar - delta a psi).  The
+// recomputation follows the forward kernel's form h' = Abar (h - v) + v, v = -B x / a,
+// or, in a block holding an |a| < 2^-10, phi1's series for |delta a| < 1/16.
+// Per-element sums over a channel's lanes use transposed shuffle butterflies over
+// blocks of steps; dB and dC (t, n) are summed over the
 // warp's channels with shuffles, over the CTA's warps in shared memory, and added to
 // fp32 accumulators in global memory.
 #include <cuda_runtime.h>
@@ -33,6 +35,7 @@ constexpr int kXTB = 8;  // steps per tile (= the checkpoint spacing)
 constexpr int kXWarps = 4;
 constexpr int kXThreads = kXWarps * 32;
 constexpr int kXCG = 2;  // complex states per lane
+constexpr float kXSmallA = 9.765625e-4f;  // |a| below 2^-10: the block recomputes with phi1's series
 
 template <int NG>
 struct XCfg {
@@ -45,8 +48,30 @@ __device__ __forceinline__ float2 cmul(float2 p, float2 q) {
     return make_float2(fmaf(p.x, q.x, -p.y * q.y), fmaf(p.x, q.y, p.y * q.x));
 }
 
+// Sum per-element values over a channel's NG lanes (lane bits at multiples of CW)
+// for BLK consecutive steps: a transposed butterfly over the high BLK state-group
+// bits (lane group ghi ends with step ghi of the block), then plain rounds over the
+// remaining LO = NG / BLK groups.
+template <int BLK, int LO, int CW>
+__device__ __forceinline__ float xreduce(float (&p)[BLK], int ghi) {
+#pragma unroll
+    for (int m = BLK / 2; m >= 1; m /= 2) {
+        const bool up = (ghi & m) != 0;
+#pragma unroll
+        for (int j = 0; j < m; ++j) {
+            const float keep = up ? p[m + j] : p[j];
+            const float send = up ? p[j] : p[m + j];
+            p[j] = keep + __shfl_xor_sync(0xffffffffu, send, m * LO * CW);
+        }
+    }
+    float v = p[0];
+#pragma unroll
+    for (int m = 1; m < LO; m <<= 1) v += __shfl_xor_sync(0xffffffffu, v, m * CW);
+    return v;
+}
+
 template <typename T, int NG>
-__global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g) {
+__global__ void __launch_bounds__(kXThreads, 6) bwd_complex_kernel(ComplexBwdArgs g) {
     const ComplexArgs& a = g.f;
     using C = XCfg<NG>;
     __shared__ float2 sdx[kXTB * C::DC];   // (delta, x)
@@ -71,6 +96,7 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
     const bool cvalid = d < a.D;
     const int nvalid = cvalid ? (N - gq * kXCG < kXCG ? N - gq * kXCG : kXCG) : 0;
     float2 av[kXCG], aq[kXCG], ia[kXCG], lam[kXCG], gA[kXCG];
+    bool small_a = false;
 #pragma unroll
     for (int j = 0; j < kXCG; ++j) {
         const int n = gq * kXCG + j;
@@ -78,12 +104,15 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
         const float ar = ok ? __ldg(a.A + (d * N + n) * 2) : -1.f;
         const float ai = ok ? __ldg(a.A + (d * N + n) * 2 + 1) : 0.f;
         const float m2 = ar * ar + ai * ai;
+        small_a |= ok && m2 < kXSmallA * kXSmallA;
         av[j] = make_float2(ar, ai);
         aq[j] = make_float2(ar * kLog2e, ai);
         const float inv = m2 > 0.f ? 1.f / m2 : 0.f;
         ia[j] = make_float2(ar * inv, -ai * inv);
         lam[j] = gA[j] = make_float2(0.f, 0.f);
     }
+    // one CTA-wide choice of the recomputation's form (block-uniform branch)
+    const bool acc = __syncthreads_or(small_a ? 1 : 0) != 0;
     const float dsk = (cvalid && a.Dskip) ? __ldg(a.Dskip + d) : 0.f;
     float dD_acc = 0.f, db_acc = 0.f;
     const int ntile = (int)((a.L + kXTB - 1) / kXTB);
@@ -138,7 +167,24 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
                                              g.ckpt[(((b * g.nck + it) * a.D + d) * N + n) * 2 + 1])
                                : make_float2(0.f, 0.f);
         }
-        {
+        if (!acc) {
+            // the forward kernel's form: h' = Abar (h - v) + v with v = -B x / a
+            float2 h[kXCG] = {hk[0], hk[1]};
+            for (int t = 0; t < tl; ++t) {
+                const float2 dx = sdx[t * C::DC + cw];
+#pragma unroll
+                for (int j = 0; j < kXCG; ++j) {
+                    const float2 cs = cplx::cis(dx.x * aq[j].y);
+                    const float e = ex2(dx.x * aq[j].x);
+                    const float2 ab = make_float2(e * cs.x, e * cs.y);
+                    const float bx = sB[t * C::NS + gq * kXCG + j] * dx.y;
+                    const float2 nh = cmul(ab, make_float2(fmaf(bx, ia[j].x, h[j].x), fmaf(bx, ia[j].y, h[j].y)));
+                    h[j] = make_float2(fmaf(-bx, ia[j].x, nh.x), fmaf(-bx, ia[j].y, nh.y));
+                }
+                shs[t * kXThreads + tid] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+            }
+        } else {
+            // |a| < 2^-10 somewhere in the block: Bbar from phi1's series where delta a is small
             float2 h[kXCG] = {hk[0], hk[1]};
             for (int t = 0; t < tl; ++t) {
                 const float2 dx = sdx[t * C::DC + cw];
@@ -169,8 +215,16 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
             }
         }
 
-        // ---- reverse sweep
-        for (int t = tl - 1; t >= 0; --t) {
+        // ---- reverse sweep, in blocks of BLK steps whose per-element sums are reduced together
+        constexpr int BLK = NG > 4 ? 4 : NG, LO = NG / BLK;
+        const int ghi = gq / LO, glo = gq % LO;
+        for (int tb = ((tl - 1) / BLK) * BLK; tb >= 0; tb -= BLK) {
+          float p1[BLK], p2[BLK], p3[BLK];
+#pragma unroll
+          for (int kk = BLK - 1; kk >= 0; --kk) {
+            const int t = tb + kk;
+            p1[kk] = p2[kk] = p3[kk] = 0.f;
+            if (t >= tl) continue;
             const float2 dx = sdx[t * C::DC + cw];
             const float4 q4 = sq[t * C::DC + cw];
             const float delta = dx.x, x = dx.y, dy = q4.x;
@@ -227,22 +281,9 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
                 yp = fmaf(Cn, hc[j].x, yp);
                 lam[j] = make_float2(fmaf(ab.x, l.x, ab.y * l.y), fmaf(ab.x, l.y, -ab.y * l.x));  // conj(ab) l
             }
-            // per-element sums over the NG lanes of the channel (lane bits at multiples of CW)
-#pragma unroll
-            for (int m = 1; m < NG; m <<= 1) {
-                dxp += __shfl_xor_sync(0xffffffffu, dxp, m * C::CW);
-                ddp += __shfl_xor_sync(0xffffffffu, ddp, m * C::CW);
-                yp += __shfl_xor_sync(0xffffffffu, yp, m * C::CW);
-            }
-            if (gq == 0 && cvalid) {
-                const int64_t gi = (b * a.L + t0 + t) * a.D + d;
-                const float ddr = ddp * q4.z;
-                IO<T>::store(static_cast<T*>(g.du), gi, fmaf(dsk, dy, dxp));
-                IO<T>::store(static_cast<T*>(g.ddelta_raw), gi, ddr);
-                if (g.dz) IO<T>::store(static_cast<T*>(g.dz), gi, q4.y * fmaf(dsk, x, yp));
-                dD_acc = fmaf(dy, x, dD_acc);
-                db_acc += ddr;
-            }
+            p1[kk] = dxp;
+            p2[kk] = ddp;
+            p3[kk] = yp;
             // dB, dC of step t summed over the warp's channels (the low lane bits)
 #pragma unroll
             for (int j = 0; j < kXCG; ++j) {
@@ -256,6 +297,23 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
                     sacc[warp][t * C::NS + gq * kXCG + j][1] = dcv[j];
                 }
             }
+          }
+          // the block's per-element sums: lane group ghi finishes step tb + ghi
+          const float sdu = xreduce<BLK, LO, C::CW>(p1, ghi);
+          const float sdd = xreduce<BLK, LO, C::CW>(p2, ghi);
+          const float syp = xreduce<BLK, LO, C::CW>(p3, ghi);
+          const int t = tb + ghi;
+          if (glo == 0 && t < tl && cvalid) {
+              const float2 dx = sdx[t * C::DC + cw];
+              const float4 q4 = sq[t * C::DC + cw];
+              const int64_t gi = (b * a.L + t0 + t) * a.D + d;
+              const float ddr = sdd * q4.z;
+              IO<T>::store(static_cast<T*>(g.du), gi, fmaf(dsk, q4.x, sdu));
+              IO<T>::store(static_cast<T*>(g.ddelta_raw), gi, ddr);
+              if (g.dz) IO<T>::store(static_cast<T*>(g.dz), gi, q4.y * fmaf(dsk, dx.y, syp));
+              dD_acc = fmaf(q4.x, dx.y, dD_acc);
+              db_acc += ddr;
+          }
         }
         __syncthreads();
         // the tile's dB, dC: the warps' sums into the fp32 accumulators
@@ -284,6 +342,12 @@ __global__ void __launch_bounds__(kXThreads) bwd_complex_kernel(ComplexBwdArgs g
         }
         atomicAdd(g.dA + (d * N + n) * 2, gA[j].x);
         atomicAdd(g.dA + (d * N + n) * 2 + 1, gA[j].y);
+    }
+    // dD and the bias gradient: each lane group holds the steps it finished
+#pragma unroll
+    for (int m = 1; m < NG; m <<= 1) {
+        dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, m * C::CW);
+        db_acc += __shfl_xor_sync(0xffffffffu, db_acc, m * C::CW);
     }
     if (gq == 0 && cvalid) {
         if (g.dD) atomicAdd(g.dD + d, dD_acc);
