@@ -133,13 +133,13 @@ NCU_TRAFFIC = {
     "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317504 + 0,
                    "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "b7c6e53d71a0bd30",
                    "profile": "profiles/step_quad_kernel_decode2.8b_bf16.md"},
-    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152277248 + 32187392,
+    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152343296 + 32550912,
                     "sources": ("sscan_complex.cu", "sscan_complex_math.cuh", "sscan_math.cuh"),
-                    "sha256": "9aff9384dc9ba9aa",
+                    "sha256": "45ee83425d235ed2",
                     "profile": "profiles/fwd_complex_kernel_complex130m_bf16.md"},
-    "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 612145408 + 141952256,
+    "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 612188672 + 138831616,
                        "sources": ("sscan_complex_bwd.cu", "sscan_complex_math.cuh", "sscan_math.cuh"),
-                       "sha256": "bb931c335c048e9c", "profile": "profiles/bwd_complex_kernel_complexbwd130m_bf16.md"},
+                       "sha256": "9e107f54b099d7c3", "profile": "profiles/bwd_complex_kernel_complexbwd130m_bf16.md"},
 }
 
 
