@@ -435,6 +435,11 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
         e = cudaMemsetAsync(ddelta_bias, 0, (size_t)p->dim * sizeof(float), st);
     if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing gradients: %s", cudaGetErrorString(e));
     if (rows == 0) {
+        // no channels (D = 0) with batch * L * N > 0: dB and dC are sums over nothing
+        const size_t bytes = (size_t)BLN * (p->io_dtype == SSCAN_BF16 ? 2 : 4);
+        if (bytes > 0 && dB) e = cudaMemsetAsync(dB, 0, bytes, st);
+        if (e == cudaSuccess && bytes > 0 && dC) e = cudaMemsetAsync(dC, 0, bytes, st);
+        if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing dB, dC: %s", cudaGetErrorString(e));
         return SSCAN_OK;
     }
     if (p->seqlen == 0) {
@@ -624,6 +629,12 @@ sscan_status sscan_bwd_complex(const sscan_problem* p, const void* u, const void
         e = cudaMemsetAsync(ddelta_bias, 0, (size_t)p->dim * sizeof(float), st);
     if (e == cudaSuccess && rows > 0 && p->seqlen == 0 && dh0)
         e = cudaMemsetAsync(dh0, 0, (size_t)(2 * rows * p->dstate) * sizeof(float), st);
+    if (rows == 0 && BLN > 0) {
+        // no channels (D = 0) with batch * L * N > 0: dB and dC are sums over nothing
+        const size_t bytes = (size_t)BLN * (p->io_dtype == SSCAN_BF16 ? 2 : 4);
+        if (e == cudaSuccess && dB) e = cudaMemsetAsync(dB, 0, bytes, st);
+        if (e == cudaSuccess && dC) e = cudaMemsetAsync(dC, 0, bytes, st);
+    }
     if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "zeroing gradients: %s", cudaGetErrorString(e));
     if (rows == 0 || p->seqlen == 0) return SSCAN_OK;
     float* ws = static_cast<float*>(workspace);

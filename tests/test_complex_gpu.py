@@ -94,6 +94,32 @@ def test_complex130m_sampled(cuda_device):
     assert np.max(np.abs(hl - ref_h)) / np.max(np.abs(ref_h)) <= 1e-4
 
 
+def test_complex_empty_inputs(cuda_device):
+    """No steps: the final state is h0 and every gradient but the pass-through ones is
+    zero; no batch or no channels: nothing to compute, parameter gradients zero, and with
+    no channels dB and dC are zero sums.  The caching allocator is first filled with NaN
+    blocks so that outputs the library leaves unwritten show."""
+    for shape in ((2, 0, 5, 4), (0, 10, 4, 4), (2, 10, 0, 4)):
+        batch, L, D, N = shape
+        x = W.small_case(*shape, io="f32", seed=6, backward=True, complex_a=True)
+        t = to_torch(x, cuda_device)
+        A_t = torch.from_numpy(np.ascontiguousarray(x["A"].astype(np.complex64))).to(cuda_device)
+        h0 = torch.randn(batch, D, N, dtype=torch.complex64, device=cuda_device)
+        out, hl = sb.sscan_fwd_complex(t["u"], t["delta_raw"], A_t, t["B"], t["C"], t["delta_bias"], t["D_skip"],
+                                       t["z"], h0, return_last_state=True)
+        torch.cuda.synchronize()
+        assert out.numel() == batch * L * D
+        if L == 0:
+            assert torch.equal(hl, h0)
+        filler = [torch.full((1 << 16,), float("nan"), device=cuda_device) for _ in range(8)]
+        del filler
+        g = sb.sscan_bwd_complex(t["u"], t["delta_raw"], A_t, t["B"], t["C"], t["dout"], t["delta_bias"],
+                                 t["D_skip"], t["z"], h0)
+        torch.cuda.synchronize()
+        for k, v in g.items():
+            assert torch.all(v == 0), (shape, k)
+
+
 def test_complex_rejects_bad_A(cuda_device):
     x = W.small_case(1, 16, 8, 4, io="f32", seed=73, complex_a=True)
     t = to_torch(x, cuda_device)

@@ -196,6 +196,24 @@ def test_empty_batch_and_channels(cuda_device):
         assert out.numel() == 0
 
 
+def test_backward_empty_inputs(cuda_device):
+    """No steps, no batch or no channels: every gradient is a sum over nothing, so the
+    library writes zeros (the outputs start as NaN to show anything left unwritten)."""
+    for shape in ((2, 0, 5, 4), (0, 10, 4, 4), (2, 10, 0, 4)):
+        batch, L, D, N = shape
+        t = to_torch(W.small_case(*shape, io="f32", seed=5, backward=True), cuda_device)
+        h0 = torch.randn(batch, D, N, device=cuda_device)
+        nan = lambda *size: torch.full(size, float("nan"), device=cuda_device)
+        grads = {"du": nan(*t["u"].shape), "ddelta_raw": nan(*t["u"].shape), "dz": nan(*t["u"].shape),
+                 "dA": nan(D, N), "dB": nan(*t["B"].shape), "dC": nan(*t["C"].shape), "ddelta_bias": nan(D),
+                 "dD": nan(D), "dh0": nan(batch, D, N)}
+        g = sb.sscan_bwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t["delta_bias"], t["D_skip"],
+                         t["z"], h0, grads=grads)
+        torch.cuda.synchronize()
+        for k, v in g.items():
+            assert torch.all(v == 0), (shape, k)
+
+
 def test_errors_through_binding(cuda_device):
     t = to_torch(W.small_case(1, 16, 4, 4, io="f32", seed=3), cuda_device)
     with pytest.raises(sb.SscanError) as e:

@@ -71,3 +71,16 @@ def test_unaligned_state_takes_general_kernel(cuda_device, io):
                             D_skip=x["D_skip"], z=x["z"], h0=h0.astype(np.float64))
     assert normwise(to_f64(out), ref[:, 0]) <= TOL[io]
     assert normwise(to_f64(state), ref_h) <= 1e-5
+
+
+def test_step_with_no_batch_or_channels(cuda_device):
+    """batch 0 or D 0: nothing to do, an empty output and no error."""
+    for batch, D, N in ((0, 64, 16), (3, 0, 16)):
+        x = W.small_case(batch, 1, D, N, io="f32", seed=9)
+        t = to_torch(x, cuda_device)
+        state = torch.zeros(batch, D, N, device=cuda_device)
+        out = sb.sscan_step(t["u"][:, 0].contiguous(), t["delta_raw"][:, 0].contiguous(), t["A"],
+                            t["B"][:, 0].contiguous(), t["C"][:, 0].contiguous(), state, t["delta_bias"],
+                            t["D_skip"], t["z"][:, 0].contiguous())
+        torch.cuda.synchronize()
+        assert out.numel() == 0
