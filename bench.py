@@ -127,8 +127,8 @@ NCU_TRAFFIC = {
     "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 505266688 + 151573248,
                   "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "d602134642251f4d",
                   "profile": "profiles/fwd_tiled_kernel_mamba2.8b_bf16.md"},
-    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410381824 + 133053184,
-                "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "aef87df5fae5e9de",
+    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410298368 + 133372928,
+                "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "430945355610e83f",
                 "profile": "profiles/bwd_tiled_kernel_bwd130m_bf16.md"},
     "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317504 + 0,
                    "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "b7c6e53d71a0bd30",
