@@ -10,8 +10,9 @@
 // complex states (CG = 4, or 2 when the grid is small) in registers.  Per 16-step tile all threads
 // stage (delta, x) and (gate, D x gate) for the tile's channels and the tile's B
 // and C rows in shared memory with coalesced loads (phase P), then every lane
-// advances its states through the tile (phase S) and the NG lanes of a channel
-// sum their partial readouts with a butterfly; lane 0 of the channel writes out.
+// advances its states through the tile (phase S), two states per f32x2 operation, and
+// the NG lanes of a channel sum their partial readouts over blocks of NG steps with a
+// transposed butterfly, each lane writing one step's output.
 //
 // One step of one complex state a = ar + i ai, with v = -B x / a:
 //   Abar = 2^(delta ar log2 e) (cos(delta ai) + i sin(delta ai))       (eq. 2)
@@ -43,55 +44,109 @@ struct CCfg {
     static constexpr int NS = NG * CG;       // states covered (>= N)
 };
 
+__device__ __forceinline__ float2 ex2x2c(float2 q) { return make_float2(ex2(q.x), ex2(q.y)); }
+
+// A lane's CG complex states and constants, packed over pairs of states so that the
+// fast step runs on f32x2 arithmetic: hr[k] = (Re h_2k, Re h_2k+1), and likewise the
+// imaginary parts, a log2(e) split into (Re, Im), and -1/a.
+template <int CG>
+struct CLane {
+    static constexpr int P = CG / 2;
+    float2 hr[P], hi[P];  // Re h, Im h
+    float2 qr[P], qi[P];  // Re a log2 e, Im a
+    float2 nr[P], ni[P];  // Re(-1/a), Im(-1/a)
+};
+
+// Component j of a pair-packed array (j is a compile-time index after unrolling).
+template <int P>
+__device__ __forceinline__ float& comp(float2 (&v)[P], int j) {
+    return (j & 1) ? v[j >> 1].y : v[j >> 1].x;
+}
+
+// cos and sin of a pair of angles (the reduction of cplx::cis, packed).
+__device__ __forceinline__ void cis2(float2 th, float2& cs, float2& sn) {
+    const float2 m = __fmul2_rn(th, make_float2(-cplx::kInvTwoPi, -cplx::kInvTwoPi));
+    const float2 nk = make_float2(rintf(m.x), rintf(m.y));
+    float2 r = __ffma2_rn(nk, make_float2(cplx::kTwoPiHi, cplx::kTwoPiHi), th);
+    r = __ffma2_rn(nk, make_float2(cplx::kTwoPiLo, cplx::kTwoPiLo), r);
+    cs = make_float2(cplx::cos_approx(r.x), cplx::cos_approx(r.y));
+    sn = make_float2(cplx::sin_approx(r.x), cplx::sin_approx(r.y));
+}
+
 // One step of the lane's CG complex states (eq. (2) and (3a) with complex a; B, x
-// real): fast form h' = Abar (h - v) + v with v = -B x / a, or for a block with a
-// small |a| Bbar / B = delta phi1(delta a) by its series.  Returns the partial readout
-// Re(sum_j C_j h_j) over these states (eq. (3b)).
-template <int CG, bool ACC>
-__device__ __forceinline__ float cstep(float2 (&h)[CG], const float2 (&aq)[CG], const float2 (&nia)[CG],
-                                       const float2 (&ia)[CG], float delta, float x, const float* Bt,
-                                       const float* Ct) {
+// real) in the fast form h' = Abar (h - v) + v with v = -B x / a, two states per
+// packed operation.  Returns the partial readout Re(sum_j C_j h_j) (eq. (3b)).
+template <int CG>
+__device__ __forceinline__ float cstep_fast(CLane<CG>& s, float delta, float x, const float* Bt,
+                                            const float* Ct) {
+    const float2 dd = make_float2(delta, delta), xx = make_float2(x, x);
+    float2 y = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < CG / 2; ++k) {
+        const float2 e = ex2x2c(__fmul2_rn(dd, s.qr[k]));
+        float2 cs, sn;
+        cis2(__fmul2_rn(dd, s.qi[k]), cs, sn);
+        const float2 abr = __fmul2_rn(e, cs), abi = __fmul2_rn(e, sn);
+        const float2 bx = __fmul2_rn(reinterpret_cast<const float2*>(Bt)[k], xx);
+        const float2 vr = __fmul2_rn(bx, s.nr[k]), vi = __fmul2_rn(bx, s.ni[k]);
+        const float2 tr = __ffma2_rn(vr, make_float2(-1.f, -1.f), s.hr[k]);   // Re(h - v)
+        const float2 ti = __ffma2_rn(vi, make_float2(-1.f, -1.f), s.hi[k]);   // Im(h - v)
+        const float2 mti = __ffma2_rn(s.hi[k], make_float2(-1.f, -1.f), vi);  // -Im(h - v)
+        s.hr[k] = __ffma2_rn(abr, tr, __ffma2_rn(abi, mti, vr));
+        s.hi[k] = __ffma2_rn(abr, ti, __ffma2_rn(abi, tr, vi));
+        y = __ffma2_rn(reinterpret_cast<const float2*>(Ct)[k], s.hr[k], y);
+    }
+    return y.x + y.y;
+}
+
+// The same step for a block with a small |a|: Bbar / B = delta phi1(delta a) with
+// phi1's series where |delta a| < 1/16, else (Abar - 1) / a; one state at a time.
+template <int CG>
+__device__ __forceinline__ float cstep_acc(CLane<CG>& s, float delta, float x, const float* Bt, const float* Ct) {
     float y = 0.f;
 #pragma unroll
     for (int j = 0; j < CG; ++j) {
-        const float e = ex2(delta * aq[j].x);
-        const float2 cs = cplx::cis(delta * aq[j].y);
+        const float aqr = comp(s.qr, j), aqi = comp(s.qi, j);
+        const float e = ex2(delta * aqr);
+        const float2 cs = cplx::cis(delta * aqi);
         const float abr = e * cs.x, abi = e * cs.y;
         const float bx = Bt[j] * x;
-        float nr, ni;
-        if (!ACC) {
-            const float vr = bx * nia[j].x, vi = bx * nia[j].y;
-            const float tr = h[j].x - vr, ti = h[j].y - vi;
-            nr = fmaf(abr, tr, fmaf(-abi, ti, vr));
-            ni = fmaf(abr, ti, fmaf(abi, tr, vi));
-        } else {
-            // Bbar / B = delta phi1(q), q = delta a: series for |q| < 1/16, else (Abar - 1) / a
-            const float qr = delta * aq[j].x * kLn2, qi = delta * aq[j].y;
-            float cr, ci;
-            if (qr * qr + qi * qi < 0.00390625f) {
-                // phi1(q) = 1 + q/2 + q^2/6 + q^3/24 + q^4/120, Horner in complex arithmetic
-                float pr = 1.f / 120.f, pi = 0.f;
-                const float cf[4] = {1.f / 24.f, 1.f / 6.f, 0.5f, 1.f};
+        const float qr = delta * aqr * kLn2, qi = delta * aqi;
+        float cr, ci;
+        if (qr * qr + qi * qi < 0.00390625f) {
+            // phi1(q) = 1 + q/2 + q^2/6 + q^3/24 + q^4/120, Horner in complex arithmetic
+            float pr = 1.f / 120.f, pi = 0.f;
+            const float cf[4] = {1.f / 24.f, 1.f / 6.f, 0.5f, 1.f};
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float r2 = fmaf(pr, qr, fmaf(-pi, qi, cf[k]));
-                    pi = fmaf(pr, qi, pi * qr);
-                    pr = r2;
-                }
-                cr = delta * pr;
-                ci = delta * pi;
-            } else {
-                const float er = abr - 1.f;
-                cr = fmaf(er, ia[j].x, -abi * ia[j].y);
-                ci = fmaf(er, ia[j].y, abi * ia[j].x);
+            for (int k = 0; k < 4; ++k) {
+                const float r2 = fmaf(pr, qr, fmaf(-pi, qi, cf[k]));
+                pi = fmaf(pr, qi, pi * qr);
+                pr = r2;
             }
-            nr = fmaf(abr, h[j].x, fmaf(-abi, h[j].y, cr * bx));
-            ni = fmaf(abr, h[j].y, fmaf(abi, h[j].x, ci * bx));
+            cr = delta * pr;
+            ci = delta * pi;
+        } else {
+            const float er = abr - 1.f, iar = -comp(s.nr, j), iai = -comp(s.ni, j);  // 1 / a
+            cr = fmaf(er, iar, -abi * iai);
+            ci = fmaf(er, iai, abi * iar);
         }
-        h[j] = make_float2(nr, ni);
+        float& hr = comp(s.hr, j);
+        float& hi = comp(s.hi, j);
+        const float nr = fmaf(abr, hr, fmaf(-abi, hi, cr * bx));
+        const float ni = fmaf(abr, hi, fmaf(abi, hr, ci * bx));
+        hr = nr;
+        hi = ni;
         y = fmaf(Ct[j], nr, y);
     }
     return y;
+}
+
+template <int CG, bool ACC>
+__device__ __forceinline__ float cstep(CLane<CG>& s, float delta, float x, const float* Bt, const float* Ct) {
+    if constexpr (ACC)
+        return cstep_acc<CG>(s, delta, x, Bt, Ct);
+    else
+        return cstep_fast<CG>(s, delta, x, Bt, Ct);
 }
 
 // Sum the partial readouts of a channel's NG lanes (lane bits at multiples of CW)
@@ -120,10 +175,9 @@ __device__ __forceinline__ float creduce(float (&p)[NG], int g) {
 // readout.  Output pass: blocks of NG steps whose readouts are reduced together, lane
 // g finishing step tb + g; FULL tiles (kCTT steps) are unrolled with no step predicate.
 template <typename T, int NG, int CG, bool ACC, bool CKPT, bool FULL>
-__device__ __forceinline__ void scan_tile_c(float2 (&h)[CG], const float2 (&aq)[CG], const float2 (&nia)[CG],
-                                            const float2 (&ia)[CG], const float2* sdx, const float2* sgd,
-                                            const float* sB, const float* sC, int tl, int g, int cw, bool write,
-                                            T* out, int64_t out_stride, float* ck, int64_t ck_stride, int nvalid) {
+__device__ __forceinline__ void scan_tile_c(CLane<CG>& s, const float2* sdx, const float2* sgd, const float* sB,
+                                            const float* sC, int tl, int g, int cw, bool write, T* out,
+                                            int64_t out_stride, float* ck, int64_t ck_stride, int nvalid) {
     using C = CCfg<NG, CG>;
     const float* Bg = sB + g * CG;
     const float* Cg = sC + g * CG;
@@ -134,12 +188,12 @@ __device__ __forceinline__ void scan_tile_c(float2 (&h)[CG], const float2 (&aq)[
 #pragma unroll
                 for (int j = 0; j < CG; ++j)
                     if (j < nvalid) {
-                        ck[(t / 8) * ck_stride + 2 * j] = h[j].x;
-                        ck[(t / 8) * ck_stride + 2 * j + 1] = h[j].y;
+                        ck[(t / 8) * ck_stride + 2 * j] = comp(s.hr, j);
+                        ck[(t / 8) * ck_stride + 2 * j + 1] = comp(s.hi, j);
                     }
             }
             const float2 dx = sdx[t * C::DC + cw];  // (delta, x)
-            (void)cstep<CG, ACC>(h, aq, nia, ia, dx.x, dx.y, Bg + t * C::NS, Cg + t * C::NS);
+            (void)cstep<CG, ACC>(s, dx.x, dx.y, Bg + t * C::NS, Cg + t * C::NS);
         }
     } else {
 #pragma unroll(FULL ? kCTT / NG : 1)
@@ -151,7 +205,7 @@ __device__ __forceinline__ void scan_tile_c(float2 (&h)[CG], const float2 (&aq)[
                 p[k] = 0.f;
                 if (FULL || t < tl) {
                     const float2 dx = sdx[t * C::DC + cw];  // (delta, x)
-                    p[k] = cstep<CG, ACC>(h, aq, nia, ia, dx.x, dx.y, Bg + t * C::NS, Cg + t * C::NS);
+                    p[k] = cstep<CG, ACC>(s, dx.x, dx.y, Bg + t * C::NS, Cg + t * C::NS);
                 }
             }
             const float y = creduce<NG, C::CW>(p, g);
@@ -172,7 +226,8 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
     using C = CCfg<NG, CG>;
     __shared__ float2 sdx[kCTT * C::DC];  // (delta, x)
     __shared__ float2 sgd[kCTT * C::DC];  // (gate, D x gate)
-    __shared__ float sB[kCTT * C::NS], sC[kCTT * C::NS];
+    __shared__ __align__(16) float sB[kCTT * C::NS];
+    __shared__ __align__(16) float sC[kCTT * C::NS];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t ncb = (a.D + C::DC - 1) / C::DC;
     const int64_t b = blockIdx.x / ncb;
@@ -187,7 +242,7 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
     const int g = lane / C::CW, c = lane % C::CW, cw = warp * C::CW + c;
     const int64_t d = d0 + cw;
     const bool cvalid = d < a.D;
-    float2 h[CG], aq[CG], nia[CG], ia[CG];
+    CLane<CG> s;
     bool small_a = false;
 #pragma unroll
     for (int j = 0; j < CG; ++j) {
@@ -197,13 +252,14 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
         const float ai = ok ? __ldg(a.A + (d * N + n) * 2 + 1) : 0.f;
         const float m2 = ar * ar + ai * ai;
         small_a |= ok && m2 < kCSmallA * kCSmallA;
-        aq[j] = make_float2(ar * kLog2e, ai);
+        comp(s.qr, j) = ar * kLog2e;
+        comp(s.qi, j) = ai;
         const float inv = ok && m2 > 0.f ? 1.f / m2 : 0.f;
-        ia[j] = make_float2(ar * inv, -ai * inv);      // 1 / a
-        nia[j] = make_float2(-ia[j].x, -ia[j].y);      // -1 / a
-        h[j] = make_float2(0.f, 0.f);
-        if (ok && a.h0) h[j] = make_float2(__ldg(a.h0 + ((b * a.D + d) * N + n) * 2),
-                                           __ldg(a.h0 + ((b * a.D + d) * N + n) * 2 + 1));
+        comp(s.nr, j) = -ar * inv;  // -1 / a = (-ar + i ai) / |a|^2
+        comp(s.ni, j) = ai * inv;
+        const bool h0v = ok && a.h0;
+        comp(s.hr, j) = h0v ? __ldg(a.h0 + ((b * a.D + d) * N + n) * 2) : 0.f;
+        comp(s.hi, j) = h0v ? __ldg(a.h0 + ((b * a.D + d) * N + n) * 2 + 1) : 0.f;
     }
     const bool acc = __syncthreads_or(small_a ? 1 : 0) != 0;
     const int nvalid = cvalid ? (N - g * CG < CG ? N - g * CG : CG) : 0;
@@ -244,14 +300,14 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
         const int64_t ck_stride = a.D * N * 2;
         const bool wr = cvalid;
         if (acc)
-            scan_tile_c<T, NG, CG, true, CKPT, false>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck,
-                                                      ck_stride, nvalid);
+            scan_tile_c<T, NG, CG, true, CKPT, false>(s, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
+                                                      nvalid);
         else if (tl == kCTT)
-            scan_tile_c<T, NG, CG, false, CKPT, true>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck,
-                                                      ck_stride, nvalid);
+            scan_tile_c<T, NG, CG, false, CKPT, true>(s, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
+                                                      nvalid);
         else
-            scan_tile_c<T, NG, CG, false, CKPT, false>(h, aq, nia, ia, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck,
-                                                       ck_stride, nvalid);
+            scan_tile_c<T, NG, CG, false, CKPT, false>(s, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
+                                                       nvalid);
         __syncthreads();
     }
     if (a.h_last && cvalid) {
@@ -259,8 +315,8 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
         for (int j = 0; j < CG; ++j) {
             const int n = g * CG + j;
             if (n < N) {
-                a.h_last[((b * a.D + d) * N + n) * 2] = h[j].x;
-                a.h_last[((b * a.D + d) * N + n) * 2 + 1] = h[j].y;
+                a.h_last[((b * a.D + d) * N + n) * 2] = comp(s.hr, j);
+                a.h_last[((b * a.D + d) * N + n) * 2 + 1] = comp(s.hi, j);
             }
         }
     }
