@@ -2,7 +2,7 @@
  * sscan_oracle.c -- plain, slow, fp64 CPU oracle for the selective state-space
  * scan (S6) of "Mamba: Linear-Time Sequence Modeling with Selective State
  * Spaces" (Gu & Dao).  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and
- * the benchmark's CPU-baseline leg call it to judge the CUDA library; nothing
+ * the benchmark's CPU-baseline leg call it to check the CUDA library; nothing
  * in the product path links, imports or executes this file.  It shares no code,
  * header, table or helper with the CUDA path.
  *
