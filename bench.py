@@ -133,9 +133,9 @@ NCU_TRAFFIC = {
     "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317504 + 0,
                    "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "b7c6e53d71a0bd30",
                    "profile": "profiles/step_quad_kernel_decode2.8b_bf16.md"},
-    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152343296 + 32550912,
+    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152319232 + 31278080,
                     "sources": ("sscan_complex.cu", "sscan_complex_math.cuh", "sscan_math.cuh"),
-                    "sha256": "45ee83425d235ed2",
+                    "sha256": "2c181ea6f7027cff",
                     "profile": "profiles/fwd_complex_kernel_complex130m_bf16.md"},
     "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 612188672 + 138831616,
                        "sources": ("sscan_complex_bwd.cu", "sscan_complex_math.cuh", "sscan_math.cuh"),
