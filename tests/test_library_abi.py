@@ -84,6 +84,23 @@ def test_workspace_is_required_when_planned(lib):
     assert lib.sscan_workspace_size(ctypes.byref(_p()), 9) == 0
 
 
+def test_backward_workspaces_hold_their_documented_contents(lib):
+    """Host-side sizing only (no device work): the complex backward's workspace is the
+    fp32 dB, dC accumulators (2 x batch L N) plus the complex state before every 8th step
+    (batch x ceil(L/8) x D x N x 2 floats), rounded up to 256 bytes; the real backward's
+    holds at least the accumulators and the fp32 checkpoints (batch x ceil(L/8) x D x N);
+    empty problems need none."""
+    for batch, L, D, N in ((8, 2048, 1536, 16), (2, 777, 40, 8), (1, 9, 5, 1)):
+        p = _p(batch=batch, L=L, D=D, N=N, io=1)
+        nck = -(-L // 8)
+        floats = 2 * batch * L * N + batch * nck * D * N * 2
+        assert lib.sscan_workspace_size(ctypes.byref(p), 4) == -(-floats * 4 // 256) * 256
+        need = lib.sscan_workspace_size(ctypes.byref(p), 2)
+        assert need >= (2 * batch * L * N + batch * nck * D * N) * 4 and need % 256 == 0
+    for batch, L, D in ((0, 10, 4), (2, 0, 4), (2, 10, 0)):
+        assert lib.sscan_workspace_size(ctypes.byref(_p(batch=batch, L=L, D=D, N=4)), 4) == 0
+
+
 def test_last_state_and_bwd_reject_bad_arguments(lib):
     p = _p()
     fake = ctypes.c_void_p(0x10000)
