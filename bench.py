@@ -282,15 +282,15 @@ def cpu_oracle_rate(x: dict, w: W.Workload, target_s: float, seed: int = 0, with
 
 
 def cpu_oracle_rate_1thread(x: dict, w: W.Workload, target_s: float = 2.0, seed: int = 1):
-    """The same oracle on one host thread, for scale (Gelem/s, rows, seconds)."""
+    """The same oracle on one host thread, for scale (Gelem/s, rows, seconds, passes)."""
     import oracle
     threads = oracle.set_threads(0)
     oracle.set_threads(1)
     try:
-        rate, _, rows, secs = cpu_oracle_rate(x, w, target_s, seed)
+        rate, _, rows, secs, passes = cpu_oracle_rate(x, w, target_s, seed, with_passes=True)
     finally:
         oracle.set_threads(threads)
-    return rate, rows, secs
+    return rate, rows, secs, passes
 
 
 def reference_arm(args, w: W.Workload):
@@ -573,13 +573,15 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
     cpu = None
     if world == 1 and not args.no_cpu_baseline and not w.backward and not w.decode and not w.complex_a:
         rate, cores, rows, secs, passes = cpu_oracle_rate(x, w, args.cpu_seconds, with_passes=True)
-        rate1, rows1, secs1 = cpu_oracle_rate_1thread(x, w)
+        rate1, rows1, secs1, passes1 = cpu_oracle_rate_1thread(x, w)
         what = (f"{passes} passes over all {rows} rows" if passes > 1 else
                 f"{rows} random rows of {w.batch * w.dim}")
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{what} x L={w.seqlen} ({passes * rows * w.seqlen} elements, {secs:.1f} s)",
                "single_thread": {"value": rate1, "unit": UNIT,
-                                 "sample": f"{rows1} random rows x L={w.seqlen}, {secs1:.1f} s on 1 thread"}}
+                                 "sample": f"{rows1} random rows x L={w.seqlen}"
+                                           + (f", {passes1} passes" if passes1 > 1 else "")
+                                           + f", {secs1:.1f} s on 1 thread"}}
     line = {
         "metric": (METRIC_COMPLEX_BWD if w.backward and w.complex_a else METRIC_BWD if w.backward
                    else METRIC_STEP if w.decode else METRIC_COMPLEX if w.complex_a else METRIC), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
