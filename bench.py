@@ -293,6 +293,48 @@ def cpu_oracle_rate_1thread(x: dict, w: W.Workload, target_s: float = 2.0, seed:
     return rate, rows, secs, passes
 
 
+def block_rows(w: W.Workload, per_block: int, seed: int, dc: int = 32) -> np.ndarray:
+    """(batch, channel) rows covering every block of ``dc`` consecutive channels (the
+    tiled kernel's CTA width at N = 16): ``per_block`` random channels of each block,
+    each in a random batch."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    for c0 in range(0, w.dim, dc):
+        width = min(dc, w.dim - c0)
+        ch = c0 + rng.choice(width, size=min(per_block, width), replace=False)
+        rows.extend(rng.integers(0, w.batch, size=ch.size) * w.dim + ch)
+    return np.unique(np.asarray(rows, np.int64))
+
+
+def error_measures(got: np.ndarray, ref: np.ndarray, floor: float = 1e-3) -> dict:
+    """Normwise max|got - ref| / max|ref|, and the pointwise max |got - ref| / |ref| over
+    the elements with |ref| >= floor * max|ref|."""
+    a = np.abs(ref)
+    mx = float(a.max()) if a.size else 0.0
+    err = np.abs(got - ref)
+    keep = a >= floor * mx
+    return {"normwise": float(err.max() / mx) if mx > 0 else float(err.max(initial=0.0)),
+            "pointwise": float((err[keep] / a[keep]).max()) if keep.any() else 0.0}
+
+
+def oracle_parity(x: dict, w: W.Workload, out, per_block: int = 2, seed: int = 77) -> dict:
+    """The timed run's own output against the fp64 oracle on a row sample that covers
+    every channel block (``per_block`` rows per 32-channel block, each a whole
+    sequence)."""
+    import oracle
+    import torch
+    rows = block_rows(w, per_block, seed)
+    b = torch.as_tensor(rows // w.dim, device=out.device)
+    d = torch.as_tensor(rows % w.dim, device=out.device)
+    got = out[b, :, d].double().cpu().numpy()
+    ref, _ = oracle.fwd(x["u"], x["delta_raw"], x["A"], x["B"], x["C"], delta_bias=x["delta_bias"],
+                        D_skip=x["D_skip"], z=x.get("z"), rows=rows)
+    tol = 2e-2 if w.io == "bf16" else 1e-4
+    m = error_measures(got, ref)
+    return {**m, "tolerance_normwise": tol, "ok": bool(m["normwise"] <= tol),
+            "sample": f"{rows.size} rows ({per_block} per 32-channel block, every block) x L={w.seqlen}"}
+
+
 def reference_arm(args, w: W.Workload):
     """The oracle as it stands, timed on the host cores: K timed steps (after W
     warm-up steps), each a bounded random sample of the workload's rows."""
@@ -492,8 +534,62 @@ def gpu_arm(args, w: W.Workload):
         e2e_value, h2d, d2h = e2e_leg(args, t, out, ws, st, units, world, dev)
     if rank != 0:
         return
+    secondary = None
+    if world == 1 and args.workload == DEFAULT_WORKLOAD and not args.no_secondary:
+        del t
+        secondary = fp32_record(args, lib, dev)
     finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk, e2e_value, h2d, d2h,
-           launches_per_step, world, l2_note)
+           launches_per_step, world, l2_note, out=out if not (w.backward or w.decode or w.complex_a) else None,
+           secondary=secondary)
+
+
+def fp32_record(args, lib, dev) -> dict:
+    """The same layer with fp32 I/O (the headline shape's second precision): K timed
+    forward passes after the warm-up, their per-launch time, Gelem/s, roofline fraction
+    and the output's error against the oracle on a row sample covering every channel
+    block.  Runs after the bf16 measurement, once its tensors are released."""
+    import torch
+
+    from selective_state_space_33_b200 import binding as sb
+    w = W.WORKLOADS["mamba2.8b-f32"]
+    x = W.make_inputs(w)
+    t = W.to_device(x, dev)
+    out = torch.empty_like(t["u"])
+    prob = sb.make_problem(w.batch, w.seqlen, w.dim, w.dstate, sb.SSCAN_F32)
+    ws = torch.empty(max(sb.sscan_workspace_size(prob, sb.SSCAN_OP_FWD), 256), dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+
+    def step():
+        sb.sscan_fwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["delta_bias"], t["D_skip"], t["z"],
+                     out=out, workspace=ws, stream=st)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        a.record(st)
+        step()
+        b.record(st)
+    torch.cuda.synchronize()
+    per_launch = statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e-3
+    total = ev[0][0].elapsed_time(ev[-1][1]) * 1e-3
+    units = roofline_units(w)
+    peaks = measured_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", HBM_FALLBACK_GBS))
+    mufu = SM_COUNT * MUFU_PER_SM_CLK * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    rec = {"workload": f"{w.name}: {w.description}", "io_dtype": "f32",
+           "value": aggregate(units["elements"], args.steps, 1, total), "unit": UNIT,
+           "ms_per_step": total / args.steps * 1e3, "steps": args.steps,
+           "roofline": {"bound": "alu", "pipe": "MUFU ex2", "achieved": units["exps"] / per_launch / 1e9,
+                        "peak": mufu / 1e9, "unit": "Gexp/s", "frac": units["exps"] / per_launch / mufu,
+                        "per_launch_ms": per_launch * 1e3, "alg_exps_per_launch": units["exps"],
+                        "hbm": {"achieved": units["bytes"] / per_launch / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                                "frac": units["bytes"] / per_launch / 1e9 / hbm_peak,
+                                "alg_bytes_per_launch": units["bytes"]}}}
+    if not args.no_cpu_baseline:
+        rec["parity"] = oracle_parity(x, w, out)
+    return rec
 
 
 def e2e_leg(args, t, out, ws, st, units, world, dev):
@@ -557,7 +653,7 @@ def e2e_leg(args, t, out, ws, st, units, world, dev):
 
 
 def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk, e2e_value, h2d, d2h,
-           launches_per_step, world, l2_note):
+           launches_per_step, world, l2_note, out=None, secondary=None):
     peaks = measured_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", HBM_FALLBACK_GBS))
     hbm_src = "measured" if "hbm_gbs" in peaks else "fallback"
@@ -582,6 +678,8 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
                                  "sample": f"{rows1} random rows x L={w.seqlen}"
                                            + (f", {passes1} passes" if passes1 > 1 else "")
                                            + f", {secs1:.1f} s on 1 thread"}}
+        if out is not None:
+            cpu["parity"] = oracle_parity(x, w, out)
     line = {
         "metric": (METRIC_COMPLEX_BWD if w.backward and w.complex_a else METRIC_BWD if w.backward
                    else METRIC_STEP if w.decode else METRIC_COMPLEX if w.complex_a else METRIC), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -609,6 +707,10 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
         },
         "cpu_baseline": cpu,
     }
+    if cpu is not None and "parity" in cpu:
+        line["parity"] = cpu["parity"]
+    if secondary is not None:
+        line["secondary"] = secondary
     print(json.dumps(line), flush=True)
 
 
@@ -617,6 +719,19 @@ def hbm_roofline(units, launch_s, hbm_peak, hbm_src, traffic=None):
     return {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
             "traffic": traffic, "source": hbm_src, "per_launch_ms": launch_s * 1e3,
             "alg_bytes_per_launch": units["bytes"]}
+
+
+def launch_ranks(n: int, argv: list):
+    """Run this script as ``n`` ranks on one node (one process per GPU) through
+    torch.distributed.run on the loopback address; replaces the current process."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + argv
+    sys.stdout.flush()
+    os.execv(sys.executable, cmd)
 
 
 def main(argv=None):
@@ -628,10 +743,17 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the fp32-I/O record that follows the default (bf16) workload")
     ap.add_argument("--profile-run", action="store_true",
                     help="timed steps only (no clock tail, end-to-end leg, probe or CPU baseline): "
                          "the command line used under ncu")
     args = ap.parse_args(argv)
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        launch_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv))
+    if world_env is not None and int(world_env) != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but the launcher started WORLD_SIZE={world_env} ranks")
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":
         reference_arm(args, w)

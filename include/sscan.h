@@ -133,8 +133,9 @@ SSCAN_API sscan_status sscan_last_state(const sscan_problem* problem, const void
  * than that (possible only on the general path for unaligned tensors) returns
  * SSCAN_ERR_WORKSPACE before anything is launched.  The first call on each
  * device looks up the array's device address (cudaGetSymbolAddress, with that
- * device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array and it keeps the last call's
+ * device current) and caches it for the process; make that first call before any
+ * stream capture.  A cudaDeviceReset between calls is not supported (the cached
+ * address would be stale).  All calls share the one array and it keeps the last call's
  * contents; the kernels overwrite every scratch byte they later read, so nothing
  * needs clearing.  Calls whose work overlaps on the GPU (different streams, or
  * different host threads without ordering) race on the scratch: serialise them.

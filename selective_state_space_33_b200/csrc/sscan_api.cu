@@ -272,12 +272,29 @@ void cast_out(const float* src, void* dst, int64_t n, cudaStream_t st) {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+// The bound above, from plan_tiled's own constants: a split plan has cols < kTiledMinCols
+// CTA columns of DC channels and ceil(kTiledTargetCtas / cols) chunks, i.e. fewer than
+// kTiledTargetCtas + kTiledMinCols column-chunks, each holding DC * (N + 1) floats
+// (the chunk's end states and delta sum); DC * (N + 1) is largest at N = 4 (DC = 128).
+constexpr size_t tiled_scratch_bound() {
+    size_t worst = 0;
+    for (int n = 1; n <= sscan::kMaxState; ++n) {
+        const size_t dc = n <= 4 ? 128 : (n <= 8 ? 64 : 32);
+        const size_t b = (size_t)(sscan::kTiledTargetCtas + sscan::kTiledMinCols - 1) * dc * (n + 1) * 4 + 255;
+        worst = b > worst ? b : worst;
+    }
+    return worst;
+}
+static_assert(tiled_scratch_bound() <= kNoAllocScratchBytes,
+              "the static scratch must hold every plan of the tiled forward path");
+
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
 // Device address of the scratch on the current device, looked up once per device
-// (with that device current) and cached.
+// (with that device current) and cached for the process.  A cudaDeviceReset between
+// calls would leave a stale address behind, so it is not supported.
 sscan_status noalloc_scratch(void** ptr) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);

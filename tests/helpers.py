@@ -25,4 +25,21 @@ def normwise(got, ref) -> float:
     return float(err / denom) if denom > 0 else float(err)
 
 
+def pointwise(got, ref, floor: float = 1e-3) -> float:
+    """max |got - ref| / |ref| over the elements with |ref| >= floor * max |ref|.
+
+    Reported beside the normwise error: outputs gated by SiLU(z) with z near 0, or
+    whose readout and skip term nearly cancel, sit close to zero, where a relative
+    error says little; the floor leaves those out."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    if ref.size == 0:
+        return 0.0
+    a = np.abs(ref)
+    keep = a >= floor * a.max()
+    if not keep.any():
+        return 0.0
+    return float(np.max(np.abs(got[keep] - ref[keep]) / a[keep]))
+
+
 TOL = {"f32": 1e-4, "bf16": 2e-2}

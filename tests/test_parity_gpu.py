@@ -1,6 +1,8 @@
 """GPU parity: the CUDA library (through its C ABI) against the fp64 CPU oracle on
 the same seeded inputs.  Tolerance (normwise, per tensor): max|gpu - ref| / max|ref|
-<= 1e-4 for fp32 I/O and <= 2e-2 for bf16 I/O."""
+<= 1e-4 for fp32 I/O and <= 2e-2 for bf16 I/O.  The pointwise relative error over
+the elements with |ref| >= 1e-3 max|ref| is reported beside it (and bounded where
+a test says so)."""
 import math
 
 import numpy as np
@@ -11,7 +13,7 @@ import oracle
 from selective_state_space_33_b200 import binding as sb
 from selective_state_space_33_b200 import workloads as W
 
-from .helpers import TOL, normwise, to_f64, to_torch
+from .helpers import TOL, normwise, pointwise, to_f64, to_torch
 
 pytestmark = pytest.mark.gpu
 
@@ -52,40 +54,115 @@ def test_mamba130m_bf16_full(cuda_device):
     _check_full(x, "bf16", cuda_device)
 
 
-def _sampled_rows(w, k, seed):
+def _block_rows(w, per_block, seed, dc=32):
+    """(batch, channel) rows covering every block of ``dc`` consecutive channels (the
+    tiled kernel's CTA width at N = 16): ``per_block`` random channels of each block,
+    each in a random batch, plus the first and last channel of the first and last
+    batch."""
     rng = np.random.default_rng(seed)
-    rows = rng.choice(w.batch * w.dim, size=k, replace=False)
-    # always include the first and last channel of the first and last batch
-    extra = [0, w.dim - 1, (w.batch - 1) * w.dim, w.batch * w.dim - 1]
-    return np.unique(np.concatenate([rows, extra]))
+    rows = []
+    for c0 in range(0, w.dim, dc):
+        width = min(dc, w.dim - c0)
+        ch = c0 + rng.choice(width, size=min(per_block, width), replace=False)
+        rows.extend(rng.integers(0, w.batch, size=ch.size) * w.dim + ch)
+    rows.extend([0, w.dim - 1, (w.batch - 1) * w.dim, w.batch * w.dim - 1])
+    return np.unique(np.asarray(rows, np.int64))
 
 
-def _check_sampled(w, dev, k=96):
+def _report(name, **errs):
+    print(f"[parity] {name}: " + ", ".join(f"{k}={v:.3e}" for k, v in errs.items()))
+
+
+# Pointwise bounds (|ref| >= 1e-3 max|ref|).  fp32 arithmetic leaves a normwise error
+# near 1e-6, which an element at 1e-3 of the maximum sees as up to ~1e-3 relative;
+# bf16 I/O adds the output's own rounding (2^-9 relative).  Measured on B200: fp32
+# out 2.3e-4, bf16 out 4.0e-3, final states up to 3.2e-3.
+POINTWISE = {"f32": 1e-3, "bf16": 2e-2, "state": 1e-2}
+
+
+def _check_whole(w, dev):
+    """Every output element and every final state of a full-size workload against the
+    oracle (about a second of oracle time per pass on a 16-core host)."""
     x = W.make_inputs(w)
     t = to_torch(x, dev)
     out, hl = _gpu_fwd(t, return_last_state=True)
     torch.cuda.synchronize()
-    rows = _sampled_rows(w, k, w.seed)
-    ref, ref_h = _oracle_fwd(x, rows=rows)
-    b, d = rows // w.dim, rows % w.dim
-    got = to_f64(out[b, :, d])                     # (rows, L)
-    got_h = to_f64(hl.reshape(-1, w.dstate)[rows])
+    del t
+    got, got_h = to_f64(out), to_f64(hl)
+    del out, hl
+    ref, ref_h = _oracle_fwd(x)
     e_out, e_h = normwise(got, ref), normwise(got_h, ref_h)
+    p_out, p_h = pointwise(got, ref), pointwise(got_h, ref_h)
+    _report(w.name, out_normwise=e_out, out_pointwise=p_out, h_normwise=e_h, h_pointwise=p_h)
+    assert np.isfinite(got).all()
     assert e_out <= TOL[w.io], e_out
     assert e_h <= TOL[w.io], e_h
-    assert torch.isfinite(out.float()).all()
+    assert p_out <= POINTWISE[w.io], p_out
+    assert p_h <= POINTWISE["state"], p_h
+    return p_out, p_h
 
 
-def test_mamba2p8b_bf16_sampled(cuda_device):
-    _check_sampled(W.WORKLOADS["mamba2.8b"], cuda_device)
+def test_mamba2p8b_bf16_whole(cuda_device):
+    _check_whole(W.WORKLOADS["mamba2.8b"], cuda_device)
 
 
-def test_mamba2p8b_fp32_sampled(cuda_device):
-    _check_sampled(W.WORKLOADS["mamba2.8b-f32"], cuda_device)
+def test_mamba2p8b_fp32_whole(cuda_device):
+    _check_whole(W.WORKLOADS["mamba2.8b-f32"], cuda_device)
 
 
 def test_million_length_sampled(cuda_device):
-    _check_sampled(W.WORKLOADS["million"], cuda_device, k=16)
+    """L = 2^20 over 1536 channels: the sequence is split into chunks joined by the
+    cross-chunk carry.  Three rows of every 32-channel block (144 rows, about 150 M
+    elements of oracle work) and their final states."""
+    w = W.WORKLOADS["million"]
+    x = W.make_inputs(w)
+    t = to_torch(x, cuda_device)
+    out, hl = _gpu_fwd(t, return_last_state=True)
+    torch.cuda.synchronize()
+    rows = _block_rows(w, 3, w.seed)
+    assert rows.size >= 144
+    b, d = rows // w.dim, rows % w.dim
+    got = to_f64(out[b, :, d])                     # (rows, L)
+    got_h = to_f64(hl.reshape(-1, w.dstate)[rows])
+    del out, t
+    ref, ref_h = _oracle_fwd(x, rows=rows)
+    e_out, e_h = normwise(got, ref), normwise(got_h, ref_h)
+    p_out, p_h = pointwise(got, ref), pointwise(got_h, ref_h)
+    _report(w.name, rows=rows.size, out_normwise=e_out, out_pointwise=p_out, h_normwise=e_h, h_pointwise=p_h)
+    assert e_out <= TOL[w.io], e_out
+    assert e_h <= TOL[w.io], e_h
+    assert p_out <= POINTWISE[w.io], p_out
+    assert p_h <= POINTWISE["state"], p_h
+    assert np.isfinite(got).all()
+
+
+@pytest.mark.parametrize("variant", ["skip_gate", "bare"])
+@pytest.mark.parametrize("shape", [(1, 65536, 64, 16), (4, 2047, 96, 16)])
+def test_fp32_small_delta_long_sequence(cuda_device, variant, shape):
+    """fp32 I/O with delta log-uniform in [1e-4, 1e-2] and A = -(n+1), the million-step
+    workload's regime, where |delta A| reaches 1e-4 and a step's increment
+    (Abar - 1)(h - v) is a small difference: held to the fp32 tolerance.  The long
+    case (2^16 steps, 64 channels) runs through the sequence split and carry, the
+    other through one pass per row.  'bare' drops the skip term and the gate, so the
+    output is the readout C.h alone and no larger term hides an error in the state."""
+    batch, L, D, N = shape
+    x = W.small_case(batch, L, D, N, io="f32", seed=L + D, dt_min=1e-4, dt_max=1e-2, dskip="ones")
+    if variant == "bare":
+        del x["z"], x["D_skip"]
+    t = to_torch(x, cuda_device)
+    out, hl = _gpu_fwd(t, return_last_state=True)
+    torch.cuda.synchronize()
+    ref, ref_h = _oracle_fwd(x)
+    got, got_h = to_f64(out), to_f64(hl)
+    e_out, e_h = normwise(got, ref), normwise(got_h, ref_h)
+    p_out, p_h = pointwise(got, ref), pointwise(got_h, ref_h)
+    _report(f"small-delta {shape} {variant}", out_normwise=e_out, out_pointwise=p_out, h_normwise=e_h,
+            h_pointwise=p_h)
+    assert e_out <= TOL["f32"], e_out
+    assert e_h <= TOL["f32"], e_h
+    assert p_h <= POINTWISE["state"], p_h
+    if variant == "skip_gate":
+        assert p_out <= POINTWISE["f32"], p_out
 
 
 # ---------------------------------------------------------------- tails, options, N

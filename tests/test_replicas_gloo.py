@@ -58,7 +58,8 @@ def _ref_worker(rank, world, port, q):
     import bench
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
-        bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"])
+        bench.main(["--gpus", str(world), "--impl", "reference", "--workload", "tiny", "--steps", "1",
+                    "--warmup", "0"])
     q.put((rank, buf.getvalue()))
 
 
@@ -77,3 +78,27 @@ def test_reference_arm_prints_on_rank0_only():
     line = json.loads(res[0].strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert res[1].strip() == ""
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """``bench.py --gpus 2`` started without a launcher runs itself as 2 ranks (one
+    process per GPU) and reports n_gpus 2; the reference arm needs no GPU."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, timeout=600, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    assert json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_gpus_flag_must_match_the_launcher():
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode != 0 and "WORLD_SIZE=1" in r.stderr
