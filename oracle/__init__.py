@@ -24,7 +24,8 @@ _lib = None
 class _Problem(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
                 ("dim", ctypes.c_int64), ("dstate", ctypes.c_int64),
-                ("io_dtype", ctypes.c_int32), ("delta_softplus", ctypes.c_int32)]
+                ("io_dtype", ctypes.c_int32), ("delta_softplus", ctypes.c_int32),
+                ("input_silu", ctypes.c_int32)]
 
 
 def _load():
@@ -89,12 +90,14 @@ def _ptr(a):
 
 
 def fwd(u, delta_raw, A, B, C, *, delta_bias=None, D_skip=None, z=None, h0=None,
-        delta_softplus=True, rows=None, want_out=True):
+        delta_softplus=True, rows=None, want_out=True, input_silu=False):
     """Forward scan in fp64.  Returns (out, h_last).
 
     rows=None: out (batch, L, D), h_last (batch, D, N).
     rows=[b*D+d, ...]: out (len(rows), L), h_last (len(rows), N) for those rows only.
     want_out=False computes only h_last (the last-state operation).
+    input_silu=True feeds x = SiLU(u) to the scan instead of u (the input-branch
+    activation of the Mamba block, Fig. 3 caption).
     """
     (u, delta_raw, B, C, z), code = _ios(u, delta_raw, B, C, z)
     batch, L, D = u.shape
@@ -112,7 +115,7 @@ def fwd(u, delta_raw, A, B, C, *, delta_bias=None, D_skip=None, z=None, h0=None,
         nr = 0
         out = np.empty((batch, L, D), np.float64) if want_out else None
         h_last = np.empty((batch, D, N), np.float64)
-    prob = _Problem(batch, L, D, N, code, 1 if delta_softplus else 0)
+    prob = _Problem(batch, L, D, N, code, 1 if delta_softplus else 0, 1 if input_silu else 0)
     rc = _load().orc_fwd(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias), _ptr(A),
                          _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h0), _ptr(rows), nr,
                          _ptr(out), _ptr(h_last))
@@ -122,7 +125,7 @@ def fwd(u, delta_raw, A, B, C, *, delta_bias=None, D_skip=None, z=None, h0=None,
 
 
 def bwd(u, delta_raw, A, B, C, dout, *, delta_bias=None, D_skip=None, z=None, h0=None,
-        delta_softplus=True):
+        delta_softplus=True, input_silu=False):
     """Reverse-mode gradients of sum(out * dout) in fp64.
 
     Returns a dict with du, ddelta_raw (batch, L, D); dA (D, N); dB, dC (batch, L, N);
@@ -140,7 +143,7 @@ def bwd(u, delta_raw, A, B, C, dout, *, delta_bias=None, D_skip=None, z=None, h0
     g["ddelta_bias"] = np.empty(D) if delta_bias is not None else None
     g["dD"] = np.empty(D) if D_skip is not None else None
     g["dz"] = np.empty((batch, L, D)) if z is not None else None
-    prob = _Problem(batch, L, D, N, code, 1 if delta_softplus else 0)
+    prob = _Problem(batch, L, D, N, code, 1 if delta_softplus else 0, 1 if input_silu else 0)
     rc = _load().orc_bwd(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias), _ptr(A),
                          _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h0), _ptr(dout),
                          _ptr(g["du"]), _ptr(g["ddelta_raw"]), _ptr(g["ddelta_bias"]),
@@ -164,7 +167,7 @@ def _interleave(c, shape):
 
 
 def fwd_complex(u, delta_raw, A, B, C, *, delta_bias=None, D_skip=None, z=None, h0=None,
-                delta_softplus=True, want_out=True):
+                delta_softplus=True, want_out=True, input_silu=False):
     """Forward scan with a complex diagonal A in fp64.  A: (D, N) complex (or (D, N, 2)
     real pairs); h0: (batch, D, N) complex or None.  B, C real (batch, L, N).
     Returns (out (batch, L, D) real, h_last (batch, D, N) complex128)."""
@@ -176,7 +179,7 @@ def fwd_complex(u, delta_raw, A, B, C, *, delta_bias=None, D_skip=None, z=None, 
     delta_bias, D_skip = _f64(delta_bias), _f64(D_skip)
     out = np.empty((batch, L, D), np.float64) if want_out else None
     h_last = np.empty((batch, D, N, 2), np.float64)
-    prob = _Problem(batch, L, D, N, code, 1 if delta_softplus else 0)
+    prob = _Problem(batch, L, D, N, code, 1 if delta_softplus else 0, 1 if input_silu else 0)
     rc = _load().orc_fwd_complex(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias), _ptr(A2),
                                  _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h02), _ptr(out), _ptr(h_last))
     if rc != 0:
@@ -185,7 +188,7 @@ def fwd_complex(u, delta_raw, A, B, C, *, delta_bias=None, D_skip=None, z=None, 
 
 
 def bwd_complex(u, delta_raw, A, B, C, dout, *, delta_bias=None, D_skip=None, z=None, h0=None,
-                delta_softplus=True):
+                delta_softplus=True, input_silu=False):
     """Reverse-mode gradients of sum(out * dout) for the complex-A scan, fp64.
     dA (D, N) and dh0 (batch, D, N) are complex128 (dL/dRe + i dL/dIm); the rest real,
     keyed as in ``bwd``."""
@@ -201,7 +204,7 @@ def bwd_complex(u, delta_raw, A, B, C, dout, *, delta_bias=None, D_skip=None, z=
     g["ddelta_bias"] = np.empty(D) if delta_bias is not None else None
     g["dD"] = np.empty(D) if D_skip is not None else None
     g["dz"] = np.empty((batch, L, D)) if z is not None else None
-    prob = _Problem(batch, L, D, N, code, 1 if delta_softplus else 0)
+    prob = _Problem(batch, L, D, N, code, 1 if delta_softplus else 0, 1 if input_silu else 0)
     rc = _load().orc_bwd_complex(ctypes.byref(prob), _ptr(u), _ptr(delta_raw), _ptr(delta_bias), _ptr(A2),
                                  _ptr(B), _ptr(C), _ptr(D_skip), _ptr(z), _ptr(h02), _ptr(dout),
                                  _ptr(g["du"]), _ptr(g["ddelta_raw"]), _ptr(g["ddelta_bias"]),

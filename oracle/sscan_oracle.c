@@ -14,7 +14,9 @@
  *   sec. 2.1 eq. (3a)/(3b)  recurrence h_t = Abar h_{t-1} + Bbar x_t, y_t = C h_t
  *   sec. 3.2                delta, B, C are functions of the input; delta passes
  *                           through softplus
- *   Fig. 3 caption          the block's gate uses SiLU
+ *   Fig. 3 caption          the block's gate uses SiLU, and the block replaces
+ *                           the first multiplicative gate with an activation
+ *                           (SiLU) on the input branch ahead of the SSM
  *   sec. 4.1                the scan reads (delta, A, B, C) and writes only
  *                           (B, L, D) outputs
  * Readings where the pages are silent (all marked again at the use site):
@@ -26,6 +28,10 @@
  *   - a skip term D_skip[d]*x_t is added to y_t, and the result is multiplied
  *     by SiLU(z_t) when a gate input z is given: out = (C.h + D x) * SiLU(z).
  *   - h_{-1} is zero unless an initial state h0 is given.
+ *   - with the input-activation flag the scan's input is x_t = SiLU(u_t) (the
+ *     activation of the Fig. 3 input branch; the pages give no convolution or
+ *     projection around it, so none is applied), used both in Bbar x_t and in
+ *     the skip term; otherwise x_t = u_t.
  *   - layouts are dense row-major: u, delta_raw, z, out: (batch, L, D);
  *     B, C: (batch, L, N) shared by all D channels; A: (D, N);
  *     h0 / h_last: (batch, D, N).
@@ -49,6 +55,7 @@ typedef struct {
     int64_t batch, seqlen, dim, dstate;
     int32_t io_dtype;       /* element type of u, delta_raw, z, B, C, dout */
     int32_t delta_softplus; /* nonzero: delta = softplus(delta_raw + bias) */
+    int32_t input_silu;     /* nonzero: the scan's input is x = SiLU(u)          */
 } orc_problem;
 
 /* Widen one element of an input array to double (exact for all three types). */
@@ -72,6 +79,20 @@ static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
 
 /* SiLU(v) = v * sigmoid(v) (Fig. 3 caption: the gate activation). */
 static double silu(double v) { return v * sigmoid(v); }
+
+/* d SiLU / dv = sigmoid(v) (1 + v (1 - sigmoid(v))). */
+static double dsilu(double v)
+{
+    const double s = sigmoid(v);
+    return s * (1.0 + v * (1.0 - s));
+}
+
+/* The scan's input x_t for the stored u_t: SiLU(u_t) when the input-branch
+ * activation of Fig. 3 is requested, else u_t itself. */
+static double scan_input(const orc_problem* p, double uv) { return p->input_silu ? silu(uv) : uv; }
+
+/* dx_t/du_t for scan_input. */
+static double scan_input_grad(const orc_problem* p, double uv) { return p->input_silu ? dsilu(uv) : 1.0; }
 
 /* Bbar / B for one state, from eq. (2) with diagonal A: expm1(d*a)/a,
  * and its limit d when a == 0. */
@@ -136,7 +157,7 @@ int orc_fwd(const orc_problem* p, const void* u, const void* delta_raw,
         for (int64_t t = 0; t < L; ++t) {
             const int64_t e = (b * L + t) * D + d; /* (batch, L, D) element */
             const int64_t s = (b * L + t) * N;     /* (batch, L, N) row     */
-            const double x = ld(u, dt, e);
+            const double x = scan_input(p, ld(u, dt, e));
             const double r = ld(delta_raw, dt, e) + (delta_bias ? delta_bias[d] : 0.0);
             const double delta = p->delta_softplus ? softplus(r) : r;
             double y = 0.0;
@@ -219,7 +240,7 @@ int orc_bwd(const orc_problem* p, const void* u, const void* delta_raw,
             for (int64_t n = 0; n < N; ++n) hs[n] = h0 ? h0[row * N + n] : 0.0;
             for (int64_t t = 0; t < L; ++t) {
                 const int64_t e = (b * L + t) * D + d, s = (b * L + t) * N;
-                const double x = ld(u, dt, e);
+                const double x = scan_input(p, ld(u, dt, e));
                 const double r = ld(delta_raw, dt, e) + bias;
                 const double delta = p->delta_softplus ? softplus(r) : r;
                 double y = 0.0;
@@ -236,7 +257,7 @@ int orc_bwd(const orc_problem* p, const void* u, const void* delta_raw,
             for (int64_t n = 0; n < N; ++n) lam[n] = 0.0; /* Abar_{t+1} lam_{t+1} */
             for (int64_t t = L - 1; t >= 0; --t) {
                 const int64_t e = (b * L + t) * D + d, s = (b * L + t) * N;
-                const double x = ld(u, dt, e);
+                const double x = scan_input(p, ld(u, dt, e));
                 const double r = ld(delta_raw, dt, e) + bias;
                 const double delta = p->delta_softplus ? softplus(r) : r;
                 const double g = ld(dout, dt, e);
@@ -266,7 +287,7 @@ int orc_bwd(const orc_problem* p, const void* u, const void* delta_raw,
                     lam[n] = abar * l;
                 }
                 const double dr = p->delta_softplus ? ddelta * sigmoid(r) : ddelta;
-                du[e] = dx;
+                du[e] = dx * scan_input_grad(p, ld(u, dt, e));
                 ddelta_raw[e] = dr;
                 pbias[row] += dr;
             }
@@ -338,7 +359,7 @@ int orc_fwd_complex(const orc_problem* p, const void* u, const void* delta_raw,
         for (int64_t t = 0; t < L; ++t) {
             const int64_t e = (b * L + t) * D + d;
             const int64_t s = (b * L + t) * N;
-            const double x = ld(u, dt, e);
+            const double x = scan_input(p, ld(u, dt, e));
             const double r = ld(delta_raw, dt, e) + (delta_bias ? delta_bias[d] : 0.0);
             const double delta = p->delta_softplus ? softplus(r) : r;
             double y = 0.0;
@@ -448,7 +469,7 @@ int orc_bwd_complex(const orc_problem* p, const void* u, const void* delta_raw,
             h[n] = h0 ? h0[(row * N + n) * 2] + I * h0[(row * N + n) * 2 + 1] : 0.0;
         for (int64_t t = 0; t < L; ++t) {
             const int64_t e = (b * L + t) * D + d, s = (b * L + t) * N;
-            const double x = ld(u, dt, e);
+            const double x = scan_input(p, ld(u, dt, e));
             const double r = ld(delta_raw, dt, e) + (delta_bias ? delta_bias[d] : 0.0);
             const double delta = p->delta_softplus ? softplus(r) : r;
             for (int64_t n = 0; n < N; ++n) {
@@ -463,7 +484,7 @@ int orc_bwd_complex(const orc_problem* p, const void* u, const void* delta_raw,
         double dDacc = 0.0, dbacc = 0.0;
         for (int64_t t = L - 1; t >= 0; --t) {
             const int64_t e = (b * L + t) * D + d, s = (b * L + t) * N;
-            const double x = ld(u, dt, e);
+            const double x = scan_input(p, ld(u, dt, e));
             const double r = ld(delta_raw, dt, e) + (delta_bias ? delta_bias[d] : 0.0);
             const double delta = p->delta_softplus ? softplus(r) : r;
             const double go = ld(dout, dt, e);
@@ -497,7 +518,7 @@ int orc_bwd_complex(const orc_problem* p, const void* u, const void* delta_raw,
                 lam[n] = conj(abar) * l;
             }
             const double drr = p->delta_softplus ? ddelta * sigmoid(r) : ddelta;
-            du[e] = dx;
+            du[e] = dx * scan_input_grad(p, ld(u, dt, e));
             ddelta_raw[e] = drr;
             dbacc += drr;
         }

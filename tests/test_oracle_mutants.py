@@ -48,6 +48,8 @@ MUTANTS = {
     "complex_bwd_dA_imag_sign": ("dA[(d * N + n) * 2 + 1] -= cimag(g);", "dA[(d * N + n) * 2 + 1] += cimag(g);"),
     "complex_bwd_psi_term": ("q * (1.0 / 8.0 + q * (1.0 / 30.0 + q * (1.0 / 144.0))));\n    return (q * cexp(q)",
                              "q * (1.0 / 6.0 + q * (1.0 / 30.0 + q * (1.0 / 144.0))));\n    return (q * cexp(q)"),
+    "input_silu_skip_raw": ("if (D_skip) y += D_skip[d] * x;", "if (D_skip) y += D_skip[d] * ld(u, dt, e);"),
+    "input_silu_no_chain": ("du[e] = dx * scan_input_grad(p, ld(u, dt, e));", "du[e] = dx;"),
     "complex_bwd_ddelta_drop": ("ddelta += creal(conj(l) * (a * abar * hp + abar * Bn * x));",
                                 "ddelta += creal(conj(l) * (abar * Bn * x));"),
 }

@@ -353,3 +353,86 @@ def test_single_step_against_decimal_arithmetic(delta, a):
     g = oracle.bwd(one, np.full((1, 1, 1), delta), np.array([[a]]), one, one, one, delta_softplus=False)
     assert abs(out.item() - y_ref) <= 4e-16 * abs(y_ref)
     assert abs(g["dA"].item() - dA_ref) <= 1e-12 * abs(dA_ref), (g["dA"].item(), dA_ref)
+
+
+# ---------------------------------------------------------------- input-branch activation (Fig. 3)
+def test_input_silu_equals_scan_of_activated_input():
+    """With the input-branch activation the scan's input is x = SiLU(u) (Fig. 3
+    caption: the block's first gate becomes an activation, sigma = SiLU).  Forming
+    u * expit(u) with scipy and scanning it without the flag must give the same
+    outputs and final states, in the state update and the skip term alike."""
+    from scipy.special import expit
+    x = W.small_case(2, 40, 6, 5, io="f32", seed=31)
+    u = x["u"].astype(np.float64)
+    h0 = np.random.default_rng(31).standard_normal((2, 6, 5))
+    kw = dict(delta_bias=x["delta_bias"], D_skip=x["D_skip"], z=x["z"], h0=h0)
+    o1, l1 = oracle.fwd(u, x["delta_raw"], x["A"], x["B"], x["C"], input_silu=True, **kw)
+    o2, l2 = oracle.fwd(u * expit(u), x["delta_raw"].astype(np.float64), x["A"], x["B"].astype(np.float64),
+                        x["C"].astype(np.float64), **kw)
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(l1, l2, rtol=1e-13, atol=1e-15)
+    # the flag changes the result (it is not ignored)
+    o3, _ = oracle.fwd(u, x["delta_raw"], x["A"], x["B"], x["C"], **kw)
+    assert np.max(np.abs(o3 - o1)) > 1e-3
+
+
+def test_input_silu_complex_equals_scan_of_activated_input():
+    from scipy.special import expit
+    x = W.small_case(1, 30, 4, 3, io="f32", seed=32, complex_a=True)
+    u = x["u"].astype(np.float64)
+    kw = dict(delta_bias=x["delta_bias"], D_skip=x["D_skip"], z=x["z"])
+    o1, l1 = oracle.fwd_complex(u, x["delta_raw"], x["A"], x["B"], x["C"], input_silu=True, **kw)
+    o2, l2 = oracle.fwd_complex(u * expit(u), x["delta_raw"].astype(np.float64), x["A"],
+                                x["B"].astype(np.float64), x["C"].astype(np.float64), **kw)
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(l1, l2, rtol=1e-13, atol=1e-15)
+
+
+def _loss_silu(p, dout, complex_a=False):
+    f = oracle.fwd_complex if complex_a else oracle.fwd
+    out, _ = f(p["u"], p["delta_raw"], p["A"], p["B"], p["C"], delta_bias=p["delta_bias"], D_skip=p["D_skip"],
+               z=p["z"], h0=p.get("h0"), input_silu=True)
+    return float(np.sum(out * dout))
+
+
+def _central(p, name, dout, **kw):
+    fd = np.empty_like(p[name])
+    flat = p[name].reshape(-1)
+    for i in range(flat.size):
+        v = flat[i]
+        step = 1e-6 * max(1.0, abs(v))
+        flat[i] = v + step
+        lp = _loss_silu(p, dout, **kw)
+        flat[i] = v - step
+        lm = _loss_silu(p, dout, **kw)
+        flat[i] = v
+        fd.reshape(-1)[i] = (lp - lm) / (2 * step)
+    return fd
+
+
+def test_input_silu_backward_matches_central_differences():
+    """Every gradient of the scan with the input activation, against central
+    differences of the forward oracle at the config-0 shape."""
+    p, dout = _fd_case(seed=3)
+    g = oracle.bwd(p["u"], p["delta_raw"], p["A"], p["B"], p["C"], dout, delta_bias=p["delta_bias"],
+                   D_skip=p["D_skip"], z=p["z"], h0=p["h0"], input_silu=True)
+    names = {"u": "du", "delta_raw": "ddelta_raw", "z": "dz", "B": "dB", "C": "dC", "A": "dA",
+             "delta_bias": "ddelta_bias", "D_skip": "dD", "h0": "dh0"}
+    for pn, gn in names.items():
+        fd = _central(p, pn, dout)
+        err = np.max(np.abs(fd - g[gn])) / max(np.max(np.abs(g[gn])), 1e-300)
+        assert err < 1e-6, (pn, err)
+
+
+def test_input_silu_complex_backward_matches_central_differences():
+    w = W.WORKLOADS["tiny"]
+    x = W.make_inputs(w.with_(seed=4, complex_a=True))
+    p = {k: x[k].astype(np.float64) for k in ("u", "delta_raw", "z", "B", "C", "delta_bias", "D_skip")}
+    p["A"] = x["A"]
+    dout = np.random.default_rng(44).standard_normal((w.batch, w.seqlen, w.dim))
+    g = oracle.bwd_complex(p["u"], p["delta_raw"], p["A"], p["B"], p["C"], dout, delta_bias=p["delta_bias"],
+                           D_skip=p["D_skip"], z=p["z"], input_silu=True)
+    for pn, gn in {"u": "du", "delta_raw": "ddelta_raw", "B": "dB"}.items():
+        fd = _central(p, pn, dout, complex_a=True)
+        err = np.max(np.abs(fd - g[gn])) / max(np.max(np.abs(g[gn])), 1e-300)
+        assert err < 1e-6, (pn, err)
