@@ -69,6 +69,11 @@ typedef enum sscan_dtype { SSCAN_F32 = 0, SSCAN_BF16 = 1 } sscan_dtype;
 
 /* problem->flags */
 #define SSCAN_DELTA_SOFTPLUS 1u
+/* The scan's input is x_t = SiLU(u_t) instead of u_t, in the state update and the
+ * skip term alike: the activation of the block's input branch ahead of the SSM
+ * (Fig. 3 caption: the block replaces its first multiplicative gate with an
+ * activation, sigma = SiLU).  Backward: du receives dL/dx * SiLU'(u). */
+#define SSCAN_INPUT_SILU 2u
 
 typedef struct sscan_problem {
     int64_t batch;    /* >= 0 */
@@ -76,7 +81,7 @@ typedef struct sscan_problem {
     int64_t dim;      /* D >= 0, channels */
     int64_t dstate;   /* N, 1..16 */
     int32_t io_dtype; /* sscan_dtype of the (batch,L,D) and (batch,L,N) tensors */
-    uint32_t flags;   /* SSCAN_DELTA_SOFTPLUS or 0 */
+    uint32_t flags;   /* OR of SSCAN_DELTA_SOFTPLUS, SSCAN_INPUT_SILU, or 0 */
 } sscan_problem;
 
 typedef enum sscan_op {

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libsscan.so")
 
 SSCAN_F32, SSCAN_BF16 = 0, 1
 SSCAN_DELTA_SOFTPLUS = 1
+SSCAN_INPUT_SILU = 2
 SSCAN_OP_FWD, SSCAN_OP_LAST_STATE, SSCAN_OP_BWD, SSCAN_OP_SUMMARY, SSCAN_OP_BWD_COMPLEX = 0, 1, 2, 3, 4
 SSCAN_ERR_TIMEOUT = 5
 
@@ -98,12 +99,13 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def make_problem(batch, seqlen, dim, dstate, io_dtype, delta_softplus=True) -> Problem:
+def make_problem(batch, seqlen, dim, dstate, io_dtype, delta_softplus=True, input_silu=False) -> Problem:
+    """input_silu: the scan's input is SiLU(u) (the block's input-branch activation)."""
     return Problem(int(batch), int(seqlen), int(dim), int(dstate), int(io_dtype),
-                   SSCAN_DELTA_SOFTPLUS if delta_softplus else 0)
+                   (SSCAN_DELTA_SOFTPLUS if delta_softplus else 0) | (SSCAN_INPUT_SILU if input_silu else 0))
 
 
-def _io_problem(u, B, delta_softplus):
+def _io_problem(u, B, delta_softplus, input_silu=False):
     if u.dim() != 3 or B.dim() != 3:
         raise ValueError("u must be (batch, L, D) and B (batch, L, N)")
     if u.dtype not in _IO_CODES:
@@ -111,7 +113,7 @@ def _io_problem(u, B, delta_softplus):
     batch, L, D = u.shape
     if B.shape[0] != batch or B.shape[1] != L:
         raise ValueError(f"B has shape {tuple(B.shape)}, expected ({batch}, {L}, N)")
-    return make_problem(batch, L, D, B.shape[2], _IO_CODES[u.dtype], delta_softplus)
+    return make_problem(batch, L, D, B.shape[2], _IO_CODES[u.dtype], delta_softplus, input_silu)
 
 
 def _expect(t, name, shape, dtype, device):
@@ -158,10 +160,10 @@ def _check_inputs(prob, u, delta_raw, A, B, C, delta_bias, D_skip, z, h0):
 
 
 def sscan_fwd(u, delta_raw, A, B, C, delta_bias=None, D_skip=None, z=None, h0=None, *,
-              delta_softplus=True, out=None, h_last=None, return_last_state=False,
+              delta_softplus=True, input_silu=False, out=None, h_last=None, return_last_state=False,
               workspace=None, stream=None):
     """Forward selective scan.  Returns ``out`` or ``(out, h_last)``."""
-    prob = _io_problem(u, B, delta_softplus)
+    prob = _io_problem(u, B, delta_softplus, input_silu)
     _check_inputs(prob, u, delta_raw, A, B, C, delta_bias, D_skip, z, h0)
     if out is None:
         out = torch.empty_like(u)
@@ -189,11 +191,11 @@ def _as_pairs(t, name, shape, dev):
 
 
 def sscan_fwd_complex(u, delta_raw, A, B, C, delta_bias=None, D_skip=None, z=None, h0=None, *,
-                      delta_softplus=True, out=None, return_last_state=False, stream=None):
+                      delta_softplus=True, input_silu=False, out=None, return_last_state=False, stream=None):
     """Forward scan with a complex diagonal A: (D, N) complex64 or (D, N, 2) float32
     (re, im) pairs; h0 likewise (batch, D, N).  B, C real.  Returns ``out`` or
     ``(out, h_last)`` with h_last (batch, D, N) complex64."""
-    prob = _io_problem(u, B, delta_softplus)
+    prob = _io_problem(u, B, delta_softplus, input_silu)
     dev = u.device
     _check_inputs(prob, u, delta_raw, None, B, C, delta_bias, D_skip, z, None)
     A2 = _as_pairs(A, "A", (prob.dim, prob.dstate), dev)
@@ -210,11 +212,11 @@ def sscan_fwd_complex(u, delta_raw, A, B, C, delta_bias=None, D_skip=None, z=Non
 
 
 def sscan_bwd_complex(u, delta_raw, A, B, C, dout, delta_bias=None, D_skip=None, z=None, h0=None, *,
-                      delta_softplus=True, want_dh0=True, workspace=None, stream=None):
+                      delta_softplus=True, input_silu=False, want_dh0=True, workspace=None, stream=None):
     """Gradients of sum(out * dout) for the complex-A scan.  Returns a dict keyed du,
     ddelta_raw, dA (D, N) complex64, dB, dC and, when the matching input is given,
     ddelta_bias, dD, dz; dh0 (batch, D, N) complex64 when ``want_dh0``."""
-    prob = _io_problem(u, B, delta_softplus)
+    prob = _io_problem(u, B, delta_softplus, input_silu)
     dev = u.device
     _check_inputs(prob, u, delta_raw, None, B, C, delta_bias, D_skip, z, None)
     _expect(dout, "dout", u.shape, u.dtype, dev)
@@ -243,10 +245,10 @@ def sscan_bwd_complex(u, delta_raw, A, B, C, dout, delta_bias=None, D_skip=None,
     return g
 
 
-def sscan_last_state(u, delta_raw, A, B, delta_bias=None, h0=None, *, delta_softplus=True,
+def sscan_last_state(u, delta_raw, A, B, delta_bias=None, h0=None, *, delta_softplus=True, input_silu=False,
                      h_last=None, workspace=None, stream=None):
     """Final state h_{L-1} (batch, D, N) only."""
-    prob = _io_problem(u, B, delta_softplus)
+    prob = _io_problem(u, B, delta_softplus, input_silu)
     _check_inputs(prob, u, delta_raw, A, B, None, delta_bias, None, None, h0)
     if h_last is None:
         h_last = torch.empty((prob.batch, prob.dim, prob.dstate), dtype=torch.float32, device=u.device)
@@ -259,11 +261,11 @@ def sscan_last_state(u, delta_raw, A, B, delta_bias=None, h0=None, *, delta_soft
 
 
 def sscan_bwd(u, delta_raw, A, B, C, dout, delta_bias=None, D_skip=None, z=None, h0=None, *,
-              delta_softplus=True, want_dh0=True, grads=None, workspace=None, stream=None):
+              delta_softplus=True, input_silu=False, want_dh0=True, grads=None, workspace=None, stream=None):
     """Gradients of sum(out * dout).  Returns a dict keyed du, ddelta_raw, dA, dB, dC and,
     when the matching input is given, ddelta_bias, dD, dz; dh0 when ``want_dh0``.
     ``grads`` may supply preallocated outputs under the same keys."""
-    prob = _io_problem(u, B, delta_softplus)
+    prob = _io_problem(u, B, delta_softplus, input_silu)
     _check_inputs(prob, u, delta_raw, A, B, C, delta_bias, D_skip, z, h0)
     _expect(dout, "dout", u.shape, u.dtype, u.device)
     f32 = dict(dtype=torch.float32, device=u.device)
@@ -298,7 +300,7 @@ def sscan_bwd(u, delta_raw, A, B, C, dout, delta_bias=None, D_skip=None, z=None,
     return {k: v for k, v in g.items() if v is not None}
 
 
-def sscan_step(u, delta_raw, A, B, C, state, delta_bias=None, D_skip=None, z=None, *, delta_softplus=True,
+def sscan_step(u, delta_raw, A, B, C, state, delta_bias=None, D_skip=None, z=None, *, delta_softplus=True, input_silu=False,
                out=None, stream=None):
     """One generation step: u, delta_raw, z (batch, D); B, C (batch, N); state (batch, D, N)
     fp32 updated in place.  Returns out (batch, D)."""
@@ -308,7 +310,7 @@ def sscan_step(u, delta_raw, A, B, C, state, delta_bias=None, D_skip=None, z=Non
         raise TypeError(f"I/O tensors must be float32 or bfloat16, got {u.dtype}")
     batch, D = u.shape
     N = B.shape[1]
-    prob = make_problem(batch, 1, D, N, _IO_CODES[u.dtype], delta_softplus)
+    prob = make_problem(batch, 1, D, N, _IO_CODES[u.dtype], delta_softplus, input_silu)
     dev, io = u.device, u.dtype
     if dev.type != "cuda":
         raise ValueError("libsscan works on CUDA tensors only")
@@ -328,11 +330,11 @@ def sscan_step(u, delta_raw, A, B, C, state, delta_bias=None, D_skip=None, z=Non
     return out
 
 
-def sscan_chunk_summary(u, delta_raw, A, B, delta_bias=None, *, delta_softplus=True, workspace=None,
+def sscan_chunk_summary(u, delta_raw, A, B, delta_bias=None, *, delta_softplus=True, input_silu=False, workspace=None,
                         stream=None):
     """(P, H), each (batch, D, N) fp32: the stretch u[:, 0:L] acts on its initial state as
     h -> P h + H (P = exp(A * sum of delta), H = final state from zero)."""
-    prob = _io_problem(u, B, delta_softplus)
+    prob = _io_problem(u, B, delta_softplus, input_silu)
     _check_inputs(prob, u, delta_raw, A, B, None, delta_bias, None, None, None)
     f32 = dict(dtype=torch.float32, device=u.device)
     P = torch.empty((prob.batch, prob.dim, prob.dstate), **f32)

@@ -42,8 +42,9 @@ sscan_status check_problem(const sscan_problem* p) {
         return fail(SSCAN_ERR_UNSUPPORTED, "dstate %lld > %d", (long long)p->dstate, sscan::kMaxState);
     if (p->io_dtype != SSCAN_F32 && p->io_dtype != SSCAN_BF16)
         return fail(SSCAN_ERR_INVALID_ARG, "unknown io_dtype %d", (int)p->io_dtype);
-    if (p->flags & ~SSCAN_DELTA_SOFTPLUS)
-        return fail(SSCAN_ERR_INVALID_ARG, "unknown flag bits 0x%x", (unsigned)p->flags);
+    if (p->flags & ~(SSCAN_DELTA_SOFTPLUS | SSCAN_INPUT_SILU))
+        return fail(SSCAN_ERR_INVALID_ARG, "unknown flag bits 0x%x",
+                    (unsigned)(p->flags & ~(SSCAN_DELTA_SOFTPLUS | SSCAN_INPUT_SILU)));
     return SSCAN_OK;
 }
 
@@ -113,6 +114,7 @@ sscan::ScanArgs make_args(const sscan_problem* p, const void* u, const void* del
     a.out = out;
     a.h_last = h_last;
     a.softplus = (p->flags & SSCAN_DELTA_SOFTPLUS) ? 1 : 0;
+    a.input_silu = (p->flags & SSCAN_INPUT_SILU) ? 1 : 0;
     a.chunk_len = p->seqlen;
     a.nchunks = 1;
     return a;
@@ -161,6 +163,7 @@ sscan_status run_tiled(const sscan_problem* p, const sscan::ScanArgs& a, void* w
     t.D = p->dim;
     t.N = (int)p->dstate;
     t.softplus = a.softplus;
+    t.input_silu = a.input_silu;
     t.has_z = a.z != nullptr;
     t.bias = a.bias;
     t.A = a.A;
@@ -479,6 +482,7 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
         t.D = p->dim;
         t.N = (int)p->dstate;
         t.softplus = (p->flags & SSCAN_DELTA_SOFTPLUS) ? 1 : 0;
+        t.input_silu = (p->flags & SSCAN_INPUT_SILU) ? 1 : 0;
         t.has_z = 0;
         t.bias = delta_bias;
         t.A = A;
@@ -496,6 +500,7 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
         ba.D = p->dim;
         ba.N = (int)p->dstate;
         ba.softplus = t.softplus;
+        ba.input_silu = t.input_silu;
         ba.has_z = z != nullptr;
         ba.bias = delta_bias;
         ba.A = A;
@@ -603,6 +608,7 @@ sscan_status sscan_fwd_complex(const sscan_problem* p, const void* u, const void
     a.D = p->dim;
     a.N = (int)p->dstate;
     a.softplus = (p->flags & SSCAN_DELTA_SOFTPLUS) ? 1 : 0;
+    a.input_silu = (p->flags & SSCAN_INPUT_SILU) ? 1 : 0;
     a.u = u;
     a.delta_raw = delta_raw;
     a.bias = delta_bias;
@@ -664,6 +670,7 @@ sscan_status sscan_bwd_complex(const sscan_problem* p, const void* u, const void
     a.D = p->dim;
     a.N = (int)p->dstate;
     a.softplus = (p->flags & SSCAN_DELTA_SOFTPLUS) ? 1 : 0;
+    a.input_silu = (p->flags & SSCAN_INPUT_SILU) ? 1 : 0;
     a.u = u;
     a.delta_raw = delta_raw;
     a.bias = delta_bias;
@@ -721,6 +728,7 @@ sscan_status sscan_step(const sscan_problem* p, const void* u, const void* delta
     a.D = p->dim;
     a.N = (int)p->dstate;
     a.softplus = (p->flags & SSCAN_DELTA_SOFTPLUS) ? 1 : 0;
+    a.input_silu = (p->flags & SSCAN_INPUT_SILU) ? 1 : 0;
     a.u = u;
     a.delta_raw = delta_raw;
     a.bias = delta_bias;
@@ -772,6 +780,7 @@ sscan_status sscan_chunk_summary(const sscan_problem* p, const void* u, const vo
         t.D = p->dim;
         t.N = (int)p->dstate;
         t.softplus = a.softplus;
+        t.input_silu = a.input_silu;
         t.bias = delta_bias;
         t.A = A;
         t.B = B;

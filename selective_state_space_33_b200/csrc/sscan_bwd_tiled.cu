@@ -72,7 +72,8 @@ struct BCfg {
     static constexpr int OFF_DY = OFF_DX + kTB * DC * 8;        // float  dy                [kTB][DC]
     static constexpr int OFF_DQ = OFF_DY + kTB * DC * 4;        // float2 (dzf, sr)         [kTB][DC]
     static constexpr int OFF_DD = OFF_DQ + kTB * DC * 8;        // float2 (D dy, D x)       [kTB][DC]
-    static constexpr int OFF_B = OFF_DD + kTB * DC * 8;         // float [kTB][NS]
+    static constexpr int OFF_SU = OFF_DD + kTB * DC * 8;        // float  SiLU'(u)          [kTB][DC]
+    static constexpr int OFF_B = OFF_SU + kTB * DC * 4;         // float [kTB][NS]
     static constexpr int OFF_C = OFF_B + kTB * NS * 4;          // float [kTB][NS]
     static constexpr int OFF_HS = OFF_C + kTB * NS * 4;         // float4 [kTB][kThreadsB] recomputed states
     static constexpr int OFF_ACC = OFF_HS + kTB * kThreadsB * 16;  // float [warp][kTB][NS][2] dB, dC of the tile
@@ -272,6 +273,7 @@ __global__ void __launch_bounds__(kThreadsB, 5)
             float2* sdy = reinterpret_cast<float2*>(smem + C::OFF_DY);
             float4* sdq = reinterpret_cast<float4*>(smem + C::OFF_DQ);
             float4* sdd = reinterpret_cast<float4*>(smem + C::OFF_DD);
+            float2* ssu = reinterpret_cast<float2*>(smem + C::OFF_SU);
             const float pb0 = (a.bias && pd < a.D) ? __ldg(a.bias + pd) : 0.f;
             const float pb1 = (a.bias && pd + 1 < a.D) ? __ldg(a.bias + pd + 1) : 0.f;
             const float pk0 = (a.Dskip && pd < a.D) ? __ldg(a.Dskip + pd) : 0.f;
@@ -280,7 +282,12 @@ __global__ void __launch_bounds__(kThreadsB, 5)
             for (int q = tid; q < C::PAIRS; q += kThreadsB) {
                 const int t = q / (C::DC / 2);
                 const bool tv = t < tile_len;
-                const float2 x = BPair<T>::f(ru[q]);
+                const float2 uv = BPair<T>::f(ru[q]);
+                float2 x = uv;
+                if (a.input_silu) {
+                    x = g2(silu(uv.x), silu(uv.y));
+                    ssu[(t * C::DC + pc) / 2] = make_float2(dsilu(uv.x), dsilu(uv.y));
+                }
                 const float2 r = BPair<T>::f(rd[q]);
                 const float2 go = BPair<T>::f(rg[q]);
                 float dl0 = r.x + pb0, dl1 = r.y + pb1, s0 = 1.f, s1 = 1.f;
@@ -477,7 +484,8 @@ __global__ void __launch_bounds__(kThreadsB, 5)
             if (t < tile_len && g < NG) {
                 const float2 dq = sdq[t * C::DC];  // (dz factor, softplus')
                 const float2 ddv = sdd[t * C::DC];
-                const float du = sdu + ddv.x;
+                float du = sdu + ddv.x;
+                if (a.input_silu) du *= reinterpret_cast<const float*>(smem + C::OFF_SU)[t * C::DC + cw];
                 const float ddr = sdd_ * dq.y;
                 const float dz = dq.x * (sy + ddv.y);
                 so[t * C::DC + cw] = from_f32<T>(du);

@@ -273,7 +273,8 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
             float2 dx = make_float2(0.f, 0.f), gd = make_float2(0.f, 0.f);
             if (t < tl && dd < a.D) {
                 const int64_t gi = (b * a.L + t0 + t) * a.D + dd;
-                const float x = IO<T>::load(u, gi);
+                const float uv = IO<T>::load(u, gi);
+                const float x = a.input_silu ? silu(uv) : uv;
                 const float r = IO<T>::load(dr, gi) + (a.bias ? __ldg(a.bias + dd) : 0.f);
                 const float gate = zz ? silu(IO<T>::load(zz, gi)) : 1.f;
                 const float dsk = a.Dskip ? __ldg(a.Dskip + dd) : 0.f;

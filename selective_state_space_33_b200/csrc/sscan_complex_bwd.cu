@@ -130,7 +130,8 @@ __global__ void __launch_bounds__(kXThreads, 6) bwd_complex_kernel(ComplexBwdArg
             float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
             if (t < tl && dd < a.D) {
                 const int64_t gi = (b * a.L + t0 + t) * a.D + dd;
-                const float x = IO<T>::load(u, gi);
+                const float uv = IO<T>::load(u, gi);
+                const float x = a.input_silu ? silu(uv) : uv;
                 const float r = IO<T>::load(dr, gi) + (a.bias ? __ldg(a.bias + dd) : 0.f);
                 const float o = IO<T>::load(go, gi);
                 float dy = o, dzf = 0.f;
@@ -140,7 +141,7 @@ __global__ void __launch_bounds__(kXThreads, 6) bwd_complex_kernel(ComplexBwdArg
                     dzf = o * s * fmaf(zv, 1.f - s, 1.f);
                 }
                 dx = make_float2(a.softplus ? softplus(r) : r, x);
-                q = make_float4(dy, dzf, a.softplus ? sigmoid(r) : 1.f, 0.f);
+                q = make_float4(dy, dzf, a.softplus ? sigmoid(r) : 1.f, a.input_silu ? dsilu(uv) : 1.f);
             }
             sdx[e] = dx;
             sq[e] = q;
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(kXThreads, 6) bwd_complex_kernel(ComplexBwdArg
               const float4 q4 = sq[t * C::DC + cw];
               const int64_t gi = (b * a.L + t0 + t) * a.D + d;
               const float ddr = sdd * q4.z;
-              IO<T>::store(static_cast<T*>(g.du), gi, fmaf(dsk, q4.x, sdu));
+              IO<T>::store(static_cast<T*>(g.du), gi, fmaf(dsk, q4.x, sdu) * q4.w);
               IO<T>::store(static_cast<T*>(g.ddelta_raw), gi, ddr);
               if (g.dz) IO<T>::store(static_cast<T*>(g.dz), gi, q4.y * fmaf(dsk, dx.y, syp));
               dD_acc = fmaf(q4.x, dx.y, dD_acc);

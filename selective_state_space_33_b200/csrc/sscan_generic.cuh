@@ -26,6 +26,7 @@ struct ScanArgs {
     void* out;           // (batch, L, D) or null
     float* h_last;       // (batch, D, N) or null
     int softplus;
+    int input_silu;      // the scan's input is SiLU(u)
     // sequence split: chunk c covers steps [c*chunk_len, min(L, (c+1)*chunk_len))
     int64_t chunk_len;
     int64_t nchunks;
@@ -81,7 +82,8 @@ __global__ void __launch_bounds__(128) fwd_rows_kernel(ScanArgs a) {
     for (int64_t t = t0; t < t1; ++t) {
         const int64_t e = (b * a.L + t) * a.D + d;
         const int64_t s = (b * a.L + t) * N;
-        const float x = IO<T>::load(u, e);
+        const float uv = IO<T>::load(u, e);
+        const float x = a.input_silu ? silu(uv) : uv;
         const float r = IO<T>::load(dr, e) + bias;
         const float delta = a.softplus ? softplus(r) : r;
         if (MODE == kModeAggregate) dsum += delta;

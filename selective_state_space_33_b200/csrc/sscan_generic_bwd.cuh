@@ -89,7 +89,8 @@ __global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
                 if (n < N) ck[(t / kSeg) * N + n] = h[n];
         }
         const int64_t e = (b * a.L + t) * a.D + d, s = (b * a.L + t) * N;
-        const float x = IO<T>::load(u, e);
+        const float uv = IO<T>::load(u, e);
+            const float x = a.input_silu ? silu(uv) : uv;
         const float r = IO<T>::load(dr, e) + bias;
         const float delta = a.softplus ? softplus(r) : r;
 #pragma unroll
@@ -116,7 +117,8 @@ __global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
         for (int k = 0; k < len; ++k) {
             const int64_t t = t0 + k;
             const int64_t e = (b * a.L + t) * a.D + d, s = (b * a.L + t) * N;
-            const float x = IO<T>::load(u, e);
+            const float uv = IO<T>::load(u, e);
+            const float x = a.input_silu ? silu(uv) : uv;
             const float r = IO<T>::load(dr, e) + bias;
             const float delta = a.softplus ? softplus(r) : r;
 #pragma unroll
@@ -131,7 +133,8 @@ __global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
         for (int k = len - 1; k >= 0; --k) {
             const int64_t t = t0 + k;
             const int64_t e = (b * a.L + t) * a.D + d, s = (b * a.L + t) * N;
-            const float x = IO<T>::load(u, e);
+            const float uv = IO<T>::load(u, e);
+            const float x = a.input_silu ? silu(uv) : uv;
             const float r = IO<T>::load(dr, e) + bias;
             const float delta = a.softplus ? softplus(r) : r;
             const float go = IO<T>::load(dout, e);
@@ -169,7 +172,7 @@ __global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
                 }
             }
             const float drr = a.softplus ? ddelta * sigmoid(r) : ddelta;
-            IO<T>::store(static_cast<T*>(g.du), e, dx);
+            IO<T>::store(static_cast<T*>(g.du), e, a.input_silu ? dx * dsilu(uv) : dx);
             IO<T>::store(static_cast<T*>(g.ddelta_raw), e, drr);
             dbacc += drr;
         }

@@ -12,6 +12,7 @@ struct TiledArgs {
     int64_t batch, L, D;
     int N;
     int softplus;
+    int input_silu;       // the scan's input is SiLU(u)
     int has_z;
     int bc_tma;           // set by the launcher: B and C tiles travel by TMA
     const float* bias;    // (D) or null
@@ -56,6 +57,7 @@ struct StepArgs {
     int64_t batch, D;
     int N;
     int softplus;
+    int input_silu;         // the scan's input is SiLU(u)
     const void* u;          // (batch, D)
     const void* delta_raw;  // (batch, D)
     const float* bias;      // (D) or null
@@ -75,6 +77,7 @@ struct ComplexArgs {
     int64_t batch, L, D;
     int N;
     int softplus;
+    int input_silu;         // the scan's input is SiLU(u)
     const void* u;          // (batch, L, D)
     const void* delta_raw;  // (batch, L, D)
     const float* bias;      // (D) or null
@@ -117,6 +120,7 @@ struct BwdTiledArgs {
     int64_t batch, L, D;
     int N;
     int softplus;
+    int input_silu;      // the scan's input is SiLU(u); du gets the SiLU' factor
     int has_z;
     const float* bias;   // (D) or null
     const float* A;      // (D, N)

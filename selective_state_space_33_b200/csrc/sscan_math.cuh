@@ -53,6 +53,12 @@ __device__ __forceinline__ float sigmoid(float r) { return rcp(1.f + ex2(-r * kL
 // SiLU(v) = v * sigmoid(v)  (Fig. 3: the block's gate activation).
 __device__ __forceinline__ float silu(float v) { return v * sigmoid(v); }
 
+// d SiLU / dv = s (1 + v (1 - s)), s = sigmoid(v).
+__device__ __forceinline__ float dsilu(float v) {
+    const float s = sigmoid(v);
+    return s * fmaf(v, 1.f - s, 1.f);
+}
+
 // phi1(q) = expm1(q) / q for |q| < 1/16, by the Taylor series 1 + q/2 + q^2/6 + q^3/24
 // + q^4/120 (the dropped q^5/720 term is < 1.3e-9 relative).
 __device__ __forceinline__ float phi1_series(float q) {

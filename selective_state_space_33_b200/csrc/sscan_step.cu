@@ -41,7 +41,8 @@ __global__ void __launch_bounds__(128) step_kernel(StepArgs a) {
         Bv[n] = n < N ? IO<T>::load(Bm, n) : 0.f;
         Cv[n] = n < N ? IO<T>::load(Cm, n) : 0.f;
     }
-    const float x = IO<T>::load(static_cast<const T*>(a.u), row);
+    const float uv = IO<T>::load(static_cast<const T*>(a.u), row);
+    const float x = a.input_silu ? silu(uv) : uv;
     const float r = IO<T>::load(static_cast<const T*>(a.delta_raw), row) + (a.bias ? __ldg(a.bias + d) : 0.f);
     const float dsk = a.Dskip ? __ldg(a.Dskip + d) : 0.f;
     const float gz = a.z ? IO<T>::load(static_cast<const T*>(a.z), row) : 0.f;
@@ -106,7 +107,8 @@ __global__ void __launch_bounds__(256) step_quad_kernel(StepArgs a) {
         Bn[4 * v] = Bv.x, Bn[4 * v + 1] = Bv.y, Bn[4 * v + 2] = Bv.z, Bn[4 * v + 3] = Bv.w;
         Cn[4 * v] = Cv.x, Cn[4 * v + 1] = Cv.y, Cn[4 * v + 2] = Cv.z, Cn[4 * v + 3] = Cv.w;
     }
-    const float x = IO<T>::load(static_cast<const T*>(a.u), row);
+    const float uv = IO<T>::load(static_cast<const T*>(a.u), row);
+    const float x = a.input_silu ? silu(uv) : uv;
     const float r = IO<T>::load(static_cast<const T*>(a.delta_raw), row) + (a.bias ? __ldg(a.bias + d) : 0.f);
     const float dsk = a.Dskip ? __ldg(a.Dskip + d) : 0.f;
     const float gz = a.z ? IO<T>::load(static_cast<const T*>(a.z), row) : 0.f;

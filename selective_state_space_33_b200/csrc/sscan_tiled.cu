@@ -418,7 +418,8 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
             for (int qi = 0; qi < C::PAIRS / kThreads; ++qi) {
                 const int q = tid + qi * kThreads;
                 const int t = q / (C::DC / 2);
-                const float2 x = Pair<T>::f(ru[q]);
+                float2 x = Pair<T>::f(ru[q]);
+                if (a.input_silu) x = silu_x2(x);
                 float2 dl = __fadd2_rn(Pair<T>::f(rd[q]), pbias);
                 if (a.softplus) dl = softplus_x2(dl);
                 sdx[(t * C::DC + pc) / 2] = make_float4(dl.x, x.x, dl.y, x.y);

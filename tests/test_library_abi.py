@@ -62,6 +62,11 @@ def test_fwd_rejects_bad_arguments(lib):
     assert b"dstate" in lib.sscan_last_error()
     assert _fwd(lib, _p(io=7)) == 1
     assert _fwd(lib, _p(flags=6)) == 1
+    assert b"0x4" in lib.sscan_last_error()
+    # SSCAN_DELTA_SOFTPLUS | SSCAN_INPUT_SILU is a valid flag set: validation goes on to
+    # the pointers
+    assert _fwd(lib, _p(flags=3), u=None) == 1
+    assert b"required" in lib.sscan_last_error()
     assert _fwd(lib, _p(), u=None) == 1
     assert _fwd(lib, _p(), out=None, h_last=None) == 1
     assert b"both NULL" in lib.sscan_last_error()
