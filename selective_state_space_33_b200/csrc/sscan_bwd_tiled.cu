@@ -6,22 +6,27 @@
 // the sequence in reverse, 8 steps (one tile) at a time:
 //   TMA brings u, delta_raw, z, dout and the B, C rows of the tile into a 2-stage
 //   ring (bounded mbarrier waits);
-//   phase P turns them into fp32 (delta, x), (dy, dz factor, softplus') and the
-//   skip terms -- dy = dout SiLU(z), dz = dout y SiLU'(z), SiLU' = s (1 + z (1 - s));
+//   phase P turns them into fp32 operand pairs (delta, delta, x, x) and (dy, dy)
+//   plus the epilogue terms -- dy = dout SiLU(z),
+//   dz factor = dout SiLU'(z), softplus' = sigmoid(r), SiLU'(u) with the input
+//   activation -- with packed f32x2 arithmetic;
 //   each lane recomputes its 4 states through the tile from the checkpoint,
 //   keeping h_t in shared memory, then runs the adjoint recurrence backwards:
 //     lam_t = C_t dy_t + Abar_{t+1} lam_{t+1}
-//     dx   += lam beta B,   dB += lam beta x,   dC += dy h_t        (beta = Bbar / B)
+//     w     = delta^2 psi(delta A),  psi(q) = (q e^q - expm1(q)) / q^2
+//             (its Taylor series for |q| < 1/2, where the closed form cancels;
+//             (1 + Abar (q - 1)) / A^2 elsewhere)
+//     lam beta = delta lam Abar - A lam w        (beta = Bbar / B = delta Abar - A w)
+//     dx   += lam beta B,   dB += lam beta x,   dC += dy h_t
 //     d delta += lam Abar (A h_{t-1} + B x)
-//     dA   += delta lam Abar h_{t-1} + lam B x delta^2 psi(delta A)
-//   with psi(q) = (q e^q - expm1(q)) / q^2 (its Taylor series for |q| < 1/2, where the
-//   closed form would cancel) and beta = delta phi1(delta A), phi1 = Abar - q psi there
-//   (no cancellation) and (Abar - 1) / A elsewhere;
-//   and the per-element sums over a channel's lanes, and the (t, n) sums over the
-//   channels of a warp, are formed with shuffles before anything touches memory.
-// dB and dC of a tile are stored per warp in shared memory, summed across the CTA's
-// warps and then added to fp32 accumulators in global memory; dA, dD and the bias gradient are
-// per-channel sums added once at the end.
+//     dA   += delta lam Abar h_{t-1} + lam w B x
+//   so one evaluation of w per state gives both beta and the A-gradient term;
+//   the per-element sums over a channel's lanes use transposed shuffle butterflies,
+//   and the (t, n) sums of dB, dC over a warp's channels a padded shared-memory
+//   transpose, before anything touches global memory.
+// dB and dC of a tile are summed across the CTA's warps in shared memory (shared
+// atomic adds) and then added to fp32 accumulators in global memory; dA, dD and the bias
+// gradient are per-channel sums added once at the end.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -67,17 +72,22 @@ struct BCfg {
     static constexpr int STAGE = 4 * RAW + 2 * RAWBC;     // u, delta_raw, z, dout, B, C
     static constexpr int STAGES = 2;
     static constexpr int PAIRS = kTB * DC / 2;
+    static_assert(PAIRS % kThreadsB == 0, "phase P runs a fixed number of channel pairs per thread");
+    // dB / dC transpose (NG == 4): per warp, NG rows of CW lanes x 8 values, rows padded to
+    // 8 (CW + 1) floats so that the column reads of a warp hit 32 distinct banks
+    static constexpr int TR_ROW = 8 * (CW + 1);
+    static constexpr int TR_WARP = NG * TR_ROW;
     static constexpr int OFF_RAW = 0;
-    static constexpr int OFF_DX = OFF_RAW + STAGES * STAGE;     // float2 (d, x)            [kTB][DC]
-    static constexpr int OFF_DY = OFF_DX + kTB * DC * 8;        // float  dy                [kTB][DC]
-    static constexpr int OFF_DQ = OFF_DY + kTB * DC * 4;        // float2 (dzf, sr)         [kTB][DC]
-    static constexpr int OFF_DD = OFF_DQ + kTB * DC * 8;        // float2 (D dy, D x)       [kTB][DC]
-    static constexpr int OFF_SU = OFF_DD + kTB * DC * 8;        // float  SiLU'(u)          [kTB][DC]
+    static constexpr int OFF_DX = OFF_RAW + STAGES * STAGE;     // float4 (d, d, x, x)      [kTB][DC]
+    static constexpr int OFF_DY = OFF_DX + kTB * DC * 16;       // float2 (dy, dy)          [kTB][DC]
+    static constexpr int OFF_EP = OFF_DY + kTB * DC * 8;        // float4 (D dy, dzf, sr, D x) [kTB][DC]
+    static constexpr int OFF_SU = OFF_EP + kTB * DC * 16;       // float  SiLU'(u)          [kTB][DC]
     static constexpr int OFF_B = OFF_SU + kTB * DC * 4;         // float [kTB][NS]
     static constexpr int OFF_C = OFF_B + kTB * NS * 4;          // float [kTB][NS]
     static constexpr int OFF_HS = OFF_C + kTB * NS * 4;         // float4 [kTB][kThreadsB] recomputed states
-    static constexpr int OFF_ACC = OFF_HS + kTB * kThreadsB * 16;  // float [warp][kTB][NS][2] dB, dC of the tile
-    static constexpr int OFF_OUT = OFF_ACC + kWarpsB * kTB * NS * 2 * 4;  // [2 buffers][3 tensors][RAW]
+    static constexpr int OFF_TR = OFF_HS + kTB * kThreadsB * 16;  // float [warp][TR_WARP]
+    static constexpr int OFF_ACC = OFF_TR + (NG == 4 ? kWarpsB * TR_WARP * 4 : 0);  // float [kTB][NS][2]
+    static constexpr int OFF_OUT = OFF_ACC + kTB * NS * 2 * 4;  // [2 buffers][3 tensors][RAW]
     static constexpr int OFF_BAR = OFF_OUT + 2 * 3 * RAW;
     static constexpr int SMEM = OFF_BAR + STAGES * 8;
 };
@@ -144,15 +154,116 @@ __device__ __forceinline__ float2 bbar2(float2 dd, float2 A2, float2 iA) {
     return g2(fabsf(q.x) < 0.0625f ? bs.x : bl.x, fabsf(q.y) < 0.0625f ? bs.y : bl.y);
 }
 
-// softplus(r) and its derivative sigmoid(r) from one exponential (regions as in
-// sscan::softplus).
-__device__ __forceinline__ float2 softplus_dsig(float r) {
-    const float u = ex2(fminf(r, 30.f) * kLog2e);
-    const float ser = u * fmaf(u, fmaf(u, fmaf(u, fmaf(u, 0.2f, -0.25f), 1.f / 3.f), -0.5f), 1.f);
-    const float lg = kLn2 * lg2(1.f + u);
-    const float v = u < 0.03125f ? ser : lg;
-    const float sig = r > 20.f ? 1.f : u * rcp(1.f + u);
-    return g2(r > 20.f ? r : v, sig);
+// softplus(r) and its derivative sigmoid(r) for two values, from one exponential
+// u = e^r each, in the three regions of sscan::softplus: r > 20: r; u < 2^-5: the
+// log1p series u - u^2/2 + ... + u^5/5 (lg2.approx near 1 carries an absolute,
+// not a relative, error); else ln2 log2(1 + u).  sigmoid(r) = u / (1 + u).
+__device__ __forceinline__ void softplus_sig_x2(float2 r, float2& sp, float2& sg) {
+    const float2 u = ex2p(g2(fminf(r.x, 20.f) * kLog2e, fminf(r.y, 20.f) * kLog2e));
+    float2 ser = __ffma2_rn(u, g2(0.2f, 0.2f), g2(-0.25f, -0.25f));
+    ser = __ffma2_rn(ser, u, g2(1.f / 3.f, 1.f / 3.f));
+    ser = __ffma2_rn(ser, u, g2(-0.5f, -0.5f));
+    ser = __ffma2_rn(ser, u, g2(1.f, 1.f));
+    ser = __fmul2_rn(ser, u);
+    const float2 w = __fadd2_rn(u, g2(1.f, 1.f));
+    const float2 lg = __fmul2_rn(g2(lg2(w.x), lg2(w.y)), g2(kLn2, kLn2));
+    const float vx = u.x < 0.03125f ? ser.x : lg.x, vy = u.y < 0.03125f ? ser.y : lg.y;
+    sp = g2(r.x > 20.f ? r.x : vx, r.y > 20.f ? r.y : vy);
+    sg = __fmul2_rn(u, g2(rcp(w.x), rcp(w.y)));
+}
+
+__device__ __forceinline__ float2 sigmoid_x2(float2 z) {
+    const float2 d = __fadd2_rn(ex2p(__fmul2_rn(z, g2(-kLog2e, -kLog2e))), g2(1.f, 1.f));
+    return g2(rcp(d.x), rcp(d.y));
+}
+
+// w = delta^2 psi(q) for two states, q = delta A = q2 ln 2, psi(q) = (q e^q - expm1(q)) / q^2.
+//   |q| < 1/2 : the Taylor series sum_k (k+1)/(k+2)! q^k through q^6 (dropped tail below
+//               2e-7 q^7, ~5e-7 relative), written in q2 = q log2(e);
+//   otherwise : (1 + Abar (q - 1)) / A^2 from Abar = e^q; 1 + Abar (q - 1) = q^2 psi(q)
+//               >= 0.09 there, so the subtraction costs about 1e-6 relative.
+__device__ __forceinline__ float2 wpsi_x2(float2 q2, float2 ab, float2 d2, float2 iA2) {
+    constexpr float l1 = 0.6931471805599453f, l2 = l1 * l1, l3 = l2 * l1, l4 = l3 * l1, l5 = l4 * l1, l6 = l5 * l1;
+    float2 ps = __ffma2_rn(q2, g2(l6 / 5760.f, l6 / 5760.f), g2(l5 / 840.f, l5 / 840.f));
+    ps = __ffma2_rn(ps, q2, g2(l4 / 144.f, l4 / 144.f));
+    ps = __ffma2_rn(ps, q2, g2(l3 / 30.f, l3 / 30.f));
+    ps = __ffma2_rn(ps, q2, g2(l2 / 8.f, l2 / 8.f));
+    ps = __ffma2_rn(ps, q2, g2(l1 / 3.f, l1 / 3.f));
+    ps = __ffma2_rn(ps, q2, g2(0.5f, 0.5f));
+    const float2 ws = __fmul2_rn(d2, ps);
+    const float2 qm1 = __ffma2_rn(q2, g2(l1, l1), g2(-1.f, -1.f));
+    const float2 wc = __fmul2_rn(__ffma2_rn(ab, qm1, g2(1.f, 1.f)), iA2);
+    constexpr float kT = 0.5f * 1.4426950408889634f;  // |q| = 1/2 in log2 units
+    return g2(fabsf(q2.x) < kT ? ws.x : wc.x, fabsf(q2.y) < kT ? ws.y : wc.y);
+}
+
+// Per-lane constants and accumulators of the reverse sweep for its 4 states (2 pairs).
+struct RevLane {
+    float2 A2[2];    // A log2(e)
+    float2 niA[2];   // -1 / A (0 when A == 0)
+    float2 nA[2];    // -A
+    float2 iA2[2];   // 1 / A^2 (0 when A == 0)
+    float2 lam[2];   // Abar_{t+1} lam_{t+1}
+    float2 P1[2];    // sum_t delta lam Abar h_{t-1}
+    float2 P2[2];    // sum_t lam w B x
+};
+
+// One reverse step for the lane's 4 states.  dx = (d, d, x, x), dy2 = (dy, dy),
+// Bv / Cv the lane's 4 values of B_t / C_t, hc = h_t, hp = h_{t-1}.  Returns the
+// lane's partial sums for du, d delta, and the readout y_t; writes its dB, dC values.
+__device__ __forceinline__ void rev_step(RevLane& s, float4 dx, float2 dyy, float4 Bv, float4 Cv, float4 hc,
+                                         float4 hp, float& pdu, float& pdd, float& py, float (&vbc)[8]) {
+    const float2 dd = g2(dx.x, dx.y), xx = g2(dx.z, dx.w), d2 = __fmul2_rn(dd, dd);
+    const float2 Bp[2] = {g2(Bv.x, Bv.y), g2(Bv.z, Bv.w)};
+    const float2 Cp[2] = {g2(Cv.x, Cv.y), g2(Cv.z, Cv.w)};
+    const float2 hcv[2] = {g2(hc.x, hc.y), g2(hc.z, hc.w)};
+    const float2 hpv[2] = {g2(hp.x, hp.y), g2(hp.z, hp.w)};
+    float2 du2 = g2(0.f, 0.f), S1 = g2(0.f, 0.f), S2 = g2(0.f, 0.f), y2 = g2(0.f, 0.f);
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        const float2 q2 = __fmul2_rn(dd, s.A2[p]);
+        const float2 ab = ex2p(q2);
+        const float2 l = __ffma2_rn(Cp[p], dyy, s.lam[p]);
+        const float2 la = __fmul2_rn(l, ab);
+        const float2 w = wpsi_x2(q2, ab, d2, s.iA2[p]);
+        const float2 m = __fmul2_rn(l, w);
+        const float2 lb = __ffma2_rn(s.nA[p], m, __fmul2_rn(dd, la));  // lam beta
+        du2 = __ffma2_rn(lb, Bp[p], du2);
+        const float2 dBv = __fmul2_rn(lb, xx);
+        const float2 dCv = __fmul2_rn(dyy, hcv[p]);
+        vbc[2 * p] = dBv.x;
+        vbc[2 * p + 1] = dBv.y;
+        vbc[4 + 2 * p] = dCv.x;
+        vbc[4 + 2 * p + 1] = dCv.y;
+        const float2 lah = __fmul2_rn(la, hpv[p]);
+        S1 = __ffma2_rn(s.A2[p], lah, S1);
+        S2 = __ffma2_rn(la, Bp[p], S2);
+        s.P1[p] = __ffma2_rn(dd, lah, s.P1[p]);
+        s.P2[p] = __ffma2_rn(m, __fmul2_rn(Bp[p], xx), s.P2[p]);
+        y2 = __ffma2_rn(Cp[p], hcv[p], y2);
+        s.lam[p] = la;
+    }
+    pdu = du2.x + du2.y;
+    pdd = fmaf(kLn2, S1.x + S1.y, dx.z * (S2.x + S2.y));
+    py = y2.x + y2.y;
+}
+
+// Sum 8 values over the 8 channel lanes (low lane bits) of each state group of a warp
+// through a padded shared-memory transpose: lane (g, c) leaves with value c of its
+// group summed over the group's lanes.  tr is the warp's scratch of TR_WARP floats.
+template <int CW>
+__device__ __forceinline__ float tr_reduce8(const float (&v)[8], float* tr, int g, int c) {
+    constexpr int ROW = 8 * (CW + 1);
+    float* mine = tr + g * ROW + c * 8;
+    reinterpret_cast<float4*>(mine)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(mine)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    __syncwarp();
+    const float* col = tr + g * ROW + c;
+    float r = col[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) r += col[8 * k];
+    __syncwarp();
+    return r;
 }
 
 template <typename T, int NG, int MODE>
@@ -205,31 +316,32 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         for (int k = 0; k < C::STAGES && k < ntb; ++k) issue(k);
     }
-    // per-warp tile sums of dB and dC: every slot a tile reads was written in that tile
+    // the tile's dB, dC summed over the CTA's channels: zero here, and zeroed again by
+    // the thread that drains each entry into global memory
     float* sacc = reinterpret_cast<float*>(smem + C::OFF_ACC);
-    constexpr int kAccWarp = kTB * C::NS * 2;
+    for (int e = tid; e < kTB * C::NS * 2; e += kThreadsB) sacc[e] = 0.f;
 
     // lane state: channel cw, states g*4 .. g*4+3
     const int g = lane / C::CW, c = lane % C::CW, cw = warp * C::CW + c;
     const int64_t d = d0 + cw;
     const bool cvalid = d < a.D;
-    float2 A2[2], iA[2], lam[2], P1[2], P2v[2];
+    RevLane s;
     bool small_a = false;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-        float av[2], ia[2];
+        float av[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int n = g * 4 + 2 * k + j;
             const bool ok = cvalid && n < N;
-            const float An = ok ? __ldg(a.A + d * N + n) : 0.f;
-            small_a |= ok && fabsf(An) < kSmallAB;
-            av[j] = An * kLog2e;
-            ia[j] = An != 0.f ? 1.f / An : 0.f;
+            av[j] = ok ? __ldg(a.A + d * N + n) : 0.f;
+            small_a |= ok && fabsf(av[j]) < kSmallAB;
         }
-        A2[k] = g2(av[0], av[1]);
-        iA[k] = g2(ia[0], ia[1]);
-        lam[k] = P1[k] = P2v[k] = g2(0.f, 0.f);
+        s.A2[k] = g2(av[0] * kLog2e, av[1] * kLog2e);
+        s.niA[k] = g2(av[0] != 0.f ? -1.f / av[0] : 0.f, av[1] != 0.f ? -1.f / av[1] : 0.f);
+        s.nA[k] = g2(-av[0], -av[1]);
+        s.iA2[k] = g2(av[0] != 0.f ? 1.f / (av[0] * av[0]) : 0.f, av[1] != 0.f ? 1.f / (av[1] * av[1]) : 0.f);
+        s.lam[k] = s.P1[k] = s.P2[k] = g2(0.f, 0.f);
     }
     if (MODE == kBwdFull && a.nseg > 1) {
         // the adjoint state the segments to the right pass in
@@ -239,16 +351,21 @@ __global__ void __launch_bounds__(kThreadsB, 5)
             const int n = g * 4 + j;
             lv[j] = cvalid && n < N ? a.ws_lam[(((int64_t)b * a.nseg + seg) * a.D + d) * N + n] : 0.f;
         }
-        lam[0] = g2(lv[0], lv[1]);
-        lam[1] = g2(lv[2], lv[3]);
+        s.lam[0] = g2(lv[0], lv[1]);
+        s.lam[1] = g2(lv[2], lv[3]);
     }
     float dsum = 0.f;
     const int nvalid = cvalid ? min(4, N - g * 4) : 0;
     float dbias_acc = 0.f;
-    // phase-P channel pair of this thread
+    // phase-P channel pair of this thread (fixed: PAIRS is a multiple of the thread count)
     const int pc = 2 * (tid % (C::DC / 2));
     const int64_t pd = d0 + pc;
+    const float2 pbias = g2((a.bias && pd < a.D) ? __ldg(a.bias + pd) : 0.f,
+                            (a.bias && pd + 1 < a.D) ? __ldg(a.bias + pd + 1) : 0.f);
+    const float2 pdsk = g2((a.Dskip && pd < a.D) ? __ldg(a.Dskip + pd) : 0.f,
+                           (a.Dskip && pd + 1 < a.D) ? __ldg(a.Dskip + pd + 1) : 0.f);
     float2 dD_acc = g2(0.f, 0.f);
+    float* tr = reinterpret_cast<float*>(smem + C::OFF_TR) + warp * C::TR_WARP;
 
     if (tid == 0 && ntb > 0) bad = !mbar_wait(bar0, 0);
     // one CTA-wide choice of the recomputation's Bbar form (block-uniform branch)
@@ -262,57 +379,52 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         const int t0 = it * kTB;
         const int tile_len = (int)(a.L - t0 < kTB ? a.L - t0 : kTB);
         const unsigned char* raw = smem + C::OFF_RAW + st * C::STAGE;
-        // ---- phase P
+        // ---- phase P: operand pairs of every (step, channel) of the tile
         {
             const P2* ru = reinterpret_cast<const P2*>(raw);
             const P2* rd = reinterpret_cast<const P2*>(raw + C::RAW);
             const P2* rz = reinterpret_cast<const P2*>(raw + 2 * C::RAW);
             const P2* rg = reinterpret_cast<const P2*>(raw + 3 * C::RAW);
-            // two channels per thread: one contiguous 16-byte (or 8-byte) store per array
             float4* sdx = reinterpret_cast<float4*>(smem + C::OFF_DX);
             float2* sdy = reinterpret_cast<float2*>(smem + C::OFF_DY);
-            float4* sdq = reinterpret_cast<float4*>(smem + C::OFF_DQ);
-            float4* sdd = reinterpret_cast<float4*>(smem + C::OFF_DD);
+            float4* sep = reinterpret_cast<float4*>(smem + C::OFF_EP);
             float2* ssu = reinterpret_cast<float2*>(smem + C::OFF_SU);
-            const float pb0 = (a.bias && pd < a.D) ? __ldg(a.bias + pd) : 0.f;
-            const float pb1 = (a.bias && pd + 1 < a.D) ? __ldg(a.bias + pd + 1) : 0.f;
-            const float pk0 = (a.Dskip && pd < a.D) ? __ldg(a.Dskip + pd) : 0.f;
-            const float pk1 = (a.Dskip && pd + 1 < a.D) ? __ldg(a.Dskip + pd + 1) : 0.f;
 #pragma unroll
-            for (int q = tid; q < C::PAIRS; q += kThreadsB) {
+            for (int qi = 0; qi < C::PAIRS / kThreadsB; ++qi) {
+                const int q = tid + qi * kThreadsB;
                 const int t = q / (C::DC / 2);
                 const bool tv = t < tile_len;
                 const float2 uv = BPair<T>::f(ru[q]);
                 float2 x = uv;
                 if (a.input_silu) {
-                    x = g2(silu(uv.x), silu(uv.y));
-                    ssu[(t * C::DC + pc) / 2] = make_float2(dsilu(uv.x), dsilu(uv.y));
+                    const float2 su = sigmoid_x2(uv);
+                    x = __fmul2_rn(uv, su);
+                    // SiLU'(u) = s (1 + u (1 - s))
+                    const float2 om = __ffma2_rn(su, g2(-1.f, -1.f), g2(1.f, 1.f));
+                    ssu[(t * C::DC + pc) / 2] = __fmul2_rn(su, __ffma2_rn(uv, om, g2(1.f, 1.f)));
                 }
-                const float2 r = BPair<T>::f(rd[q]);
+                const float2 r = __fadd2_rn(BPair<T>::f(rd[q]), pbias);
+                float2 dl = r, sr = g2(1.f, 1.f);
+                if (a.softplus) softplus_sig_x2(r, dl, sr);
                 const float2 go = BPair<T>::f(rg[q]);
-                float dl0 = r.x + pb0, dl1 = r.y + pb1, s0 = 1.f, s1 = 1.f;
-                if (a.softplus) {
-                    const float2 p0 = softplus_dsig(dl0), p1 = softplus_dsig(dl1);
-                    dl0 = p0.x;
-                    s0 = p0.y;
-                    dl1 = p1.x;
-                    s1 = p1.y;
-                }
-                float dy0 = go.x, dy1 = go.y, dz0 = 0.f, dz1 = 0.f;
+                float2 dy = go, dzf = g2(0.f, 0.f);
                 if (has_z) {
                     const float2 zz = BPair<T>::f(rz[q]);
-                    const float sz0 = sigmoid(zz.x), sz1 = sigmoid(zz.y);
-                    dy0 = go.x * zz.x * sz0;
-                    dy1 = go.y * zz.y * sz1;
-                    dz0 = go.x * sz0 * fmaf(zz.x, 1.f - sz0, 1.f);
-                    dz1 = go.y * sz1 * fmaf(zz.y, 1.f - sz1, 1.f);
+                    const float2 sz = sigmoid_x2(zz);
+                    const float2 gs = __fmul2_rn(go, sz);
+                    dy = __fmul2_rn(gs, zz);
+                    // dz factor: dout s (1 + z (1 - s))
+                    dzf = __fmul2_rn(gs, __ffma2_rn(zz, __ffma2_rn(sz, g2(-1.f, -1.f), g2(1.f, 1.f)), g2(1.f, 1.f)));
                 }
-                if (!tv) dy0 = dy1 = dz0 = dz1 = 0.f;
-                sdx[(t * C::DC + pc) / 2] = make_float4(dl0, x.x, dl1, x.y);
-                sdy[(t * C::DC + pc) / 2] = make_float2(dy0, dy1);
-                sdq[(t * C::DC + pc) / 2] = make_float4(dz0, s0, dz1, s1);
-                sdd[(t * C::DC + pc) / 2] = make_float4(pk0 * dy0, pk0 * x.x, pk1 * dy1, pk1 * x.y);
-                if (tv) dD_acc = g2(fmaf(dy0, x.x, dD_acc.x), fmaf(dy1, x.y, dD_acc.y));
+                if (!tv) dy = dzf = g2(0.f, 0.f);
+                const int e = t * C::DC + pc;
+                sdx[e] = make_float4(dl.x, dl.x, x.x, x.x);
+                sdx[e + 1] = make_float4(dl.y, dl.y, x.y, x.y);
+                reinterpret_cast<float4*>(sdy)[e / 2] = make_float4(dy.x, dy.x, dy.y, dy.y);
+                const float2 kdy = __fmul2_rn(pdsk, dy), kx = __fmul2_rn(pdsk, x);
+                sep[e] = make_float4(kdy.x, dzf.x, sr.x, kx.x);
+                sep[e + 1] = make_float4(kdy.y, dzf.y, sr.y, kx.y);
+                dD_acc = __ffma2_rn(dy, x, dD_acc);
             }
             const T* rB = reinterpret_cast<const T*>(raw + 4 * C::RAW);
             const T* rC = reinterpret_cast<const T*>(raw + 4 * C::RAW + C::RAWBC);
@@ -328,20 +440,21 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         __syncthreads();
         if (tid == 0 && k + C::STAGES < ntb) issue(k + C::STAGES);
 
+        const float4* sdx = reinterpret_cast<const float4*>(smem + C::OFF_DX) + cw;
+        const float2* sdy = reinterpret_cast<const float2*>(smem + C::OFF_DY) + cw;
+        const float4* sB = reinterpret_cast<const float4*>(smem + C::OFF_B) + g;
+        const float4* sC = reinterpret_cast<const float4*>(smem + C::OFF_C) + g;
         if constexpr (MODE == kBwdSummary) {
             // adjoint only: lam <- Abar_t (C_t dy_t + lam), from the right end of the segment
-            const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
-            const float* sdy = reinterpret_cast<const float*>(smem + C::OFF_DY) + cw;
-            const float4* sC = reinterpret_cast<const float4*>(smem + C::OFF_C) + g;
             for (int t = tile_len - 1; t >= 0; --t) {
-                const float2 dx = sdx[t * C::DC];
-                const float dy = sdy[t * C::DC];
+                const float4 dx = sdx[t * C::DC];
+                const float dy = sdy[t * C::DC].x;
                 const float4 Cv = sC[t * NG];
-                const float2 dd = g2(dx.x, dx.x), dyy = g2(dy, dy);
+                const float2 dd = g2(dx.x, dx.y), dyy = g2(dy, dy);
                 const float2 Cp[2] = {g2(Cv.x, Cv.y), g2(Cv.z, Cv.w)};
 #pragma unroll
                 for (int p = 0; p < 2; ++p)
-                    lam[p] = __fmul2_rn(__ffma2_rn(Cp[p], dyy, lam[p]), ex2p(__fmul2_rn(dd, A2[p])));
+                    s.lam[p] = __fmul2_rn(__ffma2_rn(Cp[p], dyy, s.lam[p]), ex2p(__fmul2_rn(dd, s.A2[p])));
                 dsum += dx.x;
             }
             if (tid == 0 && k + 1 < ntb)
@@ -351,147 +464,97 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         }
 
         // ---- recompute the tile's states from the checkpoint
-        const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
-        const float* sdy = reinterpret_cast<const float*>(smem + C::OFF_DY) + cw;
-        const float2* sdq = reinterpret_cast<const float2*>(smem + C::OFF_DQ) + cw;
-        const float2* sdd = reinterpret_cast<const float2*>(smem + C::OFF_DD) + cw;
-        const float4* sB = reinterpret_cast<const float4*>(smem + C::OFF_B) + g;
-        const float4* sC = reinterpret_cast<const float4*>(smem + C::OFF_C) + g;
         float4* shs = reinterpret_cast<float4*>(smem + C::OFF_HS) + tid;
-        float2 hk[2];
+        float4 hk;
         {
             const float* ck = a.ws_ckpt + (((int64_t)b * a.nck + it) * a.D + d) * N + g * 4;
             float hv[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) hv[j] = j < nvalid ? ck[j] : 0.f;
-            hk[0] = g2(hv[0], hv[1]);
-            hk[1] = g2(hv[2], hv[3]);
+            hk = make_float4(hv[0], hv[1], hv[2], hv[3]);
         }
-        if (!acc) {
-            // the forward kernel's form: h' = Abar (h - v) + v with v = -B x / A
-            float2 h0 = hk[0], h1 = hk[1];
-            for (int t = 0; t < tile_len; ++t) {
-                const float2 dx = sdx[t * C::DC];
-                const float4 Bv = sB[t * NG];
-                const float2 dd = g2(dx.x, dx.x), xx = g2(dx.y, dx.y);
-                const float2 v0 = __fmul2_rn(__fmul2_rn(g2(Bv.x, Bv.y), xx), __fmul2_rn(iA[0], g2(-1.f, -1.f)));
-                const float2 v1 = __fmul2_rn(__fmul2_rn(g2(Bv.z, Bv.w), xx), __fmul2_rn(iA[1], g2(-1.f, -1.f)));
-                h0 = __ffma2_rn(ex2p(__fmul2_rn(dd, A2[0])), __ffma2_rn(v0, g2(-1.f, -1.f), h0), v0);
-                h1 = __ffma2_rn(ex2p(__fmul2_rn(dd, A2[1])), __ffma2_rn(v1, g2(-1.f, -1.f), h1), v1);
-                shs[t * kThreadsB] = make_float4(h0.x, h0.y, h1.x, h1.y);
-            }
-        } else {
-            // |A| < 2^-10 somewhere in the block: Bbar from phi1's series where delta A is small
-            float2 h0 = hk[0], h1 = hk[1];
-            for (int t = 0; t < tile_len; ++t) {
-                const float2 dx = sdx[t * C::DC];
-                const float4 Bv = sB[t * NG];
-                const float2 dd = g2(dx.x, dx.x), xx = g2(dx.y, dx.y);
-                const float2 Bx0 = __fmul2_rn(g2(Bv.x, Bv.y), xx), Bx1 = __fmul2_rn(g2(Bv.z, Bv.w), xx);
-                h0 = __ffma2_rn(ex2p(__fmul2_rn(dd, A2[0])), h0, __fmul2_rn(bbar2(dd, A2[0], iA[0]), Bx0));
-                h1 = __ffma2_rn(ex2p(__fmul2_rn(dd, A2[1])), h1, __fmul2_rn(bbar2(dd, A2[1], iA[1]), Bx1));
-                shs[t * kThreadsB] = make_float4(h0.x, h0.y, h1.x, h1.y);
+        {
+            float2 h0 = g2(hk.x, hk.y), h1 = g2(hk.z, hk.w);
+            if (!acc) {
+                // the forward kernel's form: h' = Abar (h - v) + v with v = -B x / A
+                for (int t = 0; t < tile_len; ++t) {
+                    const float4 dx = sdx[t * C::DC];
+                    const float4 Bv = sB[t * NG];
+                    const float2 dd = g2(dx.x, dx.y), xx = g2(dx.z, dx.w);
+                    const float2 v0 = __fmul2_rn(g2(Bv.x, Bv.y), __fmul2_rn(xx, s.niA[0]));
+                    const float2 v1 = __fmul2_rn(g2(Bv.z, Bv.w), __fmul2_rn(xx, s.niA[1]));
+                    h0 = __ffma2_rn(ex2p(__fmul2_rn(dd, s.A2[0])), __ffma2_rn(v0, g2(-1.f, -1.f), h0), v0);
+                    h1 = __ffma2_rn(ex2p(__fmul2_rn(dd, s.A2[1])), __ffma2_rn(v1, g2(-1.f, -1.f), h1), v1);
+                    shs[t * kThreadsB] = make_float4(h0.x, h0.y, h1.x, h1.y);
+                }
+            } else {
+                // |A| < 2^-10 somewhere in the block: Bbar from phi1's series where delta A is small
+                const float2 iA[2] = {g2(-s.niA[0].x, -s.niA[0].y), g2(-s.niA[1].x, -s.niA[1].y)};
+                for (int t = 0; t < tile_len; ++t) {
+                    const float4 dx = sdx[t * C::DC];
+                    const float4 Bv = sB[t * NG];
+                    const float2 dd = g2(dx.x, dx.y), xx = g2(dx.z, dx.w);
+                    const float2 Bx0 = __fmul2_rn(g2(Bv.x, Bv.y), xx), Bx1 = __fmul2_rn(g2(Bv.z, Bv.w), xx);
+                    h0 = __ffma2_rn(ex2p(__fmul2_rn(dd, s.A2[0])), h0, __fmul2_rn(bbar2(dd, s.A2[0], iA[0]), Bx0));
+                    h1 = __ffma2_rn(ex2p(__fmul2_rn(dd, s.A2[1])), h1, __fmul2_rn(bbar2(dd, s.A2[1], iA[1]), Bx1));
+                    shs[t * kThreadsB] = make_float4(h0.x, h0.y, h1.x, h1.y);
+                }
             }
         }
         // ---- reverse sweep in blocks of NG steps (last block first); the state loaded as
         // h_{t-1} at step t is the h_t of step t-1, so it is carried in registers
         T* so = reinterpret_cast<T*>(smem + C::OFF_OUT + (k & 1) * 3 * C::RAW);
+        const float4* sep = reinterpret_cast<const float4*>(smem + C::OFF_EP) + cw;
+        const float* ssu = reinterpret_cast<const float*>(smem + C::OFF_SU) + cw;
         float4 hnext = tile_len > 0 ? shs[(tile_len - 1) * kThreadsB] : make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int tb = ((tile_len - 1) / NG) * NG; tb >= 0; tb -= NG) {
-            float pdu[NG], pdd[NG], py[NG];
-#pragma unroll
-            for (int kk = NG - 1; kk >= 0; --kk) {
-                const int t = tb + kk;
-                pdu[kk] = pdd[kk] = py[kk] = 0.f;
-                float vbc[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) vbc[j] = 0.f;
-                if (t < tile_len) {
-                    const float2 dx = sdx[t * C::DC];
-                    const float dy = sdy[t * C::DC];
-                    const float4 Bv = sB[t * NG], Cv = sC[t * NG];
-                    const float4 hc = hnext;
-                    float2 hp[2];
-                    if (t > 0) {
-                        hnext = shs[(t - 1) * kThreadsB];
-                        hp[0] = g2(hnext.x, hnext.y);
-                        hp[1] = g2(hnext.z, hnext.w);
-                    } else {
-                        hp[0] = hk[0];
-                        hp[1] = hk[1];
-                    }
-                    const float2 dd = g2(dx.x, dx.x), xx = g2(dx.y, dx.y), dyy = g2(dy, dy);
-                    const float2 hcv[2] = {g2(hc.x, hc.y), g2(hc.z, hc.w)};
-                    const float2 Bp[2] = {g2(Bv.x, Bv.y), g2(Bv.z, Bv.w)};
-                    const float2 Cp[2] = {g2(Cv.x, Cv.y), g2(Cv.z, Cv.w)};
-                    float2 du2 = g2(0.f, 0.f), S1 = g2(0.f, 0.f), S2 = g2(0.f, 0.f), y2 = g2(0.f, 0.f);
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        const float2 q2 = __fmul2_rn(dd, A2[p]);
-                        const float2 q = __fmul2_rn(q2, g2(kLn2, kLn2));
-                        const float2 ab = ex2p(q2);
-                        const float2 l = __ffma2_rn(Cp[p], dyy, lam[p]);
-                        const float2 la = __fmul2_rn(l, ab);
-                        // beta = Bbar / B = expm1(q) / A: series delta phi1(q) near q = 0
-                        // -psi(q), psi(q) = (q e^q - expm1(q)) / q^2, by its series (|q| < 1/2 uses it)
-                        float2 nps = __ffma2_rn(q, g2(-1.f / 840.f, -1.f / 840.f), g2(-1.f / 144.f, -1.f / 144.f));
-                        nps = __ffma2_rn(nps, q, g2(-1.f / 30.f, -1.f / 30.f));
-                        nps = __ffma2_rn(nps, q, g2(-0.125f, -0.125f));
-                        nps = __ffma2_rn(nps, q, g2(-1.f / 3.f, -1.f / 3.f));
-                        nps = __ffma2_rn(nps, q, g2(-0.5f, -0.5f));
-                        // beta = Bbar / B: for |q| < 1/2, delta phi1(q) with phi1 = Abar - q psi (no
-                        // cancellation); else (Abar - 1) / A
-                        const float2 bs = __fmul2_rn(dd, __ffma2_rn(q, nps, ab));
-                        const float2 bl = __fmul2_rn(__fadd2_rn(ab, g2(-1.f, -1.f)), iA[p]);
-                        const bool sx = fabsf(q.x) < 0.5f, sy = fabsf(q.y) < 0.5f;
-                        const float2 beta = g2(sx ? bs.x : bl.x, sy ? bs.y : bl.y);
-                        // -(delta Abar - beta) / A = -delta^2 psi(q): the series where |q| < 1/2
-                        const float2 nt2s = __fmul2_rn(__fmul2_rn(dd, dd), nps);
-                        const float2 nt2c = __fmul2_rn(__ffma2_rn(dd, g2(-ab.x, -ab.y), beta), iA[p]);
-                        const float2 nt2 = g2(sx ? nt2s.x : nt2c.x, sy ? nt2s.y : nt2c.y);
-                        const float2 lb = __fmul2_rn(l, beta);
-                        const float2 dBv = __fmul2_rn(lb, xx);
-                        const float2 dCv = __fmul2_rn(dyy, hcv[p]);
-                        vbc[2 * p] = dBv.x;
-                        vbc[2 * p + 1] = dBv.y;
-                        vbc[4 + 2 * p] = dCv.x;
-                        vbc[4 + 2 * p + 1] = dCv.y;
-                        du2 = __ffma2_rn(lb, Bp[p], du2);
-                        const float2 lah = __fmul2_rn(la, hp[p]);
-                        S1 = __ffma2_rn(A2[p], lah, S1);
-                        S2 = __ffma2_rn(la, Bp[p], S2);
-                        const float2 Bx = __fmul2_rn(Bp[p], xx);
-                        P1[p] = __ffma2_rn(dd, lah, P1[p]);
-                        P2v[p] = __ffma2_rn(__fmul2_rn(l, Bx), nt2, P2v[p]);  // minus the psi term
-                        y2 = __ffma2_rn(Cp[p], hcv[p], y2);
-                        lam[p] = la;
-                    }
-                    pdu[kk] = du2.x + du2.y;
-                    pdd[kk] = fmaf(kLn2, S1.x + S1.y, dx.y * (S2.x + S2.y));
-                    py[kk] = y2.x + y2.y;
-                }
-                // dB, dC of step t summed over this warp's channels, then over the CTA in smem
-                const float v = treduce_c8<C::CW>(vbc, c);
-                if (c < 8 && t < tile_len) {
-                    const int which = c >> 2, j = c & 3;
-                    sacc[warp * kAccWarp + (t * C::NS + g * 4 + j) * 2 + which] = v;
-                }
+        auto step = [&](int t, float& pdu, float& pdd, float& py) {
+            float vbc[8];
+            const float4 hc = hnext;
+            hnext = t > 0 ? shs[(t - 1) * kThreadsB] : hk;
+            rev_step(s, sdx[t * C::DC], sdy[t * C::DC], sB[t * NG], sC[t * NG], hc, hnext, pdu, pdd, py, vbc);
+            // dB, dC of step t summed over this warp's channels, then over the CTA in smem
+            float v;
+            if constexpr (NG == 4) v = tr_reduce8<C::CW>(vbc, tr, g, c);
+            else v = treduce_c8<C::CW>(vbc, c);
+            if (c < 8) {
+                const int which = c >> 2, j = c & 3;
+                atomicAdd(&sacc[(t * C::NS + g * 4 + j) * 2 + which], v);
             }
+        };
+        auto finish = [&](int tb, float (&pdu)[NG], float (&pdd)[NG], float (&py)[NG]) {
             const float sdu = treduce_g<NG, C::CW>(pdu, g);
             const float sdd_ = treduce_g<NG, C::CW>(pdd, g);
             const float sy = treduce_g<NG, C::CW>(py, g);
             const int t = tb + g;
             if (t < tile_len && g < NG) {
-                const float2 dq = sdq[t * C::DC];  // (dz factor, softplus')
-                const float2 ddv = sdd[t * C::DC];
-                float du = sdu + ddv.x;
-                if (a.input_silu) du *= reinterpret_cast<const float*>(smem + C::OFF_SU)[t * C::DC + cw];
-                const float ddr = sdd_ * dq.y;
-                const float dz = dq.x * (sy + ddv.y);
+                const float4 ep = sep[t * C::DC];  // (D dy, dz factor, softplus', D x)
+                float du = sdu + ep.x;
+                if (a.input_silu) du *= ssu[t * C::DC];
+                const float ddr = sdd_ * ep.z;
                 so[t * C::DC + cw] = from_f32<T>(du);
                 so[C::RAW / (int)sizeof(T) + t * C::DC + cw] = from_f32<T>(ddr);
-                so[2 * C::RAW / (int)sizeof(T) + t * C::DC + cw] = from_f32<T>(dz);
+                so[2 * C::RAW / (int)sizeof(T) + t * C::DC + cw] = from_f32<T>(ep.y * (sy + ep.w));
                 if (cvalid) dbias_acc += ddr;
+            }
+        };
+        if (tile_len == kTB) {
+#pragma unroll
+            for (int tb = kTB - NG; tb >= 0; tb -= NG) {
+                float pdu[NG], pdd[NG], py[NG];
+#pragma unroll
+                for (int kk = NG - 1; kk >= 0; --kk) step(tb + kk, pdu[kk], pdd[kk], py[kk]);
+                finish(tb, pdu, pdd, py);
+            }
+        } else {
+            // the sequence's last, partial tile
+            for (int tb = ((tile_len - 1) / NG) * NG; tb >= 0; tb -= NG) {
+                float pdu[NG], pdd[NG], py[NG];
+#pragma unroll
+                for (int kk = NG - 1; kk >= 0; --kk) {
+                    pdu[kk] = pdd[kk] = py[kk] = 0.f;
+                    if (tb + kk < tile_len) step(tb + kk, pdu[kk], pdd[kk], py[kk]);
+                }
+                finish(tb, pdu, pdd, py);
             }
         }
         fence_proxy_async();
@@ -506,21 +569,18 @@ __global__ void __launch_bounds__(kThreadsB, 5)
             tma_commit();
             tma_store_wait_read_1();
         }
-        // the tile's dB, dC: the warps' sums into the fp32 accumulators
+        // the tile's dB, dC into the fp32 accumulators (the next tile adds into sacc only
+        // after its phase-P barrier)
         for (int e = tid; e < tile_len * C::NS; e += kThreadsB) {
             const int t = e / C::NS, n = e % C::NS;
+            float2* slot = reinterpret_cast<float2*>(sacc) + e;
             if (n < N) {
-                float2 v = reinterpret_cast<const float2*>(sacc)[e];
-#pragma unroll
-                for (int w = 1; w < kWarpsB; ++w) {
-                    const float2 u = reinterpret_cast<const float2*>(sacc + w * kAccWarp)[e];
-                    v.x += u.x;
-                    v.y += u.y;
-                }
+                const float2 v = *slot;
                 const int64_t gi = ((int64_t)b * a.L + t0 + t) * N + n;
                 atomicAdd(a.dB32 + gi, v.x);
                 atomicAdd(a.dC32 + gi, v.y);
             }
+            *slot = make_float2(0.f, 0.f);
         }
     }
     if (tid == 0) tma_store_wait_all();
@@ -531,7 +591,7 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         }
         return;
     }
-    const float lamv[4] = {lam[0].x, lam[0].y, lam[1].x, lam[1].y};
+    const float lamv[4] = {s.lam[0].x, s.lam[0].y, s.lam[1].x, s.lam[1].y};
     if constexpr (MODE == kBwdSummary) {
         // the segment's summary: adjoint state passed on from zero, and its sum of delta
 #pragma unroll
@@ -541,7 +601,7 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         return;
     }
     // per-channel sums
-    const float dAv[4] = {P1[0].x - P2v[0].x, P1[0].y - P2v[0].y, P1[1].x - P2v[1].x, P1[1].y - P2v[1].y};
+    const float dAv[4] = {s.P1[0].x + s.P2[0].x, s.P1[0].y + s.P2[0].y, s.P1[1].x + s.P2[1].x, s.P1[1].y + s.P2[1].y};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         if (j >= nvalid) continue;
