@@ -256,13 +256,20 @@ SSCAN_API const char* sscan_last_error(void);
  * not counted). */
 SSCAN_API int sscan_last_launch_count(void);
 
+/* 1 in the debug build of the library (libsscan_debug.so), whose kernels check every
+ * index they compute into a workspace, parameter or state array and report a bad one
+ * through bit 3 of sscan_device_status (skipping the access) instead of touching the
+ * memory; 0 in the release build, where those checks are compiled out. */
+SSCAN_API int sscan_debug_bounds(void);
+
 /*
  * Device-side status of the library's kernels on the current device: *flags
  * receives the OR of every error bit raised since the last clear (bit 0: in a
  * forward kernel, bit 1: in the backward kernel, a bounded wait for an
  * asynchronous tile copy gave up, so that kernel stopped early and its outputs
  * are incomplete; bit 2: sscan_probe_wait_timeout's wait ran out, as it is meant
- * to).  Returns SSCAN_ERR_TIMEOUT when any bit is set, SSCAN_OK when none is.
+ * to; bit 3, debug build only: an index out of its array's range was caught and the
+ * access skipped).  Returns SSCAN_ERR_TIMEOUT when any bit is set, SSCAN_OK when none is.
  * clear != 0 resets the word after reading.  Synchronous: it waits for work
  * already submitted to the device.  Every wait in the library's kernels is
  * bounded, so a failed copy surfaces here instead of hanging the device.

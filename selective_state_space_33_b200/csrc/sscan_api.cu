@@ -833,14 +833,23 @@ const char* sscan_last_error(void) { return g_err; }
 
 int sscan_last_launch_count(void) { return g_launches; }
 
+int sscan_debug_bounds(void) {
+#ifdef SSCAN_DEBUG_BOUNDS
+    return 1;
+#else
+    return 0;
+#endif
+}
+
 sscan_status sscan_device_status(int clear, unsigned int* flags) {
     g_err[0] = 0;
     if (!flags) return fail(SSCAN_ERR_INVALID_ARG, "flags is NULL");
-    unsigned int f1 = 0, f2 = 0;
+    unsigned int f1 = 0, f2 = 0, f3 = 0;
     cudaError_t e = sscan::read_device_error(&f1, clear);
     if (e == cudaSuccess) e = sscan::read_device_error_bwd(&f2, clear);
+    if (e == cudaSuccess) e = sscan::read_device_error_cx(&f3, clear);
     if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
-    *flags = f1 | f2;
+    *flags = f1 | f2 | f3;
     return *flags ? SSCAN_ERR_TIMEOUT : SSCAN_OK;
 }
 

@@ -35,6 +35,7 @@
 
 #include "sscan_launch.h"
 #include "sscan_affine.cuh"
+#include "sscan_check.cuh"
 #include "sscan_math.cuh"
 #include "sscan_tma.cuh"
 
@@ -287,6 +288,9 @@ __global__ void __launch_bounds__(kThreadsB, 5)
     const int b = (int)(rest / nsl);
     const int N = a.N;
     const int d0 = cb * C::DC;
+    // extents of the arrays indexed below (checked in the debug build only)
+    const int64_t ext_seg = a.batch * a.nseg * a.D * N, ext_ckpt = a.batch * a.nck * a.D * N;
+    const int64_t ext_bln = a.batch * a.L * N;
     const int tiles_all = (int)((a.L + kTB - 1) / kTB);
     const int tile_lo = seg * (int)(a.seg_len / kTB);
     const int tile_hi = min(tiles_all, tile_lo + (int)((a.seg_len + kTB - 1) / kTB));
@@ -334,7 +338,7 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         for (int j = 0; j < 2; ++j) {
             const int n = g * 4 + 2 * k + j;
             const bool ok = cvalid && n < N;
-            av[j] = ok ? __ldg(a.A + d * N + n) : 0.f;
+            av[j] = ok && in_range(d * N + n, a.D * N) ? __ldg(a.A + d * N + n) : 0.f;
             small_a |= ok && fabsf(av[j]) < kSmallAB;
         }
         s.A2[k] = g2(av[0] * kLog2e, av[1] * kLog2e);
@@ -349,7 +353,8 @@ __global__ void __launch_bounds__(kThreadsB, 5)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int n = g * 4 + j;
-            lv[j] = cvalid && n < N ? a.ws_lam[(((int64_t)b * a.nseg + seg) * a.D + d) * N + n] : 0.f;
+            const int64_t il = (((int64_t)b * a.nseg + seg) * a.D + d) * N + n;
+            lv[j] = cvalid && n < N && in_range(il, ext_seg) ? a.ws_lam[il] : 0.f;
         }
         s.lam[0] = g2(lv[0], lv[1]);
         s.lam[1] = g2(lv[2], lv[3]);
@@ -467,10 +472,10 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         float4* shs = reinterpret_cast<float4*>(smem + C::OFF_HS) + tid;
         float4 hk;
         {
-            const float* ck = a.ws_ckpt + (((int64_t)b * a.nck + it) * a.D + d) * N + g * 4;
+            const int64_t ic = (((int64_t)b * a.nck + it) * a.D + d) * N + g * 4;
             float hv[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) hv[j] = j < nvalid ? ck[j] : 0.f;
+            for (int j = 0; j < 4; ++j) hv[j] = j < nvalid && in_range(ic + j, ext_ckpt) ? a.ws_ckpt[ic + j] : 0.f;
             hk = make_float4(hv[0], hv[1], hv[2], hv[3]);
         }
         {
@@ -577,8 +582,10 @@ __global__ void __launch_bounds__(kThreadsB, 5)
             if (n < N) {
                 const float2 v = *slot;
                 const int64_t gi = ((int64_t)b * a.L + t0 + t) * N + n;
-                atomicAdd(a.dB32 + gi, v.x);
-                atomicAdd(a.dC32 + gi, v.y);
+                if (in_range(gi, ext_bln)) {
+                    atomicAdd(a.dB32 + gi, v.x);
+                    atomicAdd(a.dC32 + gi, v.y);
+                }
             }
             *slot = make_float2(0.f, 0.f);
         }
@@ -595,9 +602,12 @@ __global__ void __launch_bounds__(kThreadsB, 5)
     if constexpr (MODE == kBwdSummary) {
         // the segment's summary: adjoint state passed on from zero, and its sum of delta
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (j < nvalid) a.ws_lam[(((int64_t)b * a.nseg + seg) * a.D + d) * N + g * 4 + j] = lamv[j];
-        if (g == 0 && cvalid) a.ws_dsum[((int64_t)b * a.nseg + seg) * a.D + d] = dsum;
+        for (int j = 0; j < 4; ++j) {
+            const int64_t il = (((int64_t)b * a.nseg + seg) * a.D + d) * N + g * 4 + j;
+            if (j < nvalid && in_range(il, ext_seg)) a.ws_lam[il] = lamv[j];
+        }
+        const int64_t idsum = ((int64_t)b * a.nseg + seg) * a.D + d;
+        if (g == 0 && cvalid && in_range(idsum, a.batch * a.nseg * a.D)) a.ws_dsum[idsum] = dsum;
         return;
     }
     // per-channel sums
@@ -606,14 +616,15 @@ __global__ void __launch_bounds__(kThreadsB, 5)
     for (int j = 0; j < 4; ++j) {
         if (j >= nvalid) continue;
         const int n = g * 4 + j;
-        if (a.dh0 && seg == 0) a.dh0[((int64_t)b * a.D + d) * N + n] = lamv[j];
+        const int64_t is = ((int64_t)b * a.D + d) * N + n;
+        if (a.dh0 && seg == 0 && in_range(is, a.batch * a.D * N)) a.dh0[is] = lamv[j];
         // dA = sum_t [delta lam Abar h_{t-1} + lam B x delta^2 psi(delta A)]
-        atomicAdd(a.dA + d * N + n, dAv[j]);
+        if (in_range(d * N + n, a.D * N)) atomicAdd(a.dA + d * N + n, dAv[j]);
     }
-    if (a.dbias && cvalid) atomicAdd(a.dbias + d, dbias_acc);
+    if (a.dbias && cvalid && in_range(d, a.D)) atomicAdd(a.dbias + d, dbias_acc);
     if (a.dD && pd < a.D) {
-        atomicAdd(a.dD + pd, dD_acc.x);
-        if (pd + 1 < a.D) atomicAdd(a.dD + pd + 1, dD_acc.y);
+        if (in_range(pd, a.D)) atomicAdd(a.dD + pd, dD_acc.x);
+        if (pd + 1 < a.D && in_range(pd + 1, a.D)) atomicAdd(a.dD + pd + 1, dD_acc.y);
     }
 }
 
@@ -695,11 +706,16 @@ __global__ void __launch_bounds__(128) bwd_carry_kernel(BwdTiledArgs a, int W) {
         a.nseg - 1, 0.f, W, valid,
         [&](int64_t j, float& p, float& q) {
             const int64_t s = a.nseg - 1 - j;
-            p = ex2(A2 * a.ws_dsum[(b * a.nseg + s) * a.D + d]);
-            q = a.ws_lam[((b * a.nseg + s) * a.D + d) * a.N + n];
+            const int64_t id = (b * a.nseg + s) * a.D + d, il = id * a.N + n;
+            p = in_range(id, a.batch * a.nseg * a.D) ? ex2(A2 * a.ws_dsum[id]) : 0.f;
+            q = in_range(il, a.batch * a.nseg * a.D * a.N) ? a.ws_lam[il] : 0.f;
         },
-        [&](int64_t j, float v) { a.ws_lam[((b * a.nseg + (a.nseg - 1 - j)) * a.D + d) * a.N + n] = v; });
-    if (valid && (threadIdx.x & (W - 1)) == 0) a.ws_lam[((b * a.nseg) * a.D + d) * a.N + n] = lam0;
+        [&](int64_t j, float v) {
+            const int64_t il = ((b * a.nseg + (a.nseg - 1 - j)) * a.D + d) * a.N + n;
+            if (in_range(il, a.batch * a.nseg * a.D * a.N)) a.ws_lam[il] = v;
+        });
+    const int64_t i0 = ((b * a.nseg) * a.D + d) * a.N + n;
+    if (valid && (threadIdx.x & (W - 1)) == 0 && in_range(i0, a.batch * a.nseg * a.D * a.N)) a.ws_lam[i0] = lam0;
 }
 
 }  // namespace

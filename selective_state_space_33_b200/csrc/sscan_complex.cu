@@ -7,9 +7,13 @@
 //
 // Work decomposition (as the real tiled kernel): a CTA of 4 warps owns one batch
 // and DC channels for the whole sequence; the NG lanes of a channel each hold CG
-// complex states (CG = 4, or 2 when the grid is small) in registers.  Per 16-step tile all threads
-// stage (delta, x) and (gate, D x gate) for the tile's channels and the tile's B
-// and C rows in shared memory with coalesced loads (phase P), then every lane
+// complex states (CG = 4, or 2 when the grid is small) in registers.  Per 16-step
+// tile, TMA 3-D tile copies bring u, delta_raw, z (and the B, C rows) into a 2-stage
+// shared-memory ring -- the next tile's copy lands while the current one is scanned;
+// mbarrier completion, every wait bounded -- or, for tensors whose rows or bases are
+// not 16-byte aligned, every thread loads them directly; all threads then stage
+// (delta, x) and (gate, D x gate) for the tile's channels and the tile's B and C rows
+// in shared memory (phase P), then every lane
 // advances its states through the tile (phase S), two states per f32x2 operation, and
 // the NG lanes of a channel sum their partial readouts over blocks of NG steps with a
 // transposed butterfly, each lane writing one step's output.
@@ -21,16 +25,23 @@
 // two-part 2 pi before the MUFU sine and cosine.  A CTA whose block holds an
 // |a| < 2^-10 (a = 0 included) takes Bbar / B = delta phi1(delta a) with phi1's
 // Taylor series in complex arithmetic where |delta a| < 1/16 instead.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "sscan_launch.h"
 #include "sscan_complex_math.cuh"
 #include "sscan_math.cuh"
 #include "sscan_plan.h"
+#include "sscan_tma.cuh"
 
 namespace sscan {
+
+__device__ unsigned int g_device_error_cx = 0;
+
 namespace {
 
 constexpr int kCTT = 16;           // steps per tile
@@ -42,6 +53,20 @@ struct CCfg {
     static constexpr int CW = 32 / NG;       // channels per warp
     static constexpr int DC = CW * kCWarps;  // channels per CTA
     static constexpr int NS = NG * CG;       // states covered (>= N)
+};
+
+// Dynamic shared memory of the TMA path: a 2-stage ring of raw tiles (u, delta_raw, z,
+// then B and C when their rows travel by TMA), 128-byte aligned, and its mbarriers.
+template <typename T, int NG, int CG>
+struct CRing {
+    static constexpr int DC = CCfg<NG, CG>::DC, NS = CCfg<NG, CG>::NS;
+    static constexpr int RAW = kCTT * DC * (int)sizeof(T);
+    static constexpr int RAWBC = (kCTT * NS * (int)sizeof(T) + 127) / 128 * 128;  // one B or C tile (N <= NS)
+    static constexpr int STAGE = (3 * RAW + 2 * RAWBC + 127) / 128 * 128;
+    static constexpr int STAGES = 2;
+    static constexpr int OFF_BAR = STAGES * STAGE;
+    static constexpr int SMEM = OFF_BAR + STAGES * 8;
+    static_assert(RAW % 128 == 0, "raw tiles start 128-byte aligned");
 };
 
 __device__ __forceinline__ float2 ex2x2c(float2 q) { return make_float2(ex2(q.x), ex2(q.y)); }
@@ -220,14 +245,22 @@ __device__ __forceinline__ void scan_tile_c(CLane<CG>& s, const float2* sdx, con
 
 // CKPT: the checkpoint pass of the backward (states before every 8th step, no output);
 // otherwise the forward with outputs.  Separate instantiations keep the per-step
-// checkpoint test out of the output kernel's loop.
-template <typename T, int NG, int CG, bool CKPT>
-__global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, float* ckpt, int64_t nck) {
+// checkpoint test out of the output kernel's loop.  TMA: the tiles come through the
+// TMA ring (maps m[0..4] = u, delta_raw, z, B, C; bc_tma says whether B and C do);
+// otherwise every thread loads them directly.
+template <typename T, int NG, int CG, bool CKPT, bool TMA>
+__global__ void __launch_bounds__(kCThreads)
+    fwd_complex_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dr,
+                       const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_B,
+                       const __grid_constant__ CUtensorMap tm_C, ComplexArgs a, float* ckpt, int64_t nck,
+                       int bc_tma) {
     using C = CCfg<NG, CG>;
+    using R = CRing<T, NG, CG>;
     __shared__ float2 sdx[kCTT * C::DC];  // (delta, x)
     __shared__ float2 sgd[kCTT * C::DC];  // (gate, D x gate)
     __shared__ __align__(16) float sB[kCTT * C::NS];
     __shared__ __align__(16) float sC[kCTT * C::NS];
+    extern __shared__ __align__(128) unsigned char ring[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t ncb = (a.D + C::DC - 1) / C::DC;
     const int64_t b = blockIdx.x / ncb;
@@ -238,6 +271,34 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
     const T* zz = static_cast<const T*>(a.z);
     const T* Bg = static_cast<const T*>(a.B);
     const T* Cg = static_cast<const T*>(a.C);
+    const int ntile = (int)((a.L + kCTT - 1) / kCTT);
+    const bool has_z = zz != nullptr;
+    const uint32_t bar0 = TMA ? smem_u32(ring + R::OFF_BAR) : 0u;
+    const uint32_t stage_bytes = (has_z ? 3u : 2u) * R::RAW + (bc_tma ? 2u * (uint32_t)(kCTT * N * (int)sizeof(T)) : 0u);
+
+    // the TMA copies of tile `it` into its ring stage (elected thread only)
+    auto issue = [&](int it) {
+        const int st = it % R::STAGES;
+        const uint32_t bar = bar0 + 8 * st;
+        const uint32_t base = smem_u32(ring + st * R::STAGE);
+        const int t0 = it * kCTT;
+        mbar_expect_tx(bar, stage_bytes);
+        tma_load_3d(base, &tm_u, (int)d0, t0, (int)b, bar);
+        tma_load_3d(base + R::RAW, &tm_dr, (int)d0, t0, (int)b, bar);
+        if (has_z) tma_load_3d(base + 2 * R::RAW, &tm_z, (int)d0, t0, (int)b, bar);
+        if (bc_tma) {
+            tma_load_3d(base + 3 * R::RAW, &tm_B, 0, t0, (int)b, bar);
+            tma_load_3d(base + 3 * R::RAW + R::RAWBC, &tm_C, 0, t0, (int)b, bar);
+        }
+    };
+    int bad = 0;
+    if constexpr (TMA) {
+        if (tid == 0) {
+            for (int st = 0; st < R::STAGES; ++st) mbar_init(bar0 + 8 * st, 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            for (int it = 0; it < R::STAGES && it < ntile; ++it) issue(it);
+        }
+    }
 
     const int g = lane / C::CW, c = lane % C::CW, cw = warp * C::CW + c;
     const int64_t d = d0 + cw;
@@ -261,22 +322,36 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
         comp(s.hr, j) = h0v ? __ldg(a.h0 + ((b * a.D + d) * N + n) * 2) : 0.f;
         comp(s.hi, j) = h0v ? __ldg(a.h0 + ((b * a.D + d) * N + n) * 2 + 1) : 0.f;
     }
-    const bool acc = __syncthreads_or(small_a ? 1 : 0) != 0;
+    if (TMA && tid == 0 && ntile > 0) bad = !mbar_wait(bar0, 0);
+    const int flags = __syncthreads_or((small_a ? 1 : 0) | (bad ? 2 : 0));
+    const bool acc = (flags & 1) != 0;
+    bool failed = (flags & 2) != 0;
     const int nvalid = cvalid ? (N - g * CG < CG ? N - g * CG : CG) : 0;
 
-    for (int64_t t0 = 0; t0 < a.L; t0 += kCTT) {
+    for (int it = 0; it < ntile && !failed; ++it) {
+        const int64_t t0 = (int64_t)it * kCTT;
         const int tl = (int)(a.L - t0 < kCTT ? a.L - t0 : kCTT);
+        const unsigned char* raw = ring + (it % R::STAGES) * R::STAGE;
         // phase P: (delta, x), (gate, D x gate), and the tile's B and C rows
         for (int e = tid; e < kCTT * C::DC; e += kCThreads) {
             const int t = e / C::DC, cc = e % C::DC;
             const int64_t dd = d0 + cc;
             float2 dx = make_float2(0.f, 0.f), gd = make_float2(0.f, 0.f);
             if (t < tl && dd < a.D) {
-                const int64_t gi = (b * a.L + t0 + t) * a.D + dd;
-                const float uv = IO<T>::load(u, gi);
+                float uv, rv, zv = 0.f;
+                if constexpr (TMA) {
+                    uv = to_f32<T>(reinterpret_cast<const T*>(raw)[e]);
+                    rv = to_f32<T>(reinterpret_cast<const T*>(raw + R::RAW)[e]);
+                    if (has_z) zv = to_f32<T>(reinterpret_cast<const T*>(raw + 2 * R::RAW)[e]);
+                } else {
+                    const int64_t gi = (b * a.L + t0 + t) * a.D + dd;
+                    uv = IO<T>::load(u, gi);
+                    rv = IO<T>::load(dr, gi);
+                    if (has_z) zv = IO<T>::load(zz, gi);
+                }
                 const float x = a.input_silu ? silu(uv) : uv;
-                const float r = IO<T>::load(dr, gi) + (a.bias ? __ldg(a.bias + dd) : 0.f);
-                const float gate = zz ? silu(IO<T>::load(zz, gi)) : 1.f;
+                const float r = rv + (a.bias ? __ldg(a.bias + dd) : 0.f);
+                const float gate = has_z ? silu(zv) : 1.f;
                 const float dsk = a.Dskip ? __ldg(a.Dskip + dd) : 0.f;
                 dx = make_float2(a.softplus ? softplus(r) : r, x);
                 gd = make_float2(gate, dsk * x * gate);
@@ -288,14 +363,22 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
             const int t = e / C::NS, n = e % C::NS;
             float bv = 0.f, cv = 0.f;
             if (t < tl && n < N) {
-                const int64_t gi = (b * a.L + t0 + t) * N + n;
-                bv = IO<T>::load(Bg, gi);
-                cv = IO<T>::load(Cg, gi);
+                if (TMA && bc_tma) {
+                    bv = to_f32<T>(reinterpret_cast<const T*>(raw + 3 * R::RAW)[t * N + n]);
+                    cv = to_f32<T>(reinterpret_cast<const T*>(raw + 3 * R::RAW + R::RAWBC)[t * N + n]);
+                } else {
+                    const int64_t gi = (b * a.L + t0 + t) * N + n;
+                    bv = IO<T>::load(Bg, gi);
+                    cv = IO<T>::load(Cg, gi);
+                }
             }
             sB[e] = bv;
             sC[e] = cv;
         }
+        if constexpr (TMA) fence_proxy_async();
         __syncthreads();
+        // the stage just consumed takes the tile two ahead
+        if (TMA && tid == 0 && it + R::STAGES < ntile) issue(it + R::STAGES);
         T* out = CKPT ? nullptr : static_cast<T*>(a.out) + (b * a.L + t0) * a.D + d;
         float* ck = CKPT ? ckpt + (((b * nck + t0 / 8) * a.D + d) * N + g * CG) * 2 : nullptr;
         const int64_t ck_stride = a.D * N * 2;
@@ -309,7 +392,18 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
         else
             scan_tile_c<T, NG, CG, false, CKPT, false>(s, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
                                                        nvalid);
-        __syncthreads();
+        // the next tile's raw data (or a wait that gave up); shared memory free again
+        if (TMA && tid == 0 && it + 1 < ntile)
+            bad = !mbar_wait(bar0 + 8 * ((it + 1) % R::STAGES), ((it + 1) / R::STAGES) & 1);
+        failed = __syncthreads_or(bad) != 0;
+    }
+    if (failed) {
+        if (tid == 0) {
+            atomicOr(&g_device_error_cx, 1u);
+            // let the copies still in flight land before the CTA's shared memory is released
+            for (int st = 0; st < R::STAGES; ++st) (void)mbar_wait(bar0 + 8 * st, 0), (void)mbar_wait(bar0 + 8 * st, 1);
+        }
+        return;
     }
     if (a.h_last && cvalid) {
 #pragma unroll
@@ -323,15 +417,79 @@ __global__ void __launch_bounds__(kCThreads) fwd_complex_kernel(ComplexArgs a, f
     }
 }
 
+// 3-D map over a (batch, L, W) tensor, box [1][kCTT][box_w], zero fill outside.
+template <typename T>
+bool make_map_c(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int64_t W, int box_w) {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)L, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)(W * sizeof(T)), (cuuint64_t)(L * W * sizeof(T))};
+    const cuuint32_t box[3] = {(cuuint32_t)box_w, (cuuint32_t)kCTT, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapDataType ty =
+        sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    return fn(m, ty, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16c(const void* q) { return q == nullptr || reinterpret_cast<uintptr_t>(q) % 16 == 0; }
+
+template <typename T, int NG, int CG, bool CKPT, bool TMA>
+cudaError_t launch_ck(const CUtensorMap (&m)[5], const ComplexArgs& a, float* ckpt, int64_t nck, int bc_tma,
+                      int64_t blocks, cudaStream_t st) {
+    using R = CRing<T, NG, CG>;
+    auto kern = fwd_complex_kernel<T, NG, CG, CKPT, TMA>;
+    const int smem = TMA ? R::SMEM : 0;
+    if (TMA) {
+        // function attributes are per device: set them once on each device used
+        static bool configured[kMaxDevices] = {};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        if (!configured[dev]) {
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            configured[dev] = true;
+        }
+    }
+    kern<<<(unsigned)blocks, kCThreads, smem, st>>>(m[0], m[1], m[2], m[3], m[4], a, ckpt, nck, bc_tma);
+    return cudaGetLastError();
+}
+
 template <typename T, int NG, int CG>
 cudaError_t launch_c(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream_t st) {
-    const int64_t blocks = a.batch * ((a.D + CCfg<NG, CG>::DC - 1) / CCfg<NG, CG>::DC);
+    using C = CCfg<NG, CG>;
+    const int64_t blocks = a.batch * ((a.D + C::DC - 1) / C::DC);
     if (blocks <= 0) return cudaGetLastError();
-    if (ckpt)
-        fwd_complex_kernel<T, NG, CG, true><<<(unsigned)blocks, kCThreads, 0, st>>>(a, ckpt, nck);
-    else
-        fwd_complex_kernel<T, NG, CG, false><<<(unsigned)blocks, kCThreads, 0, st>>>(a, nullptr, 0);
-    return cudaGetLastError();
+    // the TMA ring needs 16-byte aligned bases and row pitches of the (batch, L, D) tensors
+    CUtensorMap m[5];
+    bool tma = (a.D * (int64_t)sizeof(T)) % 16 == 0 && aligned16c(a.u) && aligned16c(a.delta_raw) &&
+               aligned16c(a.z) && a.L < (int64_t(1) << 31) && a.D < (int64_t(1) << 31);
+    int bc_tma = 0;
+    if (tma) {
+        tma = make_map_c<T>(&m[0], a.u, a.batch, a.L, a.D, C::DC) &&
+              make_map_c<T>(&m[1], a.delta_raw, a.batch, a.L, a.D, C::DC) &&
+              make_map_c<T>(&m[2], a.z ? a.z : a.u, a.batch, a.L, a.D, C::DC);
+        // B and C rows by TMA when a row of N values is a whole number of 16-byte units
+        if (tma && (a.N * (int64_t)sizeof(T)) % 16 == 0 && aligned16c(a.B) && aligned16c(a.C) &&
+            make_map_c<T>(&m[3], a.B, a.batch, a.L, a.N, a.N) && make_map_c<T>(&m[4], a.C ? a.C : a.B, a.batch, a.L, a.N, a.N))
+            bc_tma = 1;
+        else
+            m[3] = m[4] = m[0];
+    }
+    if (!tma) {
+        std::memset(m, 0, sizeof m);
+        return ckpt ? launch_ck<T, NG, CG, true, false>(m, a, ckpt, nck, 0, blocks, st)
+                    : launch_ck<T, NG, CG, false, false>(m, a, nullptr, 0, 0, blocks, st);
+    }
+    return ckpt ? launch_ck<T, NG, CG, true, true>(m, a, ckpt, nck, bc_tma, blocks, st)
+                : launch_ck<T, NG, CG, false, true>(m, a, nullptr, 0, bc_tma, blocks, st);
 }
 
 // Four complex states per lane, or two (twice the lanes per channel, half the
@@ -357,6 +515,15 @@ cudaError_t launch_ct(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream
 
 cudaError_t launch_fwd_complex(const ComplexArgs& a, float* ckpt, int64_t nck, int io_bf16, cudaStream_t st) {
     return io_bf16 ? launch_ct<__nv_bfloat16>(a, ckpt, nck, st) : launch_ct<float>(a, ckpt, nck, st);
+}
+
+cudaError_t read_device_error_cx(unsigned int* value, int clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(value, g_device_error_cx, sizeof(unsigned int));
+    if (e == cudaSuccess && clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error_cx, &zero, sizeof(unsigned int));
+    }
+    return e;
 }
 
 }  // namespace sscan

@@ -8,6 +8,7 @@
 #pragma once
 
 #include "sscan_affine.cuh"
+#include "sscan_check.cuh"
 #include "sscan_math.cuh"
 
 namespace sscan {
@@ -62,16 +63,18 @@ __global__ void __launch_bounds__(128) fwd_rows_kernel(ScanArgs a) {
     float h[NMAX], Al[NMAX], A2[NMAX], invA[NMAX];
 #pragma unroll
     for (int n = 0; n < NMAX; ++n) {
-        const float An = n < N ? __ldg(a.A + d * N + n) : 0.f;
+        const float An = n < N && in_range(d * N + n, a.D * N) ? __ldg(a.A + d * N + n) : 0.f;
         Al[n] = An;
         A2[n] = An * kLog2e;
         invA[n] = An != 0.f ? 1.f / An : 0.f;
         float h_init = 0.f;
         if (MODE == kModeOutput && n < N) {
             if (a.nchunks > 1)
-                h_init = a.ws_state[((b * a.nchunks + c) * a.D + d) * N + n];
+                h_init = in_range(((b * a.nchunks + c) * a.D + d) * N + n, a.batch * a.nchunks * a.D * N)
+                             ? a.ws_state[((b * a.nchunks + c) * a.D + d) * N + n]
+                             : 0.f;
             else if (a.h0)
-                h_init = __ldg(a.h0 + row * N + n);
+                h_init = in_range(row * N + n, a.batch * a.D * N) ? __ldg(a.h0 + row * N + n) : 0.f;
         }
         h[n] = h_init;
     }
@@ -106,12 +109,14 @@ __global__ void __launch_bounds__(128) fwd_rows_kernel(ScanArgs a) {
     if (MODE == kModeAggregate) {
 #pragma unroll
         for (int n = 0; n < NMAX; ++n)
-            if (n < N) a.ws_state[((b * a.nchunks + c) * a.D + d) * N + n] = h[n];
-        a.ws_dsum[(b * a.nchunks + c) * a.D + d] = dsum;
+            if (n < N && in_range(((b * a.nchunks + c) * a.D + d) * N + n, a.batch * a.nchunks * a.D * N))
+                a.ws_state[((b * a.nchunks + c) * a.D + d) * N + n] = h[n];
+        if (in_range((b * a.nchunks + c) * a.D + d, a.batch * a.nchunks * a.D))
+            a.ws_dsum[(b * a.nchunks + c) * a.D + d] = dsum;
     } else if (a.h_last && c == a.nchunks - 1) {
 #pragma unroll
         for (int n = 0; n < NMAX; ++n)
-            if (n < N) a.h_last[row * N + n] = h[n];
+            if (n < N && in_range(row * N + n, a.batch * a.D * N)) a.h_last[row * N + n] = h[n];
     }
 }
 
@@ -133,10 +138,14 @@ __global__ void __launch_bounds__(128) carry_kernel(ScanArgs a, int W) {
     const float h = affine_carry_warp(
         a.nchunks, h0, W, valid,
         [&](int64_t c, float& p, float& q) {
-            p = ex2(A2 * a.ws_dsum[(b * a.nchunks + c) * a.D + d]);
-            q = a.ws_state[((b * a.nchunks + c) * a.D + d) * a.N + n];
+            const int64_t id = (b * a.nchunks + c) * a.D + d;
+            p = in_range(id, a.batch * a.nchunks * a.D) ? ex2(A2 * a.ws_dsum[id]) : 0.f;
+            q = in_range(id * a.N + n, a.batch * a.nchunks * a.D * a.N) ? a.ws_state[id * a.N + n] : 0.f;
         },
-        [&](int64_t c, float v) { a.ws_state[((b * a.nchunks + c) * a.D + d) * a.N + n] = v; });
+        [&](int64_t c, float v) {
+            const int64_t is = ((b * a.nchunks + c) * a.D + d) * a.N + n;
+            if (in_range(is, a.batch * a.nchunks * a.D * a.N)) a.ws_state[is] = v;
+        });
     if (valid && a.h_last && (threadIdx.x & (W - 1)) == 0) a.h_last[w] = h;
 }
 

@@ -12,6 +12,7 @@
 // with psi(q) = (q e^q - expm1(q)) / q^2; dy = dout SiLU(z), dz = dout y SiLU'(z).
 #pragma once
 
+#include "sscan_check.cuh"
 #include "sscan_generic.cuh"
 #include "sscan_plan.h"
 
@@ -71,11 +72,11 @@ __global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
     float Al[NMAX], A2[NMAX], invA[NMAX], h[NMAX];
 #pragma unroll
     for (int n = 0; n < NMAX; ++n) {
-        const float An = n < N ? __ldg(a.A + d * N + n) : 0.f;
+        const float An = n < N && in_range(d * N + n, a.D * N) ? __ldg(a.A + d * N + n) : 0.f;
         Al[n] = An;
         A2[n] = An * kLog2e;
         invA[n] = An != 0.f ? 1.f / An : 0.f;
-        h[n] = (a.h0 && n < N) ? __ldg(a.h0 + row * N + n) : 0.f;
+        h[n] = (a.h0 && n < N && in_range(row * N + n, a.batch * a.D * N)) ? __ldg(a.h0 + row * N + n) : 0.f;
     }
     const float bias = a.bias ? __ldg(a.bias + d) : 0.f;
     const float dsk = a.Dskip ? __ldg(a.Dskip + d) : 0.f;
@@ -86,7 +87,8 @@ __global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
         if (t % kSeg == 0) {
 #pragma unroll
             for (int n = 0; n < NMAX; ++n)
-                if (n < N) ck[(t / kSeg) * N + n] = h[n];
+                if (n < N && in_range(row * g.nseg * N + (t / kSeg) * N + n, a.batch * a.D * g.nseg * N))
+                    ck[(t / kSeg) * N + n] = h[n];
         }
         const int64_t e = (b * a.L + t) * a.D + d, s = (b * a.L + t) * N;
         const float uv = IO<T>::load(u, e);
@@ -113,7 +115,9 @@ __global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
         const int64_t t0 = sg * kSeg;
         const int len = (int)(a.L - t0 < kSeg ? a.L - t0 : kSeg);
 #pragma unroll
-        for (int n = 0; n < NMAX; ++n) hs[0][n] = n < N ? ck[sg * N + n] : 0.f;
+        for (int n = 0; n < NMAX; ++n)
+            hs[0][n] = n < N && in_range(row * g.nseg * N + sg * N + n, a.batch * a.D * g.nseg * N) ? ck[sg * N + n]
+                                                                                                 : 0.f;
         for (int k = 0; k < len; ++k) {
             const int64_t t = t0 + k;
             const int64_t e = (b * a.L + t) * a.D + d, s = (b * a.L + t) * N;
@@ -163,8 +167,10 @@ __global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
                     const float l = fmaf(Cn, dy, lam[n]);
                     const float dab = l * hs[k][n];
                     const float dbeta = l * Bn * x;
-                    atomicAdd(g.dC32 + s + n, dy * hs[k + 1][n]);
-                    atomicAdd(g.dB32 + s + n, l * beta * x);
+                    if (in_range(s + n, a.batch * a.L * N)) {
+                        atomicAdd(g.dC32 + s + n, dy * hs[k + 1][n]);
+                        atomicAdd(g.dB32 + s + n, l * beta * x);
+                    }
                     dx = fmaf(l * beta, Bn, dx);
                     ddelta = fmaf(dab * Al[n] + dbeta, abar, ddelta);
                     dAacc[n] += dab * delta * abar + dbeta * delta * delta * psi(q, abar);
@@ -180,8 +186,8 @@ __global__ void __launch_bounds__(128) bwd_rows_kernel(BwdArgs g) {
 #pragma unroll
     for (int n = 0; n < NMAX; ++n) {
         if (n < N) {
-            if (g.dh0) g.dh0[row * N + n] = lam[n];
-            atomicAdd(g.dA + d * N + n, dAacc[n]);
+            if (g.dh0 && in_range(row * N + n, a.batch * a.D * N)) g.dh0[row * N + n] = lam[n];
+            if (in_range(d * N + n, a.D * N)) atomicAdd(g.dA + d * N + n, dAacc[n]);
         }
     }
     if (g.dD) atomicAdd(g.dD + d, dDacc);

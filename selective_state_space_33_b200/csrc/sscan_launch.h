@@ -95,6 +95,9 @@ struct ComplexArgs {
 // state before every 8th step (the backward's checkpoint pass, a.out unused).  Kept
 // out of ComplexArgs: the kernel's parameter block stays as small as the forward needs.
 cudaError_t launch_fwd_complex(const ComplexArgs& a, float* ckpt, int64_t nck, int io_bf16, cudaStream_t st);
+// Read (and optionally clear) the complex forward kernel's error word (bit 0: a bounded
+// wait for a TMA tile copy gave up).  Synchronous.
+cudaError_t read_device_error_cx(unsigned int* value, int clear);
 
 // Backward of the complex-A scan (sscan_complex_bwd.cu).
 struct ComplexBwdArgs {

@@ -30,6 +30,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "sscan_check.cuh"
 #include "sscan_launch.h"
 #include "sscan_math.cuh"
 #include "sscan_tma.cuh"
@@ -168,7 +169,8 @@ __device__ __forceinline__ float transpose_reduce(float (&p)[NG], int g) {
 // the last, partial tile of a chunk takes the predicated form.
 template <typename T, int NG, int G, int MODE, bool ACC, bool FULL>
 __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
-                                          float& dsum, float* ck, int64_t ck_stride, int nvalid) {
+                                          float& dsum, float* ck, int64_t ck_stride, int nvalid,
+                                          const float* ck_base, int64_t ck_extent) {
     using C = Cfg<T, NG, G, MODE>;
     constexpr bool WANT_Y = MODE == kOut;
     const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
@@ -182,7 +184,7 @@ __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int 
             float* dst = ck + (tb / kCkStep) * ck_stride;
 #pragma unroll
             for (int j = 0; j < G; ++j)
-                if (j < nvalid) dst[j] = (j & 1) ? s.h[j / 2].y : s.h[j / 2].x;
+                if (j < nvalid && in_range(dst + j - ck_base, ck_extent)) dst[j] = (j & 1) ? s.h[j / 2].y : s.h[j / 2].x;
         }
         float p[NG];
 #pragma unroll
@@ -264,7 +266,8 @@ __device__ __forceinline__ void scan_tile_pipe(LaneG<G>& s, unsigned char* smem,
 }
 template <typename T, int NG, int G, int MODE, bool ACC>
 __device__ __forceinline__ void scan_tile_any(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
-                                              float& dsum, float* ck, int64_t ck_stride, int nvalid) {
+                                              float& dsum, float* ck, int64_t ck_stride, int nvalid,
+                                              const float* ck_base, int64_t ck_extent) {
     if constexpr (MODE == kOut && !ACC) {
         if (tile_len == kTT) {
             scan_tile_pipe<T, NG, G>(s, smem, g, cw, sout);
@@ -272,9 +275,11 @@ __device__ __forceinline__ void scan_tile_any(LaneG<G>& s, unsigned char* smem, 
         }
     }
     if (tile_len == kTT)
-        scan_tile<T, NG, G, MODE, ACC, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid);
+        scan_tile<T, NG, G, MODE, ACC, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid, ck_base,
+                                             ck_extent);
     else
-        scan_tile<T, NG, G, MODE, ACC, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid);
+        scan_tile<T, NG, G, MODE, ACC, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid, ck_base,
+                                              ck_extent);
 }
 
 // softplus and SiLU of two values at once: the exponentials, logarithm and
@@ -325,6 +330,9 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
     const int N = a.N;
     const int d0 = cb * C::DC;
     constexpr bool want_out = MODE == kOut;
+    // extents of the arrays indexed below (checked in the debug build only)
+    const int64_t ext_state = a.batch * a.D * N, ext_chunks = a.batch * a.nchunks * a.D * N;
+    const int64_t ext_ckpt = a.batch * a.nck * a.D * N;
     const bool has_z = want_out && a.has_z;
     const bool bc_tma = a.bc_tma != 0;
     const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
@@ -365,12 +373,14 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
     for (int j = 0; j < G; ++j) {
         const int n = g * G + j;
         const bool ok = cvalid && n < N;
-        const float An = ok ? __ldg(a.A + d * N + n) : -1.f;
+        const float An = ok && in_range(d * N + n, a.D * N) ? __ldg(a.A + d * N + n) : -1.f;
         small_a |= ok && fabsf(An) < kSmallA;
         float h = 0.f;
         if (ok && MODE != kAgg) {
-            if (a.nchunks > 1) h = a.ws_state[(((int64_t)b * a.nchunks + chunk) * a.D + d) * N + n];
-            else if (a.h0) h = __ldg(a.h0 + ((int64_t)b * a.D + d) * N + n);
+            const int64_t ic = (((int64_t)b * a.nchunks + chunk) * a.D + d) * N + n;
+            const int64_t is = ((int64_t)b * a.D + d) * N + n;
+            if (a.nchunks > 1) h = in_range(ic, ext_chunks) ? a.ws_state[ic] : 0.f;
+            else if (a.h0) h = in_range(is, ext_state) ? __ldg(a.h0 + is) : 0.f;
         }
         const float A2 = ok ? An * kLog2e : 0.f;
         const float niA = ok && An != 0.f ? -1.f / An : 0.f;
@@ -464,8 +474,10 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
                             if (want_out) cv = to_f32<T>(rC[t * N + n]);
                         } else if (tt + t < t_end) {
                             const int64_t gi = ((int64_t)b * a.L + tt + t) * N + n;
-                            bv = to_f32<T>(Bg[gi]);
-                            if (want_out) cv = to_f32<T>(Cg[gi]);
+                            if (in_range(gi, a.batch * a.L * N)) {
+                                bv = to_f32<T>(Bg[gi]);
+                                if (want_out) cv = to_f32<T>(Cg[gi]);
+                            }
                         }
                     }
                     sBf[e] = bv;
@@ -486,9 +498,11 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
         const int64_t ck_stride = (int64_t)a.D * N;
         const int nvalid = cvalid ? min(G, N - g * G) : 0;
         if (acc)
-            scan_tile_any<T, NG, G, MODE, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid);
+            scan_tile_any<T, NG, G, MODE, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid,
+                                                a.ws_ckpt, ext_ckpt);
         else
-            scan_tile_any<T, NG, G, MODE, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid);
+            scan_tile_any<T, NG, G, MODE, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid,
+                                                 a.ws_ckpt, ext_ckpt);
         if (want_out) fence_proxy_async();
         // the next tile's data, then one barrier for: outputs complete, tile buffers free,
         // next raw tile landed (or a wait that gave up)
@@ -512,12 +526,16 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
         const int n = g * G + j;
         if (!cvalid || n >= N) continue;
         const float hf = (j & 1) ? s.h[j / 2].y : s.h[j / 2].x;
-        if (MODE == kAgg)
-            a.ws_state[(((int64_t)b * a.nchunks + chunk) * a.D + d) * N + n] = hf;
-        else if (a.h_last && chunk == a.nchunks - 1)
-            a.h_last[((int64_t)b * a.D + d) * N + n] = hf;
+        const int64_t ic = (((int64_t)b * a.nchunks + chunk) * a.D + d) * N + n;
+        const int64_t is = ((int64_t)b * a.D + d) * N + n;
+        if (MODE == kAgg) {
+            if (in_range(ic, ext_chunks)) a.ws_state[ic] = hf;
+        } else if (a.h_last && chunk == a.nchunks - 1) {
+            if (in_range(is, ext_state)) a.h_last[is] = hf;
+        }
     }
-    if (MODE == kAgg && g == 0 && cvalid) a.ws_dsum[((int64_t)b * a.nchunks + chunk) * a.D + d] = dsum;
+    const int64_t idsum = ((int64_t)b * a.nchunks + chunk) * a.D + d;
+    if (MODE == kAgg && g == 0 && cvalid && in_range(idsum, a.batch * a.nchunks * a.D)) a.ws_dsum[idsum] = dsum;
 }
 
 // --------------------------------------------------------------------------- host side

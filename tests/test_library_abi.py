@@ -143,3 +143,17 @@ def test_step_requires_single_token(lib):
     args = [fake] * 10
     args[8] = None  # state
     assert lib.sscan_step(ctypes.byref(p), *args, None) == 1
+
+
+def test_debug_build_exports_the_same_interface(lib):
+    """The debug build (index checks compiled in, reported through the device status
+    word) exports the same symbols and says which build it is; the release build
+    compiles the checks out."""
+    path = lib_build.build(debug=True)
+    dbg = sb.load_library(path)
+    for n in _declared_symbols():
+        assert hasattr(dbg, n), n
+    dbg.sscan_debug_bounds.restype = ctypes.c_int
+    lib.sscan_debug_bounds.restype = ctypes.c_int
+    assert dbg.sscan_debug_bounds() == 1
+    assert lib.sscan_debug_bounds() == 0
