@@ -125,22 +125,21 @@ def roofline_units(w: W.Workload) -> dict:
 # keyed by the SHA-256 of those source files (with comments and blank lines removed,
 # so that only code counts) and reported as null once the code changes.
 NCU_TRAFFIC = {
-    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 505266688 + 151573248,
-                  "sources": ("sscan_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "d602134642251f4d",
-                  "profile": "profiles/fwd_tiled_kernel_mamba2.8b_bf16.md"},
-    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410298368 + 133372928,
-                "sources": ("sscan_bwd_tiled.cu", "sscan_tma.cuh", "sscan_math.cuh"), "sha256": "430945355610e83f",
-                "profile": "profiles/bwd_tiled_kernel_bwd130m_bf16.md"},
-    "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317504 + 0,
-                   "sources": ("sscan_step.cu", "sscan_math.cuh"), "sha256": "b7c6e53d71a0bd30",
-                   "profile": "profiles/step_quad_kernel_decode2.8b_bf16.md"},
-    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152319232 + 31278080,
-                    "sources": ("sscan_complex.cu", "sscan_complex_math.cuh", "sscan_math.cuh"),
-                    "sha256": "2c181ea6f7027cff",
-                    "profile": "profiles/fwd_complex_kernel_complex130m_bf16.md"},
-    "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 612188672 + 138831616,
-                       "sources": ("sscan_complex_bwd.cu", "sscan_complex_math.cuh", "sscan_math.cuh"),
-                       "sha256": "9e107f54b099d7c3", "profile": "profiles/bwd_complex_kernel_complexbwd130m_bf16.md"},
+    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 505390080 + 151158272,
+        "sources": ('sscan_tiled.cu', 'sscan_tma.cuh', 'sscan_math.cuh', 'sscan_check.cuh'), "sha256": "a7dfbf4ffeaeecac",
+        "profile": "profiles/fwd_tiled_kernel_mamba2.8b_bf16.md"},
+    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410679296 + 133782528,
+        "sources": ('sscan_bwd_tiled.cu', 'sscan_tma.cuh', 'sscan_math.cuh', 'sscan_check.cuh'), "sha256": "a8acc2a5f68ebfa5",
+        "profile": "profiles/bwd_tiled_kernel_bwd130m_bf16.md"},
+    "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317504 + 256,
+        "sources": ('sscan_step.cu', 'sscan_math.cuh'), "sha256": "c1a451e4bc5a2b5e",
+        "profile": "profiles/step_quad_kernel_decode2.8b_bf16.md"},
+    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152569856 + 30774528,
+        "sources": ('sscan_complex.cu', 'sscan_complex_math.cuh', 'sscan_math.cuh', 'sscan_tma.cuh'), "sha256": "4098bc4b952ac034",
+        "profile": "profiles/fwd_complex_kernel_complex130m_bf16.md"},
+    "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 612771328 + 138951424,
+        "sources": ('sscan_complex_bwd.cu', 'sscan_complex_math.cuh', 'sscan_math.cuh'), "sha256": "b6f7471f16370f79",
+        "profile": "profiles/bwd_complex_kernel_complexbwd130m_bf16.md"},
 }
 
 
