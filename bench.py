@@ -533,13 +533,69 @@ def gpu_arm(args, w: W.Workload):
         e2e_value, h2d, d2h = e2e_leg(args, t, out, ws, st, units, world, dev)
     if rank != 0:
         return
-    secondary = None
+    secondary, others = None, None
     if world == 1 and args.workload == DEFAULT_WORKLOAD and not args.no_secondary:
         del t
         secondary = fp32_record(args, lib, dev)
+        others = [other_record(args, W.WORKLOADS[name]) for name in ("mamba130m", "bwd130m")]
     finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk, e2e_value, h2d, d2h,
            launches_per_step, world, l2_note, out=out if not (w.backward or w.decode or w.complex_a) else None,
-           secondary=secondary)
+           secondary=secondary, others=others)
+
+
+def other_record(args, w: W.Workload) -> dict:
+    """A further workload timed the same way after the headline (K steps after the
+    warm-up, CUDA events per step): its Gelem/s, per-launch time and MUFU roofline
+    fraction; for a forward workload also the output's error against the oracle on a
+    row sample covering every channel block."""
+    import torch
+
+    from selective_state_space_33_b200 import binding as sb
+    x = W.make_inputs(w)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    t = W.to_device(x, dev)
+    st = torch.cuda.current_stream()
+    prob = sb.make_problem(w.batch, w.seqlen, w.dim, w.dstate, sb.SSCAN_BF16 if w.io == "bf16" else sb.SSCAN_F32)
+    op = sb.SSCAN_OP_BWD if w.backward else sb.SSCAN_OP_FWD
+    ws = torch.empty(max(sb.sscan_workspace_size(prob, op), 256), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(t["u"])
+    grads = None
+    if w.backward:
+        grads = sb.sscan_bwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t["delta_bias"],
+                             t["D_skip"], t["z"], workspace=ws)
+
+    def step():
+        if w.backward:
+            sb.sscan_bwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t["delta_bias"], t["D_skip"],
+                         t["z"], grads=grads, workspace=ws, stream=st)
+        else:
+            sb.sscan_fwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["delta_bias"], t["D_skip"], t["z"],
+                         out=out, workspace=ws, stream=st)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        a.record(st)
+        step()
+        b.record(st)
+    torch.cuda.synchronize()
+    per_launch = statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e-3
+    total = ev[0][0].elapsed_time(ev[-1][1]) * 1e-3
+    units = roofline_units(w)
+    mufu = SM_COUNT * MUFU_PER_SM_CLK * float(measured_peaks().get("sm_max_mhz", 1965.0)) * 1e6
+    rec = {"workload": f"{w.name}: {w.description}", "io_dtype": w.io,
+           "metric": METRIC_BWD if w.backward else METRIC,
+           "value": aggregate(units["elements"], args.steps, 1, total), "unit": UNIT,
+           "ms_per_step": total / args.steps * 1e3,
+           "roofline": {"bound": "alu", "pipe": "MUFU ex2", "achieved": units["exps"] / per_launch / 1e9,
+                        "peak": mufu / 1e9, "unit": "Gexp/s", "frac": units["exps"] / per_launch / mufu,
+                        "per_launch_ms": per_launch * 1e3, "alg_exps_per_launch": units["exps"],
+                        "alg_bytes_per_launch": units["bytes"]}}
+    if not w.backward and not args.no_cpu_baseline:
+        rec["parity"] = oracle_parity(x, w, out)
+    return rec
 
 
 def fp32_record(args, lib, dev) -> dict:
@@ -652,7 +708,7 @@ def e2e_leg(args, t, out, ws, st, units, world, dev):
 
 
 def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk, e2e_value, h2d, d2h,
-           launches_per_step, world, l2_note, out=None, secondary=None):
+           launches_per_step, world, l2_note, out=None, secondary=None, others=None):
     peaks = measured_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", HBM_FALLBACK_GBS))
     hbm_src = "measured" if "hbm_gbs" in peaks else "fallback"
@@ -710,6 +766,8 @@ def finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk,
         line["parity"] = cpu["parity"]
     if secondary is not None:
         line["secondary"] = secondary
+    if others:
+        line["others"] = others
     print(json.dumps(line), flush=True)
 
 
@@ -743,7 +801,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-secondary", action="store_true",
-                    help="skip the fp32-I/O record that follows the default (bf16) workload")
+                    help="skip the records that follow the default (bf16) workload: fp32 I/O, the "
+                         "Mamba-130M-shaped forward and backward")
     ap.add_argument("--profile-run", action="store_true",
                     help="timed steps only (no clock tail, end-to-end leg, probe or CPU baseline): "
                          "the command line used under ncu")

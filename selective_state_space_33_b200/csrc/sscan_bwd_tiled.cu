@@ -480,16 +480,35 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         }
         {
             float2 h0 = g2(hk.x, hk.y), h1 = g2(hk.z, hk.w);
-            if (!acc) {
-                // the forward kernel's form: h' = Abar (h - v) + v with v = -B x / A
+            // the forward kernel's form: h' = Abar (h - v) + v with v = -B x / A; the
+            // exponentials and v of step t + 1 are prepared before the update of step t
+            auto prep = [&](int t, float2& a0, float2& a1, float2& v0, float2& v1) {
+                const float4 dx = sdx[t * C::DC];
+                const float4 Bv = sB[t * NG];
+                const float2 dd = g2(dx.x, dx.y), xx = g2(dx.z, dx.w);
+                a0 = ex2p(__fmul2_rn(dd, s.A2[0]));
+                a1 = ex2p(__fmul2_rn(dd, s.A2[1]));
+                v0 = __fmul2_rn(g2(Bv.x, Bv.y), __fmul2_rn(xx, s.niA[0]));
+                v1 = __fmul2_rn(g2(Bv.z, Bv.w), __fmul2_rn(xx, s.niA[1]));
+            };
+            if (!acc && tile_len == kTB) {
+                float2 a0, a1, v0, v1;
+                prep(0, a0, a1, v0, v1);
+#pragma unroll
+                for (int t = 0; t < kTB; ++t) {
+                    float2 b0 = a0, b1 = a1, w0 = v0, w1 = v1;
+                    if (t + 1 < kTB) prep(t + 1, b0, b1, w0, w1);
+                    h0 = __ffma2_rn(a0, __ffma2_rn(v0, g2(-1.f, -1.f), h0), v0);
+                    h1 = __ffma2_rn(a1, __ffma2_rn(v1, g2(-1.f, -1.f), h1), v1);
+                    shs[t * kThreadsB] = make_float4(h0.x, h0.y, h1.x, h1.y);
+                    a0 = b0, a1 = b1, v0 = w0, v1 = w1;
+                }
+            } else if (!acc) {
                 for (int t = 0; t < tile_len; ++t) {
-                    const float4 dx = sdx[t * C::DC];
-                    const float4 Bv = sB[t * NG];
-                    const float2 dd = g2(dx.x, dx.y), xx = g2(dx.z, dx.w);
-                    const float2 v0 = __fmul2_rn(g2(Bv.x, Bv.y), __fmul2_rn(xx, s.niA[0]));
-                    const float2 v1 = __fmul2_rn(g2(Bv.z, Bv.w), __fmul2_rn(xx, s.niA[1]));
-                    h0 = __ffma2_rn(ex2p(__fmul2_rn(dd, s.A2[0])), __ffma2_rn(v0, g2(-1.f, -1.f), h0), v0);
-                    h1 = __ffma2_rn(ex2p(__fmul2_rn(dd, s.A2[1])), __ffma2_rn(v1, g2(-1.f, -1.f), h1), v1);
+                    float2 a0, a1, v0, v1;
+                    prep(t, a0, a1, v0, v1);
+                    h0 = __ffma2_rn(a0, __ffma2_rn(v0, g2(-1.f, -1.f), h0), v0);
+                    h1 = __ffma2_rn(a1, __ffma2_rn(v1, g2(-1.f, -1.f), h1), v1);
                     shs[t * kThreadsB] = make_float4(h0.x, h0.y, h1.x, h1.y);
                 }
             } else {
