@@ -29,6 +29,7 @@ sys.path.insert(0, ROOT)
 from selective_state_space_33_b200 import workloads as W  # noqa: E402
 
 METRIC = "selective-scan fwd Gelem/s (B·L·D) & % of HBM/MUFU roofline at 2.8B-layer shape"
+METRIC_FWD = "selective-scan fwd Gelem/s (B·L·D)"
 METRIC_BWD = "selective-scan bwd Gelem/s (B·L·D), states recomputed on chip"
 METRIC_STEP = "selective-scan generation step Gelem/s (batch·D per token), state read and written in HBM"
 METRIC_COMPLEX = "selective-scan fwd with complex diagonal A, Gelem/s (B·L·D)"
@@ -586,7 +587,7 @@ def other_record(args, w: W.Workload) -> dict:
     units = roofline_units(w)
     mufu = SM_COUNT * MUFU_PER_SM_CLK * float(measured_peaks().get("sm_max_mhz", 1965.0)) * 1e6
     rec = {"workload": f"{w.name}: {w.description}", "io_dtype": w.io,
-           "metric": METRIC_BWD if w.backward else METRIC,
+           "metric": METRIC_BWD if w.backward else METRIC_FWD,
            "value": aggregate(units["elements"], args.steps, 1, total), "unit": UNIT,
            "ms_per_step": total / args.steps * 1e3,
            "roofline": {"bound": "alu", "pipe": "MUFU ex2", "achieved": units["exps"] / per_launch / 1e9,
