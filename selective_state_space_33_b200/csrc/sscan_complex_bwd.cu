@@ -48,6 +48,100 @@ __device__ __forceinline__ float2 cmul(float2 p, float2 q) {
     return make_float2(fmaf(p.x, q.x, -p.y * q.y), fmaf(p.x, q.y, p.y * q.x));
 }
 
+__device__ __forceinline__ float2 x2(float a, float b) { return make_float2(a, b); }
+
+// The lane's two complex states side by side: re = (Re z_0, Re z_1), im = (Im z_0, Im z_1),
+// so that complex arithmetic on both states runs on f32x2 operations.
+struct XP {
+    float2 re, im;
+};
+
+// p q for both states; nqi = -Im q (passed in so that no packed operand is negated).
+__device__ __forceinline__ XP xmul(XP p, XP q, float2 nqi) {
+    return {__ffma2_rn(p.im, nqi, __fmul2_rn(p.re, q.re)), __ffma2_rn(p.re, q.im, __fmul2_rn(p.im, q.re))};
+}
+
+// cos and sin of a pair of angles (reduction to [-pi, pi] by a two-part 2 pi, packed).
+__device__ __forceinline__ void xcis(float2 th, float2& cs, float2& sn) {
+    const float2 m = __fmul2_rn(th, x2(-cplx::kInvTwoPi, -cplx::kInvTwoPi));
+    const float2 nk = x2(rintf(m.x), rintf(m.y));
+    float2 r = __ffma2_rn(nk, x2(cplx::kTwoPiHi, cplx::kTwoPiHi), th);
+    r = __ffma2_rn(nk, x2(cplx::kTwoPiLo, cplx::kTwoPiLo), r);
+    cs = x2(cplx::cos_approx(r.x), cplx::cos_approx(r.y));
+    sn = x2(cplx::sin_approx(r.x), cplx::sin_approx(r.y));
+}
+
+// Per-lane constants and accumulators of the two complex states, packed.
+struct XLane {
+    float2 aq, ai;      // Re a log2(e), Im a
+    float2 ar, nai;     // Re a, -Im a
+    float2 nar;         // -Re a
+    float2 nr, ni;      // Re(-1/a), Im(-1/a)
+    float2 i2r, i2i, ni2i;  // Re(1/a^2), Im(1/a^2), -Im(1/a^2)
+    XP lam, gA;         // adjoint state, A-gradient accumulator (dL/dRe a, dL/dIm a)
+};
+
+// One reverse step of the lane's two complex states (eq. (2), (3) in complex arithmetic,
+// adjoint lam_t = C_t dy_t + conj(Abar_{t+1}) lam_{t+1}).  w = delta^2 psi(delta a) is
+// evaluated once per state -- psi's series for |delta a| < 1/2, else
+// (1 + Abar (q - 1)) / a^2 -- and gives beta = delta Abar - a w as well as the A-gradient
+// term.  Returns the lane's partial sums for du, d delta and the readout; dB and dC values
+// of the two states in dbv / dcv.
+__device__ __forceinline__ void xrev_step(XLane& s, float delta, float x, float dy, float2 Bp, float2 Cp, XP hc,
+                                          XP hp, float& pdu, float& pdd, float& py, float2& dbv, float2& dcv) {
+    const float2 dd = x2(delta, delta), xx = x2(x, x), dyy = x2(dy, dy);
+    const float2 e = x2(ex2(delta * s.aq.x), ex2(delta * s.aq.y));
+    float2 cs, sn;
+    xcis(__fmul2_rn(dd, s.ai), cs, sn);
+    const XP ab = {__fmul2_rn(e, cs), __fmul2_rn(e, sn)};
+    const float2 nabi = __fmul2_rn(e, __fmul2_rn(sn, x2(-1.f, -1.f)));
+    const XP l = {__ffma2_rn(Cp, dyy, s.lam.re), s.lam.im};
+    const XP q = {__fmul2_rn(dd, s.ar), __fmul2_rn(dd, s.ai)};
+    const float2 nqi = __fmul2_rn(dd, s.nai);
+    const float2 qq = __ffma2_rn(q.re, q.re, __fmul2_rn(q.im, q.im));
+    // series: psi(q) = 1/2 + q/3 + q^2/8 + q^3/30 + q^4/144 + q^5/840 (dropped tail < 2.7e-6 at |q| = 1/2)
+    XP p = {__ffma2_rn(q.re, x2(1.f / 840.f, 1.f / 840.f), x2(1.f / 144.f, 1.f / 144.f)),
+            __fmul2_rn(q.im, x2(1.f / 840.f, 1.f / 840.f))};
+    const float cf[4] = {1.f / 30.f, 0.125f, 1.f / 3.f, 0.5f};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const XP pq = xmul(p, q, nqi);
+        p = {__fadd2_rn(pq.re, x2(cf[k], cf[k])), pq.im};
+    }
+    const float2 d2 = __fmul2_rn(dd, dd);
+    const XP ws = {__fmul2_rn(d2, p.re), __fmul2_rn(d2, p.im)};
+    // closed form: w = (1 + Abar (q - 1)) / a^2
+    const float2 qm1 = __fadd2_rn(q.re, x2(-1.f, -1.f));
+    const XP t = {__ffma2_rn(ab.re, qm1, __ffma2_rn(nabi, q.im, x2(1.f, 1.f))),
+                  __ffma2_rn(ab.re, q.im, __fmul2_rn(ab.im, qm1))};
+    const XP wc = {__ffma2_rn(t.im, s.ni2i, __fmul2_rn(t.re, s.i2r)), __ffma2_rn(t.re, s.i2i, __fmul2_rn(t.im, s.i2r))};
+    const bool s0 = qq.x < 0.25f, s1 = qq.y < 0.25f;
+    const XP w = {x2(s0 ? ws.re.x : wc.re.x, s1 ? ws.re.y : wc.re.y), x2(s0 ? ws.im.x : wc.im.x, s1 ? ws.im.y : wc.im.y)};
+    // beta = delta Abar - a w (= Bbar / B)
+    const XP naw = {__ffma2_rn(s.nar, w.re, __fmul2_rn(s.ai, w.im)), __ffma2_rn(s.nar, w.im, __fmul2_rn(s.nai, w.re))};
+    const XP beta = {__ffma2_rn(dd, ab.re, naw.re), __ffma2_rn(dd, ab.im, naw.im)};
+    const float2 lb = __ffma2_rn(l.re, beta.re, __fmul2_rn(l.im, beta.im));  // Re(conj(l) beta)
+    const float2 du2 = __fmul2_rn(lb, Bp);
+    dbv = __fmul2_rn(lb, xx);
+    const float2 bx = __fmul2_rn(Bp, xx);
+    // dh/d delta = Abar (a h_{t-1} + B x)
+    const XP ah = {__ffma2_rn(s.ar, hp.re, __ffma2_rn(s.nai, hp.im, bx)), __ffma2_rn(s.ar, hp.im, __fmul2_rn(s.ai, hp.re))};
+    const XP dhd = xmul(ah, ab, nabi);
+    const float2 dd2 = __ffma2_rn(l.re, dhd.re, __fmul2_rn(l.im, dhd.im));
+    // dh/da = delta Abar h_{t-1} + w B x;  dA += conj(conj(l) dh/da)
+    const XP abh = xmul(hp, ab, nabi);
+    const XP dha = {__ffma2_rn(dd, abh.re, __fmul2_rn(w.re, bx)), __ffma2_rn(dd, abh.im, __fmul2_rn(w.im, bx))};
+    s.gA.re = __ffma2_rn(l.re, dha.re, __ffma2_rn(l.im, dha.im, s.gA.re));
+    s.gA.im = __ffma2_rn(l.im, dha.re, __ffma2_rn(__fmul2_rn(l.re, x2(-1.f, -1.f)), dha.im, s.gA.im));
+    dcv = __fmul2_rn(dyy, hc.re);
+    const float2 y2 = __fmul2_rn(Cp, hc.re);
+    // lam_{t-1} side: conj(Abar) l
+    s.lam = {__ffma2_rn(ab.re, l.re, __fmul2_rn(ab.im, l.im)), __ffma2_rn(ab.re, l.im, __fmul2_rn(nabi, l.re))};
+    pdu = du2.x + du2.y;
+    pdd = dd2.x + dd2.y;
+    py = y2.x + y2.y;
+}
+
 // Sum per-element values over a channel's NG lanes (lane bits at multiples of CW)
 // for BLK consecutive steps: a transposed butterfly over the high BLK state-group
 // bits (lane group ghi ends with step ghi of the block), then plain rounds over the
@@ -76,7 +170,8 @@ __global__ void __launch_bounds__(kXThreads, 6) bwd_complex_kernel(ComplexBwdArg
     using C = XCfg<NG>;
     __shared__ float2 sdx[kXTB * C::DC];   // (delta, x)
     __shared__ float4 sq[kXTB * C::DC];    // (dy, dz factor, softplus', -)
-    __shared__ float sB[kXTB * C::NS], sC[kXTB * C::NS];
+    __shared__ __align__(16) float sB[kXTB * C::NS];
+    __shared__ __align__(16) float sC[kXTB * C::NS];
     __shared__ float4 shs[kXTB * kXThreads];                 // recomputed h_t of each lane
     __shared__ float sacc[kXWarps][kXTB * C::NS][2];         // per-warp dB, dC of the tile
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -95,21 +190,41 @@ __global__ void __launch_bounds__(kXThreads, 6) bwd_complex_kernel(ComplexBwdArg
     const int64_t d = d0 + cw;
     const bool cvalid = d < a.D;
     const int nvalid = cvalid ? (N - gq * kXCG < kXCG ? N - gq * kXCG : kXCG) : 0;
-    float2 av[kXCG], aq[kXCG], ia[kXCG], lam[kXCG], gA[kXCG];
+    static_assert(kXCG == 2, "the packed step covers two complex states per lane");
+    XLane s;
     bool small_a = false;
+    float arv[kXCG], aiv[kXCG];
 #pragma unroll
     for (int j = 0; j < kXCG; ++j) {
         const int n = gq * kXCG + j;
         const bool ok = j < nvalid;
-        const float ar = ok ? __ldg(a.A + (d * N + n) * 2) : -1.f;
-        const float ai = ok ? __ldg(a.A + (d * N + n) * 2 + 1) : 0.f;
-        const float m2 = ar * ar + ai * ai;
-        small_a |= ok && m2 < kXSmallA * kXSmallA;
-        av[j] = make_float2(ar, ai);
-        aq[j] = make_float2(ar * kLog2e, ai);
-        const float inv = m2 > 0.f ? 1.f / m2 : 0.f;
-        ia[j] = make_float2(ar * inv, -ai * inv);
-        lam[j] = gA[j] = make_float2(0.f, 0.f);
+        arv[j] = ok ? __ldg(a.A + (d * N + n) * 2) : -1.f;
+        aiv[j] = ok ? __ldg(a.A + (d * N + n) * 2 + 1) : 0.f;
+        small_a |= ok && arv[j] * arv[j] + aiv[j] * aiv[j] < kXSmallA * kXSmallA;
+    }
+    {
+        float nr[2], ni[2], i2r[2], i2i[2];
+#pragma unroll
+        for (int j = 0; j < kXCG; ++j) {
+            const float m2 = arv[j] * arv[j] + aiv[j] * aiv[j];
+            const float inv = m2 > 0.f ? 1.f / m2 : 0.f;
+            const float iar = arv[j] * inv, iai = -aiv[j] * inv;  // 1 / a
+            nr[j] = -iar;
+            ni[j] = -iai;
+            i2r[j] = iar * iar - iai * iai;  // 1 / a^2
+            i2i[j] = 2.f * iar * iai;
+        }
+        s.aq = x2(arv[0] * kLog2e, arv[1] * kLog2e);
+        s.ai = x2(aiv[0], aiv[1]);
+        s.ar = x2(arv[0], arv[1]);
+        s.nai = x2(-aiv[0], -aiv[1]);
+        s.nar = x2(-arv[0], -arv[1]);
+        s.nr = x2(nr[0], nr[1]);
+        s.ni = x2(ni[0], ni[1]);
+        s.i2r = x2(i2r[0], i2r[1]);
+        s.i2i = x2(i2i[0], i2i[1]);
+        s.ni2i = x2(-i2i[0], -i2i[1]);
+        s.lam = s.gA = XP{x2(0.f, 0.f), x2(0.f, 0.f)};
     }
     // one CTA-wide choice of the recomputation's form (block-uniform branch)
     const bool acc = __syncthreads_or(small_a ? 1 : 0) != 0;
@@ -160,59 +275,69 @@ __global__ void __launch_bounds__(kXThreads, 6) bwd_complex_kernel(ComplexBwdArg
         __syncthreads();
 
         // ---- recompute the tile's states from its checkpoint
-        float2 hk[kXCG];
+        XP hk;
+        {
+            float hv[4];
 #pragma unroll
-        for (int j = 0; j < kXCG; ++j) {
-            const int n = gq * kXCG + j;
-            hk[j] = j < nvalid ? make_float2(g.ckpt[(((b * g.nck + it) * a.D + d) * N + n) * 2],
-                                             g.ckpt[(((b * g.nck + it) * a.D + d) * N + n) * 2 + 1])
-                               : make_float2(0.f, 0.f);
+            for (int j = 0; j < kXCG; ++j) {
+                const int n = gq * kXCG + j;
+                const int64_t ic = (((b * g.nck + it) * a.D + d) * N + n) * 2;
+                hv[2 * j] = j < nvalid ? g.ckpt[ic] : 0.f;
+                hv[2 * j + 1] = j < nvalid ? g.ckpt[ic + 1] : 0.f;
+            }
+            hk = {x2(hv[0], hv[2]), x2(hv[1], hv[3])};
         }
         if (!acc) {
-            // the forward kernel's form: h' = Abar (h - v) + v with v = -B x / a
-            float2 h[kXCG] = {hk[0], hk[1]};
+            // the forward kernel's form: h' = Abar (h - v) + v with v = -B x / a, both states packed
+            XP h = hk;
             for (int t = 0; t < tl; ++t) {
                 const float2 dx = sdx[t * C::DC + cw];
-#pragma unroll
-                for (int j = 0; j < kXCG; ++j) {
-                    const float2 cs = cplx::cis(dx.x * aq[j].y);
-                    const float e = ex2(dx.x * aq[j].x);
-                    const float2 ab = make_float2(e * cs.x, e * cs.y);
-                    const float bx = sB[t * C::NS + gq * kXCG + j] * dx.y;
-                    const float2 nh = cmul(ab, make_float2(fmaf(bx, ia[j].x, h[j].x), fmaf(bx, ia[j].y, h[j].y)));
-                    h[j] = make_float2(fmaf(-bx, ia[j].x, nh.x), fmaf(-bx, ia[j].y, nh.y));
-                }
-                shs[t * kXThreads + tid] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+                const float2 dd = x2(dx.x, dx.x);
+                const float2 e = x2(ex2(dx.x * s.aq.x), ex2(dx.x * s.aq.y));
+                float2 cs, sn;
+                xcis(__fmul2_rn(dd, s.ai), cs, sn);
+                const float2 abr = __fmul2_rn(e, cs), abi = __fmul2_rn(e, sn);
+                const float2 bx = __fmul2_rn(*reinterpret_cast<const float2*>(&sB[t * C::NS + gq * kXCG]), x2(dx.y, dx.y));
+                const float2 vr = __fmul2_rn(bx, s.nr), vi = __fmul2_rn(bx, s.ni);
+                const float2 tr = __ffma2_rn(vr, x2(-1.f, -1.f), h.re);   // Re(h - v)
+                const float2 ti = __ffma2_rn(vi, x2(-1.f, -1.f), h.im);   // Im(h - v)
+                const float2 mti = __ffma2_rn(h.im, x2(-1.f, -1.f), vi);  // -Im(h - v)
+                h.re = __ffma2_rn(abr, tr, __ffma2_rn(abi, mti, vr));
+                h.im = __ffma2_rn(abr, ti, __ffma2_rn(abi, tr, vi));
+                shs[t * kXThreads + tid] = make_float4(h.re.x, h.re.y, h.im.x, h.im.y);
             }
         } else {
             // |a| < 2^-10 somewhere in the block: Bbar from phi1's series where delta a is small
-            float2 h[kXCG] = {hk[0], hk[1]};
+            float2 h[kXCG] = {x2(hk.re.x, hk.im.x), x2(hk.re.y, hk.im.y)};
             for (int t = 0; t < tl; ++t) {
                 const float2 dx = sdx[t * C::DC + cw];
 #pragma unroll
                 for (int j = 0; j < kXCG; ++j) {
-                    const float2 cs = cplx::cis(dx.x * aq[j].y);
-                    const float e = ex2(dx.x * aq[j].x);
+                    const float aqr = j ? s.aq.y : s.aq.x, ai = j ? s.ai.y : s.ai.x, ar = j ? s.ar.y : s.ar.x;
+                    const float2 cs = cplx::cis(dx.x * ai);
+                    const float e = ex2(dx.x * aqr);
                     const float2 ab = make_float2(e * cs.x, e * cs.y);
-                    const float2 q = make_float2(dx.x * av[j].x, dx.x * av[j].y);
+                    const float2 q = make_float2(dx.x * ar, dx.x * ai);
                     float2 beta;
                     if (q.x * q.x + q.y * q.y < 0.00390625f) {
-                        float2 p = make_float2(1.f / 120.f, 0.f);
+                        float2 pc = make_float2(1.f / 120.f, 0.f);
                         const float cf[4] = {1.f / 24.f, 1.f / 6.f, 0.5f, 1.f};
 #pragma unroll
                         for (int m = 0; m < 4; ++m) {
-                            p = cmul(p, q);
-                            p.x += cf[m];
+                            pc = cmul(pc, q);
+                            pc.x += cf[m];
                         }
-                        beta = make_float2(dx.x * p.x, dx.x * p.y);
+                        beta = make_float2(dx.x * pc.x, dx.x * pc.y);
                     } else {
-                        beta = cmul(make_float2(ab.x - 1.f, ab.y), ia[j]);
+                        // (Abar - 1) / a, 1 / a = -(nr + i ni)
+                        const float2 ia = make_float2(-(j ? s.nr.y : s.nr.x), -(j ? s.ni.y : s.ni.x));
+                        beta = cmul(make_float2(ab.x - 1.f, ab.y), ia);
                     }
                     const float bx = sB[t * C::NS + gq * kXCG + j] * dx.y;
                     const float2 nh = cmul(ab, h[j]);
                     h[j] = make_float2(fmaf(beta.x, bx, nh.x), fmaf(beta.y, bx, nh.y));
                 }
-                shs[t * kXThreads + tid] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+                shs[t * kXThreads + tid] = make_float4(h[0].x, h[1].x, h[0].y, h[1].y);
             }
         }
 
@@ -227,61 +352,18 @@ __global__ void __launch_bounds__(kXThreads, 6) bwd_complex_kernel(ComplexBwdArg
             p1[kk] = p2[kk] = p3[kk] = 0.f;
             if (t >= tl) continue;
             const float2 dx = sdx[t * C::DC + cw];
-            const float4 q4 = sq[t * C::DC + cw];
-            const float delta = dx.x, x = dx.y, dy = q4.x;
+            const float dy = sq[t * C::DC + cw].x;
             const float4 hc4 = shs[t * kXThreads + tid];
-            const float4 hp4 = t > 0 ? shs[(t - 1) * kXThreads + tid] : make_float4(hk[0].x, hk[0].y, hk[1].x, hk[1].y);
-            const float2 hc[kXCG] = {make_float2(hc4.x, hc4.y), make_float2(hc4.z, hc4.w)};
-            const float2 hp[kXCG] = {make_float2(hp4.x, hp4.y), make_float2(hp4.z, hp4.w)};
-            float dxp = 0.f, ddp = 0.f, yp = 0.f, dbv[kXCG], dcv[kXCG];
-#pragma unroll
-            for (int j = 0; j < kXCG; ++j) {
-                const float Bn = sB[t * C::NS + gq * kXCG + j], Cn = sC[t * C::NS + gq * kXCG + j];
-                const float2 cs = cplx::cis(delta * aq[j].y);
-                const float e = ex2(delta * aq[j].x);
-                const float2 ab = make_float2(e * cs.x, e * cs.y);
-                const float2 q = make_float2(delta * av[j].x, delta * av[j].y);
-                const float qq = q.x * q.x + q.y * q.y;
-                // beta = Bbar / B and the dA term delta^2 psi(q), psi(q) = (q e^q - (e^q - 1)) / q^2.
-                // |q| < 1/2: psi by its series, beta = delta phi1(q) = delta (Abar - q psi) (no
-                // cancellation); else beta = (Abar - 1) / a and delta^2 psi = (delta Abar - beta) / a,
-                // whose cancellation costs at most a few 1e-6 relative there.  One branch per state.
-                float2 beta, d2psi;
-                if (qq < 0.25f) {
-                    float2 p = make_float2(1.f / 840.f, 0.f);
-                    const float cf[5] = {1.f / 144.f, 1.f / 30.f, 0.125f, 1.f / 3.f, 0.5f};
-#pragma unroll
-                    for (int m = 0; m < 5; ++m) {
-                        p = cmul(p, q);
-                        p.x += cf[m];
-                    }
-                    const float2 qp = cmul(q, p);
-                    beta = make_float2(delta * (ab.x - qp.x), delta * (ab.y - qp.y));
-                    const float dd2 = delta * delta;
-                    d2psi = make_float2(dd2 * p.x, dd2 * p.y);
-                } else {
-                    beta = cmul(make_float2(ab.x - 1.f, ab.y), ia[j]);
-                    d2psi = cmul(make_float2(fmaf(delta, ab.x, -beta.x), fmaf(delta, ab.y, -beta.y)), ia[j]);
-                }
-                const float2 l = make_float2(fmaf(Cn, dy, lam[j].x), lam[j].y);
-                const float lb = fmaf(l.x, beta.x, l.y * beta.y);  // Re(conj(l) beta)
-                const float bx = Bn * x;
-                dxp = fmaf(lb, Bn, dxp);
-                dbv[j] = lb * x;
-                // dh/d delta = Abar (a h_{t-1} + B x)
-                const float2 ah = cmul(av[j], hp[j]);
-                const float2 dhd = cmul(ab, make_float2(ah.x + bx, ah.y));
-                ddp = fmaf(l.x, dhd.x, fmaf(l.y, dhd.y, ddp));
-                // dh/da = delta Abar h_{t-1} + delta^2 psi B x
-                const float2 abh = cmul(ab, hp[j]);
-                const float2 dha = make_float2(fmaf(delta, abh.x, bx * d2psi.x), fmaf(delta, abh.y, bx * d2psi.y));
-                // conj(conj(l) dha): (Re, -Im) of conj(l) dha
-                gA[j].x = fmaf(l.x, dha.x, fmaf(l.y, dha.y, gA[j].x));
-                gA[j].y = fmaf(-l.x, dha.y, fmaf(l.y, dha.x, gA[j].y));
-                dcv[j] = dy * hc[j].x;
-                yp = fmaf(Cn, hc[j].x, yp);
-                lam[j] = make_float2(fmaf(ab.x, l.x, ab.y * l.y), fmaf(ab.x, l.y, -ab.y * l.x));  // conj(ab) l
-            }
+            const XP hc = {x2(hc4.x, hc4.y), x2(hc4.z, hc4.w)};
+            const XP hp = t > 0 ? XP{x2(shs[(t - 1) * kXThreads + tid].x, shs[(t - 1) * kXThreads + tid].y),
+                                     x2(shs[(t - 1) * kXThreads + tid].z, shs[(t - 1) * kXThreads + tid].w)}
+                                : hk;
+            const float2 Bp = *reinterpret_cast<const float2*>(&sB[t * C::NS + gq * kXCG]);
+            const float2 Cp = *reinterpret_cast<const float2*>(&sC[t * C::NS + gq * kXCG]);
+            float dxp, ddp, yp;
+            float2 dbp, dcp;
+            xrev_step(s, dx.x, dx.y, dy, Bp, Cp, hc, hp, dxp, ddp, yp, dbp, dcp);
+            float dbv[kXCG] = {dbp.x, dbp.y}, dcv[kXCG] = {dcp.x, dcp.y};
             p1[kk] = dxp;
             p2[kk] = ddp;
             p3[kk] = yp;
@@ -338,11 +420,11 @@ __global__ void __launch_bounds__(kXThreads, 6) bwd_complex_kernel(ComplexBwdArg
         if (j >= nvalid) continue;
         const int n = gq * kXCG + j;
         if (g.dh0) {
-            g.dh0[((b * a.D + d) * N + n) * 2] = lam[j].x;
-            g.dh0[((b * a.D + d) * N + n) * 2 + 1] = lam[j].y;
+            g.dh0[((b * a.D + d) * N + n) * 2] = j ? s.lam.re.y : s.lam.re.x;
+            g.dh0[((b * a.D + d) * N + n) * 2 + 1] = j ? s.lam.im.y : s.lam.im.x;
         }
-        atomicAdd(g.dA + (d * N + n) * 2, gA[j].x);
-        atomicAdd(g.dA + (d * N + n) * 2 + 1, gA[j].y);
+        atomicAdd(g.dA + (d * N + n) * 2, j ? s.gA.re.y : s.gA.re.x);
+        atomicAdd(g.dA + (d * N + n) * 2 + 1, j ? s.gA.im.y : s.gA.im.x);
     }
     // dD and the bias gradient: each lane group holds the steps it finished
 #pragma unroll
