@@ -138,8 +138,8 @@ NCU_TRAFFIC = {
     "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152569856 + 30774528,
         "sources": ('sscan_complex.cu', 'sscan_complex_math.cuh', 'sscan_math.cuh', 'sscan_tma.cuh'), "sha256": "4098bc4b952ac034",
         "profile": "profiles/fwd_complex_kernel_complex130m_bf16.md"},
-    "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 612771328 + 138951424,
-        "sources": ('sscan_complex_bwd.cu', 'sscan_complex_math.cuh', 'sscan_math.cuh'), "sha256": "b6f7471f16370f79",
+    "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 613000192 + 139654656,
+        "sources": ('sscan_complex_bwd.cu', 'sscan_complex_math.cuh', 'sscan_math.cuh'), "sha256": "72ceb8f7a14ce8a2",
         "profile": "profiles/bwd_complex_kernel_complexbwd130m_bf16.md"},
 }
 
