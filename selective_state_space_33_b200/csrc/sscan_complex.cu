@@ -91,7 +91,7 @@ __device__ __forceinline__ float& comp(float2 (&v)[P], int j) {
 // cos and sin of a pair of angles (the reduction of cplx::cis, packed).
 __device__ __forceinline__ void cis2(float2 th, float2& cs, float2& sn) {
     const float2 m = __fmul2_rn(th, make_float2(-cplx::kInvTwoPi, -cplx::kInvTwoPi));
-    const float2 nk = make_float2(rintf(m.x), rintf(m.y));
+    const float2 nk = cplx::round2_fma(m);
     float2 r = __ffma2_rn(nk, make_float2(cplx::kTwoPiHi, cplx::kTwoPiHi), th);
     r = __ffma2_rn(nk, make_float2(cplx::kTwoPiLo, cplx::kTwoPiLo), r);
     cs = make_float2(cplx::cos_approx(r.x), cplx::cos_approx(r.y));

@@ -64,7 +64,7 @@ __device__ __forceinline__ XP xmul(XP p, XP q, float2 nqi) {
 // cos and sin of a pair of angles (reduction to [-pi, pi] by a two-part 2 pi, packed).
 __device__ __forceinline__ void xcis(float2 th, float2& cs, float2& sn) {
     const float2 m = __fmul2_rn(th, x2(-cplx::kInvTwoPi, -cplx::kInvTwoPi));
-    const float2 nk = x2(rintf(m.x), rintf(m.y));
+    const float2 nk = cplx::round2_fma(m);
     float2 r = __ffma2_rn(nk, x2(cplx::kTwoPiHi, cplx::kTwoPiHi), th);
     r = __ffma2_rn(nk, x2(cplx::kTwoPiLo, cplx::kTwoPiLo), r);
     cs = x2(cplx::cos_approx(r.x), cplx::cos_approx(r.y));

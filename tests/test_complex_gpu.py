@@ -67,6 +67,33 @@ def test_complex_general_A_values(cuda_device, io):
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_complex_large_angles(cuda_device, io):
+    """Im(a) up to 2000, so delta Im(a) reaches ~200 rad: the angle reduction takes multiples
+    of 2 pi up to ~30 turns before the MUFU sine and cosine (the turn count is rounded on the
+    FMA pipe), forward and backward."""
+    x = W.small_case(2, 70, 32, 16, io=io, seed=77, complex_a=True)
+    rng = np.random.default_rng(77)
+    A = (-np.exp(rng.uniform(-3, 1, size=(32, 16))) + 1j * rng.uniform(-2000, 2000, size=(32, 16)))
+    e_out, e_h = _run(x, io, cuda_device, A=A)
+    assert e_out <= TOL[io], e_out
+    assert e_h <= 1e-4, e_h
+    # The gradients that sum a Abar h over states (d delta, d bias, dh0, dA) are ill-conditioned
+    # at such angles: a relative change of A of 2^-23 (its fp32 rounding) already moves the
+    # oracle's own values by ~1e-3.  Their bound is ten times that measured spread.
+    xb = W.small_case(2, 70, 32, 16, io=io, seed=77, backward=True, complex_a=True)
+    A64 = A.astype(np.complex64).astype(np.complex128)
+
+    def orc(Av):
+        return oracle.bwd_complex(xb["u"], xb["delta_raw"], Av, xb["B"], xb["C"], xb["dout"],
+                                  delta_bias=xb["delta_bias"], D_skip=xb["D_skip"], z=xb.get("z"))
+
+    ref = orc(A64)
+    pert = orc(A64 * (1 + 2.0 ** -23 * np.random.default_rng(78).standard_normal(A64.shape)))
+    spread = {k: float(np.max(np.abs(pert[k] - ref[k])) / max(np.max(np.abs(ref[k])), 1e-300)) for k in ref}
+    _check_complex_bwd(xb, io, cuda_device, A=A, tol={k: 10 * v for k, v in spread.items()})
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_complex_tma_and_plain_load_paths_agree(cuda_device, io):
     """16-byte aligned rows travel through the TMA ring; a copy starting one element
     past the boundary takes the plain-load path.  Both match the oracle and each other,
@@ -166,7 +193,7 @@ def test_complex_rejects_bad_A(cuda_device):
 
 
 # ---------------------------------------------------------------- backward
-def _check_complex_bwd(x, io, dev, A=None, h0=None):
+def _check_complex_bwd(x, io, dev, A=None, h0=None, tol=None):
     t = to_torch(x, dev)
     A_np = (x["A"] if A is None else A).astype(np.complex64)
     A_t = torch.from_numpy(np.ascontiguousarray(A_np)).to(dev)
@@ -182,7 +209,7 @@ def _check_complex_bwd(x, io, dev, A=None, h0=None):
         got = g[k].detach().cpu()
         got = got.numpy().astype(np.complex128) if got.is_complex() else to_f64(g[k])
         errs[k] = float(np.max(np.abs(got - r)) / max(np.max(np.abs(r)), 1e-300))
-    bad = {k: e for k, e in errs.items() if not e <= TOL[io]}
+    bad = {k: e for k, e in errs.items() if not e <= max(TOL[io], (tol or {}).get(k, 0.0))}
     assert not bad, errs
     return errs
 
