@@ -10,6 +10,8 @@ namespace sscan {
 
 constexpr int kMaxState = 16;
 constexpr int kSmCount = 148;               // B200
+constexpr int64_t kSmemPerSm = 228 * 1024;  // shared memory per SM (B200)
+constexpr int64_t kSmemPerCtaReserved = 1024;  // reserved by the system per resident CTA
 constexpr int64_t kRowsFillGpu = 16384;     // rows that keep every sub-partition busy
 constexpr int64_t kTargetThreads = (int64_t)kSmCount * 4 * 32 * 4;  // 4 warps per sub-partition
 constexpr int64_t kMinChunk = 512;          // shortest sequence chunk worth a carry
@@ -49,7 +51,7 @@ inline FwdPlan plan_fwd(int64_t batch, int64_t L, int64_t D, int64_t N) {
 constexpr int64_t kTiledMinCols = 2 * kSmCount;     // below this, split the sequence
 constexpr int64_t kTiledTargetCtas = 8 * kSmCount;  // CTAs resident at once (8 per SM)
 constexpr int64_t kTiledMinChunk = 1024;            // steps
-constexpr int64_t kTiledStep = 16;                  // chunk lengths are whole tiles
+constexpr int64_t kTiledStep = 64;                  // chunk lengths are whole tiles of any length
 
 inline FwdPlan plan_tiled(int64_t batch, int64_t L, int64_t D, int64_t N, int64_t DC) {
     FwdPlan p{1, L, 0, 0};

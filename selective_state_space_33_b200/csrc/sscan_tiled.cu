@@ -1,14 +1,15 @@
 // sscan_tiled.cu -- the fast forward kernel of the selective scan for sm_100a.
 //
 // Work decomposition.  A CTA owns one batch b, a block of DC consecutive channels
-// and one sequence chunk; it walks the chunk in tiles of kTT steps.  Its four
+// and one sequence chunk; it walks the chunk in tiles of TT steps (16, 32 or 64:
+// longer tiles where the grid leaves few CTAs per SM, see launch_geom).  Its four
 // warps each own CW = 32/NG channels; the NG lanes of a channel each hold G = 4
 // of the N <= 4*NG fp32 states in registers for the whole chunk (lane =
 // g*CW + c), so the recurrence h_t = Abar h_{t-1} + Bbar x_t (sec. 2.1, eq. (3a))
 // runs sequentially in t with no state ever leaving the SM (sec. 4.1).
 //
 // Per tile:
-//   TMA 3-D loads bring the u, delta_raw (and z) tiles [kTT x DC] into a 2-stage
+//   TMA 3-D loads bring the u, delta_raw (and z) tiles [TT x DC] into a 2-stage
 //   shared-memory ring (mbarrier completion, one elected thread issues and waits,
 //   every wait bounded);
 //   phase P: all threads turn the raw tile into fp32 (delta, x) pairs and the SiLU
@@ -33,6 +34,7 @@
 #include "sscan_check.cuh"
 #include "sscan_launch.h"
 #include "sscan_math.cuh"
+#include "sscan_plan.h"
 #include "sscan_tma.cuh"
 
 namespace sscan {
@@ -41,7 +43,6 @@ __device__ unsigned int g_device_error = 0;
 
 namespace {
 
-constexpr int kTT = 16;       // steps per tile
 constexpr int kWarps = 4;     // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr float kSmallA = 9.765625e-4f;  // |A| below 2^-10 takes the series form of Bbar
@@ -65,26 +66,26 @@ template <> struct Pair<__nv_bfloat16> {
 // beside other kernels and keeps two.  Measured, bf16: one stage 0.583 against
 // 0.592 ms at the 2.8B-layer shape and 0.254 against 0.259 ms at the 130M shape;
 // two stages for the checkpoint pass 1.374 against 1.386 ms per backward call.
-template <typename T, int NG, int G, int MODE>
+template <typename T, int NG, int G, int MODE, int TT>
 struct Cfg {
     static constexpr int CW = 32 / NG;                     // channels per warp
     static constexpr int DC = CW * kWarps;                 // channels per CTA
     static constexpr int NS = NG * G;                      // states covered (>= N)
     static constexpr int STAGES = (sizeof(T) == 2 && MODE == kCkpt) ? 2 : 1;
-    static constexpr int RAW = kTT * DC * (int)sizeof(T);  // bytes of one raw (batch, L, D) tile
-    static constexpr int RAWBC = kTT * NS * (int)sizeof(T);  // bytes reserved for one raw B or C tile
+    static constexpr int RAW = TT * DC * (int)sizeof(T);  // bytes of one raw (batch, L, D) tile
+    static constexpr int RAWBC = TT * NS * (int)sizeof(T);  // bytes reserved for one raw B or C tile
     static constexpr int STAGE = 3 * RAW + 2 * RAWBC;      // u, delta_raw, z, B, C
     static constexpr int GD_PITCH = DC;                    // float2 row pitch of the epilogue operands
-    static constexpr int BC_ENTRIES = kTT * NS;
-    static constexpr int PAIRS = kTT * DC / 2;             // channel pairs of phase P
+    static constexpr int BC_ENTRIES = TT * NS;
+    static constexpr int PAIRS = TT * DC / 2;             // channel pairs of phase P
     static_assert(PAIRS % kThreads == 0, "phase P runs a fixed number of pairs per thread");
     // shared-memory layout (byte offsets, all 128-aligned)
     static constexpr int OFF_RAW = 0;                                     // [STAGES][STAGE]
-    static constexpr int OFF_DX = OFF_RAW + STAGES * STAGE;               // float2 (delta, x) [kTT][DC]
-    static constexpr int OFF_GD = OFF_DX + kTT * DC * 8;                  // float2 (gate, D x gate) [kTT][GD_PITCH]
-    static constexpr int OFF_B = OFF_GD + kTT * GD_PITCH * 8;             // float  [kTT][NS]
-    static constexpr int OFF_C = OFF_B + kTT * NS * 4;                    // float  [kTT][NS]
-    static constexpr int OFF_OUT = OFF_C + kTT * NS * 4;                  // [RAW] output tile
+    static constexpr int OFF_DX = OFF_RAW + STAGES * STAGE;               // float2 (delta, x) [TT][DC]
+    static constexpr int OFF_GD = OFF_DX + TT * DC * 8;                  // float2 (gate, D x gate) [TT][GD_PITCH]
+    static constexpr int OFF_B = OFF_GD + TT * GD_PITCH * 8;             // float  [TT][NS]
+    static constexpr int OFF_C = OFF_B + TT * NS * 4;                    // float  [TT][NS]
+    static constexpr int OFF_OUT = OFF_C + TT * NS * 4;                  // [RAW] output tile
     static constexpr int OFF_BAR = OFF_OUT + RAW;                         // uint64 [STAGES]
     static constexpr int SMEM = OFF_BAR + STAGES * 8;
 };
@@ -165,20 +166,20 @@ __device__ __forceinline__ float transpose_reduce(float (&p)[NG], int g) {
 
 // Phase S over one tile, NG steps per block (the readouts of a block are reduced
 // together); with outputs, two blocks per loop iteration so that one block's
-// reduction overlaps the next block's steps.  FULL tiles (kTT valid steps) need no per-step predicate;
+// reduction overlaps the next block's steps.  FULL tiles (TT valid steps) need no per-step predicate;
 // the last, partial tile of a chunk takes the predicated form.
-template <typename T, int NG, int G, int MODE, bool ACC, bool FULL>
+template <typename T, int NG, int G, int MODE, int TT, bool ACC, bool FULL>
 __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
                                           float& dsum, float* ck, int64_t ck_stride, int nvalid,
                                           const float* ck_base, int64_t ck_extent) {
-    using C = Cfg<T, NG, G, MODE>;
+    using C = Cfg<T, NG, G, MODE, TT>;
     constexpr bool WANT_Y = MODE == kOut;
     const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
     const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
     const float* sB = reinterpret_cast<const float*>(smem + C::OFF_B) + g * G;
     const float* sC = reinterpret_cast<const float*>(smem + C::OFF_C) + g * G;
 #pragma unroll(MODE == kOut ? 2 : 1)
-    for (int tb = 0; tb < kTT; tb += NG) {
+    for (int tb = 0; tb < TT; tb += NG) {
         if (MODE == kCkpt && tb % kCkStep == 0 && (FULL || tb < tile_len)) {
             // state before step tb, the starting point of one backward recomputation
             float* dst = ck + (tb / kCkStep) * ck_stride;
@@ -239,22 +240,22 @@ __device__ __forceinline__ float upd_step(LaneG<G>& s, const Prep<G>& P, const f
     return y.x + y.y;
 }
 
-template <typename T, int NG, int G>
+template <typename T, int NG, int G, int TT>
 __device__ __forceinline__ void scan_tile_pipe(LaneG<G>& s, unsigned char* smem, int g, int cw, T* sout) {
-    using C = Cfg<T, NG, G, kOut>;
+    using C = Cfg<T, NG, G, kOut, TT>;
     const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
     const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
     const float* sB = reinterpret_cast<const float*>(smem + C::OFF_B) + g * G;
     const float* sC = reinterpret_cast<const float*>(smem + C::OFF_C) + g * G;
     Prep<G> P = prep_step<G>(s, sdx[0], sB);
 #pragma unroll
-    for (int tb = 0; tb < kTT; tb += NG) {
+    for (int tb = 0; tb < TT; tb += NG) {
         float p[NG];
 #pragma unroll
         for (int k = 0; k < NG; ++k) {
             const int t = tb + k;
             Prep<G> Pn = P;
-            if (t + 1 < kTT) Pn = prep_step<G>(s, sdx[(t + 1) * C::DC], sB + (t + 1) * C::NS);
+            if (t + 1 < TT) Pn = prep_step<G>(s, sdx[(t + 1) * C::DC], sB + (t + 1) * C::NS);
             p[k] = upd_step<G>(s, P, sC + t * C::NS);
             P = Pn;
         }
@@ -264,21 +265,21 @@ __device__ __forceinline__ void scan_tile_pipe(LaneG<G>& s, unsigned char* smem,
         sout[t * C::DC + cw] = from_f32<T>(fmaf(y, gd.x, gd.y));
     }
 }
-template <typename T, int NG, int G, int MODE, bool ACC>
+template <typename T, int NG, int G, int MODE, int TT, bool ACC>
 __device__ __forceinline__ void scan_tile_any(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
                                               float& dsum, float* ck, int64_t ck_stride, int nvalid,
                                               const float* ck_base, int64_t ck_extent) {
     if constexpr (MODE == kOut && !ACC) {
-        if (tile_len == kTT) {
-            scan_tile_pipe<T, NG, G>(s, smem, g, cw, sout);
+        if (tile_len == TT) {
+            scan_tile_pipe<T, NG, G, TT>(s, smem, g, cw, sout);
             return;
         }
     }
-    if (tile_len == kTT)
-        scan_tile<T, NG, G, MODE, ACC, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid, ck_base,
+    if (tile_len == TT)
+        scan_tile<T, NG, G, MODE, TT, ACC, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid, ck_base,
                                              ck_extent);
     else
-        scan_tile<T, NG, G, MODE, ACC, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid, ck_base,
+        scan_tile<T, NG, G, MODE, TT, ACC, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid, ck_base,
                                               ck_extent);
 }
 
@@ -308,13 +309,13 @@ __device__ __forceinline__ float2 silu_x2(float2 z) {
 
 template <int G> struct Occupancy { static constexpr int kCtas = G == 4 ? 9 : 5; };
 
-template <typename T, int NG, int G, int MODE>
+template <typename T, int NG, int G, int MODE, int TT>
 __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
     fwd_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dr,
                      const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_out,
                      const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
                      TiledArgs a) {
-    using C = Cfg<T, NG, G, MODE>;
+    using C = Cfg<T, NG, G, MODE, TT>;
     using P2 = typename Pair<T>::type;
     extern __shared__ __align__(128) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
     const int b = (int)(bc / a.nchunks);
     const int64_t t_begin = (int64_t)chunk * a.chunk_len;
     const int64_t t_end = min(a.L, t_begin + a.chunk_len);
-    const int ntile = (int)((t_end - t_begin + kTT - 1) / kTT);
+    const int ntile = (int)((t_end - t_begin + TT - 1) / TT);
     const int N = a.N;
     const int d0 = cb * C::DC;
     constexpr bool want_out = MODE == kOut;
@@ -337,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
     const bool bc_tma = a.bc_tma != 0;
     const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
     const uint32_t raw_bytes = (has_z ? 3u : 2u) * C::RAW;
-    const uint32_t bc_bytes = (uint32_t)(kTT * N * (int)sizeof(T));
+    const uint32_t bc_bytes = (uint32_t)(TT * N * (int)sizeof(T));
     const uint32_t stage_bytes = raw_bytes + (bc_tma ? (want_out ? 2u : 1u) * bc_bytes : 0u);
 
     // issue the TMA copies of tile `it` into its ring stage (elected thread only)
@@ -345,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
         const int st = it % C::STAGES;
         const uint32_t bar = bar0 + 8 * st;
         const uint32_t base = smem_u32(smem + C::OFF_RAW + st * C::STAGE);
-        const int tt = (int)(t_begin + (int64_t)it * kTT);
+        const int tt = (int)(t_begin + (int64_t)it * TT);
         mbar_expect_tx(bar, stage_bytes);
         tma_load_3d(base, &tm_u, d0, tt, b, bar);
         tma_load_3d(base + C::RAW, &tm_dr, d0, tt, b, bar);
@@ -413,8 +414,8 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
 
     for (int it = 0; it < ntile && !failed; ++it) {
         const int st = it % C::STAGES;
-        const int64_t tt = t_begin + (int64_t)it * kTT;
-        const int tile_len = (int)(t_end - tt < kTT ? t_end - tt : kTT);
+        const int64_t tt = t_begin + (int64_t)it * TT;
+        const int tile_len = (int)(t_end - tt < TT ? t_end - tt : TT);
         // phase P: raw tile -> (delta, x) pairs and (gate, D x gate); B and C rows as fp32
         {
             const unsigned char* raw = smem + C::OFF_RAW + st * C::STAGE;
@@ -444,11 +445,13 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
             const T* rB = reinterpret_cast<const T*>(raw + 3 * C::RAW);
             const T* rC = reinterpret_cast<const T*>(raw + 3 * C::RAW + C::RAWBC);
             if (bc_tma && N == C::NS) {
-                // dense [kTT][N] tiles: one thread converts 4 consecutive values of B
-                // (threads 0 .. V-1) or of C (V .. 2V-1)
+                // dense [TT][N] tiles: 4-value groups, those of B (0 .. V-1) then of C
+                // (V .. 2V-1), one per thread per round
                 constexpr int V = C::BC_ENTRIES / 4;
-                static_assert(2 * V <= kThreads, "one 4-value group per thread");
-                const int which = tid / V, v = tid % V;
+                static_assert((2 * V) % kThreads == 0 || 2 * V < kThreads, "whole rounds of 4-value groups");
+#pragma unroll
+                for (int gq = tid; gq < 2 * V; gq += kThreads) {
+                const int which = gq / V, v = gq % V;
                 if (which == 0 || (which == 1 && want_out)) {
                     const T* src = which ? rC : rB;
                     float4 f;
@@ -460,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
                                         __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
                     }
                     reinterpret_cast<float4*>(which ? sCf : sBf)[v] = f;
+                }
                 }
             } else {
 #pragma unroll
@@ -498,10 +502,10 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
         const int64_t ck_stride = (int64_t)a.D * N;
         const int nvalid = cvalid ? min(G, N - g * G) : 0;
         if (acc)
-            scan_tile_any<T, NG, G, MODE, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid,
+            scan_tile_any<T, NG, G, MODE, TT, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid,
                                                 a.ws_ckpt, ext_ckpt);
         else
-            scan_tile_any<T, NG, G, MODE, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid,
+            scan_tile_any<T, NG, G, MODE, TT, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid,
                                                  a.ws_ckpt, ext_ckpt);
         if (want_out) fence_proxy_async();
         // the next tile's data, then one barrier for: outputs complete, tile buffers free,
@@ -552,14 +556,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3-D map over a (batch, L, D) tensor, box [1][kTT][DC], zero fill outside.
+// 3-D map over a (batch, L, D) tensor, box [1][TT][DC], zero fill outside.
 template <typename T>
-bool make_map(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int64_t D, int DC) {
+bool make_map(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int64_t D, int DC, int TT) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)batch};
     const cuuint64_t strides[2] = {(cuuint64_t)(D * sizeof(T)), (cuuint64_t)(L * D * sizeof(T))};
-    const cuuint32_t box[3] = {(cuuint32_t)DC, (cuuint32_t)kTT, 1};
+    const cuuint32_t box[3] = {(cuuint32_t)DC, (cuuint32_t)TT, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapDataType ty =
         sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
@@ -576,26 +580,26 @@ bool bc_by_tma(const TiledArgs& a) {
            (a.C == nullptr || reinterpret_cast<uintptr_t>(a.C) % 16 == 0);
 }
 
-template <typename T, int NG, int G, int MODE>
+template <typename T, int NG, int G, int MODE, int TT>
 cudaError_t launch_mode(const TiledArgs& args, const TiledPtrs& p, cudaStream_t st) {
-    using C = Cfg<T, NG, G, MODE>;
+    using C = Cfg<T, NG, G, MODE, TT>;
     TiledArgs a = args;
     a.bc_tma = bc_by_tma<T>(a) ? 1 : 0;
     CUtensorMap mu, md, mz, mo, mb, mc;
     const void* zsrc = p.z ? p.z : p.u;      // an unused map still needs a valid address
     const void* osrc = p.out ? p.out : p.u;
-    if (!make_map<T>(&mu, p.u, a.batch, a.L, a.D, C::DC) || !make_map<T>(&md, p.delta_raw, a.batch, a.L, a.D, C::DC) ||
-        !make_map<T>(&mz, zsrc, a.batch, a.L, a.D, C::DC) || !make_map<T>(&mo, osrc, a.batch, a.L, a.D, C::DC))
+    if (!make_map<T>(&mu, p.u, a.batch, a.L, a.D, C::DC, TT) || !make_map<T>(&md, p.delta_raw, a.batch, a.L, a.D, C::DC, TT) ||
+        !make_map<T>(&mz, zsrc, a.batch, a.L, a.D, C::DC, TT) || !make_map<T>(&mo, osrc, a.batch, a.L, a.D, C::DC, TT))
         return cudaErrorInvalidValue;
     if (a.bc_tma) {
-        if (!make_map<T>(&mb, a.B, a.batch, a.L, a.N, a.N) ||
-            !make_map<T>(&mc, a.C ? a.C : a.B, a.batch, a.L, a.N, a.N))
+        if (!make_map<T>(&mb, a.B, a.batch, a.L, a.N, a.N, TT) ||
+            !make_map<T>(&mc, a.C ? a.C : a.B, a.batch, a.L, a.N, a.N, TT))
             return cudaErrorInvalidValue;
     } else {
         mb = mu;
         mc = mu;
     }
-    auto kern = fwd_tiled_kernel<T, NG, G, MODE>;
+    auto kern = fwd_tiled_kernel<T, NG, G, MODE, TT>;
     // function attributes are per device: set them once on each device used
     static bool configured[kMaxDevices] = {};
     int dev = 0;
@@ -611,12 +615,27 @@ cudaError_t launch_mode(const TiledArgs& args, const TiledPtrs& p, cudaStream_t 
     return cudaGetLastError();
 }
 
+// Steps per tile.  Each tile costs two CTA-wide barriers and one phase P whose latency
+// the other CTAs of the SM must hide; longer tiles halve that per step but need more
+// shared memory, so fewer CTAs fit an SM.  Measured (bf16 / fp32 I/O, ms per launch,
+// tiles of 16 / 32 / 64 steps): Mamba-130M layer 0.255 / 0.225 / 0.214 and 0.252 / 0.223 /
+// 0.299; Mamba-2.8B layer 0.587 / 0.556 / 0.622 and 0.573 / 0.565 / 0.774; the million-step
+// split 20.9 / 19.6 / 21.6.  So 64 when the whole grid fits the GPU at once with 64-step
+// tiles, else 32.  The backward's checkpoint pass, which runs beside the reverse kernel's
+// summary pass, keeps 16 (its backward call 1.253 / 1.271 / 1.278 ms).
 template <typename T, int NG, int G>
 cudaError_t launch_geom(const TiledArgs& a, const TiledPtrs& p, int mode, cudaStream_t st) {
-    if (mode == kTiledOut) return launch_mode<T, NG, G, kOut>(a, p, st);
-    if (mode == kTiledAgg) return launch_mode<T, NG, G, kAgg>(a, p, st);
-    if (mode == kTiledCkpt) return launch_mode<T, NG, G, kCkpt>(a, p, st);
-    return launch_mode<T, NG, G, kLast>(a, p, st);
+    if (mode == kTiledCkpt) return launch_mode<T, NG, G, kCkpt, 16>(a, p, st);
+    const int64_t ctas = a.batch * a.nchunks * ((a.D + 32 / NG * kWarps - 1) / (32 / NG * kWarps));
+    const int64_t fit64 = kSmemPerSm / (Cfg<T, NG, G, kOut, 64>::SMEM + kSmemPerCtaReserved);
+    if (ctas <= fit64 * kSmCount) {
+        if (mode == kTiledOut) return launch_mode<T, NG, G, kOut, 64>(a, p, st);
+        if (mode == kTiledAgg) return launch_mode<T, NG, G, kAgg, 64>(a, p, st);
+        return launch_mode<T, NG, G, kLast, 64>(a, p, st);
+    }
+    if (mode == kTiledOut) return launch_mode<T, NG, G, kOut, 32>(a, p, st);
+    if (mode == kTiledAgg) return launch_mode<T, NG, G, kAgg, 32>(a, p, st);
+    return launch_mode<T, NG, G, kLast, 32>(a, p, st);
 }
 
 template <typename T>
