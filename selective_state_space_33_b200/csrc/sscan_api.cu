@@ -521,21 +521,22 @@ sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_
         if (plan.nsegs > 1) {
             // the reverse sweep split in time: segment summaries and their carry on the
             // second stream, the checkpoint pass on the caller's, joined before the
-            // reverse kernel
+            // reverse kernel.  The checkpoint pass, the longer of the two, is launched
+            // first so that its CTAs are placed before the summaries fill the SMs.
             std::lock_guard<std::mutex> lock(g_aux_mutex);
             AuxStream* ax = nullptr;
             if ((e = aux_stream(&ax)) != cudaSuccess || (e = cudaEventRecord(ax->fork, st)) != cudaSuccess ||
                 (e = cudaStreamWaitEvent(ax->stream, ax->fork, 0)) != cudaSuccess)
                 return fail(SSCAN_ERR_CUDA, "backward stream fork: %s", cudaGetErrorString(e));
             ++g_launches;
+            e = sscan::launch_fwd_tiled(t, tp, geo, bf16, sscan::kTiledCkpt, st);
+            if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "checkpoint kernel: %s", cudaGetErrorString(e));
+            ++g_launches;
             e = sscan::launch_bwd_tiled(ba, bp, bf16, sscan::kBwdSummary, ax->stream);
             if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "backward summary kernel: %s", cudaGetErrorString(e));
             ++g_launches;
             e = sscan::launch_bwd_carry(ba, ax->stream);
             if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "backward carry kernel: %s", cudaGetErrorString(e));
-            ++g_launches;
-            e = sscan::launch_fwd_tiled(t, tp, geo, bf16, sscan::kTiledCkpt, st);
-            if (e != cudaSuccess) return fail(SSCAN_ERR_CUDA, "checkpoint kernel: %s", cudaGetErrorString(e));
             if ((e = cudaEventRecord(ax->join, ax->stream)) != cudaSuccess ||
                 (e = cudaStreamWaitEvent(st, ax->join, 0)) != cudaSuccess)
                 return fail(SSCAN_ERR_CUDA, "backward stream join: %s", cudaGetErrorString(e));

@@ -91,6 +91,10 @@ struct BCfg {
     static constexpr int OFF_OUT = OFF_ACC + kTB * NS * 2 * 4;  // [2 buffers][3 tensors][RAW]
     static constexpr int OFF_BAR = OFF_OUT + 2 * 3 * RAW;
     static constexpr int SMEM = OFF_BAR + STAGES * 8;
+    // the summary pass uses the ring, the (delta, dy) operands and C only: its barriers
+    // follow C and its launch asks for that much shared memory
+    static constexpr int OFF_BAR_SUM = OFF_HS;
+    static constexpr int SMEM_SUM = OFF_BAR_SUM + STAGES * 8;
 };
 
 // Transposed butterfly over the NG lanes of a channel (lane bits at multiples of CW),
@@ -296,8 +300,10 @@ __global__ void __launch_bounds__(kThreadsB, 5)
     const int tile_hi = min(tiles_all, tile_lo + (int)((a.seg_len + kTB - 1) / kTB));
     const int ntb = tile_hi - tile_lo;  // tiles of this segment
     const bool has_z = a.has_z != 0;
-    const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
-    const uint32_t stage_bytes = (has_z ? 4u : 3u) * C::RAW + 2u * (uint32_t)(kTB * N * (int)sizeof(T));
+    constexpr bool kSum = MODE == kBwdSummary;  // the summary pass reads neither u nor B
+    const uint32_t bar0 = smem_u32(smem + (kSum ? C::OFF_BAR_SUM : C::OFF_BAR));
+    const uint32_t stage_bytes = ((has_z ? 4u : 3u) - (kSum ? 1u : 0u)) * C::RAW +
+                                 (kSum ? 1u : 2u) * (uint32_t)(kTB * N * (int)sizeof(T));
 
     // tiles are taken in reverse: processing index k covers tile tile_hi - 1 - k
     auto issue = [&](int k) {
@@ -306,11 +312,11 @@ __global__ void __launch_bounds__(kThreadsB, 5)
         const uint32_t base = smem_u32(smem + C::OFF_RAW + st * C::STAGE);
         const int t0 = (tile_hi - 1 - k) * kTB;
         mbar_expect_tx(bar, stage_bytes);
-        tma_load_3d(base, &tm_u, d0, t0, b, bar);
+        if (!kSum) tma_load_3d(base, &tm_u, d0, t0, b, bar);
         tma_load_3d(base + C::RAW, &tm_dr, d0, t0, b, bar);
         if (has_z) tma_load_3d(base + 2 * C::RAW, &tm_z, d0, t0, b, bar);
         tma_load_3d(base + 3 * C::RAW, &tm_g, d0, t0, b, bar);
-        tma_load_3d(base + 4 * C::RAW, &tm_B, 0, t0, b, bar);
+        if (!kSum) tma_load_3d(base + 4 * C::RAW, &tm_B, 0, t0, b, bar);
         tma_load_3d(base + 4 * C::RAW + C::RAWBC, &tm_C, 0, t0, b, bar);
     };
 
@@ -323,7 +329,8 @@ __global__ void __launch_bounds__(kThreadsB, 5)
     // the tile's dB, dC summed over the CTA's channels: zero here, and zeroed again by
     // the thread that drains each entry into global memory
     float* sacc = reinterpret_cast<float*>(smem + C::OFF_ACC);
-    for (int e = tid; e < kTB * C::NS * 2; e += kThreadsB) sacc[e] = 0.f;
+    if (!kSum)
+        for (int e = tid; e < kTB * C::NS * 2; e += kThreadsB) sacc[e] = 0.f;
 
     // lane state: channel cw, states g*4 .. g*4+3
     const int g = lane / C::CW, c = lane % C::CW, cw = warp * C::CW + c;
@@ -399,6 +406,23 @@ __global__ void __launch_bounds__(kThreadsB, 5)
                 const int q = tid + qi * kThreadsB;
                 const int t = q / (C::DC / 2);
                 const bool tv = t < tile_len;
+                if constexpr (kSum) {
+                    // the summary pass needs delta and dy only
+                    const float2 r = __fadd2_rn(BPair<T>::f(rd[q]), pbias);
+                    float2 dl = r, sr;
+                    if (a.softplus) softplus_sig_x2(r, dl, sr);
+                    float2 dy = BPair<T>::f(rg[q]);
+                    if (has_z) {
+                        const float2 zz = BPair<T>::f(rz[q]);
+                        dy = __fmul2_rn(__fmul2_rn(dy, sigmoid_x2(zz)), zz);
+                    }
+                    if (!tv) dy = g2(0.f, 0.f);
+                    const int e = t * C::DC + pc;
+                    sdx[e] = make_float4(dl.x, dl.x, 0.f, 0.f);
+                    sdx[e + 1] = make_float4(dl.y, dl.y, 0.f, 0.f);
+                    reinterpret_cast<float4*>(sdy)[e / 2] = make_float4(dy.x, dy.x, dy.y, dy.y);
+                    continue;
+                }
                 const float2 uv = BPair<T>::f(ru[q]);
                 float2 x = uv;
                 if (a.input_silu) {
@@ -437,7 +461,7 @@ __global__ void __launch_bounds__(kThreadsB, 5)
             float* sCf = reinterpret_cast<float*>(smem + C::OFF_C);
             for (int e = tid; e < kTB * C::NS; e += kThreadsB) {
                 const int t = e / C::NS, n = e % C::NS;
-                sBf[e] = n < N ? to_f32<T>(rB[t * N + n]) : 0.f;
+                if (!kSum) sBf[e] = n < N ? to_f32<T>(rB[t * N + n]) : 0.f;
                 sCf[e] = n < N ? to_f32<T>(rC[t * N + n]) : 0.f;
             }
         }
@@ -678,15 +702,16 @@ cudaError_t launch_bwd_kernel(const CUtensorMap (&m)[9], const BwdTiledArgs& a, 
     static bool configured[kMaxDevices] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    constexpr int smem = MODE == kBwdSummary ? C::SMEM_SUM : C::SMEM;
     if (!configured[dev]) {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         configured[dev] = true;
     }
     const int64_t segs = MODE == kBwdSummary ? a.nseg - 1 : a.nseg;
     const int64_t blocks = a.batch * segs * ((a.D + C::DC - 1) / C::DC);
     if (blocks > 0)
-        kern<<<(unsigned)blocks, kThreadsB, C::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], m[8], a);
+        kern<<<(unsigned)blocks, kThreadsB, smem, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], m[8], a);
     return cudaGetLastError();
 }
 

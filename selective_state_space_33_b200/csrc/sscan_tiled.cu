@@ -621,11 +621,12 @@ cudaError_t launch_mode(const TiledArgs& args, const TiledPtrs& p, cudaStream_t 
 // tiles of 16 / 32 / 64 steps): Mamba-130M layer 0.255 / 0.225 / 0.214 and 0.252 / 0.223 /
 // 0.299; Mamba-2.8B layer 0.587 / 0.556 / 0.622 and 0.573 / 0.565 / 0.774; the million-step
 // split 20.9 / 19.6 / 21.6.  So 64 when the whole grid fits the GPU at once with 64-step
-// tiles, else 32.  The backward's checkpoint pass, which runs beside the reverse kernel's
-// summary pass, keeps 16 (its backward call 1.253 / 1.271 / 1.278 ms).
+// tiles, else 32.  The backward's checkpoint pass runs beside the reverse kernel's summary
+// pass; launched before it, it takes 32 (backward call 1.254 ms with 16-step tiles, 1.204 ms
+// with 32; 64-step tiles of the two-stage checkpoint ring need 76 KB).
 template <typename T, int NG, int G>
 cudaError_t launch_geom(const TiledArgs& a, const TiledPtrs& p, int mode, cudaStream_t st) {
-    if (mode == kTiledCkpt) return launch_mode<T, NG, G, kCkpt, 16>(a, p, st);
+    if (mode == kTiledCkpt) return launch_mode<T, NG, G, kCkpt, 32>(a, p, st);
     const int64_t ctas = a.batch * a.nchunks * ((a.D + 32 / NG * kWarps - 1) / (32 / NG * kWarps));
     const int64_t fit64 = kSmemPerSm / (Cfg<T, NG, G, kOut, 64>::SMEM + kSmemPerCtaReserved);
     if (ctas <= fit64 * kSmCount) {
