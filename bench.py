@@ -126,20 +126,20 @@ def roofline_units(w: W.Workload) -> dict:
 # keyed by the SHA-256 of those source files (with comments and blank lines removed,
 # so that only code counts) and reported as null once the code changes.
 NCU_TRAFFIC = {
-    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 505390080 + 151158272,
-        "sources": ('sscan_tiled.cu', 'sscan_tma.cuh', 'sscan_math.cuh', 'sscan_check.cuh'), "sha256": "a7dfbf4ffeaeecac",
+    "mamba2.8b": {"kernel": "fwd_tiled_kernel", "bytes": 506067968 + 151158016,
+        "sources": ('sscan_tiled.cu', 'sscan_tma.cuh', 'sscan_math.cuh', 'sscan_check.cuh', 'sscan_plan.h'), "sha256": "e94bf6f48cf8dec3",
         "profile": "profiles/fwd_tiled_kernel_mamba2.8b_bf16.md"},
-    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410679296 + 133782528,
-        "sources": ('sscan_bwd_tiled.cu', 'sscan_tma.cuh', 'sscan_math.cuh', 'sscan_check.cuh'), "sha256": "a8acc2a5f68ebfa5",
+    "bwd130m": {"kernel": "bwd_tiled_kernel", "bytes": 410449408 + 133641984,
+        "sources": ('sscan_bwd_tiled.cu', 'sscan_tma.cuh', 'sscan_math.cuh', 'sscan_check.cuh'), "sha256": "5a0552a6bbd9fdb2",
         "profile": "profiles/bwd_tiled_kernel_bwd130m_bf16.md"},
-    "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317504 + 256,
+    "decode2.8b": {"kernel": "step_quad_kernel", "bytes": 23317760 + 0,
         "sources": ('sscan_step.cu', 'sscan_math.cuh'), "sha256": "c1a451e4bc5a2b5e",
         "profile": "profiles/step_quad_kernel_decode2.8b_bf16.md"},
-    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152569856 + 30774528,
-        "sources": ('sscan_complex.cu', 'sscan_complex_math.cuh', 'sscan_math.cuh', 'sscan_tma.cuh'), "sha256": "4098bc4b952ac034",
+    "complex130m": {"kernel": "fwd_complex_kernel", "bytes": 152337152 + 31579136,
+        "sources": ('sscan_complex.cu', 'sscan_complex_math.cuh', 'sscan_math.cuh', 'sscan_tma.cuh'), "sha256": "a5b8c078e8916124",
         "profile": "profiles/fwd_complex_kernel_complex130m_bf16.md"},
-    "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 613000192 + 139654656,
-        "sources": ('sscan_complex_bwd.cu', 'sscan_complex_math.cuh', 'sscan_math.cuh'), "sha256": "72ceb8f7a14ce8a2",
+    "complexbwd130m": {"kernel": "bwd_complex_kernel", "bytes": 614110976 + 140454400,
+        "sources": ('sscan_complex_bwd.cu', 'sscan_complex_math.cuh', 'sscan_math.cuh'), "sha256": "1324535f04cda675",
         "profile": "profiles/bwd_complex_kernel_complexbwd130m_bf16.md"},
 }
 

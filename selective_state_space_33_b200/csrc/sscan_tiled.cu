@@ -75,15 +75,14 @@ struct Cfg {
     static constexpr int RAW = TT * DC * (int)sizeof(T);  // bytes of one raw (batch, L, D) tile
     static constexpr int RAWBC = TT * NS * (int)sizeof(T);  // bytes reserved for one raw B or C tile
     static constexpr int STAGE = 3 * RAW + 2 * RAWBC;      // u, delta_raw, z, B, C
-    static constexpr int GD_PITCH = DC;                    // float2 row pitch of the epilogue operands
     static constexpr int BC_ENTRIES = TT * NS;
     static constexpr int PAIRS = TT * DC / 2;             // channel pairs of phase P
     static_assert(PAIRS % kThreads == 0, "phase P runs a fixed number of pairs per thread");
     // shared-memory layout (byte offsets, all 128-aligned)
     static constexpr int OFF_RAW = 0;                                     // [STAGES][STAGE]
     static constexpr int OFF_DX = OFF_RAW + STAGES * STAGE;               // float2 (delta, x) [TT][DC]
-    static constexpr int OFF_GD = OFF_DX + TT * DC * 8;                  // float2 (gate, D x gate) [TT][GD_PITCH]
-    static constexpr int OFF_B = OFF_GD + TT * GD_PITCH * 8;             // float  [TT][NS]
+    static constexpr int OFF_GD = OFF_DX + TT * DC * 8;                  // float  gate [TT][DC]
+    static constexpr int OFF_B = OFF_GD + TT * DC * 4;                   // float  [TT][NS]
     static constexpr int OFF_C = OFF_B + TT * NS * 4;                    // float  [TT][NS]
     static constexpr int OFF_OUT = OFF_C + TT * NS * 4;                  // [RAW] output tile
     static constexpr int OFF_BAR = OFF_OUT + RAW;                         // uint64 [STAGES]
@@ -170,12 +169,12 @@ __device__ __forceinline__ float transpose_reduce(float (&p)[NG], int g) {
 // the last, partial tile of a chunk takes the predicated form.
 template <typename T, int NG, int G, int MODE, int TT, bool ACC, bool FULL>
 __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
-                                          float& dsum, float* ck, int64_t ck_stride, int nvalid,
+                                          float dskc, float& dsum, float* ck, int64_t ck_stride, int nvalid,
                                           const float* ck_base, int64_t ck_extent) {
     using C = Cfg<T, NG, G, MODE, TT>;
     constexpr bool WANT_Y = MODE == kOut;
     const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
-    const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
+    const float* sgt = reinterpret_cast<const float*>(smem + C::OFF_GD) + cw;
     const float* sB = reinterpret_cast<const float*>(smem + C::OFF_B) + g * G;
     const float* sC = reinterpret_cast<const float*>(smem + C::OFF_C) + g * G;
 #pragma unroll(MODE == kOut ? 2 : 1)
@@ -203,8 +202,7 @@ __device__ __forceinline__ void scan_tile(LaneG<G>& s, unsigned char* smem, int 
             const float y = transpose_reduce<NG, C::CW>(p, g);
             const int t = tb + g;
             if (FULL || t < tile_len) {
-                const float2 gd = sgd[t * C::GD_PITCH];
-                sout[t * C::DC + cw] = from_f32<T>(fmaf(y, gd.x, gd.y));
+                sout[t * C::DC + cw] = from_f32<T>(sgt[t * C::DC] * fmaf(dskc, sdx[t * C::DC].y, y));
             }
         }
     }
@@ -241,10 +239,11 @@ __device__ __forceinline__ float upd_step(LaneG<G>& s, const Prep<G>& P, const f
 }
 
 template <typename T, int NG, int G, int TT>
-__device__ __forceinline__ void scan_tile_pipe(LaneG<G>& s, unsigned char* smem, int g, int cw, T* sout) {
+__device__ __forceinline__ void scan_tile_pipe(LaneG<G>& s, unsigned char* smem, int g, int cw, T* sout,
+                                               float dskc) {
     using C = Cfg<T, NG, G, kOut, TT>;
     const float2* sdx = reinterpret_cast<const float2*>(smem + C::OFF_DX) + cw;
-    const float2* sgd = reinterpret_cast<const float2*>(smem + C::OFF_GD) + cw;
+    const float* sgt = reinterpret_cast<const float*>(smem + C::OFF_GD) + cw;
     const float* sB = reinterpret_cast<const float*>(smem + C::OFF_B) + g * G;
     const float* sC = reinterpret_cast<const float*>(smem + C::OFF_C) + g * G;
     Prep<G> P = prep_step<G>(s, sdx[0], sB);
@@ -261,26 +260,25 @@ __device__ __forceinline__ void scan_tile_pipe(LaneG<G>& s, unsigned char* smem,
         }
         const float y = transpose_reduce<NG, C::CW>(p, g);
         const int t = tb + g;
-        const float2 gd = sgd[t * C::GD_PITCH];
-        sout[t * C::DC + cw] = from_f32<T>(fmaf(y, gd.x, gd.y));
+        sout[t * C::DC + cw] = from_f32<T>(sgt[t * C::DC] * fmaf(dskc, sdx[t * C::DC].y, y));
     }
 }
 template <typename T, int NG, int G, int MODE, int TT, bool ACC>
 __device__ __forceinline__ void scan_tile_any(LaneG<G>& s, unsigned char* smem, int tile_len, int g, int cw, T* sout,
-                                              float& dsum, float* ck, int64_t ck_stride, int nvalid,
+                                              float dskc, float& dsum, float* ck, int64_t ck_stride, int nvalid,
                                               const float* ck_base, int64_t ck_extent) {
     if constexpr (MODE == kOut && !ACC) {
         if (tile_len == TT) {
-            scan_tile_pipe<T, NG, G, TT>(s, smem, g, cw, sout);
+            scan_tile_pipe<T, NG, G, TT>(s, smem, g, cw, sout, dskc);
             return;
         }
     }
     if (tile_len == TT)
-        scan_tile<T, NG, G, MODE, TT, ACC, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid, ck_base,
-                                             ck_extent);
+        scan_tile<T, NG, G, MODE, TT, ACC, true>(s, smem, tile_len, g, cw, sout, dskc, dsum, ck, ck_stride, nvalid,
+                                                 ck_base, ck_extent);
     else
-        scan_tile<T, NG, G, MODE, TT, ACC, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid, ck_base,
-                                              ck_extent);
+        scan_tile<T, NG, G, MODE, TT, ACC, false>(s, smem, tile_len, g, cw, sout, dskc, dsum, ck, ck_stride, nvalid,
+                                                  ck_base, ck_extent);
 }
 
 // softplus and SiLU of two values at once: the exponentials, logarithm and
@@ -404,13 +402,13 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
     // phase-P channel pair of this thread (fixed, since kThreads is a multiple of DC/2)
     const int pc = 2 * (tid % (C::DC / 2));
     const int64_t pd = d0 + pc;
+    // skip weight D of this lane's channel (the epilogue forms gate * (y + D x))
+    const float dskc = (want_out && a.Dskip && cvalid) ? __ldg(a.Dskip + d) : 0.f;
     const T* Bg = static_cast<const T*>(a.B);
     const T* Cg = static_cast<const T*>(a.C);
     float dsum = 0.f;
     const float2 pbias = f2((a.bias && pd < a.D) ? __ldg(a.bias + pd) : 0.f,
                             (a.bias && pd + 1 < a.D) ? __ldg(a.bias + pd + 1) : 0.f);
-    const float2 pdsk = f2((want_out && a.Dskip && pd < a.D) ? __ldg(a.Dskip + pd) : 0.f,
-                           (want_out && a.Dskip && pd + 1 < a.D) ? __ldg(a.Dskip + pd + 1) : 0.f);
 
     for (int it = 0; it < ntile && !failed; ++it) {
         const int st = it % C::STAGES;
@@ -423,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
             const P2* rd = reinterpret_cast<const P2*>(raw + C::RAW);
             const P2* rz = reinterpret_cast<const P2*>(raw + 2 * C::RAW);
             float4* sdx = reinterpret_cast<float4*>(smem + C::OFF_DX);
-            float4* sgd = reinterpret_cast<float4*>(smem + C::OFF_GD);
+            float2* sgt = reinterpret_cast<float2*>(smem + C::OFF_GD);
             // a fixed trip count (PAIRS is a multiple of kThreads for every geometry)
 #pragma unroll
             for (int qi = 0; qi < C::PAIRS / kThreads; ++qi) {
@@ -436,8 +434,7 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
                 sdx[(t * C::DC + pc) / 2] = make_float4(dl.x, x.x, dl.y, x.y);
                 if (want_out) {
                     const float2 gt = has_z ? silu_x2(Pair<T>::f(rz[q])) : f2(1.f, 1.f);
-                    const float2 dxg = __fmul2_rn(__fmul2_rn(pdsk, x), gt);
-                    sgd[(t * C::GD_PITCH + pc) / 2] = make_float4(gt.x, dxg.x, gt.y, dxg.y);
+                    sgt[(t * C::DC + pc) / 2] = gt;
                 }
             }
             float* sBf = reinterpret_cast<float*>(smem + C::OFF_B);
@@ -502,10 +499,10 @@ __global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
         const int64_t ck_stride = (int64_t)a.D * N;
         const int nvalid = cvalid ? min(G, N - g * G) : 0;
         if (acc)
-            scan_tile_any<T, NG, G, MODE, TT, true>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid,
+            scan_tile_any<T, NG, G, MODE, TT, true>(s, smem, tile_len, g, cw, sout, dskc, dsum, ck, ck_stride, nvalid,
                                                 a.ws_ckpt, ext_ckpt);
         else
-            scan_tile_any<T, NG, G, MODE, TT, false>(s, smem, tile_len, g, cw, sout, dsum, ck, ck_stride, nvalid,
+            scan_tile_any<T, NG, G, MODE, TT, false>(s, smem, tile_len, g, cw, sout, dskc, dsum, ck, ck_stride, nvalid,
                                                  a.ws_ckpt, ext_ckpt);
         if (want_out) fence_proxy_async();
         // the next tile's data, then one barrier for: outputs complete, tile buffers free,
