@@ -31,8 +31,10 @@
 
 #include <cstdint>
 #include <cstring>
+#include <type_traits>
 
 #include "sscan_launch.h"
+#include "sscan_act.cuh"
 #include "sscan_complex_math.cuh"
 #include "sscan_math.cuh"
 #include "sscan_plan.h"
@@ -44,7 +46,6 @@ __device__ unsigned int g_device_error_cx = 0;
 
 namespace {
 
-constexpr int kCTT = 16;           // steps per tile
 constexpr int kCWarps = 4;
 constexpr int kCThreads = kCWarps * 32;
 constexpr float kCSmallA = 9.765625e-4f;
@@ -55,19 +56,32 @@ struct CCfg {
     static constexpr int NS = NG * CG;       // states covered (>= N)
 };
 
-// Dynamic shared memory of the TMA path: a 2-stage ring of raw tiles (u, delta_raw, z,
-// then B and C when their rows travel by TMA), 128-byte aligned, and its mbarriers.
-template <typename T, int NG, int CG>
-struct CRing {
+// Dynamic shared memory of a TT-step tile: phase P's staging -- (delta, x) pairs and the
+// SiLU gate per (step, channel), the tile's B and C rows -- then, on the TMA path, a
+// 2-stage ring of raw tiles (u, delta_raw, z, then B and C when their rows travel by
+// TMA) and its mbarriers; 128-byte aligned sections.
+template <typename T, int NG, int CG, int TT>
+struct CSmem {
     static constexpr int DC = CCfg<NG, CG>::DC, NS = CCfg<NG, CG>::NS;
-    static constexpr int RAW = kCTT * DC * (int)sizeof(T);
-    static constexpr int RAWBC = (kCTT * NS * (int)sizeof(T) + 127) / 128 * 128;  // one B or C tile (N <= NS)
+    static constexpr int OFF_DX = 0;                                             // float2 [TT][DC]
+    static constexpr int OFF_GT = OFF_DX + TT * DC * 8;                          // float  [TT][DC]
+    static constexpr int OFF_B = OFF_GT + (TT * DC * 4 + 127) / 128 * 128;       // float  [TT][NS]
+    static constexpr int OFF_C = OFF_B + (TT * NS * 4 + 127) / 128 * 128;        // float  [TT][NS]
+    static constexpr int OFF_RING = OFF_C + (TT * NS * 4 + 127) / 128 * 128;
+    static constexpr int RAW = TT * DC * (int)sizeof(T);
+    static constexpr int RAWBC = (TT * NS * (int)sizeof(T) + 127) / 128 * 128;  // one B or C tile (N <= NS)
     static constexpr int STAGE = (3 * RAW + 2 * RAWBC + 127) / 128 * 128;
     static constexpr int STAGES = 2;
-    static constexpr int OFF_BAR = STAGES * STAGE;
-    static constexpr int SMEM = OFF_BAR + STAGES * 8;
-    static_assert(RAW % 128 == 0, "raw tiles start 128-byte aligned");
+    static constexpr int OFF_BAR = OFF_RING + STAGES * STAGE;
+    static constexpr int SMEM_PLAIN = OFF_RING;          // plain loads: no ring
+    static constexpr int SMEM_TMA = OFF_BAR + STAGES * 8;
+    static constexpr int PAIRS = TT * DC / 2;            // channel pairs of phase P
+    static_assert(RAW % 128 == 0 && (TT * DC * 8) % 128 == 0, "sections start 128-byte aligned");
+    static_assert(PAIRS % kCThreads == 0, "phase P runs a fixed number of channel pairs per thread");
 };
+
+__device__ __forceinline__ float2 to_f32x2(float2 v) { return v; }
+__device__ __forceinline__ float2 to_f32x2(__nv_bfloat162 v) { return __bfloat1622float2(v); }
 
 __device__ __forceinline__ float2 ex2x2c(float2 q) { return make_float2(ex2(q.x), ex2(q.y)); }
 
@@ -100,28 +114,52 @@ __device__ __forceinline__ void cis2(float2 th, float2& cs, float2& sn) {
 
 // One step of the lane's CG complex states (eq. (2) and (3a) with complex a; B, x
 // real) in the fast form h' = Abar (h - v) + v with v = -B x / a, two states per
-// packed operation.  Returns the partial readout Re(sum_j C_j h_j) (eq. (3b)).
+// packed operation, in two parts: cprep forms Abar and v (the MUFU work: 2^(delta Re a),
+// cos and sin of delta Im a), cupd updates the states and returns the partial readout
+// Re(sum_j C_j h_j) (eq. (3b)).  Full output tiles issue the cprep of step t + 1 before
+// the cupd of step t.
 template <int CG>
-__device__ __forceinline__ float cstep_fast(CLane<CG>& s, float delta, float x, const float* Bt,
-                                            const float* Ct) {
+struct CPrep {
+    float2 abr[CG / 2], abi[CG / 2], vr[CG / 2], vi[CG / 2];
+};
+
+template <int CG>
+__device__ __forceinline__ CPrep<CG> cprep(const CLane<CG>& s, float delta, float x, const float* Bt) {
+    CPrep<CG> P;
     const float2 dd = make_float2(delta, delta), xx = make_float2(x, x);
-    float2 y = make_float2(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < CG / 2; ++k) {
         const float2 e = ex2x2c(__fmul2_rn(dd, s.qr[k]));
         float2 cs, sn;
         cis2(__fmul2_rn(dd, s.qi[k]), cs, sn);
-        const float2 abr = __fmul2_rn(e, cs), abi = __fmul2_rn(e, sn);
+        P.abr[k] = __fmul2_rn(e, cs);
+        P.abi[k] = __fmul2_rn(e, sn);
         const float2 bx = __fmul2_rn(reinterpret_cast<const float2*>(Bt)[k], xx);
-        const float2 vr = __fmul2_rn(bx, s.nr[k]), vi = __fmul2_rn(bx, s.ni[k]);
-        const float2 tr = __ffma2_rn(vr, make_float2(-1.f, -1.f), s.hr[k]);   // Re(h - v)
-        const float2 ti = __ffma2_rn(vi, make_float2(-1.f, -1.f), s.hi[k]);   // Im(h - v)
-        const float2 mti = __ffma2_rn(s.hi[k], make_float2(-1.f, -1.f), vi);  // -Im(h - v)
-        s.hr[k] = __ffma2_rn(abr, tr, __ffma2_rn(abi, mti, vr));
-        s.hi[k] = __ffma2_rn(abr, ti, __ffma2_rn(abi, tr, vi));
+        P.vr[k] = __fmul2_rn(bx, s.nr[k]);
+        P.vi[k] = __fmul2_rn(bx, s.ni[k]);
+    }
+    return P;
+}
+
+template <int CG>
+__device__ __forceinline__ float cupd(CLane<CG>& s, const CPrep<CG>& P, const float* Ct) {
+    float2 y = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < CG / 2; ++k) {
+        const float2 tr = __ffma2_rn(P.vr[k], make_float2(-1.f, -1.f), s.hr[k]);   // Re(h - v)
+        const float2 ti = __ffma2_rn(P.vi[k], make_float2(-1.f, -1.f), s.hi[k]);   // Im(h - v)
+        const float2 mti = __ffma2_rn(s.hi[k], make_float2(-1.f, -1.f), P.vi[k]);  // -Im(h - v)
+        s.hr[k] = __ffma2_rn(P.abr[k], tr, __ffma2_rn(P.abi[k], mti, P.vr[k]));
+        s.hi[k] = __ffma2_rn(P.abr[k], ti, __ffma2_rn(P.abi[k], tr, P.vi[k]));
         y = __ffma2_rn(reinterpret_cast<const float2*>(Ct)[k], s.hr[k], y);
     }
     return y.x + y.y;
+}
+
+template <int CG>
+__device__ __forceinline__ float cstep_fast(CLane<CG>& s, float delta, float x, const float* Bt,
+                                            const float* Ct) {
+    return cupd<CG>(s, cprep<CG>(s, delta, x, Bt), Ct);
 }
 
 // The same step for a block with a small |a|: Bbar / B = delta phi1(delta a) with
@@ -198,11 +236,13 @@ __device__ __forceinline__ float creduce(float (&p)[NG], int g) {
 
 // Phase S over one tile.  Checkpoint pass: the state before every 8th step, no
 // readout.  Output pass: blocks of NG steps whose readouts are reduced together, lane
-// g finishing step tb + g; FULL tiles (kCTT steps) are unrolled with no step predicate.
-template <typename T, int NG, int CG, bool ACC, bool CKPT, bool FULL>
-__device__ __forceinline__ void scan_tile_c(CLane<CG>& s, const float2* sdx, const float2* sgd, const float* sB,
+// g finishing step tb + g (gate (y + D x), with the lane's own skip weight dskc); FULL
+// tiles (TT steps) are unrolled with no step predicate.
+template <typename T, int NG, int CG, int TT, bool ACC, bool CKPT, bool FULL>
+__device__ __forceinline__ void scan_tile_c(CLane<CG>& s, const float2* sdx, const float* sgt, const float* sB,
                                             const float* sC, int tl, int g, int cw, bool write, T* out,
-                                            int64_t out_stride, float* ck, int64_t ck_stride, int nvalid) {
+                                            int64_t out_stride, float dskc, float* ck, int64_t ck_stride,
+                                            int nvalid) {
     using C = CCfg<NG, CG>;
     const float* Bg = sB + g * CG;
     const float* Cg = sC + g * CG;
@@ -221,8 +261,8 @@ __device__ __forceinline__ void scan_tile_c(CLane<CG>& s, const float2* sdx, con
             (void)cstep<CG, ACC>(s, dx.x, dx.y, Bg + t * C::NS, Cg + t * C::NS);
         }
     } else {
-#pragma unroll(FULL ? kCTT / NG : 1)
-        for (int tb = 0; tb < (FULL ? kCTT : tl); tb += NG) {
+#pragma unroll(FULL ? TT / NG : 1)
+        for (int tb = 0; tb < (FULL ? TT : tl); tb += NG) {
             float p[NG];
 #pragma unroll
             for (int k = 0; k < NG; ++k) {
@@ -235,11 +275,41 @@ __device__ __forceinline__ void scan_tile_c(CLane<CG>& s, const float2* sdx, con
             }
             const float y = creduce<NG, C::CW>(p, g);
             const int t = tb + g;
-            if (write && (FULL || t < tl)) {
-                const float2 gd = sgd[t * C::DC + cw];
-                IO<T>::store(out, (int64_t)t * out_stride, fmaf(y, gd.x, gd.y));
-            }
+            if (write && (FULL || t < tl))
+                IO<T>::store(out, (int64_t)t * out_stride, sgt[t * C::DC + cw] * fmaf(dskc, sdx[t * C::DC + cw].y, y));
         }
+    }
+}
+
+// Full output tiles of the fast form, software-pipelined: the exponentials, cosines and
+// sines of step t + 1 (cprep) are issued before the state update of step t (cupd), so
+// their MUFU latency overlaps the dependent fmas; the arithmetic is that of cstep_fast.
+template <typename T, int NG, int CG, int TT>
+__device__ __forceinline__ void scan_tile_c_pipe(CLane<CG>& s, const float2* sdx, const float* sgt, const float* sB,
+                                                 const float* sC, int g, int cw, bool write, T* out,
+                                                 int64_t out_stride, float dskc) {
+    using C = CCfg<NG, CG>;
+    const float* Bg = sB + g * CG;
+    const float* Cg = sC + g * CG;
+    const float2 dx0 = sdx[cw];
+    CPrep<CG> P = cprep<CG>(s, dx0.x, dx0.y, Bg);
+#pragma unroll
+    for (int tb = 0; tb < TT; tb += NG) {
+        float p[NG];
+#pragma unroll
+        for (int k = 0; k < NG; ++k) {
+            const int t = tb + k;
+            CPrep<CG> Pn = P;
+            if (t + 1 < TT) {
+                const float2 dx = sdx[(t + 1) * C::DC + cw];
+                Pn = cprep<CG>(s, dx.x, dx.y, Bg + (t + 1) * C::NS);
+            }
+            p[k] = cupd<CG>(s, P, Cg + t * C::NS);
+            P = Pn;
+        }
+        const float y = creduce<NG, C::CW>(p, g);
+        const int t = tb + g;
+        if (write) IO<T>::store(out, (int64_t)t * out_stride, sgt[t * C::DC + cw] * fmaf(dskc, sdx[t * C::DC + cw].y, y));
     }
 }
 
@@ -248,19 +318,21 @@ __device__ __forceinline__ void scan_tile_c(CLane<CG>& s, const float2* sdx, con
 // checkpoint test out of the output kernel's loop.  TMA: the tiles come through the
 // TMA ring (maps m[0..4] = u, delta_raw, z, B, C; bc_tma says whether B and C do);
 // otherwise every thread loads them directly.
-template <typename T, int NG, int CG, bool CKPT, bool TMA>
+template <typename T, int NG, int CG, int TT, bool CKPT, bool TMA>
 __global__ void __launch_bounds__(kCThreads)
     fwd_complex_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dr,
                        const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_B,
                        const __grid_constant__ CUtensorMap tm_C, ComplexArgs a, float* ckpt, int64_t nck,
                        int bc_tma) {
     using C = CCfg<NG, CG>;
-    using R = CRing<T, NG, CG>;
-    __shared__ float2 sdx[kCTT * C::DC];  // (delta, x)
-    __shared__ float2 sgd[kCTT * C::DC];  // (gate, D x gate)
-    __shared__ __align__(16) float sB[kCTT * C::NS];
-    __shared__ __align__(16) float sC[kCTT * C::NS];
-    extern __shared__ __align__(128) unsigned char ring[];
+    using S = CSmem<T, NG, CG, TT>;
+    using P2 = typename std::conditional<sizeof(T) == 2, __nv_bfloat162, float2>::type;
+    extern __shared__ __align__(128) unsigned char smem[];
+    float2* sdx = reinterpret_cast<float2*>(smem + S::OFF_DX);  // (delta, x)
+    float* sgt = reinterpret_cast<float*>(smem + S::OFF_GT);    // SiLU gate
+    float* sB = reinterpret_cast<float*>(smem + S::OFF_B);
+    float* sC = reinterpret_cast<float*>(smem + S::OFF_C);
+    unsigned char* ring = smem + S::OFF_RING;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t ncb = (a.D + C::DC - 1) / C::DC;
     const int64_t b = blockIdx.x / ncb;
@@ -271,32 +343,32 @@ __global__ void __launch_bounds__(kCThreads)
     const T* zz = static_cast<const T*>(a.z);
     const T* Bg = static_cast<const T*>(a.B);
     const T* Cg = static_cast<const T*>(a.C);
-    const int ntile = (int)((a.L + kCTT - 1) / kCTT);
+    const int ntile = (int)((a.L + TT - 1) / TT);
     const bool has_z = zz != nullptr;
-    const uint32_t bar0 = TMA ? smem_u32(ring + R::OFF_BAR) : 0u;
-    const uint32_t stage_bytes = (has_z ? 3u : 2u) * R::RAW + (bc_tma ? 2u * (uint32_t)(kCTT * N * (int)sizeof(T)) : 0u);
+    const uint32_t bar0 = TMA ? smem_u32(smem + S::OFF_BAR) : 0u;
+    const uint32_t stage_bytes = (has_z ? 3u : 2u) * S::RAW + (bc_tma ? 2u * (uint32_t)(TT * N * (int)sizeof(T)) : 0u);
 
     // the TMA copies of tile `it` into its ring stage (elected thread only)
     auto issue = [&](int it) {
-        const int st = it % R::STAGES;
+        const int st = it % S::STAGES;
         const uint32_t bar = bar0 + 8 * st;
-        const uint32_t base = smem_u32(ring + st * R::STAGE);
-        const int t0 = it * kCTT;
+        const uint32_t base = smem_u32(ring + st * S::STAGE);
+        const int t0 = it * TT;
         mbar_expect_tx(bar, stage_bytes);
         tma_load_3d(base, &tm_u, (int)d0, t0, (int)b, bar);
-        tma_load_3d(base + R::RAW, &tm_dr, (int)d0, t0, (int)b, bar);
-        if (has_z) tma_load_3d(base + 2 * R::RAW, &tm_z, (int)d0, t0, (int)b, bar);
+        tma_load_3d(base + S::RAW, &tm_dr, (int)d0, t0, (int)b, bar);
+        if (has_z) tma_load_3d(base + 2 * S::RAW, &tm_z, (int)d0, t0, (int)b, bar);
         if (bc_tma) {
-            tma_load_3d(base + 3 * R::RAW, &tm_B, 0, t0, (int)b, bar);
-            tma_load_3d(base + 3 * R::RAW + R::RAWBC, &tm_C, 0, t0, (int)b, bar);
+            tma_load_3d(base + 3 * S::RAW, &tm_B, 0, t0, (int)b, bar);
+            tma_load_3d(base + 3 * S::RAW + S::RAWBC, &tm_C, 0, t0, (int)b, bar);
         }
     };
     int bad = 0;
     if constexpr (TMA) {
         if (tid == 0) {
-            for (int st = 0; st < R::STAGES; ++st) mbar_init(bar0 + 8 * st, 1);
+            for (int st = 0; st < S::STAGES; ++st) mbar_init(bar0 + 8 * st, 1);
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-            for (int it = 0; it < R::STAGES && it < ntile; ++it) issue(it);
+            for (int it = 0; it < S::STAGES && it < ntile; ++it) issue(it);
         }
     }
 
@@ -322,50 +394,54 @@ __global__ void __launch_bounds__(kCThreads)
         comp(s.hr, j) = h0v ? __ldg(a.h0 + ((b * a.D + d) * N + n) * 2) : 0.f;
         comp(s.hi, j) = h0v ? __ldg(a.h0 + ((b * a.D + d) * N + n) * 2 + 1) : 0.f;
     }
+    // skip weight D of this lane's channel (the epilogue forms gate (y + D x))
+    const float dskc = (!CKPT && a.Dskip && cvalid) ? __ldg(a.Dskip + d) : 0.f;
     if (TMA && tid == 0 && ntile > 0) bad = !mbar_wait(bar0, 0);
     const int flags = __syncthreads_or((small_a ? 1 : 0) | (bad ? 2 : 0));
     const bool acc = (flags & 1) != 0;
     bool failed = (flags & 2) != 0;
     const int nvalid = cvalid ? (N - g * CG < CG ? N - g * CG : CG) : 0;
+    // phase-P channel pair of this thread (fixed: PAIRS is a multiple of the thread count)
+    const int pc = 2 * (tid % (C::DC / 2));
+    const int64_t pd = d0 + pc;
+    const float2 pbias = make_float2((a.bias && pd < a.D) ? __ldg(a.bias + pd) : 0.f,
+                                     (a.bias && pd + 1 < a.D) ? __ldg(a.bias + pd + 1) : 0.f);
 
     for (int it = 0; it < ntile && !failed; ++it) {
-        const int64_t t0 = (int64_t)it * kCTT;
-        const int tl = (int)(a.L - t0 < kCTT ? a.L - t0 : kCTT);
-        const unsigned char* raw = ring + (it % R::STAGES) * R::STAGE;
-        // phase P: (delta, x), (gate, D x gate), and the tile's B and C rows
-        for (int e = tid; e < kCTT * C::DC; e += kCThreads) {
-            const int t = e / C::DC, cc = e % C::DC;
-            const int64_t dd = d0 + cc;
-            float2 dx = make_float2(0.f, 0.f), gd = make_float2(0.f, 0.f);
-            if (t < tl && dd < a.D) {
-                float uv, rv, zv = 0.f;
-                if constexpr (TMA) {
-                    uv = to_f32<T>(reinterpret_cast<const T*>(raw)[e]);
-                    rv = to_f32<T>(reinterpret_cast<const T*>(raw + R::RAW)[e]);
-                    if (has_z) zv = to_f32<T>(reinterpret_cast<const T*>(raw + 2 * R::RAW)[e]);
-                } else {
-                    const int64_t gi = (b * a.L + t0 + t) * a.D + dd;
-                    uv = IO<T>::load(u, gi);
-                    rv = IO<T>::load(dr, gi);
-                    if (has_z) zv = IO<T>::load(zz, gi);
-                }
-                const float x = a.input_silu ? silu(uv) : uv;
-                const float r = rv + (a.bias ? __ldg(a.bias + dd) : 0.f);
-                const float gate = has_z ? silu(zv) : 1.f;
-                const float dsk = a.Dskip ? __ldg(a.Dskip + dd) : 0.f;
-                dx = make_float2(a.softplus ? softplus(r) : r, x);
-                gd = make_float2(gate, dsk * x * gate);
+        const int64_t t0 = (int64_t)it * TT;
+        const int tl = (int)(a.L - t0 < TT ? a.L - t0 : TT);
+        const unsigned char* raw = ring + (it % S::STAGES) * S::STAGE;
+        // phase P: (delta, x) pairs and the gate of two channels per thread and row, packed
+#pragma unroll
+        for (int qi = 0; qi < S::PAIRS / kCThreads; ++qi) {
+            const int q = tid + qi * kCThreads;
+            const int t = q / (C::DC / 2);
+            float2 uv, rv, zv = make_float2(0.f, 0.f);
+            if constexpr (TMA) {
+                uv = to_f32x2(reinterpret_cast<const P2*>(raw)[q]);
+                rv = to_f32x2(reinterpret_cast<const P2*>(raw + S::RAW)[q]);
+                if (has_z) zv = to_f32x2(reinterpret_cast<const P2*>(raw + 2 * S::RAW)[q]);
+            } else {
+                const int64_t gi = (b * a.L + t0 + t) * a.D + pd;
+                const bool v0 = t < tl && pd < a.D, v1 = t < tl && pd + 1 < a.D;
+                uv = make_float2(v0 ? IO<T>::load(u, gi) : 0.f, v1 ? IO<T>::load(u, gi + 1) : 0.f);
+                rv = make_float2(v0 ? IO<T>::load(dr, gi) : 0.f, v1 ? IO<T>::load(dr, gi + 1) : 0.f);
+                if (has_z) zv = make_float2(v0 ? IO<T>::load(zz, gi) : 0.f, v1 ? IO<T>::load(zz, gi + 1) : 0.f);
             }
-            sdx[e] = dx;
-            sgd[e] = gd;
+            const float2 x = a.input_silu ? silu_x2(uv) : uv;
+            float2 dl = __fadd2_rn(rv, pbias);
+            if (a.softplus) dl = softplus_x2(dl);
+            const float2 gt = has_z ? silu_x2(zv) : make_float2(1.f, 1.f);
+            reinterpret_cast<float4*>(sdx)[(t * C::DC + pc) / 2] = make_float4(dl.x, x.x, dl.y, x.y);
+            reinterpret_cast<float2*>(sgt)[(t * C::DC + pc) / 2] = gt;
         }
-        for (int e = tid; e < kCTT * C::NS; e += kCThreads) {
+        for (int e = tid; e < TT * C::NS; e += kCThreads) {
             const int t = e / C::NS, n = e % C::NS;
             float bv = 0.f, cv = 0.f;
             if (t < tl && n < N) {
                 if (TMA && bc_tma) {
-                    bv = to_f32<T>(reinterpret_cast<const T*>(raw + 3 * R::RAW)[t * N + n]);
-                    cv = to_f32<T>(reinterpret_cast<const T*>(raw + 3 * R::RAW + R::RAWBC)[t * N + n]);
+                    bv = to_f32<T>(reinterpret_cast<const T*>(raw + 3 * S::RAW)[t * N + n]);
+                    cv = to_f32<T>(reinterpret_cast<const T*>(raw + 3 * S::RAW + S::RAWBC)[t * N + n]);
                 } else {
                     const int64_t gi = (b * a.L + t0 + t) * N + n;
                     bv = IO<T>::load(Bg, gi);
@@ -378,30 +454,32 @@ __global__ void __launch_bounds__(kCThreads)
         if constexpr (TMA) fence_proxy_async();
         __syncthreads();
         // the stage just consumed takes the tile two ahead
-        if (TMA && tid == 0 && it + R::STAGES < ntile) issue(it + R::STAGES);
+        if (TMA && tid == 0 && it + S::STAGES < ntile) issue(it + S::STAGES);
         T* out = CKPT ? nullptr : static_cast<T*>(a.out) + (b * a.L + t0) * a.D + d;
         float* ck = CKPT ? ckpt + (((b * nck + t0 / 8) * a.D + d) * N + g * CG) * 2 : nullptr;
         const int64_t ck_stride = a.D * N * 2;
         const bool wr = cvalid;
         if (acc)
-            scan_tile_c<T, NG, CG, true, CKPT, false>(s, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
-                                                      nvalid);
-        else if (tl == kCTT)
-            scan_tile_c<T, NG, CG, false, CKPT, true>(s, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
-                                                      nvalid);
+            scan_tile_c<T, NG, CG, TT, true, CKPT, false>(s, sdx, sgt, sB, sC, tl, g, cw, wr, out, a.D, dskc, ck,
+                                                          ck_stride, nvalid);
+        else if (!CKPT && tl == TT)
+            scan_tile_c_pipe<T, NG, CG, TT>(s, sdx, sgt, sB, sC, g, cw, wr, out, a.D, dskc);
+        else if (tl == TT)
+            scan_tile_c<T, NG, CG, TT, false, CKPT, true>(s, sdx, sgt, sB, sC, tl, g, cw, wr, out, a.D, dskc, ck,
+                                                          ck_stride, nvalid);
         else
-            scan_tile_c<T, NG, CG, false, CKPT, false>(s, sdx, sgd, sB, sC, tl, g, cw, wr, out, a.D, ck, ck_stride,
-                                                       nvalid);
+            scan_tile_c<T, NG, CG, TT, false, CKPT, false>(s, sdx, sgt, sB, sC, tl, g, cw, wr, out, a.D, dskc, ck,
+                                                           ck_stride, nvalid);
         // the next tile's raw data (or a wait that gave up); shared memory free again
         if (TMA && tid == 0 && it + 1 < ntile)
-            bad = !mbar_wait(bar0 + 8 * ((it + 1) % R::STAGES), ((it + 1) / R::STAGES) & 1);
+            bad = !mbar_wait(bar0 + 8 * ((it + 1) % S::STAGES), ((it + 1) / S::STAGES) & 1);
         failed = __syncthreads_or(bad) != 0;
     }
     if (failed) {
         if (tid == 0) {
             atomicOr(&g_device_error_cx, 1u);
             // let the copies still in flight land before the CTA's shared memory is released
-            for (int st = 0; st < R::STAGES; ++st) (void)mbar_wait(bar0 + 8 * st, 0), (void)mbar_wait(bar0 + 8 * st, 1);
+            for (int st = 0; st < S::STAGES; ++st) (void)mbar_wait(bar0 + 8 * st, 0), (void)mbar_wait(bar0 + 8 * st, 1);
         }
         return;
     }
@@ -417,9 +495,9 @@ __global__ void __launch_bounds__(kCThreads)
     }
 }
 
-// 3-D map over a (batch, L, W) tensor, box [1][kCTT][box_w], zero fill outside.
+// 3-D map over a (batch, L, W) tensor, box [1][rows][box_w], zero fill outside.
 template <typename T>
-bool make_map_c(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int64_t W, int box_w) {
+bool make_map_c(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int64_t W, int box_w, int rows) {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
         void* p = nullptr;
@@ -431,7 +509,7 @@ bool make_map_c(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int6
     }
     const cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)L, (cuuint64_t)batch};
     const cuuint64_t strides[2] = {(cuuint64_t)(W * sizeof(T)), (cuuint64_t)(L * W * sizeof(T))};
-    const cuuint32_t box[3] = {(cuuint32_t)box_w, (cuuint32_t)kCTT, 1};
+    const cuuint32_t box[3] = {(cuuint32_t)box_w, (cuuint32_t)rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapDataType ty =
         sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
@@ -442,29 +520,31 @@ bool make_map_c(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int6
 
 bool aligned16c(const void* q) { return q == nullptr || reinterpret_cast<uintptr_t>(q) % 16 == 0; }
 
-template <typename T, int NG, int CG, bool CKPT, bool TMA>
+template <typename T, int NG, int CG, int TT, bool CKPT, bool TMA>
 cudaError_t launch_ck(const CUtensorMap (&m)[5], const ComplexArgs& a, float* ckpt, int64_t nck, int bc_tma,
                       int64_t blocks, cudaStream_t st) {
-    using R = CRing<T, NG, CG>;
-    auto kern = fwd_complex_kernel<T, NG, CG, CKPT, TMA>;
-    const int smem = TMA ? R::SMEM : 0;
-    if (TMA) {
-        // function attributes are per device: set them once on each device used
-        static bool configured[kMaxDevices] = {};
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-        if (!configured[dev]) {
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            configured[dev] = true;
-        }
+    using S = CSmem<T, NG, CG, TT>;
+    auto kern = fwd_complex_kernel<T, NG, CG, TT, CKPT, TMA>;
+    const int smem = TMA ? S::SMEM_TMA : S::SMEM_PLAIN;
+    // function attributes are per device: set them once on each device used
+    static bool configured[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        configured[dev] = true;
     }
     kern<<<(unsigned)blocks, kCThreads, smem, st>>>(m[0], m[1], m[2], m[3], m[4], a, ckpt, nck, bc_tma);
     return cudaGetLastError();
 }
 
+// Tiles of 32 steps: at the Mamba-130M shape 0.592 ms with 16-step tiles, 0.572 ms with 32
+// and 0.597 ms with 64 (then 5 CTAs per SM for the 768-CTA grid); the backward through its
+// checkpoint pass 3.670 / 3.635 / 3.615 ms.
 template <typename T, int NG, int CG>
 cudaError_t launch_c(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream_t st) {
     using C = CCfg<NG, CG>;
+    constexpr int TT = 32;
     const int64_t blocks = a.batch * ((a.D + C::DC - 1) / C::DC);
     if (blocks <= 0) return cudaGetLastError();
     // the TMA ring needs 16-byte aligned bases and row pitches of the (batch, L, D) tensors
@@ -473,23 +553,23 @@ cudaError_t launch_c(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream_
                aligned16c(a.z) && a.L < (int64_t(1) << 31) && a.D < (int64_t(1) << 31);
     int bc_tma = 0;
     if (tma) {
-        tma = make_map_c<T>(&m[0], a.u, a.batch, a.L, a.D, C::DC) &&
-              make_map_c<T>(&m[1], a.delta_raw, a.batch, a.L, a.D, C::DC) &&
-              make_map_c<T>(&m[2], a.z ? a.z : a.u, a.batch, a.L, a.D, C::DC);
+        tma = make_map_c<T>(&m[0], a.u, a.batch, a.L, a.D, C::DC, TT) &&
+              make_map_c<T>(&m[1], a.delta_raw, a.batch, a.L, a.D, C::DC, TT) &&
+              make_map_c<T>(&m[2], a.z ? a.z : a.u, a.batch, a.L, a.D, C::DC, TT);
         // B and C rows by TMA when a row of N values is a whole number of 16-byte units
         if (tma && (a.N * (int64_t)sizeof(T)) % 16 == 0 && aligned16c(a.B) && aligned16c(a.C) &&
-            make_map_c<T>(&m[3], a.B, a.batch, a.L, a.N, a.N) && make_map_c<T>(&m[4], a.C ? a.C : a.B, a.batch, a.L, a.N, a.N))
+            make_map_c<T>(&m[3], a.B, a.batch, a.L, a.N, a.N, TT) && make_map_c<T>(&m[4], a.C ? a.C : a.B, a.batch, a.L, a.N, a.N, TT))
             bc_tma = 1;
         else
             m[3] = m[4] = m[0];
     }
     if (!tma) {
         std::memset(m, 0, sizeof m);
-        return ckpt ? launch_ck<T, NG, CG, true, false>(m, a, ckpt, nck, 0, blocks, st)
-                    : launch_ck<T, NG, CG, false, false>(m, a, nullptr, 0, 0, blocks, st);
+        return ckpt ? launch_ck<T, NG, CG, TT, true, false>(m, a, ckpt, nck, 0, blocks, st)
+                    : launch_ck<T, NG, CG, TT, false, false>(m, a, nullptr, 0, 0, blocks, st);
     }
-    return ckpt ? launch_ck<T, NG, CG, true, true>(m, a, ckpt, nck, bc_tma, blocks, st)
-                : launch_ck<T, NG, CG, false, true>(m, a, nullptr, 0, bc_tma, blocks, st);
+    return ckpt ? launch_ck<T, NG, CG, TT, true, true>(m, a, ckpt, nck, bc_tma, blocks, st)
+                : launch_ck<T, NG, CG, TT, false, true>(m, a, nullptr, 0, bc_tma, blocks, st);
 }
 
 // Four complex states per lane, or two (twice the lanes per channel, half the
