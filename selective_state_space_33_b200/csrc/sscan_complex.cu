@@ -7,12 +7,12 @@
 //
 // Work decomposition (as the real tiled kernel): a CTA of 4 warps owns one batch
 // and DC channels for the whole sequence; the NG lanes of a channel each hold CG
-// complex states (CG = 4, or 2 when the grid is small) in registers.  Per 16-step
+// complex states (CG = 4, or 2 when the grid is small) in registers.  Per 32-step
 // tile, TMA 3-D tile copies bring u, delta_raw, z (and the B, C rows) into a 2-stage
 // shared-memory ring -- the next tile's copy lands while the current one is scanned;
 // mbarrier completion, every wait bounded -- or, for tensors whose rows or bases are
 // not 16-byte aligned, every thread loads them directly; all threads then stage
-// (delta, x) and (gate, D x gate) for the tile's channels and the tile's B and C rows
+// (delta, x) pairs and the gate for the tile's channels and the tile's B and C rows
 // in shared memory (phase P), then every lane
 // advances its states through the tile (phase S), two states per f32x2 operation, and
 // the NG lanes of a channel sum their partial readouts over blocks of NG steps with a

@@ -26,19 +26,19 @@ __device__ __forceinline__ float cos_approx(float x) {
 // leaves no fraction bits for |p| < 2^22, so the sum is rounded to an integer (ties to
 // even, as rintf) and subtracting the constant again is exact.  __fadd_rn keeps the
 // compiler from contracting the additions into an fma with the product that forms p.
-// |p| is clamped to 2^22 first: beyond that the fp32 angle has no fraction of a turn
-// left to resolve, and the clamp keeps the result a valid (if partial) reduction.
+// Beyond |p| = 2^22 the sum keeps no fraction bit and the turn count is not the nearest
+// integer (for -2^23 < p <= -2^22 it may be off by half a turn); such an angle exceeds
+// 2.6e7 rad, where the fp32 angle itself carries an error of a radian or more, so no
+// reduction could give its sine.  (A clamp of p to 2^22 cost 5% of the complex forward.)
 __device__ __forceinline__ float round_fma(float p) {
     constexpr float kShift = 12582912.f;  // 1.5 * 2^23
-    const float pc = fminf(fmaxf(p, -4194304.f), 4194304.f);
-    return __fadd_rn(__fadd_rn(pc, kShift), -kShift);
+    return __fadd_rn(__fadd_rn(p, kShift), -kShift);
 }
 
-// round_fma for two values with packed adds (the clamp stays per component).
+// round_fma for two values with packed adds.
 __device__ __forceinline__ float2 round2_fma(float2 p) {
     constexpr float kShift = 12582912.f;
-    const float2 pc = make_float2(fminf(fmaxf(p.x, -4194304.f), 4194304.f), fminf(fmaxf(p.y, -4194304.f), 4194304.f));
-    return __fadd2_rn(__fadd2_rn(pc, make_float2(kShift, kShift)), make_float2(-kShift, -kShift));
+    return __fadd2_rn(__fadd2_rn(p, make_float2(kShift, kShift)), make_float2(-kShift, -kShift));
 }
 
 // cos and sin of an angle of any size: reduce by a multiple of 2 pi first.
