@@ -32,7 +32,7 @@ def _run(x, io, dev, h0=None, A=None):
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("shape", [(2, 100, 37, 16), (1, 257, 8, 4), (3, 33, 5, 1), (2, 64, 40, 7),
-                                   (1, 40, 130, 16)])
+                                   (1, 40, 130, 16), (2, 50, 136, 2)])
 def test_complex_shapes_and_tails(cuda_device, io, shape):
     x = W.small_case(*shape, io=io, seed=sum(shape) + 5, complex_a=True)
     h0 = np.random.default_rng(3).standard_normal((shape[0], shape[2], shape[3], 2)) @ np.array([1.0, 1j]) * 0.5
@@ -215,7 +215,8 @@ def _check_complex_bwd(x, io, dev, A=None, h0=None, tol=None):
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
-@pytest.mark.parametrize("shape", [(2, 100, 37, 16), (1, 70, 8, 4), (3, 33, 5, 1), (2, 64, 40, 7), (1, 45, 130, 16)])
+@pytest.mark.parametrize("shape", [(2, 100, 37, 16), (1, 70, 8, 4), (3, 33, 5, 1), (2, 64, 40, 7), (1, 45, 130, 16),
+                                   (2, 50, 136, 2)])
 def test_complex_backward_small(cuda_device, io, shape):
     x = W.small_case(*shape, io=io, seed=sum(shape) + 9, backward=True, complex_a=True)
     h0 = np.random.default_rng(4).standard_normal((shape[0], shape[2], shape[3], 2)) @ np.array([1.0, 1j]) * 0.5
