@@ -57,9 +57,10 @@ struct CCfg {
 };
 
 // Dynamic shared memory of a TT-step tile: phase P's staging -- (delta, x) pairs and the
-// SiLU gate per (step, channel), the tile's B and C rows -- then, on the TMA path, a
-// 2-stage ring of raw tiles (u, delta_raw, z, then B and C when their rows travel by
-// TMA) and its mbarriers; 128-byte aligned sections.
+// SiLU gate per (step, channel), the tile's B and C rows -- and, on the TMA path, the
+// output tile (written back by one TMA store per tile), a 2-stage ring of raw tiles (u,
+// delta_raw, z, then B and C when their rows travel by TMA) and its mbarriers;
+// 128-byte aligned sections.
 template <typename T, int NG, int CG, int TT>
 struct CSmem {
     static constexpr int DC = CCfg<NG, CG>::DC, NS = CCfg<NG, CG>::NS;
@@ -67,7 +68,8 @@ struct CSmem {
     static constexpr int OFF_GT = OFF_DX + TT * DC * 8;                          // float  [TT][DC]
     static constexpr int OFF_B = OFF_GT + (TT * DC * 4 + 127) / 128 * 128;       // float  [TT][NS]
     static constexpr int OFF_C = OFF_B + (TT * NS * 4 + 127) / 128 * 128;        // float  [TT][NS]
-    static constexpr int OFF_RING = OFF_C + (TT * NS * 4 + 127) / 128 * 128;
+    static constexpr int OFF_OUT = OFF_C + (TT * NS * 4 + 127) / 128 * 128;    // T [TT][DC] (TMA path)
+    static constexpr int OFF_RING = OFF_OUT + (TT * DC * (int)sizeof(T) + 127) / 128 * 128;
     static constexpr int RAW = TT * DC * (int)sizeof(T);
     static constexpr int RAWBC = (TT * NS * (int)sizeof(T) + 127) / 128 * 128;  // one B or C tile (N <= NS)
     static constexpr int STAGE = (3 * RAW + 2 * RAWBC + 127) / 128 * 128;
@@ -322,10 +324,11 @@ template <typename T, int NG, int CG, int TT, bool CKPT, bool TMA>
 __global__ void __launch_bounds__(kCThreads)
     fwd_complex_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dr,
                        const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_B,
-                       const __grid_constant__ CUtensorMap tm_C, ComplexArgs a, float* ckpt, int64_t nck,
-                       int bc_tma) {
+                       const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_out,
+                       ComplexArgs a, float* ckpt, int64_t nck, int bc_tma) {
     using C = CCfg<NG, CG>;
     using S = CSmem<T, NG, CG, TT>;
+    constexpr bool kTileOut = TMA && !CKPT;  // outputs through a shared tile and a TMA store
     using P2 = typename std::conditional<sizeof(T) == 2, __nv_bfloat162, float2>::type;
     extern __shared__ __align__(128) unsigned char smem[];
     float2* sdx = reinterpret_cast<float2*>(smem + S::OFF_DX);  // (delta, x)
@@ -452,29 +455,36 @@ __global__ void __launch_bounds__(kCThreads)
             sC[e] = cv;
         }
         if constexpr (TMA) fence_proxy_async();
+        // the previous tile's output store must have read the output tile
+        if (kTileOut && tid == 0) tma_store_wait_read_0();
         __syncthreads();
         // the stage just consumed takes the tile two ahead
         if (TMA && tid == 0 && it + S::STAGES < ntile) issue(it + S::STAGES);
-        T* out = CKPT ? nullptr : static_cast<T*>(a.out) + (b * a.L + t0) * a.D + d;
+        T* const otile = reinterpret_cast<T*>(smem + S::OFF_OUT);
+        T* out = CKPT ? nullptr : kTileOut ? otile + cw : static_cast<T*>(a.out) + (b * a.L + t0) * a.D + d;
+        const int64_t ostride = kTileOut ? C::DC : a.D;
         float* ck = CKPT ? ckpt + (((b * nck + t0 / 8) * a.D + d) * N + g * CG) * 2 : nullptr;
         const int64_t ck_stride = a.D * N * 2;
-        const bool wr = cvalid;
+        const bool wr = kTileOut || cvalid;  // the TMA store drops columns past D
         if (acc)
-            scan_tile_c<T, NG, CG, TT, true, CKPT, false>(s, sdx, sgt, sB, sC, tl, g, cw, wr, out, a.D, dskc, ck,
+            scan_tile_c<T, NG, CG, TT, true, CKPT, false>(s, sdx, sgt, sB, sC, tl, g, cw, wr, out, ostride, dskc, ck,
                                                           ck_stride, nvalid);
         else if (!CKPT && tl == TT)
-            scan_tile_c_pipe<T, NG, CG, TT>(s, sdx, sgt, sB, sC, g, cw, wr, out, a.D, dskc);
+            scan_tile_c_pipe<T, NG, CG, TT>(s, sdx, sgt, sB, sC, g, cw, wr, out, ostride, dskc);
         else if (tl == TT)
-            scan_tile_c<T, NG, CG, TT, false, CKPT, true>(s, sdx, sgt, sB, sC, tl, g, cw, wr, out, a.D, dskc, ck,
+            scan_tile_c<T, NG, CG, TT, false, CKPT, true>(s, sdx, sgt, sB, sC, tl, g, cw, wr, out, ostride, dskc, ck,
                                                           ck_stride, nvalid);
         else
-            scan_tile_c<T, NG, CG, TT, false, CKPT, false>(s, sdx, sgt, sB, sC, tl, g, cw, wr, out, a.D, dskc, ck,
+            scan_tile_c<T, NG, CG, TT, false, CKPT, false>(s, sdx, sgt, sB, sC, tl, g, cw, wr, out, ostride, dskc, ck,
                                                            ck_stride, nvalid);
+        if constexpr (kTileOut) fence_proxy_async();
         // the next tile's raw data (or a wait that gave up); shared memory free again
         if (TMA && tid == 0 && it + 1 < ntile)
             bad = !mbar_wait(bar0 + 8 * ((it + 1) % S::STAGES), ((it + 1) / S::STAGES) & 1);
         failed = __syncthreads_or(bad) != 0;
+        if (kTileOut && tid == 0) tma_store_3d(&tm_out, (int)d0, (int)t0, (int)b, smem_u32(otile));
     }
+    if (kTileOut && tid == 0) tma_store_wait_all();
     if (failed) {
         if (tid == 0) {
             atomicOr(&g_device_error_cx, 1u);
@@ -521,7 +531,7 @@ bool make_map_c(CUtensorMap* m, const void* base, int64_t batch, int64_t L, int6
 bool aligned16c(const void* q) { return q == nullptr || reinterpret_cast<uintptr_t>(q) % 16 == 0; }
 
 template <typename T, int NG, int CG, int TT, bool CKPT, bool TMA>
-cudaError_t launch_ck(const CUtensorMap (&m)[5], const ComplexArgs& a, float* ckpt, int64_t nck, int bc_tma,
+cudaError_t launch_ck(const CUtensorMap (&m)[6], const ComplexArgs& a, float* ckpt, int64_t nck, int bc_tma,
                       int64_t blocks, cudaStream_t st) {
     using S = CSmem<T, NG, CG, TT>;
     auto kern = fwd_complex_kernel<T, NG, CG, TT, CKPT, TMA>;
@@ -534,7 +544,7 @@ cudaError_t launch_ck(const CUtensorMap (&m)[5], const ComplexArgs& a, float* ck
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         configured[dev] = true;
     }
-    kern<<<(unsigned)blocks, kCThreads, smem, st>>>(m[0], m[1], m[2], m[3], m[4], a, ckpt, nck, bc_tma);
+    kern<<<(unsigned)blocks, kCThreads, smem, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], a, ckpt, nck, bc_tma);
     return cudaGetLastError();
 }
 
@@ -547,15 +557,18 @@ cudaError_t launch_c(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream_
     constexpr int TT = 32;
     const int64_t blocks = a.batch * ((a.D + C::DC - 1) / C::DC);
     if (blocks <= 0) return cudaGetLastError();
-    // the TMA ring needs 16-byte aligned bases and row pitches of the (batch, L, D) tensors
-    CUtensorMap m[5];
+    // the TMA ring and the output store need 16-byte aligned bases and row pitches of the
+    // (batch, L, D) tensors
+    CUtensorMap m[6];
     bool tma = (a.D * (int64_t)sizeof(T)) % 16 == 0 && aligned16c(a.u) && aligned16c(a.delta_raw) &&
-               aligned16c(a.z) && a.L < (int64_t(1) << 31) && a.D < (int64_t(1) << 31);
+               aligned16c(a.z) && (ckpt != nullptr || aligned16c(a.out)) && a.L < (int64_t(1) << 31) &&
+               a.D < (int64_t(1) << 31);
     int bc_tma = 0;
     if (tma) {
         tma = make_map_c<T>(&m[0], a.u, a.batch, a.L, a.D, C::DC, TT) &&
               make_map_c<T>(&m[1], a.delta_raw, a.batch, a.L, a.D, C::DC, TT) &&
-              make_map_c<T>(&m[2], a.z ? a.z : a.u, a.batch, a.L, a.D, C::DC, TT);
+              make_map_c<T>(&m[2], a.z ? a.z : a.u, a.batch, a.L, a.D, C::DC, TT) &&
+              make_map_c<T>(&m[5], ckpt ? a.u : a.out, a.batch, a.L, a.D, C::DC, TT);
         // B and C rows by TMA when a row of N values is a whole number of 16-byte units
         if (tma && (a.N * (int64_t)sizeof(T)) % 16 == 0 && aligned16c(a.B) && aligned16c(a.C) &&
             make_map_c<T>(&m[3], a.B, a.batch, a.L, a.N, a.N, TT) && make_map_c<T>(&m[4], a.C ? a.C : a.B, a.batch, a.L, a.N, a.N, TT))
