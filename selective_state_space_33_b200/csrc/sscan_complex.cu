@@ -7,8 +7,8 @@
 //
 // Work decomposition (as the real tiled kernel): a CTA of 4 warps owns one batch
 // and DC channels for the whole sequence; the NG lanes of a channel each hold CG
-// complex states (CG = 4, or 2 when the grid is small) in registers.  Per 32-step
-// tile, TMA 3-D tile copies bring u, delta_raw, z (and the B, C rows) into a 2-stage
+// complex states (CG = 4, or 2 when the grid is small) in registers.  Per 32- or 64-step
+// tile, TMA 3-D tile copies bring u, delta_raw, z (and the B, C rows) into a one-stage
 // shared-memory ring -- the next tile's copy lands while the current one is scanned;
 // mbarrier completion, every wait bounded -- or, for tensors whose rows or bases are
 // not 16-byte aligned, every thread loads them directly; all threads then stage
@@ -60,7 +60,10 @@ struct CCfg {
 // SiLU gate per (step, channel), the tile's B and C rows -- and, on the TMA path, the
 // output tile (written back by one TMA store per tile), a 2-stage ring of raw tiles (u,
 // delta_raw, z, then B and C when their rows travel by TMA) and its mbarriers;
-// 128-byte aligned sections.
+// 128-byte aligned sections.  One ring stage: phase P empties it before the next tile's
+// copy is issued, and the copy lands while the tile is scanned (at the Mamba-130M shape
+// 0.496 ms with two stages and 32-step tiles, 0.491 with one; 0.511 and 0.483 ms with
+// 64-step tiles).
 template <typename T, int NG, int CG, int TT>
 struct CSmem {
     static constexpr int DC = CCfg<NG, CG>::DC, NS = CCfg<NG, CG>::NS;
@@ -73,7 +76,7 @@ struct CSmem {
     static constexpr int RAW = TT * DC * (int)sizeof(T);
     static constexpr int RAWBC = (TT * NS * (int)sizeof(T) + 127) / 128 * 128;  // one B or C tile (N <= NS)
     static constexpr int STAGE = (3 * RAW + 2 * RAWBC + 127) / 128 * 128;
-    static constexpr int STAGES = 2;
+    static constexpr int STAGES = 1;  // the next tile's copy lands during this tile's scan
     static constexpr int OFF_BAR = OFF_RING + STAGES * STAGE;
     static constexpr int SMEM_PLAIN = OFF_RING;          // plain loads: no ring
     static constexpr int SMEM_TMA = OFF_BAR + STAGES * 8;
@@ -548,13 +551,9 @@ cudaError_t launch_ck(const CUtensorMap (&m)[6], const ComplexArgs& a, float* ck
     return cudaGetLastError();
 }
 
-// Tiles of 32 steps: at the Mamba-130M shape 0.592 ms with 16-step tiles, 0.572 ms with 32
-// and 0.597 ms with 64 (then 5 CTAs per SM for the 768-CTA grid); the backward through its
-// checkpoint pass 3.670 / 3.635 / 3.615 ms.
-template <typename T, int NG, int CG>
-cudaError_t launch_c(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream_t st) {
+template <typename T, int NG, int CG, int TT>
+cudaError_t launch_c_tt(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream_t st) {
     using C = CCfg<NG, CG>;
-    constexpr int TT = 32;
     const int64_t blocks = a.batch * ((a.D + C::DC - 1) / C::DC);
     if (blocks <= 0) return cudaGetLastError();
     // the TMA ring and the output store need 16-byte aligned bases and row pitches of the
@@ -583,6 +582,18 @@ cudaError_t launch_c(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream_
     }
     return ckpt ? launch_ck<T, NG, CG, TT, true, true>(m, a, ckpt, nck, bc_tma, blocks, st)
                 : launch_ck<T, NG, CG, TT, false, true>(m, a, nullptr, 0, bc_tma, blocks, st);
+}
+
+// Steps per tile: 64 when the whole grid fits the GPU at once with 64-step tiles, else 32
+// (at the Mamba-130M shape, one ring stage: 0.491 ms with 32-step tiles, 0.483 with 64;
+// with two stages 0.592 / 0.572 / 0.597 ms for 16 / 32 / 64 before the output tile).
+template <typename T, int NG, int CG>
+cudaError_t launch_c(const ComplexArgs& a, float* ckpt, int64_t nck, cudaStream_t st) {
+    using C = CCfg<NG, CG>;
+    const int64_t blocks = a.batch * ((a.D + C::DC - 1) / C::DC);
+    const int64_t fit64 = kSmemPerSm / (CSmem<T, NG, CG, 64>::SMEM_TMA + kSmemPerCtaReserved);
+    if (blocks <= fit64 * kSmCount) return launch_c_tt<T, NG, CG, 64>(a, ckpt, nck, st);
+    return launch_c_tt<T, NG, CG, 32>(a, ckpt, nck, st);
 }
 
 // Four complex states per lane, or two (twice the lanes per channel, half the
