@@ -282,10 +282,14 @@ __device__ __forceinline__ void scan_tile_any(LaneG<G>& s, unsigned char* smem, 
                                                   ck_base, ck_extent);
 }
 
-template <int G> struct Occupancy { static constexpr int kCtas = G == 4 ? 9 : 5; };
+// Register budget (resident CTAs per SM the launch bound asks for): 9 for 4-state lanes,
+// except with 64-step tiles, which are launched only when at most 4 CTAs per SM are needed
+// and then get the registers of 4 (117, no spills: 0.2070 against 0.2107 ms at the
+// Mamba-130M shape); 5 for the 8-state lanes.
+template <int G, int TT> struct Occupancy { static constexpr int kCtas = G == 4 ? (TT == 64 ? 4 : 9) : 5; };
 
 template <typename T, int NG, int G, int MODE, int TT>
-__global__ void __launch_bounds__(kThreads, Occupancy<G>::kCtas)
+__global__ void __launch_bounds__(kThreads, Occupancy<G, TT>::kCtas)
     fwd_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dr,
                      const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_out,
                      const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -602,7 +606,8 @@ template <typename T, int NG, int G>
 cudaError_t launch_geom(const TiledArgs& a, const TiledPtrs& p, int mode, cudaStream_t st) {
     if (mode == kTiledCkpt) return launch_mode<T, NG, G, kCkpt, 32>(a, p, st);
     const int64_t ctas = a.batch * a.nchunks * ((a.D + 32 / NG * kWarps - 1) / (32 / NG * kWarps));
-    const int64_t fit64 = kSmemPerSm / (Cfg<T, NG, G, kOut, 64>::SMEM + kSmemPerCtaReserved);
+    const int64_t fit64_smem = kSmemPerSm / (Cfg<T, NG, G, kOut, 64>::SMEM + kSmemPerCtaReserved);
+    const int64_t fit64 = fit64_smem < Occupancy<G, 64>::kCtas ? fit64_smem : Occupancy<G, 64>::kCtas;
     if (ctas <= fit64 * kSmCount) {
         if (mode == kTiledOut) return launch_mode<T, NG, G, kOut, 64>(a, p, st);
         if (mode == kTiledAgg) return launch_mode<T, NG, G, kAgg, 64>(a, p, st);
