@@ -561,7 +561,8 @@ def gpu_arm(args, w: W.Workload):
     if world == 1 and args.workload == DEFAULT_WORKLOAD and not args.no_secondary:
         del t
         secondary = fp32_record(args, lib, dev)
-        others = [other_record(args, W.WORKLOADS[name]) for name in ("mamba130m", "bwd130m", "complex130m", "million")]
+        others = [other_record(args, W.WORKLOADS[name])
+                  for name in ("mamba130m", "bwd130m", "complex130m", "complexbwd130m", "million")]
     finish(args, w, x, lib, dev, torch, units, value, max_s, per_launch_ms, clk, e2e_value, h2d, d2h,
            launches_per_step, world, l2_note, out=out if not (w.backward or w.decode or w.complex_a) else None,
            secondary=secondary, others=others)
@@ -584,12 +585,18 @@ def other_record(args, w: W.Workload) -> dict:
     ws = torch.empty(max(sb.sscan_workspace_size(prob, op), 256), dtype=torch.uint8, device=dev)
     out = torch.empty_like(t["u"])
     grads = None
-    if w.backward:
+    if w.backward and not w.complex_a:
         grads = sb.sscan_bwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t["delta_bias"],
                              t["D_skip"], t["z"], workspace=ws)
+    elif w.backward:
+        cws = torch.empty(max(sb.sscan_workspace_size(prob, sb.SSCAN_OP_BWD_COMPLEX), 256), dtype=torch.uint8,
+                          device=dev)
 
     def step():
-        if w.backward:
+        if w.backward and w.complex_a:
+            sb.sscan_bwd_complex(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t["delta_bias"],
+                                 t["D_skip"], t.get("z"), workspace=cws, stream=st)
+        elif w.backward:
             sb.sscan_bwd(t["u"], t["delta_raw"], t["A"], t["B"], t["C"], t["dout"], t["delta_bias"], t["D_skip"],
                          t["z"], grads=grads, workspace=ws, stream=st)
         elif w.complex_a:
@@ -614,7 +621,8 @@ def other_record(args, w: W.Workload) -> dict:
     units = roofline_units(w)
     mufu = SM_COUNT * MUFU_PER_SM_CLK * float(measured_peaks().get("sm_max_mhz", 1965.0)) * 1e6
     rec = {"workload": f"{w.name}: {w.description}", "io_dtype": w.io,
-           "metric": METRIC_BWD if w.backward else (METRIC_COMPLEX if w.complex_a else METRIC_FWD),
+           "metric": ((METRIC_COMPLEX_BWD if w.complex_a else METRIC_BWD) if w.backward
+                      else (METRIC_COMPLEX if w.complex_a else METRIC_FWD)),
            "value": aggregate(units["elements"], steps, 1, total), "unit": UNIT, "steps": steps,
            "ms_per_step": total / steps * 1e3,
            "roofline": {"bound": "alu", "pipe": "MUFU (ex2, sin, cos)" if w.complex_a else "MUFU ex2",
