@@ -64,3 +64,40 @@ def test_cpu_sampler_repeats_a_quick_workload(bench):
     rate, threads, rows, secs, passes = bench.cpu_oracle_rate(x, w, 0.2, with_passes=True)
     assert rows == w.batch * w.dim and passes > 1 and rate > 0 and threads >= 1
     assert secs > 0.05
+
+
+def _parity_case(complex_a):
+    import dataclasses
+    base = W.WORKLOADS["complex130m" if complex_a else "mamba130m"]
+    return dataclasses.replace(base, batch=2, seqlen=40, dim=72, io="f32")
+
+
+@pytest.mark.parametrize("complex_a", [False, True])
+def test_parity_helpers_reproduce_the_oracle_and_catch_a_bad_row(bench, complex_a):
+    # The bench's parity record compares the timed output with the oracle on a row sample
+    # covering every 32-channel block.  Given the oracle's own full output (as fp32), both
+    # helpers report errors at fp32 rounding; a mistake planted in one sampled row (one
+    # channel of one batch row, the whole sequence) must fail the tolerance.
+    import numpy as np
+    import torch
+
+    import oracle
+    w = _parity_case(complex_a)
+    x = W.make_inputs(w)
+    kw = dict(delta_bias=x["delta_bias"], D_skip=x["D_skip"], z=x.get("z"))
+    if complex_a:
+        ref, _ = oracle.fwd_complex(x["u"], x["delta_raw"], x["A"], x["B"], x["C"], **kw)
+        check = bench.complex_oracle_parity
+    else:
+        ref, _ = oracle.fwd(x["u"], x["delta_raw"], x["A"], x["B"], x["C"], **kw)
+        check = bench.oracle_parity
+    out = torch.from_numpy(ref.astype(np.float32))
+    good = check(x, w, out)
+    assert good["ok"] and good["normwise"] < 1e-6, good
+    rows = bench.block_rows(w, 2, 77)
+    assert np.unique(rows % w.dim // 32).size == (w.dim + 31) // 32  # every channel block sampled
+    r = int(rows[len(rows) // 2])
+    bad_out = out.clone()
+    bad_out[r // w.dim, :, r % w.dim] += 0.01 * float(np.abs(ref).max())
+    bad = check(x, w, bad_out)
+    assert not bad["ok"] and bad["normwise"] > 1e-4, bad
