@@ -134,7 +134,10 @@ SSCAN_API sscan_status sscan_last_state(const sscan_problem* problem, const void
  * Scratch: a fixed 4 MiB array in the library's device memory (every GPU that
  * loads libsscan holds it until the process exits).  It covers every problem
  * whose (batch, L, D) tensors have 16-byte aligned bases and row pitches (the
- * TMA-tiled path needs at most 3.8 MB).  A call whose path needs more scratch
+ * TMA-tiled path needs at most 3.8 MB: this entry point splits a long sequence into
+ * fewer, longer chunks than sscan_fwd does, one wave of CTAs instead of several, so a
+ * split sequence can take somewhat longer here; results agree with sscan_fwd to the
+ * rounding of the chunk carries).  A call whose path needs more scratch
  * than that (possible only on the general path for unaligned tensors) returns
  * SSCAN_ERR_WORKSPACE before anything is launched.  The first call on each
  * device looks up the array's device address (cudaGetSymbolAddress, with that

@@ -154,9 +154,10 @@ bool tiled_ok(const sscan_problem* p, const sscan::ScanArgs& a) {
            aligned16(a.out) && p->seqlen < (int64_t(1) << 31) && p->dim < (int64_t(1) << 31);
 }
 
-sscan_status run_tiled(const sscan_problem* p, const sscan::ScanArgs& a, void* ws, cudaStream_t st) {
+sscan_status run_tiled(const sscan_problem* p, const sscan::ScanArgs& a, void* ws, cudaStream_t st,
+                       int64_t target) {
     const sscan::TiledGeom geo = sscan::tiled_geometry(p->batch, p->seqlen, p->dim, p->dstate);
-    const sscan::FwdPlan plan = sscan::plan_tiled(p->batch, p->seqlen, p->dim, p->dstate, geo.DC);
+    const sscan::FwdPlan plan = sscan::plan_tiled(p->batch, p->seqlen, p->dim, p->dstate, geo.DC, target);
     sscan::TiledArgs t{};
     t.batch = p->batch;
     t.L = p->seqlen;
@@ -240,8 +241,10 @@ cudaError_t aux_stream(AuxStream** out) {
     return cudaSuccess;
 }
 
-sscan_status run_fwd(const sscan_problem* p, const sscan::ScanArgs& a, void* ws, cudaStream_t st) {
-    if (tiled_ok(p, a)) return run_tiled(p, a, ws, st);
+// target: the split's target CTA count (kTiledTargetCtasCompact for the fixed scratch).
+sscan_status run_fwd(const sscan_problem* p, const sscan::ScanArgs& a, void* ws, cudaStream_t st,
+                     int64_t target = sscan::kTiledTargetCtas) {
+    if (tiled_ok(p, a)) return run_tiled(p, a, ws, st, target);
     return run_rows(p, a, ws, st);
 }
 
@@ -269,21 +272,22 @@ void cast_out(const float* src, void* dst, int64_t n, cudaStream_t st) {
 // Fixed device scratch for sscan_fwd_noalloc.  Every GPU that loads this library
 // holds these bytes until the process exits.  In host code the array's name is
 // only a host-side stand-in; its device address comes from cudaGetSymbolAddress.
-// 4 MiB covers every plan of the tiled path: fewer than kTiledMinCols CTA columns
-// times at most ceil(kTiledTargetCtas / cols) chunks bounds the chunk states by
+// 4 MiB covers every plan of the tiled path as this entry point plans it (with the
+// one-wave target kTiledTargetCtasCompact): fewer than kTiledMinCols CTA columns times at
+// most ceil(kTiledTargetCtasCompact / cols) chunks bounds the chunk states by
 // 1480 * DC * (N + 1) floats, at most 3.8 MB for N <= 16.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // The bound above, from plan_tiled's own constants: a split plan has cols < kTiledMinCols
-// CTA columns of DC channels and ceil(kTiledTargetCtas / cols) chunks, i.e. fewer than
-// kTiledTargetCtas + kTiledMinCols column-chunks, each holding DC * (N + 1) floats
+// CTA columns of DC channels and ceil(kTiledTargetCtasCompact / cols) chunks, i.e. fewer than
+// kTiledTargetCtasCompact + kTiledMinCols column-chunks, each holding DC * (N + 1) floats
 // (the chunk's end states and delta sum); DC * (N + 1) is largest at N = 4 (DC = 128).
 constexpr size_t tiled_scratch_bound() {
     size_t worst = 0;
     for (int n = 1; n <= sscan::kMaxState; ++n) {
         const size_t dc = n <= 4 ? 128 : (n <= 8 ? 64 : 32);
-        const size_t b = (size_t)(sscan::kTiledTargetCtas + sscan::kTiledMinCols - 1) * dc * (n + 1) * 4 + 255;
+        const size_t b = (size_t)(sscan::kTiledTargetCtasCompact + sscan::kTiledMinCols - 1) * dc * (n + 1) * 4 + 255;
         worst = b > worst ? b : worst;
     }
     return worst;
@@ -414,7 +418,8 @@ sscan_status sscan_fwd_noalloc(const sscan_problem* p, const void* u, const void
     // scratch of the path this call takes (run_fwd makes the same choice)
     const size_t need =
         tiled_ok(p, a) ? sscan::plan_tiled(p->batch, p->seqlen, p->dim, p->dstate,
-                                           sscan::tiled_geometry(p->batch, p->seqlen, p->dim, p->dstate).DC)
+                                           sscan::tiled_geometry(p->batch, p->seqlen, p->dim, p->dstate).DC,
+                                           sscan::kTiledTargetCtasCompact)
                              .workspace_bytes
                        : sscan::plan_fwd(p->batch, p->seqlen, p->dim, p->dstate).workspace_bytes;
     if (need > kNoAllocScratchBytes)
@@ -424,7 +429,7 @@ sscan_status sscan_fwd_noalloc(const sscan_problem* p, const void* u, const void
     if (need > 0) {
         if (sscan_status s = noalloc_scratch(&ws)) return s;
     }
-    return run_fwd(p, a, ws, st);
+    return run_fwd(p, a, ws, st, sscan::kTiledTargetCtasCompact);
 }
 
 sscan_status sscan_bwd(const sscan_problem* p, const void* u, const void* delta_raw,

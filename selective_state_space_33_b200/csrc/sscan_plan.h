@@ -49,15 +49,23 @@ inline FwdPlan plan_fwd(int64_t batch, int64_t L, int64_t D, int64_t N) {
 // Plan of the tiled forward kernel: CTAs cover DC channels of one batch; the
 // sequence is split only when there are too few CTA columns to occupy the GPU.
 constexpr int64_t kTiledMinCols = 2 * kSmCount;     // below this, split the sequence
-constexpr int64_t kTiledTargetCtas = 8 * kSmCount;  // CTAs resident at once (8 per SM)
+// Target CTA count of a split: chunks enough for several waves of 8 CTAs per SM.  The CTAs
+// of an SM finish in launch order, so a single wave of long chunks leaves the SMs short of
+// work for its last ~30%; shorter chunks over more waves keep them fed at the cost of a
+// longer carry (at the million-step shape: 8 per SM 19.50 ms, 16 17.49, 32 16.58, 64 16.28,
+// 128 16.26).  The fixed-scratch entry point plans with the one-wave target, which bounds
+// its chunk states (see kTiledTargetCtasCompact).
+constexpr int64_t kTiledTargetCtas = 64 * kSmCount;
+constexpr int64_t kTiledTargetCtasCompact = 8 * kSmCount;
 constexpr int64_t kTiledMinChunk = 1024;            // steps
 constexpr int64_t kTiledStep = 64;                  // chunk lengths are whole tiles of any length
 
-inline FwdPlan plan_tiled(int64_t batch, int64_t L, int64_t D, int64_t N, int64_t DC) {
+inline FwdPlan plan_tiled(int64_t batch, int64_t L, int64_t D, int64_t N, int64_t DC,
+                          int64_t target = kTiledTargetCtas) {
     FwdPlan p{1, L, 0, 0};
     const int64_t cols = batch * ((D + DC - 1) / DC);
     if (cols <= 0 || L <= 0 || cols >= kTiledMinCols) return p;
-    int64_t want = (kTiledTargetCtas + cols - 1) / cols;
+    int64_t want = (target + cols - 1) / cols;
     const int64_t most = L / kTiledMinChunk;
     if (want > most) want = most;
     if (want <= 1) return p;
